@@ -1,0 +1,206 @@
+"""The oracle -- TEST INFRASTRUCTURE, not product code.
+
+A plain CPU definition of the routed-MoE FFN forward (route -> budget ->
+dispatch -> SwiGLU expert FFN -> weighted combine + sigmoid-gated shared
+expert), written in C (``moe_oracle.c``) and wrapped here with ctypes.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline/reference
+legs of ``bench.py`` may import this package.  The CUDA library never calls
+it, and the two share no source.
+
+Each function follows a passage of the pages:
+  * SpecForge PR #943 (Qwen3.8-27B DSpark MoE drafter), "Modifications":
+    softmax router with renormalised top-k, sigmoid-gated shared expert,
+    grouped dispatch; its FFN parameter table fixes the gated FFN's shape.
+  * colibri issue_budget.md (EXPERT_BUDGET), "How it works" steps 1-5 and
+    "Safety": the batch-union expert budget.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to its source (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    i32 = ctypes.c_int32
+    lib.oracle_ffn_params.restype = ctypes.c_int64
+    lib.oracle_ffn_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    lib.oracle_route.argtypes = [i32, i32, i32, i32, P, P, P]
+    lib.oracle_budget.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P]
+    lib.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, P, P, P]
+    lib.oracle_expert_rows.argtypes = [i32, i32, P, P, P, i32, P, P, i32]
+    lib.oracle_shared_gate_row.restype = ctypes.c_double
+    lib.oracle_shared_gate_row.argtypes = [i32, P, P]
+    lib.oracle_forward.argtypes = [i32] * 8 + [P] * 9 + [i32, P, P] + [P] * 9 + [i32]
+    lib.oracle_max_threads.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def ffn_params(H: int, I: int) -> int:
+    """Parameters of one gated expert FFN (gate, up, down projections)."""
+    return int(_load().oracle_ffn_params(H, I))
+
+
+def route(logits: np.ndarray, k: int, norm_topk: bool = True):
+    """Softmax over all experts, top-k by logit, renormalised if norm_topk.
+
+    Returns (idx [T,k] int32, w [T,k] float32)."""
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    _check(_load().oracle_route(T, E, k, int(bool(norm_topk)), _ptr(logits), _ptr(idx), _ptr(w)), "route")
+    return idx, w
+
+
+def budget(idx: np.ndarray, w: np.ndarray, E: int, N: int, norm_topk: bool = True):
+    """EXPERT_BUDGET cap over the batch union (copies; inputs untouched).
+
+    Returns (idx, w, keff [T], kept [E] uint8, n_dropped)."""
+    idx = np.array(idx, np.int32, copy=True, order="C")
+    w = np.array(w, np.float32, copy=True, order="C")
+    T, k = idx.shape
+    keff = np.empty(T, np.int32)
+    kept = np.empty(E, np.uint8)
+    nd = np.zeros(1, np.int32)
+    _check(_load().oracle_budget(T, E, k, N, int(bool(norm_topk)), _ptr(idx), _ptr(w), _ptr(keff),
+                                 _ptr(kept), _ptr(nd)), "budget")
+    return idx, w, keff, kept, int(nd[0])
+
+
+def dispatch(idx: np.ndarray, keff: np.ndarray, E: int):
+    """Group kept slots by expert. Returns (counts, offsets, perm, slot_pos)."""
+    idx = _c(idx, np.int32)
+    keff = _c(keff, np.int32)
+    T, k = idx.shape
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    perm = np.full(max(T * k, 1), -1, np.int32)
+    slot_pos = np.empty(max(T * k, 1), np.int32)
+    _check(_load().oracle_dispatch(T, E, k, _ptr(idx), _ptr(keff), _ptr(counts), _ptr(offsets),
+                                   _ptr(perm), _ptr(slot_pos)), "dispatch")
+    total = int(offsets[E])
+    return counts, offsets, perm[:total].copy(), slot_pos[: T * k].copy()
+
+
+def expert_rows(wg: np.ndarray, wu: np.ndarray, wd: np.ndarray, x: np.ndarray, nthreads: int = 1):
+    """SwiGLU FFN of one expert on rows of x (all bf16 as uint16 bit patterns).
+
+    wg, wu: [I, H]; wd: [H, I]; x: [n, H].  Returns y [n, H] float64."""
+    wg, wu, wd, x = (_c(a, np.uint16) for a in (wg, wu, wd, x))
+    I, H = wg.shape
+    n = x.shape[0]
+    y = np.empty((n, H), np.float64)
+    _check(_load().oracle_expert_rows(H, I, _ptr(wg), _ptr(wu), _ptr(wd), n, _ptr(x), _ptr(y), nthreads),
+           "expert_rows")
+    return y
+
+
+def shared_gate(g: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """sigmoid(g . x_t) for every row of x (bf16 bit patterns)."""
+    g = _c(g, np.uint16)
+    x = _c(x, np.uint16)
+    lib = _load()
+    H = g.shape[0]
+    return np.array([lib.oracle_shared_gate_row(H, _ptr(g), _ptr(x[t])) for t in range(x.shape[0])])
+
+
+@dataclass
+class ForwardResult:
+    out: np.ndarray        # [n_rows, H] float64, rows in the order requested
+    idx: np.ndarray        # [T, k] int32 (after the budget)
+    w: np.ndarray          # [T, k] float32 (after the budget)
+    keff: np.ndarray       # [T] int32
+    kept: np.ndarray       # [E] uint8
+    n_dropped: int
+    counts: np.ndarray     # [E]
+    offsets: np.ndarray    # [E+1]
+    perm: np.ndarray       # [sum keff]
+    slot_pos: np.ndarray   # [T*k]
+
+
+def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, budget: int = 0,
+            ws_gate=None, ws_up=None, ws_down=None, ws_gvec=None, rows=None, nthreads: int = 1) -> ForwardResult:
+    """The whole layer. x and all weights are bf16 bit patterns (uint16).
+
+    x [T,H]; logits [T,E] f32; w_gate, w_up [E,I,H]; w_down [E,H,I];
+    shared (optional): ws_gate, ws_up [Is,H], ws_down [H,Is], ws_gvec [H].
+    rows: token ids whose output to compute (default: all)."""
+    x = _c(x, np.uint16)
+    logits = _c(logits, np.float32)
+    w_gate, w_up, w_down = (_c(a, np.uint16) for a in (w_gate, w_up, w_down))
+    T, H = x.shape
+    E, I, _ = w_gate.shape
+    Is = 0
+    if ws_gate is not None:
+        ws_gate, ws_up, ws_down, ws_gvec = (_c(a, np.uint16) for a in (ws_gate, ws_up, ws_down, ws_gvec))
+        Is = ws_gate.shape[0]
+    else:
+        ws_gate = ws_up = ws_down = ws_gvec = np.zeros(1, np.uint16)
+    rows = np.arange(T, dtype=np.int32) if rows is None else _c(rows, np.int32)
+    n_rows = rows.shape[0]
+    out = np.empty((max(n_rows, 1), H), np.float64)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    keff = np.empty(max(T, 1), np.int32)
+    kept = np.empty(E, np.uint8)
+    nd = np.zeros(1, np.int32)
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    perm = np.full(max(T * k, 1), -1, np.int32)
+    slot_pos = np.empty(max(T * k, 1), np.int32)
+    rc = _load().oracle_forward(
+        T, H, E, I, k, Is, int(bool(norm_topk)), budget,
+        _ptr(x), _ptr(logits), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec),
+        n_rows, _ptr(rows), _ptr(out),
+        _ptr(idx), _ptr(w), _ptr(keff), _ptr(kept), _ptr(nd),
+        _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(slot_pos), nthreads)
+    _check(rc, "forward")
+    total = int(offsets[E])
+    return ForwardResult(out[:n_rows], idx, w, keff[:T], kept, int(nd[0]), counts, offsets,
+                         perm[:total].copy(), slot_pos[: T * k].copy())
