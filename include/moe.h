@@ -1,0 +1,196 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed Mixture-of-Experts FFN forward.
+ *
+ * The layer, for a batch of T tokens x_t (hidden size H):
+ *   route    softmax over the E router logits of each token, the k largest
+ *            logits kept, their probabilities renormalised to sum 1 when
+ *            norm_topk is set;
+ *   budget   optional cap N on the number of distinct experts the whole
+ *            batch uses: when the batch union holds more than N experts,
+ *            only the N with the highest aggregate gate weight survive and
+ *            each token's remaining weights are renormalised;
+ *   dispatch the kept (token, slot) pairs grouped by expert;
+ *   FFN      per expert e: y = W_down[e] (silu(W_gate[e] x) * (W_up[e] x));
+ *   combine  out_t = sum_j w_tj y_tj + sigmoid(g . x_t) FFN_shared(x_t).
+ *
+ * Passages that define the operation (web pages, by title and section):
+ *   SpecForge PR #943, "Qwen3.8-27B DSpark MoE drafter with 16 x 1024 top-2
+ *     experts", section "Modifications": the config keys hidden,
+ *     n_routed_experts, moe_intermediate_size, num_experts_per_tok, the
+ *     2048-wide sigmoid-gated shared expert, the softmax router with
+ *     renormalised top-k ("qwen3_5_moe preset") and grouped_mm dispatch;
+ *     its FFN parameter table (3*H*I parameters per expert).
+ *   colibri issue_budget.md, "EXPERT_BUDGET", section "How it works", steps
+ *     1-5 (the budget) and section "Safety" (off by default, dropped experts
+ *     omitted and the rest renormalised).
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, row-major and densely packed.  bf16 values are passed as
+ *     their 16-bit patterns (moe_bf16_t).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  All
+ *     work is enqueued on it; no entry point synchronises, allocates device
+ *     or host memory, or keeps state between calls, so calls on different
+ *     streams with different buffers may run concurrently.
+ *   - T = 0 is a no-op returning MOE_OK.
+ *   - Return codes: MOE_OK, or a negative MOE_ERR_* below; nothing is
+ *     launched when an argument check fails.
+ *   - Limits: 1 <= E <= 1024; 1 <= k <= min(E, 32); H % 128 == 0;
+ *     I % 64 == 0; Is % 64 == 0 (Is = 0: no shared expert); budget >= 0;
+ *     0 <= T and T * (k + 1) * H < 2^31.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t; /* bf16 bit pattern */
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)   /* null/misaligned pointer, bad size or flag */
+#define MOE_ERR_UNSUPPORTED (-2)   /* shape outside the limits above, or no sm_100 device */
+#define MOE_ERR_WORKSPACE (-3)     /* ws_bytes < moe_workspace_bytes(cfg, T) */
+#define MOE_ERR_CUDA (-4)          /* a CUDA launch or driver call failed */
+#define MOE_ERR_DEVICE (-5)        /* a kernel reported an error in the status word */
+
+/* Bits of the device status word (see moe_status_read). */
+#define MOE_STATUS_TIMEOUT 1       /* a pipeline wait ran past its limit; results invalid */
+
+typedef struct {
+    int32_t hidden;                   /* H */
+    int32_t n_routed_experts;         /* E */
+    int32_t moe_intermediate_size;    /* I */
+    int32_t num_experts_per_tok;      /* k */
+    int32_t shared_intermediate_size; /* Is; 0 = no shared expert */
+    int32_t norm_topk;                /* 1: renormalise the kept weights to sum 1 */
+    int32_t budget;                   /* N (EXPERT_BUDGET); 0 = off */
+} moe_config_t;
+
+typedef struct {
+    const moe_bf16_t *w_gate;      /* [E, I, H] routed gate projections */
+    const moe_bf16_t *w_up;        /* [E, I, H] routed up projections */
+    const moe_bf16_t *w_down;      /* [E, H, I] routed down projections */
+    const moe_bf16_t *ws_gate;     /* [Is, H] shared gate projection, NULL if Is = 0 */
+    const moe_bf16_t *ws_up;       /* [Is, H] shared up projection, NULL if Is = 0 */
+    const moe_bf16_t *ws_down;     /* [H, Is] shared down projection, NULL if Is = 0 */
+    const moe_bf16_t *ws_gate_vec; /* [H] shared-expert gate vector g, NULL if Is = 0 */
+} moe_weights_t;
+
+/* Optional device outputs of moe_forward; any NULL member is kept inside
+ * the workspace instead. */
+typedef struct {
+    int32_t *topk_idx;     /* [T, k] */
+    float *topk_w;         /* [T, k] */
+    float *sgate;          /* [T]    (Is > 0 only) */
+    int32_t *keff;         /* [T]    */
+    uint8_t *expert_kept;  /* [E]    (written only when budget > 0) */
+    int32_t *n_dropped;    /* [1]    (written only when budget > 0) */
+    int32_t *counts;       /* [E]    */
+    int32_t *offsets;      /* [E+1]  */
+    int32_t *perm;         /* [T*k]  first offsets[E] entries valid */
+    int32_t *slot_pos;     /* [T*k]  */
+} moe_aux_t;
+
+/* Bytes of device workspace the calls below need for a batch of T tokens
+ * (0 for an invalid config).  The workspace is caller-allocated scratch;
+ * its first 256 bytes hold the status word.  Clear the status word once
+ * after allocating (moe_status_clear). */
+size_t moe_workspace_bytes(const moe_config_t *cfg, int32_t T);
+
+/* Route: for each token t, topk_idx[t, 0..k) = the k experts with the
+ * largest logits (descending; equal logits: lower expert id first),
+ * topk_w[t, j] = softmax(logits[t])[topk_idx[t, j]], divided by the sum of
+ * the k kept probabilities when cfg->norm_topk.  When sgate != NULL (needs
+ * Is > 0, x and ws_gate_vec), sgate[t] = sigmoid(ws_gate_vec . x_t).  When
+ * keff != NULL, keff[t] = k.
+ *   logits [T, E] f32; x [T, H]; ws_gate_vec [H]; topk_idx [T, k] i32;
+ *   topk_w [T, k] f32; sgate [T] f32; keff [T] i32. */
+int moe_route(const moe_config_t *cfg, int32_t T, const float *logits, const moe_bf16_t *x,
+              const moe_bf16_t *ws_gate_vec, int32_t *topk_idx, float *topk_w, float *sgate,
+              int32_t *keff, void *stream);
+
+/* Budget (EXPERT_BUDGET, colibri issue_budget.md "How it works"): works in
+ * place on the router output topk_idx/topk_w [T, k].  Let U be the set of
+ * experts any token routes to.  When cfg->budget > 0 and |U| > budget:
+ * agg[e] = sum of the weights routed to e (tokens, then slots, ascending);
+ * the budget experts first in (agg descending, id ascending) are kept;
+ * every token's kept slots move to the front in their original order, the
+ * tail becomes (idx -1, w 0), keff[t] = kept slots, and a token that lost a
+ * slot has its kept weights divided by their sum when cfg->norm_topk.
+ * Otherwise topk_idx/topk_w are unchanged and keff[t] = k.
+ * expert_kept[e] = 1 for experts of the final union; *n_dropped = |U| -
+ * budget or 0.  keff [T] i32; expert_kept [E] u8; n_dropped [1] i32 (all
+ * device).  Uses the workspace. */
+int moe_budget(const moe_config_t *cfg, int32_t T, int32_t *topk_idx, float *topk_w, int32_t *keff,
+               uint8_t *expert_kept, int32_t *n_dropped, void *ws, size_t ws_bytes, void *stream);
+
+/* Dispatch: groups the kept slots s = t*k + j (j < keff[t]; keff == NULL
+ * means every slot) by expert, bit-exactly:
+ *   counts[e] = kept slots routed to e; offsets[0] = 0,
+ *   offsets[e+1] = offsets[e] + counts[e];
+ *   perm[offsets[e] ..] = those slot ids in ascending order;
+ *   slot_pos[s] = position of slot s in perm, -1 for a dropped slot;
+ *   x_perm[p, :] = x[perm[p] / k, :] when x_perm != NULL.
+ * topk_idx [T, k]; keff [T]; x [T, H]; counts [E]; offsets [E+1];
+ * perm [T*k]; slot_pos [T*k]; x_perm [T*k, H].  Uses the workspace. */
+int moe_dispatch(const moe_config_t *cfg, int32_t T, const int32_t *topk_idx, const int32_t *keff,
+                 const moe_bf16_t *x, int32_t *counts, int32_t *offsets, int32_t *perm,
+                 int32_t *slot_pos, moe_bf16_t *x_perm, void *ws, size_t ws_bytes, void *stream);
+
+/* Expert FFN over the dispatched tokens (tcgen05 grouped GEMMs), writing the
+ * weighted per-slot outputs in token order:
+ *   ybuf[t, j, :] = topk_w[t, j] * FFN_{topk_idx[t, j]}(x_t)   for each kept slot,
+ *   ybuf[t, k, :] = sgate[t] * FFN_shared(x_t)                  when Is > 0,
+ * rounded to bf16; other rows of ybuf are left untouched.
+ * x [T, H] (read for the shared expert); x_perm [T*k, H] and offsets, perm
+ * from moe_dispatch; topk_w [T, k]; sgate [T] (Is > 0); ybuf [T, k+1, H].
+ * Uses the workspace (intermediate activations, status word). */
+int moe_expert_ffn(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                   const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                   const moe_weights_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, void *stream);
+
+/* The two phases of moe_expert_ffn, for callers that time or overlap them:
+ * gate_up computes h = silu(W_gate x) * (W_up x) for every dispatched row
+ * (and the shared expert's rows) into the workspace; down reads h from the
+ * same workspace and writes ybuf as moe_expert_ffn does.  Arguments as in
+ * moe_expert_ffn. */
+int moe_expert_gate_up(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                       const int32_t *offsets, const moe_weights_t *w, void *ws, size_t ws_bytes, void *stream);
+int moe_expert_down(const moe_config_t *cfg, int32_t T, const int32_t *offsets, const int32_t *perm,
+                    const float *topk_w, const float *sgate, const moe_weights_t *w, moe_bf16_t *ybuf, void *ws,
+                    size_t ws_bytes, void *stream);
+
+/* Combine: out[t, :] = bf16( sum_{j < keff[t]} ybuf[t, j, :] + [Is > 0] ybuf[t, k, :] ),
+ * summed in fp32 in slot order and rounded once (a token with no kept slot
+ * and no shared expert gets 0).  keff == NULL means k.
+ * ybuf [T, k+1, H]; keff [T]; out [T, H]. */
+int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, const int32_t *keff,
+                moe_bf16_t *out, void *stream);
+
+/* The whole layer: route -> budget (if cfg->budget > 0) -> dispatch ->
+ * expert FFN -> combine, enqueued on one stream with no host sync.
+ * x [T, H]; logits [T, E] f32; out [T, H]; aux may be NULL. */
+int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
+                const moe_weights_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
+                size_t ws_bytes, void *stream);
+
+/* Status word: MOE_STATUS_* bits set by kernels (sticky until cleared).
+ * moe_status_read enqueues a copy on `stream`, waits for the stream, and
+ * returns MOE_OK with *status_out filled (host pointer).  moe_status_clear
+ * enqueues a reset of the word on `stream`. */
+int moe_status_read(const void *ws, int32_t *status_out, void *stream);
+int moe_status_clear(void *ws, void *stream);
+
+/* Static text for a return code. */
+const char *moe_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H */

@@ -57,7 +57,8 @@ def _load():
     lib.oracle_expert_rows.argtypes = [i32, i32, P, P, P, i32, P, P, i32]
     lib.oracle_shared_gate_row.restype = ctypes.c_double
     lib.oracle_shared_gate_row.argtypes = [i32, P, P]
-    lib.oracle_forward.argtypes = [i32] * 8 + [P] * 9 + [i32, P, P] + [P] * 9 + [i32]
+    lib.oracle_forward.argtypes = [i32] * 8 + [P] * 9 + [i32, P, P] + [P] * 9 + [i32]  # pointer arrays pass as P
+    lib.oracle_combine_rows.argtypes = [i32] * 5 + [P] * 4 + [P] * 3 + [P] * 4 + [i32, P, P, i32]
     lib.oracle_max_threads.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -163,18 +164,43 @@ class ForwardResult:
     slot_pos: np.ndarray   # [T*k]
 
 
+def _expert_ptrs(w, E):
+    """Per-expert pointer array from a full [E, ...] array or a dict {e: array}."""
+    arr = (ctypes.c_void_p * E)()
+    keep = []
+    if isinstance(w, dict):
+        for e, a in w.items():
+            a = _c(a, np.uint16)
+            keep.append(a)
+            arr[e] = a.ctypes.data
+    else:
+        a = _c(w, np.uint16)
+        keep.append(a)
+        step = a[0].nbytes if E else 0
+        for e in range(E):
+            arr[e] = a.ctypes.data + e * step
+    return arr, keep
+
+
 def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, budget: int = 0,
-            ws_gate=None, ws_up=None, ws_down=None, ws_gvec=None, rows=None, nthreads: int = 1) -> ForwardResult:
+            ws_gate=None, ws_up=None, ws_down=None, ws_gvec=None, rows=None, nthreads: int = 1,
+            I: int = None) -> ForwardResult:
     """The whole layer. x and all weights are bf16 bit patterns (uint16).
 
-    x [T,H]; logits [T,E] f32; w_gate, w_up [E,I,H]; w_down [E,H,I];
+    x [T,H]; logits [T,E] f32; w_gate, w_up [E,I,H] and w_down [E,H,I] as full
+    arrays, or as dicts {expert: [I,H] / [H,I] array} holding only the experts
+    the requested rows route to (then pass I);
     shared (optional): ws_gate, ws_up [Is,H], ws_down [H,Is], ws_gvec [H].
     rows: token ids whose output to compute (default: all)."""
     x = _c(x, np.uint16)
     logits = _c(logits, np.float32)
-    w_gate, w_up, w_down = (_c(a, np.uint16) for a in (w_gate, w_up, w_down))
     T, H = x.shape
-    E, I, _ = w_gate.shape
+    E = logits.shape[1]
+    if I is None:
+        I = w_gate.shape[1]
+    pg, kg = _expert_ptrs(w_gate, E)
+    pu, ku = _expert_ptrs(w_up, E)
+    pd, kd = _expert_ptrs(w_down, E)
     Is = 0
     if ws_gate is not None:
         ws_gate, ws_up, ws_down, ws_gvec = (_c(a, np.uint16) for a in (ws_gate, ws_up, ws_down, ws_gvec))
@@ -195,7 +221,7 @@ def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, 
     slot_pos = np.empty(max(T * k, 1), np.int32)
     rc = _load().oracle_forward(
         T, H, E, I, k, Is, int(bool(norm_topk)), budget,
-        _ptr(x), _ptr(logits), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(x), _ptr(logits), pg, pu, pd,
         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec),
         n_rows, _ptr(rows), _ptr(out),
         _ptr(idx), _ptr(w), _ptr(keff), _ptr(kept), _ptr(nd),
@@ -204,3 +230,38 @@ def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, 
     total = int(offsets[E])
     return ForwardResult(out[:n_rows], idx, w, keff[:T], kept, int(nd[0]), counts, offsets,
                          perm[:total].copy(), slot_pos[: T * k].copy())
+
+
+def combine_rows(x, idx, w, keff, w_gate, w_up, w_down, *, I: int, ws_gate=None, ws_up=None, ws_down=None,
+                 ws_gvec=None, rows=None, nthreads: int = 1) -> np.ndarray:
+    """Expert FFN + weighted combine (+ gated shared expert) for GIVEN routing
+    (idx/w/keff, e.g. after a budget), for the listed token rows.  Weights as
+    in forward().  Returns out [n_rows, H] float64."""
+    x = _c(x, np.uint16)
+    idx = _c(idx, np.int32)
+    w = _c(w, np.float32)
+    keff = _c(keff, np.int32)
+    T, H = x.shape
+    k = idx.shape[1]
+    if isinstance(w_gate, dict):  # pointer table must cover every expert id idx can name
+        E = max(max(w_gate, default=0), int(idx.max(initial=0))) + 1
+    else:
+        E = w_gate.shape[0]
+        if idx.size and int(idx.max()) >= E:
+            raise ValueError("routing names an expert outside the weight arrays")
+    pg, kg = _expert_ptrs(w_gate, E)
+    pu, ku = _expert_ptrs(w_up, E)
+    pd, kd = _expert_ptrs(w_down, E)
+    Is = 0
+    if ws_gate is not None:
+        ws_gate, ws_up, ws_down, ws_gvec = (_c(a, np.uint16) for a in (ws_gate, ws_up, ws_down, ws_gvec))
+        Is = ws_gate.shape[0]
+    else:
+        ws_gate = ws_up = ws_down = ws_gvec = np.zeros(1, np.uint16)
+    rows = np.arange(T, dtype=np.int32) if rows is None else _c(rows, np.int32)
+    out = np.empty((max(rows.shape[0], 1), H), np.float64)
+    _check(_load().oracle_combine_rows(T, H, I, k, Is, _ptr(x), _ptr(idx), _ptr(w), _ptr(keff), pg, pu, pd,
+                                       _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec),
+                                       rows.shape[0], _ptr(rows), _ptr(out), nthreads), "combine_rows")
+    return out[: rows.shape[0]]
+

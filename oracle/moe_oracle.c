@@ -266,37 +266,27 @@ double oracle_shared_gate_row(int32_t H, const uint16_t *g, const uint16_t *x)
 }
 
 /* ---------------------------------------------------------------------- */
-/* Whole layer, for a chosen set of output rows.                           */
+/* Expert FFN + combine for given routing, for a chosen set of rows.       */
 /* ---------------------------------------------------------------------- */
-/* Routing, budget and dispatch run over all T tokens (the budget couples
- * tokens); the FFN and the combine run only for the n_rows tokens listed in
- * rows[], writing out[r, :] for token rows[r]:
- *   out_t = sum_{j < keff[t]} w[t, j] * FFN_{idx[t, j]}(x_t)
- *         + [Is > 0] * sigmoid(g . x_t) * FFN_shared(x_t).
- * Weights: w_gate, w_up [E, I, H]; w_down [E, H, I]; ws_gate, ws_up [Is, H];
- * ws_down [H, Is]; ws_gvec [H] (all bf16 bit patterns, row-major).
- * The routing outputs (idx, w, keff, kept, n_dropped) and dispatch outputs
- * (counts, offsets, perm, slot_pos) are written for the whole batch. */
-int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_t Is,
-                   int32_t norm_topk, int32_t budget,
-                   const uint16_t *x, const float *logits,
-                   const uint16_t *w_gate, const uint16_t *w_up, const uint16_t *w_down,
-                   const uint16_t *ws_gate, const uint16_t *ws_up, const uint16_t *ws_down,
-                   const uint16_t *ws_gvec,
-                   int32_t n_rows, const int32_t *rows, double *out,
-                   int32_t *idx, float *w, int32_t *keff, uint8_t *kept, int32_t *n_dropped,
-                   int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
-                   int32_t nthreads)
+/* For each listed token t = rows[r]:
+ *   out[r, :] = sum_{j < keff[t]} w[t, j] * FFN_{idx[t, j]}(x_t)
+ *             + [Is > 0] * sigmoid(g . x_t) * FFN_shared(x_t)
+ * (slots summed in order, the shared expert last, all in fp64).
+ * Weights: w_gate[e], w_up[e] point to expert e's [I, H] projections and
+ * w_down[e] to its [H, I] projection (an entry may be NULL when no listed
+ * row routes to e); ws_gate, ws_up [Is, H]; ws_down [H, Is]; ws_gvec [H]
+ * (all bf16 bit patterns, row-major). */
+int oracle_combine_rows(int32_t T, int32_t H, int32_t I, int32_t k, int32_t Is,
+                        const uint16_t *x, const int32_t *idx, const float *w, const int32_t *keff,
+                        const uint16_t *const *w_gate, const uint16_t *const *w_up,
+                        const uint16_t *const *w_down,
+                        const uint16_t *ws_gate, const uint16_t *ws_up, const uint16_t *ws_down,
+                        const uint16_t *ws_gvec,
+                        int32_t n_rows, const int32_t *rows, double *out, int32_t nthreads)
 {
-    if (T < 0 || H < 1 || E < 1 || I < 1 || k < 1 || k > E || Is < 0 || budget < 0 || n_rows < 0)
-        return ORACLE_EINVAL;
-    int rc = oracle_route(T, E, k, norm_topk, logits, idx, w);
-    if (rc) return rc;
-    rc = oracle_budget(T, E, k, budget, norm_topk, idx, w, keff, kept, n_dropped);
-    if (rc) return rc;
-    rc = oracle_dispatch(T, E, k, idx, keff, counts, offsets, perm, slot_pos);
-    if (rc) return rc;
-
+    if (T < 0 || H < 1 || I < 1 || k < 1 || Is < 0 || n_rows < 0) return ORACLE_EINVAL;
+    for (int32_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= T) return ORACLE_EINVAL;
     const int32_t per_tok = k + (Is > 0 ? 1 : 0);
     const int32_t n_jobs = n_rows * per_tok;
     double *ys = (double *)malloc(sizeof(double) * (size_t)(n_jobs > 0 ? n_jobs : 1) * H);
@@ -318,8 +308,12 @@ int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_
                 if (j < k) {
                     if (j >= keff[t]) continue;
                     int32_t e = idx[(size_t)t * k + j];
-                    swiglu_ffn(H, I, w_gate + (size_t)e * I * H, w_up + (size_t)e * I * H,
-                               w_down + (size_t)e * H * I, xt, hbuf, y);
+                    if (e < 0 || !w_gate[e] || !w_up[e] || !w_down[e]) {
+#pragma omp atomic write
+                        err = 2;
+                        continue;
+                    }
+                    swiglu_ffn(H, I, w_gate[e], w_up[e], w_down[e], xt, hbuf, y);
                 } else {
                     swiglu_ffn(H, Is, ws_gate, ws_up, ws_down, xt, hbuf, y);
                 }
@@ -327,7 +321,7 @@ int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_
         }
         free(hbuf);
     }
-    if (err) { free(ys); return ORACLE_ENOMEM; }
+    if (err) { free(ys); return err == 2 ? ORACLE_EINVAL : ORACLE_ENOMEM; }
     /* combine: weighted sum in slot order, then the gated shared expert */
     for (int32_t r = 0; r < n_rows; ++r) {
         int32_t t = rows[r];
@@ -346,6 +340,34 @@ int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_
     }
     free(ys);
     return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Whole layer: route -> budget -> dispatch over all T tokens (the budget  */
+/* couples tokens), then FFN + combine for the listed rows.                */
+/* ---------------------------------------------------------------------- */
+int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_t Is,
+                   int32_t norm_topk, int32_t budget,
+                   const uint16_t *x, const float *logits,
+                   const uint16_t *const *w_gate, const uint16_t *const *w_up,
+                   const uint16_t *const *w_down,
+                   const uint16_t *ws_gate, const uint16_t *ws_up, const uint16_t *ws_down,
+                   const uint16_t *ws_gvec,
+                   int32_t n_rows, const int32_t *rows, double *out,
+                   int32_t *idx, float *w, int32_t *keff, uint8_t *kept, int32_t *n_dropped,
+                   int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
+                   int32_t nthreads)
+{
+    if (T < 0 || H < 1 || E < 1 || I < 1 || k < 1 || k > E || Is < 0 || budget < 0 || n_rows < 0)
+        return ORACLE_EINVAL;
+    int rc = oracle_route(T, E, k, norm_topk, logits, idx, w);
+    if (rc) return rc;
+    rc = oracle_budget(T, E, k, budget, norm_topk, idx, w, keff, kept, n_dropped);
+    if (rc) return rc;
+    rc = oracle_dispatch(T, E, k, idx, keff, counts, offsets, perm, slot_pos);
+    if (rc) return rc;
+    return oracle_combine_rows(T, H, I, k, Is, x, idx, w, keff, w_gate, w_up, w_down,
+                               ws_gate, ws_up, ws_down, ws_gvec, n_rows, rows, out, nthreads);
 }
 
 int oracle_max_threads(void)

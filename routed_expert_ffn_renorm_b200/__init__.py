@@ -1,0 +1,251 @@
+"""B200 (sm_100a) routed Mixture-of-Experts FFN forward.
+
+Thin Python binding over the C ABI of ``libmoe.so`` (declared in
+``include/moe.h``): the functions below have the C entry points' names and
+only marshal arguments -- torch tensors in, device pointers and the current
+CUDA stream out.  Every step of the layer runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and a missing or unbuildable
+library raises.
+
+    cfg = MoEConfig(hidden=5120, n_routed_experts=16, moe_intermediate_size=1024,
+                    num_experts_per_tok=2, shared_intermediate_size=2048)
+    ws = torch.empty(workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    status_clear(ws)
+    moe_forward(cfg, x, logits, weights, out, ws)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional
+
+__all__ = [
+    "MoEConfig", "MoEWeights", "MoEError", "load_library", "workspace_bytes", "moe_route", "moe_budget",
+    "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_forward",
+    "status_read", "status_clear",
+    "EXPORTED_SYMBOLS", "MOE_STATUS_TIMEOUT",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+EXPORTED_SYMBOLS = (
+    "moe_workspace_bytes", "moe_route", "moe_budget", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+    "moe_forward", "moe_status_read", "moe_status_clear", "moe_error_string", "moe_expert_gate_up",
+    "moe_expert_down",
+)
+MOE_STATUS_TIMEOUT = 1
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {msg} (code {code})")
+        self.code = code
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "hidden", "n_routed_experts", "moe_intermediate_size", "num_experts_per_tok",
+        "shared_intermediate_size", "norm_topk", "budget")]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec")]
+
+
+class _Aux(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "topk_idx", "topk_w", "sgate", "keff", "expert_kept", "n_dropped", "counts", "offsets", "perm",
+        "slot_pos")]
+
+
+@dataclass(frozen=True)
+class MoEConfig:
+    """The layer's configuration keys (names as in the drafter config files)."""
+    hidden: int
+    n_routed_experts: int
+    moe_intermediate_size: int
+    num_experts_per_tok: int
+    shared_intermediate_size: int = 0
+    norm_topk: bool = True
+    budget: int = 0
+
+    def _c(self) -> _Config:
+        return _Config(self.hidden, self.n_routed_experts, self.moe_intermediate_size, self.num_experts_per_tok,
+                       self.shared_intermediate_size, int(bool(self.norm_topk)), self.budget)
+
+
+@dataclass
+class MoEWeights:
+    """Device bf16 weights: w_gate, w_up [E, I, H]; w_down [E, H, I];
+    optional shared expert ws_gate, ws_up [Is, H], ws_down [H, Is], ws_gate_vec [H]."""
+    w_gate: "torch.Tensor"
+    w_up: "torch.Tensor"
+    w_down: "torch.Tensor"
+    ws_gate: Optional["torch.Tensor"] = None
+    ws_up: Optional["torch.Tensor"] = None
+    ws_down: Optional["torch.Tensor"] = None
+    ws_gate_vec: Optional["torch.Tensor"] = None
+
+    def _c(self) -> _Weights:
+        return _Weights(*(_ptr(getattr(self, n), allow_none=True) for n in (
+            "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec")))
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library(build_if_stale: bool = True):
+    """Load libmoe.so (building it first when missing or older than its sources)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if build_if_stale:
+            from . import _build
+            if _build.stale():
+                _build.build()
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m routed_expert_ffn_renorm_b200._build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        cfg = ctypes.POINTER(_Config)
+        lib.moe_workspace_bytes.restype = sz
+        lib.moe_workspace_bytes.argtypes = [cfg, i32]
+        lib.moe_route.argtypes = [cfg, i32, P, P, P, P, P, P, P, P]
+        lib.moe_budget.argtypes = [cfg, i32, P, P, P, P, P, P, sz, P]
+        lib.moe_dispatch.argtypes = [cfg, i32, P, P, P, P, P, P, P, P, P, sz, P]
+        lib.moe_expert_ffn.argtypes = [cfg, i32, P, P, P, P, P, P, ctypes.POINTER(_Weights), P, P, sz, P]
+        lib.moe_combine.argtypes = [cfg, i32, P, P, P, P]
+        lib.moe_expert_gate_up.argtypes = [cfg, i32, P, P, P, ctypes.POINTER(_Weights), P, sz, P]
+        lib.moe_expert_down.argtypes = [cfg, i32, P, P, P, P, ctypes.POINTER(_Weights), P, P, sz, P]
+        lib.moe_forward.argtypes = [cfg, i32, P, P, ctypes.POINTER(_Weights), P, ctypes.POINTER(_Aux), P, sz, P]
+        lib.moe_status_read.argtypes = [P, ctypes.POINTER(i32), P]
+        lib.moe_status_clear.argtypes = [P, P]
+        lib.moe_error_string.restype = ctypes.c_char_p
+        lib.moe_error_string.argtypes = [ctypes.c_int]
+        for name in EXPORTED_SYMBOLS:
+            if name not in ("moe_workspace_bytes", "moe_error_string"):
+                getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _ptr(t, allow_none: bool = False):
+    if t is None:
+        if allow_none:
+            return None
+        raise ValueError("tensor argument is None")
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"expected a torch.Tensor, got {type(t).__name__}")
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        msg = load_library().moe_error_string(rc).decode()
+        raise MoEError(fn, rc, msg)
+
+
+def workspace_bytes(cfg: MoEConfig, T: int) -> int:
+    n = load_library().moe_workspace_bytes(ctypes.byref(cfg._c()), T)
+    if n == 0:
+        raise MoEError("moe_workspace_bytes", -1, "invalid configuration")
+    return int(n)
+
+
+def moe_route(cfg: MoEConfig, logits, topk_idx, topk_w, *, x=None, ws_gate_vec=None, sgate=None, keff=None,
+              stream=None):
+    T = logits.shape[0]
+    _check("moe_route", load_library().moe_route(
+        ctypes.byref(cfg._c()), T, _ptr(logits), _ptr(x, True), _ptr(ws_gate_vec, True), _ptr(topk_idx),
+        _ptr(topk_w), _ptr(sgate, True), _ptr(keff, True), _stream(stream)))
+
+
+def moe_budget(cfg: MoEConfig, topk_idx, topk_w, keff, expert_kept, n_dropped, ws, stream=None):
+    T = topk_idx.shape[0]
+    _check("moe_budget", load_library().moe_budget(
+        ctypes.byref(cfg._c()), T, _ptr(topk_idx), _ptr(topk_w), _ptr(keff), _ptr(expert_kept), _ptr(n_dropped),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_dispatch(cfg: MoEConfig, topk_idx, counts, offsets, perm, slot_pos, ws, *, keff=None, x=None, x_perm=None,
+                 stream=None):
+    T = topk_idx.shape[0]
+    _check("moe_dispatch", load_library().moe_dispatch(
+        ctypes.byref(cfg._c()), T, _ptr(topk_idx), _ptr(keff, True), _ptr(x, True), _ptr(counts), _ptr(offsets),
+        _ptr(perm), _ptr(slot_pos), _ptr(x_perm, True), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_expert_ffn(cfg: MoEConfig, x, x_perm, offsets, perm, topk_w, weights: MoEWeights, ybuf, ws, *, sgate=None,
+                   stream=None):
+    T = x.shape[0]
+    w = weights._c()
+    _check("moe_expert_ffn", load_library().moe_expert_ffn(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(perm), _ptr(topk_w),
+        _ptr(sgate, True), ctypes.byref(w), _ptr(ybuf), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_expert_gate_up(cfg: MoEConfig, x, x_perm, offsets, weights: MoEWeights, ws, stream=None):
+    T = x.shape[0]
+    w = weights._c()
+    _check("moe_expert_gate_up", load_library().moe_expert_gate_up(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(x_perm), _ptr(offsets), ctypes.byref(w), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_expert_down(cfg: MoEConfig, T: int, offsets, perm, topk_w, weights: MoEWeights, ybuf, ws, *, sgate=None,
+                    stream=None):
+    w = weights._c()
+    _check("moe_expert_down", load_library().moe_expert_down(
+        ctypes.byref(cfg._c()), T, _ptr(offsets), _ptr(perm), _ptr(topk_w), _ptr(sgate, True), ctypes.byref(w),
+        _ptr(ybuf), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_combine(cfg: MoEConfig, ybuf, out, *, keff=None, stream=None):
+    T = out.shape[0]
+    _check("moe_combine", load_library().moe_combine(
+        ctypes.byref(cfg._c()), T, _ptr(ybuf), _ptr(keff, True), _ptr(out), _stream(stream)))
+
+
+def moe_forward(cfg: MoEConfig, x, logits, weights: MoEWeights, out, ws, *, aux: Optional[dict] = None,
+                stream=None):
+    """The whole layer on the current stream.  ``aux`` may map moe_aux_t
+    member names (topk_idx, topk_w, sgate, keff, expert_kept, n_dropped,
+    counts, offsets, perm, slot_pos) to device tensors to receive them."""
+    T = x.shape[0]
+    w = weights._c()
+    a = _Aux()
+    if aux:
+        for name, t in aux.items():
+            setattr(a, name, _ptr(t))
+    _check("moe_forward", load_library().moe_forward(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(logits), ctypes.byref(w), _ptr(out), ctypes.byref(a), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def status_read(ws, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check("moe_status_read", load_library().moe_status_read(_ptr(ws), ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+def status_clear(ws, stream=None):
+    _check("moe_status_clear", load_library().moe_status_clear(_ptr(ws), _stream(stream)))

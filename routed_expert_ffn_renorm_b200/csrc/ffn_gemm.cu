@@ -1,0 +1,678 @@
+// Grouped expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA.  Two launches of one persistent, warp-specialised kernel:
+//
+//   gated (GEMM1):  h[p, i] = silu(W_gate[e] x_p)_i * (W_up[e] x_p)_i
+//   down  (GEMM2):  ybuf[row(p), :] = w_p * (W_down[e] h_p)
+//
+// for every dispatched row p of expert e (SpecForge PR #943,
+// "Modifications": gated expert FFN, grouped dispatch; its parameter table
+// fixes gate/up/down of H x I each), and the same for the shared expert,
+// whose rows are all T tokens in token order and whose weight is the
+// sigmoid gate.
+//
+// Orientation ("swap AB").  The weights sit in the MMA M slot (128 weight
+// rows per tile) and the tokens of one expert in the N slot (16..256 per
+// tile), so a group of 3 tokens costs an N=16 MMA, not a 128-row padded
+// tile: the decode-sized batches of the drafter layers stream weights and
+// barely touch the tensor pipe, the large batches fill N = 256.
+//   gated tile: A = [64 gate rows ; 64 up rows] of the same intermediate
+//               indices, so gate and up of index i land in TMEM lanes i and
+//               64 + i and the epilogue pairs them through shared memory;
+//   down tile:  A = 128 rows of W_down (128 output columns).
+// Both operands are K-major bf16 in 128-byte-swizzled shared memory, loaded
+// by TMA boxes of 64 K-elements; the accumulator is fp32 in TMEM, double
+// buffered (2 x BN columns) so the epilogue of one tile overlaps the
+// mainloop of the next.
+//
+// Roles (192 threads, one CTA per SM, persistent over a static stride of
+// work items):  warp 0 -- TMA producer (one lane); warp 1 -- TMEM
+// allocation and MMA issue (one lane); warps 2..5 -- epilogue, one TMEM lane
+// quarter each.
+//
+// Work items are (expert, weight tile r, token tile j) ordered by expert,
+// then r, then j, so the token tiles that reuse a weight tile run side by
+// side (one HBM read, L2 hits) and the tile list is derived in-kernel from
+// the dispatch offsets -- no host sync.  The token tile's TMA box height is
+// picked per tile (16, 32, 64, 128 or 256 rows) and the MMA N is the valid
+// token count rounded up to 16.
+//
+// Every wait on an mbarrier is bounded: past the limit the kernel sets
+// MOE_STATUS_TIMEOUT in the status word, the other roles see an abort flag
+// and stop, the producer waits (bounded) for its copies in flight, the MMA
+// lane for its MMAs, and TMEM is freed before exit.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBlockK = 64;                    // K elements per stage (128 B rows)
+constexpr int kTileM = 128;                    // weight rows per tile (MMA M)
+constexpr int kABytes = kTileM * kBlockK * 2;  // 16 KB
+constexpr int kNumBox = 5;                     // token box heights 16 << i
+constexpr int kThreads = 192;
+constexpr int kMaxStages = 8;
+constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
+constexpr int kXchgStride = 33;                // fp32 exchange row stride (bank-conflict free)
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+
+struct __align__(64) GemmMaps {
+    CUtensorMap a0, a1;       // routed A (gated: W_gate, W_up as [E*I, H]; down: W_down as [E*H, I])
+    CUtensorMap s0, s1;       // shared A (gated: ws_gate, ws_up [Is, H]; down: ws_down [H, Is])
+    CUtensorMap b[kNumBox];   // routed activations [T*k, K], box heights 16 << i
+    CUtensorMap bs[kNumBox];  // shared activations [T, K]
+};
+
+struct GemmParams {
+    int T, H, E, I, k, Is;
+    int BN;        // token tile (power of two, 16..256)
+    int R, Rs;     // weight tiles per routed / shared expert
+    int nk, nks;   // K steps routed / shared
+    int stages;
+    const int32_t *offsets;
+    const int32_t *perm;
+    const float *topk_w;
+    const float *sgate;
+    uint16_t *out_routed;  // gated: h_perm [T*k, I]; down: ybuf [T, k+1, H]
+    uint16_t *out_shared;  // gated: h_shared [T, Is]; down: ybuf
+    int32_t *status;
+};
+
+// ------------------------------------------------------------ PTX helpers --
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait.  Returns false when the limit passes (status + abort flag
+// set) or, if watch_abort, when another role has aborted.
+__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
+                                       bool watch_abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (watch_abort && *abort_flag) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicOr(status, MOE_STATUS_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// K-major operand in 128B-swizzled rows of 128 bytes, 8-row atoms of 1024 B.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+    d |= (uint64_t)1 << 16;                    // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: next 8-row atom
+    d |= (uint64_t)1 << 46;                    // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+    return d;
+}
+// kind::f16 instruction descriptor: fp32 D, bf16 A and B, both K-major, M = 128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// 32 lanes x 32 consecutive fp32 columns: thread i gets lane (base + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------ scheduling --
+struct Item {
+    int shared;  // 1: shared expert
+    int e;       // routed expert
+    int r;       // weight tile
+    int row0;    // first activation row of the token tile
+    int nvalid;  // valid tokens in the tile (1..BN)
+};
+
+__device__ __forceinline__ Item decode_item(int item, int routed_items, const int *item_base, const int *offs,
+                                            const GemmParams &p) {
+    Item it;
+    if (item < routed_items) {
+        int lo = 0, hi = p.E - 1;  // largest e with item_base[e] <= item
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (item_base[mid] <= item) lo = mid;
+            else hi = mid - 1;
+        }
+        const int cnt = offs[lo + 1] - offs[lo];
+        const int ntt = (cnt + p.BN - 1) / p.BN;
+        const int local = item - item_base[lo];
+        const int j = local % ntt;
+        it.shared = 0;
+        it.e = lo;
+        it.r = local / ntt;
+        it.row0 = offs[lo] + j * p.BN;
+        it.nvalid = min(p.BN, cnt - j * p.BN);
+    } else {
+        const int ntt = (p.T + p.BN - 1) / p.BN;
+        const int local = item - routed_items;
+        const int j = local % ntt;
+        it.shared = 1;
+        it.e = 0;
+        it.r = local / ntt;
+        it.row0 = j * p.BN;
+        it.nvalid = min(p.BN, p.T - j * p.BN);
+    }
+    return it;
+}
+
+__device__ __forceinline__ int box_index(int nvalid) {
+    int b = 0;
+    while ((16 << b) < nvalid) ++b;
+    return b;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+
+// --------------------------------------------------------------- kernel --
+template <bool kGated>
+__global__ void __launch_bounds__(kThreads, 1)
+    ffn_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = p.stages;
+    const int stage_bytes = kABytes + p.BN * 128;
+    uint8_t *stages = smem;
+    float *xchg = reinterpret_cast<float *>(smem + (size_t)S * stage_bytes);
+    int *item_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
+    int *offs = item_base + (p.E + 1);                                   // [E + 1]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(
+        (reinterpret_cast<uintptr_t>(offs + (p.E + 1)) + 7) & ~uintptr_t(7));
+    uint64_t *full = bars, *empty = bars + S, *tfull = bars + 2 * S, *tempty = bars + 2 * S + 2;
+    uint64_t *mma_done = bars + 2 * S + 4;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
+    int *scan_tmp = reinterpret_cast<int *>(tmem_slot + 4);  // [kThreads]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tmem_cols = 2 * p.BN;
+
+    // ---- setup: barriers, TMEM, tile schedule
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 1);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&maps.a0);
+        prefetch_tmap(&maps.s0);
+        if (kGated) {
+            prefetch_tmap(&maps.a1);
+            prefetch_tmap(&maps.s1);
+        }
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc_fence_before();
+    }
+    // item_base[e] = sum_{e' < e} ceil(count(e') / BN) * R  (block scan)
+    {
+        const int per = (p.E + kThreads - 1) / kThreads;
+        const int e0 = threadIdx.x * per, e1 = min(p.E, e0 + per);
+        int local = 0;
+        for (int e = e0; e < e1; ++e) {
+            const int o0 = __ldg(p.offsets + e), o1 = __ldg(p.offsets + e + 1);
+            offs[e] = o0;
+            if (e == p.E - 1) offs[p.E] = o1;
+            local += (o1 - o0 + p.BN - 1) / p.BN * p.R;
+        }
+        scan_tmp[threadIdx.x] = local;
+        __syncthreads();
+        if (warp == 0) {  // 192 partials, 6 per lane
+            int v[kThreads / 32];
+            int sum = 0;
+#pragma unroll
+            for (int q = 0; q < kThreads / 32; ++q) {
+                v[q] = scan_tmp[lane * (kThreads / 32) + q];
+                sum += v[q];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            int run = incl - sum;
+#pragma unroll
+            for (int q = 0; q < kThreads / 32; ++q) {
+                scan_tmp[lane * (kThreads / 32) + q] = run;
+                run += v[q];
+            }
+        }
+        __syncthreads();
+        int run = scan_tmp[threadIdx.x];
+        for (int e = e0; e < e1; ++e) {
+            item_base[e] = run;
+            run += (offs[e + 1] - offs[e] + p.BN - 1) / p.BN * p.R;
+        }
+        if (e1 == p.E && e0 < e1) item_base[p.E] = run;
+    }
+    __syncthreads();
+    tc_fence_after();
+    const int routed_items = item_base[p.E];
+    const int total_items = routed_items + (p.Is > 0 ? p.Rs * ((p.T + p.BN - 1) / p.BN) : 0);
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, last_phase = 0;
+            for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+                const Item it = decode_item(item, routed_items, item_base, offs, p);
+                const int bi = box_index(it.nvalid);
+                const CUtensorMap *ma0 = it.shared ? &maps.s0 : &maps.a0;
+                const CUtensorMap *ma1 = it.shared ? &maps.s1 : &maps.a1;
+                const CUtensorMap *mb = it.shared ? &maps.bs[bi] : &maps.b[bi];
+                const int a_row = kGated ? (it.shared ? 0 : it.e * p.I) + it.r * 64
+                                         : (it.shared ? 0 : it.e * p.H) + it.r * kTileM;
+                const int nk = it.shared ? p.nks : p.nk;
+                const uint32_t bytes = kABytes + (uint32_t)(16 << bi) * 128u;
+                bool ok = true;
+                for (int ks = 0; ks < nk; ++ks) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, true)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sA = stages + (size_t)stage * stage_bytes;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    if (kGated) {
+                        tma_load_2d(ma0, &full[stage], sA, ks * kBlockK, a_row);
+                        tma_load_2d(ma1, &full[stage], sA + kABytes / 2, ks * kBlockK, a_row);
+                    } else {
+                        tma_load_2d(ma0, &full[stage], sA, ks * kBlockK, a_row);
+                    }
+                    tma_load_2d(mb, &full[stage], sA + kABytes, ks * kBlockK, it.row0);
+                    issued |= 1u << stage;
+                    last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+            // wait for every copy still in flight before the CTA may exit
+            for (int s = 0; s < S; ++s)
+                if ((issued >> s) & 1u) mbar_wait(&full[s], (last_phase >> s) & 1u, abort_flag, p.status, false);
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            int stage = 0, local = 0;
+            uint32_t phase = 0;
+            for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++local) {
+                const Item it = decode_item(item, routed_items, item_base, offs, p);
+                const int n = (it.nvalid + 15) & ~15;
+                const uint32_t idesc = idesc_bf16(n);
+                const int acc = local & 1;
+                const uint32_t use = (uint32_t)(local >> 1);
+                if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag, p.status, true)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(acc * p.BN);
+                const int nk = it.shared ? p.nks : p.nk;
+                bool ok = true;
+                for (int ks = 0; ks < nk; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, p.status, true)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sA = smem_u32(stages + (size_t)stage * stage_bytes);
+                    const uint64_t da = sw128_desc(sA), db = sw128_desc(sA + kABytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBlockK / 16; ++kk)  // +32 bytes per K16 step
+                        umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+                    umma_commit(&empty[stage]);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+            }
+            umma_commit(mma_done);  // completes once every MMA above has
+            mbar_wait(mma_done, 0, abort_flag, p.status, false);
+        }
+    } else {
+        // ================= epilogue (warps 2..5) =================
+        const int q = warp & 3;  // TMEM lane quarter of this warp
+        const bool elected = (warp == 2 && lane == 0);
+        int local = 0;
+        for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++local) {
+            const Item it = decode_item(item, routed_items, item_base, offs, p);
+            const int acc = local & 1;
+            const uint32_t use = (uint32_t)(local >> 1);
+            if (elected) *epi_ok = mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 1 : 0;
+            named_bar_sync(1, 128);
+            if (!*epi_ok) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (uint32_t)(acc * p.BN) + ((uint32_t)(q * 32) << 16);
+            for (int c0 = 0; c0 < it.nvalid; c0 += 32) {
+                float v[32];
+                tmem_ld32(tbase + (uint32_t)c0, v);
+                if (kGated) {
+                    if (q < 2) {  // gate rows 0..63: silu(g) to the exchange buffer
+                        float *xr = xchg + (q * 32 + lane) * kXchgStride;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) xr[i] = silu(v[i]);
+                    }
+                    named_bar_sync(1, 128);
+                    if (q >= 2) {  // up rows 64..127: h = silu(g) * u
+                        const int row = (q - 2) * 32 + lane;
+                        const float *xr = xchg + row * kXchgStride;
+                        uint16_t *out = it.shared ? p.out_shared : p.out_routed;
+                        const int ld = it.shared ? p.Is : p.I;
+                        uint16_t *dst = out + (size_t)(it.row0 + c0) * ld + it.r * 64 + row;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (c0 + i < it.nvalid) dst[(size_t)i * ld] = f32_to_bf16_bits(xr[i] * v[i]);
+                    }
+                    named_bar_sync(1, 128);
+                } else {
+                    // per-token destination row of ybuf and weight, token c0 + lane
+                    int mrow = 0;
+                    float mw = 0.f;
+                    const int n = c0 + lane;
+                    if (n < it.nvalid) {
+                        if (it.shared) {
+                            const int t = it.row0 + n;
+                            mrow = t * (p.k + 1) + p.k;
+                            mw = __ldg(p.sgate + t);
+                        } else {
+                            const int slot = __ldg(p.perm + it.row0 + n);
+                            mrow = slot + slot / p.k;  // t*(k+1) + j
+                            mw = __ldg(p.topk_w + slot);
+                        }
+                    }
+                    uint16_t *out = p.out_routed + it.r * kTileM + q * 32 + lane;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int rr = __shfl_sync(0xffffffffu, mrow, i);
+                        const float ww = __shfl_sync(0xffffffffu, mw, i);
+                        if (c0 + i < it.nvalid) out[(size_t)rr * p.H] = f32_to_bf16_bits(v[i] * ww);
+                    }
+                }
+            }
+            tc_fence_before();
+            named_bar_sync(1, 128);
+            if (elected) mbar_arrive(&tempty[acc]);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------- host side --
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] tensor, box = 64 columns x box_rows rows, 128-byte swizzle.
+bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBlockK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int pick_bn(long long T, int k, int E) {
+    const long long avg = (T * k + E - 1) / E;  // mean tokens per expert
+    int bn = 64;
+    while (bn < 256 && bn < 2 * avg) bn <<= 1;
+    return bn;
+}
+
+size_t smem_bytes_for(int BN, int E, int stages) {
+    return 1024 + (size_t)stages * (kABytes + BN * 128) + 64 * kXchgStride * 4 + 2 * (size_t)(E + 1) * 4 + 8 +
+           (size_t)(2 * stages + 5) * 8 + 16 + kThreads * 4;
+}
+
+int pick_stages(int BN, int E) {
+    int s = kMaxStages;
+    while (s > 2 && smem_bytes_for(BN, E, s) > (size_t)kSmemLimit) --s;
+    return s;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    int cc_major = 0;
+};
+
+DeviceInfo device_info() {
+    static DeviceInfo cache[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceInfo{};
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev].sms == 0) {
+        cudaDeviceGetAttribute(&cache[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&cache[dev].cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    }
+    return cache[dev];
+}
+
+template <bool kGated>
+int launch_one(const GemmMaps &maps, const GemmParams &p, int sms, cudaStream_t st) {
+    const size_t smem = smem_bytes_for(p.BN, p.E, p.stages);
+    if (smem > (size_t)kSmemLimit) return MOE_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(ffn_gemm_kernel<kGated>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    // upper bound on work items (the real count is known only on the device)
+    const long long slots = (long long)p.T * p.k;
+    long long items = (std::min<long long>(p.E, slots) + (slots + p.BN - 1) / p.BN) * p.R;
+    if (p.Is > 0) items += (long long)p.Rs * ((p.T + p.BN - 1) / p.BN);
+    const int grid = (int)std::max<long long>(1, std::min<long long>(sms, items));
+    ffn_gemm_kernel<kGated><<<grid, kThreads, smem, st>>>(maps, p);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+namespace {
+
+int choose_bn(const FfnArgs &a, int *bn) {
+    *bn = pick_bn(a.T, a.k, a.E);
+    // Benchmark/test override of the token tile (config-invariance checks).
+    if (const char *f = getenv("MOE_FORCE_BN")) {
+        char *end = nullptr;
+        const long v = strtol(f, &end, 10);
+        if (*f == 0 || *end != 0 || (v != 32 && v != 64 && v != 128 && v != 256)) return MOE_ERR_INVALID_ARG;
+        *bn = (int)v;
+    }
+    return MOE_OK;
+}
+
+GemmParams base_params(const FfnArgs &a, int BN) {
+    GemmParams p{};
+    p.T = a.T;
+    p.H = a.H;
+    p.E = a.E;
+    p.I = a.I;
+    p.k = a.k;
+    p.Is = a.Is;
+    p.BN = BN;
+    p.stages = pick_stages(BN, a.E);
+    p.offsets = a.offsets;
+    p.perm = a.perm;
+    p.topk_w = a.topk_w;
+    p.sgate = a.sgate;
+    p.status = a.status;
+    return p;
+}
+
+}  // namespace
+
+int ffn_launch_gate_up(const FfnArgs &a, cudaStream_t st) {
+    const DeviceInfo di = device_info();
+    if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
+    int BN = 0;
+    if (int rc = choose_bn(a, &BN)) return rc;
+    const uint64_t Tk = (uint64_t)a.T * a.k;
+    GemmParams p = base_params(a, BN);
+    GemmMaps m;
+    memset(&m, 0, sizeof(m));
+    bool ok = encode_2d(&m.a0, a.w_gate, (uint64_t)a.E * a.I, a.H, 64) &&
+              encode_2d(&m.a1, a.w_up, (uint64_t)a.E * a.I, a.H, 64);
+    for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&m.b[b], a.x_perm, Tk, a.H, 16 << b);
+    if (a.Is > 0) {
+        ok = ok && encode_2d(&m.s0, a.ws_gate, a.Is, a.H, 64) && encode_2d(&m.s1, a.ws_up, a.Is, a.H, 64);
+        for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&m.bs[b], a.x, a.T, a.H, 16 << b);
+    } else {
+        m.s0 = m.a0;
+        m.s1 = m.a1;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    p.R = a.I / 64;
+    p.Rs = a.Is / 64;
+    p.nk = a.H / kBlockK;
+    p.nks = a.H / kBlockK;
+    p.out_routed = a.h_perm;
+    p.out_shared = a.h_shared;
+    return launch_one<true>(m, p, di.sms, st);
+}
+
+int ffn_launch_down(const FfnArgs &a, cudaStream_t st) {
+    const DeviceInfo di = device_info();
+    if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
+    int BN = 0;
+    if (int rc = choose_bn(a, &BN)) return rc;
+    const uint64_t Tk = (uint64_t)a.T * a.k;
+    GemmParams p = base_params(a, BN);
+    GemmMaps m;
+    memset(&m, 0, sizeof(m));
+    bool ok = encode_2d(&m.a0, a.w_down, (uint64_t)a.E * a.H, a.I, kTileM);
+    for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&m.b[b], a.h_perm, Tk, a.I, 16 << b);
+    if (a.Is > 0) {
+        ok = ok && encode_2d(&m.s0, a.ws_down, a.H, a.Is, kTileM);
+        for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b)
+            ok = ok && encode_2d(&m.bs[b], a.h_shared, a.T, a.Is, 16 << b);
+    } else {
+        m.s0 = m.a0;
+    }
+    m.a1 = m.a0;
+    m.s1 = m.s0;
+    if (!ok) return MOE_ERR_CUDA;
+    p.R = a.H / kTileM;
+    p.Rs = a.H / kTileM;
+    p.nk = a.I / kBlockK;
+    p.nks = a.Is / kBlockK;
+    p.out_routed = a.ybuf;
+    p.out_shared = a.ybuf;
+    return launch_one<false>(m, p, di.sms, st);
+}
+
+}  // namespace moe

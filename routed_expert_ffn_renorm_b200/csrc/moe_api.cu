@@ -1,0 +1,294 @@
+// C ABI of libmoe: argument checks, workspace layout and the launch
+// sequence.  No entry point allocates, frees or synchronises (except
+// moe_status_read, which waits for its own copy); every launch goes on the
+// caller's stream.
+#include <cstring>
+
+#include "moe_internal.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+    size_t status, idx, w, sgate, keff, kept, ndrop, counts, offsets, perm, slot_pos, hist, bagg, bcnt;
+    size_t x_perm, h_perm, h_shared, ybuf, total;
+};
+
+WsLayout ws_layout(const moe_config_t &c, int T) {
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes);
+        return o;
+    };
+    const size_t Tk = (size_t)T * c.num_experts_per_tok;
+    const size_t E = (size_t)c.n_routed_experts;
+    L.status = take(kAlign);
+    L.idx = take(Tk * 4);
+    L.w = take(Tk * 4);
+    L.sgate = take((size_t)T * 4);
+    L.keff = take((size_t)T * 4);
+    L.kept = take(E);
+    L.ndrop = take(4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 4);
+    L.perm = take(Tk * 4);
+    L.slot_pos = take(Tk * 4);
+    L.hist = take((size_t)dispatch_chunks(T) * E * 4);
+    L.bagg = take((size_t)budget_chunks(T) * E * 4);
+    L.bcnt = take((size_t)budget_chunks(T) * E * 4);
+    L.x_perm = take(Tk * c.hidden * 2);
+    L.h_perm = take(Tk * c.moe_intermediate_size * 2);
+    L.h_shared = take((size_t)T * c.shared_intermediate_size * 2);
+    L.ybuf = take((size_t)T * (c.num_experts_per_tok + 1) * c.hidden * 2);
+    L.total = off;
+    return L;
+}
+
+int check_config(const moe_config_t *c, int32_t T) {
+    if (!c || T < 0) return MOE_ERR_INVALID_ARG;
+    const int E = c->n_routed_experts, k = c->num_experts_per_tok;
+    if (E < 1 || k < 1 || k > E || c->budget < 0 || c->shared_intermediate_size < 0 || c->hidden < 1 ||
+        c->moe_intermediate_size < 1 || (c->norm_topk != 0 && c->norm_topk != 1))
+        return MOE_ERR_INVALID_ARG;
+    if (E > kMaxExperts || k > kMaxTopK || c->hidden % 128 != 0 || c->moe_intermediate_size % 64 != 0 ||
+        c->shared_intermediate_size % 64 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    if ((long long)T * (k + 1) * c->hidden >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+bool aligned(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_or_null(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_config_t *cfg, int32_t T) {
+    if (check_config(cfg, T) != MOE_OK) return 0;
+    return ws_layout(*cfg, T).total;
+}
+
+const char *moe_error_string(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or device";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA launch or driver call failed";
+        case MOE_ERR_DEVICE: return "device-side error reported in the status word";
+        default: return "unknown error";
+    }
+}
+
+int moe_route(const moe_config_t *cfg, int32_t T, const float *logits, const moe_bf16_t *x,
+              const moe_bf16_t *ws_gate_vec, int32_t *topk_idx, float *topk_w, float *sgate, int32_t *keff,
+              void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned(logits) || !aligned(topk_idx) || !aligned(topk_w) || !aligned_or_null(keff))
+        return MOE_ERR_INVALID_ARG;
+    if (sgate && (cfg->shared_intermediate_size == 0 || !aligned(x) || !aligned(ws_gate_vec) || !aligned(sgate)))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_route(T, cfg->n_routed_experts, cfg->num_experts_per_tok, cfg->norm_topk, logits,
+                                topk_idx, topk_w, keff, x, ws_gate_vec, cfg->hidden, sgate, as_stream(stream)));
+}
+
+int moe_budget(const moe_config_t *cfg, int32_t T, int32_t *topk_idx, float *topk_w, int32_t *keff,
+               uint8_t *expert_kept, int32_t *n_dropped, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned(topk_idx) || !aligned(topk_w) || !aligned(keff) || !expert_kept || !n_dropped || !aligned(ws))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    return cuda_rc(launch_budget(T, cfg->n_routed_experts, cfg->num_experts_per_tok, cfg->budget, cfg->norm_topk,
+                                 topk_idx, topk_w, keff, expert_kept, n_dropped, at<float>(ws, L.bagg),
+                                 at<int32_t>(ws, L.bcnt), as_stream(stream)));
+}
+
+int moe_dispatch(const moe_config_t *cfg, int32_t T, const int32_t *topk_idx, const int32_t *keff,
+                 const moe_bf16_t *x, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
+                 moe_bf16_t *x_perm, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned(topk_idx) || !aligned_or_null(keff) || !aligned(counts) || !aligned(offsets) || !aligned(perm) ||
+        !aligned(slot_pos) || !aligned(ws) || !aligned_or_null(x_perm) || (x_perm && !aligned(x)))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    const int E = cfg->n_routed_experts, k = cfg->num_experts_per_tok;
+    cudaStream_t st = as_stream(stream);
+    rc = cuda_rc(launch_dispatch(T, E, k, topk_idx, keff, at<int32_t>(ws, L.hist), counts, offsets, perm, slot_pos, st));
+    if (rc || !x_perm) return rc;
+    return cuda_rc(launch_gather_rows(T, k, cfg->hidden, offsets, E, perm, x, x_perm, st));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Common checks and argument block of the two FFN phases; `gate_up`
+// selects which phase's inputs are checked.
+int ffn_args(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+             const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+             const moe_weights_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, bool gate_up, FfnArgs *a) {
+    const bool sh = cfg->shared_intermediate_size > 0;
+    if (!w || !aligned(offsets) || !aligned(ws)) return MOE_ERR_INVALID_ARG;
+    if (gate_up && (!aligned(x_perm) || !aligned(w->w_gate) || !aligned(w->w_up) ||
+                    (sh && (!aligned(x) || !aligned(w->ws_gate) || !aligned(w->ws_up)))))
+        return MOE_ERR_INVALID_ARG;
+    if (!gate_up && (!aligned(perm) || !aligned(topk_w) || !aligned(ybuf) || !aligned(w->w_down) ||
+                     (sh && (!aligned(sgate) || !aligned(w->ws_down)))))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    *a = FfnArgs{};
+    a->T = T;
+    a->H = cfg->hidden;
+    a->E = cfg->n_routed_experts;
+    a->I = cfg->moe_intermediate_size;
+    a->k = cfg->num_experts_per_tok;
+    a->Is = cfg->shared_intermediate_size;
+    a->x = x;
+    a->x_perm = x_perm;
+    a->offsets = offsets;
+    a->perm = perm;
+    a->topk_w = topk_w;
+    a->sgate = sgate;
+    a->w_gate = w->w_gate;
+    a->w_up = w->w_up;
+    a->w_down = w->w_down;
+    a->ws_gate = w->ws_gate;
+    a->ws_up = w->ws_up;
+    a->ws_down = w->ws_down;
+    a->h_perm = at<uint16_t>(ws, L.h_perm);
+    a->h_shared = sh ? at<uint16_t>(ws, L.h_shared) : nullptr;
+    a->ybuf = ybuf;
+    a->status = at<int32_t>(ws, L.status);
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_expert_gate_up(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                       const int32_t *offsets, const moe_weights_t *w, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    FfnArgs a;
+    rc = ffn_args(cfg, T, x, x_perm, offsets, nullptr, nullptr, nullptr, w, nullptr, ws, ws_bytes, true, &a);
+    if (rc) return rc;
+    return ffn_launch_gate_up(a, as_stream(stream));
+}
+
+int moe_expert_down(const moe_config_t *cfg, int32_t T, const int32_t *offsets, const int32_t *perm,
+                    const float *topk_w, const float *sgate, const moe_weights_t *w, moe_bf16_t *ybuf, void *ws,
+                    size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    FfnArgs a;
+    rc = ffn_args(cfg, T, nullptr, nullptr, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, false, &a);
+    if (rc) return rc;
+    return ffn_launch_down(a, as_stream(stream));
+}
+
+int moe_expert_ffn(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                   const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                   const moe_weights_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    FfnArgs a, b;
+    rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, true, &a);
+    if (rc) return rc;
+    rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, false, &b);
+    if (rc) return rc;
+    rc = ffn_launch_gate_up(a, as_stream(stream));
+    if (rc) return rc;
+    return ffn_launch_down(b, as_stream(stream));
+}
+
+int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, const int32_t *keff, moe_bf16_t *out,
+                void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned(ybuf) || !aligned_or_null(keff) || !aligned(out)) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_combine(T, cfg->num_experts_per_tok, cfg->hidden, cfg->shared_intermediate_size > 0, ybuf,
+                                  keff, out, as_stream(stream)));
+}
+
+int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits, const moe_weights_t *w,
+                moe_bf16_t *out, const moe_aux_t *aux, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    const bool sh = cfg->shared_intermediate_size > 0;
+    if (!aligned(x) || !aligned(logits) || !aligned(out) || !aligned(ws) || !w) return MOE_ERR_INVALID_ARG;
+    if (sh && !aligned(w->ws_gate_vec)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    moe_aux_t a{};
+    if (aux) a = *aux;
+    int32_t *idx = a.topk_idx ? a.topk_idx : at<int32_t>(ws, L.idx);
+    float *tw = a.topk_w ? a.topk_w : at<float>(ws, L.w);
+    float *sgate = sh ? (a.sgate ? a.sgate : at<float>(ws, L.sgate)) : nullptr;
+    int32_t *keff = a.keff ? a.keff : at<int32_t>(ws, L.keff);
+    uint8_t *kept = a.expert_kept ? a.expert_kept : at<uint8_t>(ws, L.kept);
+    int32_t *ndrop = a.n_dropped ? a.n_dropped : at<int32_t>(ws, L.ndrop);
+    int32_t *counts = a.counts ? a.counts : at<int32_t>(ws, L.counts);
+    int32_t *offsets = a.offsets ? a.offsets : at<int32_t>(ws, L.offsets);
+    int32_t *perm = a.perm ? a.perm : at<int32_t>(ws, L.perm);
+    int32_t *slot_pos = a.slot_pos ? a.slot_pos : at<int32_t>(ws, L.slot_pos);
+    moe_bf16_t *x_perm = at<moe_bf16_t>(ws, L.x_perm);
+    moe_bf16_t *ybuf = at<moe_bf16_t>(ws, L.ybuf);
+
+    rc = moe_route(cfg, T, logits, x, sh ? w->ws_gate_vec : nullptr, idx, tw, sgate, keff, stream);
+    if (rc) return rc;
+    if (cfg->budget > 0) {
+        rc = moe_budget(cfg, T, idx, tw, keff, kept, ndrop, ws, ws_bytes, stream);
+        if (rc) return rc;
+    }
+    rc = moe_dispatch(cfg, T, idx, keff, x, counts, offsets, perm, slot_pos, x_perm, ws, ws_bytes, stream);
+    if (rc) return rc;
+    rc = moe_expert_ffn(cfg, T, x, x_perm, offsets, perm, tw, sgate, w, ybuf, ws, ws_bytes, stream);
+    if (rc) return rc;
+    return moe_combine(cfg, T, ybuf, keff, out, stream);
+}
+
+int moe_status_read(const void *ws, int32_t *status_out, void *stream) {
+    if (!aligned(ws) || !status_out) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cuda_rc(cudaStreamSynchronize(st));
+}
+
+int moe_status_clear(void *ws, void *stream) {
+    if (!aligned(ws)) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(cudaMemsetAsync(ws, 0, sizeof(int32_t), as_stream(stream)));
+}
+
+}  // extern "C"

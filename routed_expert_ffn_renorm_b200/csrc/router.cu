@@ -1,0 +1,143 @@
+// Router: softmax over the E logits of a token, top-k by logit with the
+// kept probabilities renormalised (SpecForge PR #943, "Modifications":
+// softmax router with renormalised top-k), plus the sigmoid gate of the
+// shared expert.
+//
+// One warp per token.  Lane l holds the logits of experts l, l+32, ...
+// (coalesced 128-byte loads).  Each of the k selection rounds takes a
+// lane-local best and a 5-step shuffle argmax ordered by (logit descending,
+// expert id ascending), so equal logits keep the lower id, and the winner's
+// owner lane masks it out.  The memory traffic is the logits row once; the
+// kernel is latency-bound and tiny next to the expert FFN.
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+template <int V>  // logits per lane: V * 32 >= E
+__global__ void __launch_bounds__(256) route_kernel(int T, int E, int k, int norm_topk,
+                                                    const float *__restrict__ logits,
+                                                    int32_t *__restrict__ idx, float *__restrict__ w,
+                                                    int32_t *__restrict__ keff,
+                                                    const uint16_t *__restrict__ x,
+                                                    const uint16_t *__restrict__ gvec, int H,
+                                                    float *__restrict__ sgate) {
+    const int lane = threadIdx.x & 31;
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    const float *l = logits + (size_t)t * E;
+
+    float v[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? __ldg(l + e) : -INFINITY;
+    }
+    // softmax denominator: max, then sum of exp(l - max) over all E
+    float m = v[0];
+#pragma unroll
+    for (int i = 1; i < V; ++i) m = fmaxf(m, v[i]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+        if (lane + 32 * i < E) s += expf(v[i] - m);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+
+    // k selection rounds; lane j keeps the j-th winner
+    uint32_t taken = 0;
+    int my_idx = -1;
+    float my_logit = -INFINITY;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) {
+                bv = v[i];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (better(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == j) {
+            my_idx = bi;
+            my_logit = bv;
+        }
+    }
+    // probabilities of the kept experts; renormalise with the sum taken in
+    // slot order
+    float p = (lane < k) ? expf(my_logit - m) / s : 0.f;
+    if (norm_topk) {
+        float ps = 0.f;
+        for (int j = 0; j < k; ++j) ps += __shfl_sync(0xffffffffu, p, j);
+        p = p / ps;
+    }
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = my_idx;
+        w[(size_t)t * k + lane] = p;
+    }
+    if (keff != nullptr && lane == 0) keff[t] = k;
+
+    if (sgate != nullptr) {  // sigmoid(g . x_t), 8 bf16 per 16-byte load
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+        const uint4 *gr = reinterpret_cast<const uint4 *>(gvec);
+        float z = 0.f;
+        for (int c = lane; c < H / 8; c += 32) {
+            const uint4 a = __ldg(xr + c), b = __ldg(gr + c);
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                z = fmaf(bf16_bits_to_f32((uint16_t)(av[q] & 0xffffu)),
+                         bf16_bits_to_f32((uint16_t)(bv[q] & 0xffffu)), z);
+                z = fmaf(bf16_bits_to_f32((uint16_t)(av[q] >> 16)), bf16_bits_to_f32((uint16_t)(bv[q] >> 16)), z);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+        if (lane == 0) sgate[t] = 1.f / (1.f + expf(-z));
+    }
+}
+
+template <int V>
+cudaError_t launch_v(int T, int E, int k, int norm_topk, const float *logits, int32_t *idx, float *w,
+                     int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
+                     cudaStream_t st) {
+    const int threads = 256, per_block = threads / 32;
+    route_kernel<V><<<(T + per_block - 1) / per_block, threads, 0, st>>>(T, E, k, norm_topk, logits, idx, w,
+                                                                          keff, x, gvec, H, sgate);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route(int T, int E, int k, int norm_topk, const float *logits, int32_t *idx, float *w,
+                         int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
+                         cudaStream_t st) {
+    if (E <= 32) return launch_v<1>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
+    if (E <= 64) return launch_v<2>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
+    if (E <= 128) return launch_v<4>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
+    if (E <= 256) return launch_v<8>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
+    if (E <= 512) return launch_v<16>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
+    return launch_v<32>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,166 @@
+"""Helpers for the GPU parity tests: run the CUDA path through the C ABI and
+the CPU oracle on the same seeded inputs, and compare them.
+
+Comparison rules (the tolerance is the one stated for the layer output):
+  * routing indices, budget drops, counts, offsets, perm, slot_pos: bit-exact;
+  * routing weights: fp32 within 2e-6 relative (GPU and CPU exp differ by ulps);
+  * the layer output: relative L2 error <= 5e-3 over the compared rows
+    (bf16 inputs/outputs, fp32 accumulation on the GPU, fp64 in the oracle).
+  * budget near-ties: when the GPU keeps a different expert set, the
+    oracle's aggregate gap between the last kept and first dropped expert
+    must be <= 1e-5 of the largest aggregate; the downstream comparison then
+    runs the oracle on the GPU's post-budget routing.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+import oracle
+import routed_expert_ffn_renorm_b200 as moe
+from routed_expert_ffn_renorm_b200 import workloads as W
+
+REL_L2_TOL = 5e-3
+W_RTOL = 2e-6
+NEAR_TIE = 1e-5
+
+
+def lib_config(cfg: W.MoEConfig) -> moe.MoEConfig:
+    return moe.MoEConfig(cfg.H, cfg.E, cfg.I, cfg.k, cfg.Is, cfg.norm_topk, cfg.budget)
+
+
+def weights_of(inp: W.MoEInputs) -> moe.MoEWeights:
+    return moe.MoEWeights(inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec)
+
+
+@dataclass
+class GpuResult:
+    out: np.ndarray       # [T, H] float32 (bf16 values)
+    idx: np.ndarray
+    w: np.ndarray
+    keff: np.ndarray
+    kept: np.ndarray
+    n_dropped: int
+    counts: np.ndarray
+    offsets: np.ndarray
+    perm: np.ndarray      # [sum keff]
+    slot_pos: np.ndarray
+    sgate: Optional[np.ndarray]
+    status: int
+    out_bits: np.ndarray  # raw bf16 bits, for bit-identity checks
+
+
+def gpu_forward(cfg: W.MoEConfig, inp: W.MoEInputs, ws: Optional[torch.Tensor] = None) -> GpuResult:
+    dev = inp.x.device
+    T, k, E = cfg.T, cfg.k, cfg.E
+    c = lib_config(cfg)
+    if ws is None:
+        ws = torch.empty(moe.workspace_bytes(c, T), dtype=torch.uint8, device=dev)
+        moe.status_clear(ws)
+    aux = dict(
+        topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+        topk_w=torch.empty((T, k), dtype=torch.float32, device=dev),
+        keff=torch.empty(T, dtype=torch.int32, device=dev),
+        expert_kept=torch.zeros(E, dtype=torch.uint8, device=dev),
+        n_dropped=torch.zeros(1, dtype=torch.int32, device=dev),
+        counts=torch.empty(E, dtype=torch.int32, device=dev),
+        offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+        perm=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
+        slot_pos=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
+    )
+    if cfg.Is:
+        aux["sgate"] = torch.empty(T, dtype=torch.float32, device=dev)
+    out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    moe.moe_forward(c, inp.x, inp.logits, weights_of(inp), out, ws, aux=aux)
+    status = moe.status_read(ws)
+    torch.cuda.synchronize()
+    h = {n: t.cpu().numpy() for n, t in aux.items()}
+    total = int(h["offsets"][E])
+    return GpuResult(out.float().cpu().numpy(), h["topk_idx"], h["topk_w"], h["keff"], h["expert_kept"],
+                     int(h["n_dropped"][0]), h["counts"], h["offsets"], h["perm"][:total], h["slot_pos"][: T * k],
+                     h.get("sgate"), status, W.bf16_bits(out))
+
+
+def rel_l2(a: np.ndarray, ref: np.ndarray) -> float:
+    a = np.asarray(a, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(a - ref) / den) if den > 0 else float(np.linalg.norm(a))
+
+
+def sample_rows(T: int, n: int, seed: int = 1) -> np.ndarray:
+    """First, last and n-2 seeded tokens in between (all tokens if n >= T)."""
+    if n >= T:
+        return np.arange(T, dtype=np.int32)
+    rng = np.random.default_rng(seed)
+    mid = rng.choice(np.arange(1, T - 1), size=max(n - 2, 0), replace=False)
+    return np.unique(np.concatenate([[0, T - 1], mid])).astype(np.int32)
+
+
+def _expert_dicts(inp: W.MoEInputs, experts):
+    bits = W.bf16_bits
+    return ({e: bits(inp.w_gate[e]) for e in experts}, {e: bits(inp.w_up[e]) for e in experts},
+            {e: bits(inp.w_down[e]) for e in experts})
+
+
+def check_layer(cfg: W.MoEConfig, inp: W.MoEInputs, g: GpuResult, rows: Optional[np.ndarray] = None,
+                nthreads: Optional[int] = None) -> dict:
+    """Compare a GPU forward with the oracle; returns diagnostics, asserts."""
+    assert g.status == 0, f"device status {g.status}"
+    T, k, E = cfg.T, cfg.k, cfg.E
+    nthreads = nthreads or oracle.max_threads()
+    logits = inp.logits.cpu().numpy()
+    # route (bit-exact indices, fp32 weights within ulps)
+    idx_o, w_o = oracle.route(logits, k, cfg.norm_topk)
+    diag = {}
+    if cfg.budget == 0:
+        assert (g.idx == idx_o).all(), "routing indices differ"
+        np.testing.assert_allclose(g.w, w_o, rtol=W_RTOL, atol=1e-7)
+        assert (g.keff == k).all()
+        idx_b, w_b, keff_b = idx_o, w_o, np.full(T, k, np.int32)
+    else:
+        # the budget on the oracle's own routing
+        idx_b, w_b, keff_b, kept_b, nd_b = oracle.budget(idx_o, w_o, E, cfg.budget, cfg.norm_topk)
+        if (kept_b == g.kept).all():
+            assert g.n_dropped == nd_b
+            assert (g.idx == idx_b).all() and (g.keff == keff_b).all()
+            np.testing.assert_allclose(g.w, w_b, rtol=W_RTOL, atol=1e-7)
+        else:
+            agg = np.zeros(E)
+            np.add.at(agg, idx_o.ravel(), w_o.ravel().astype(np.float64))
+            union = np.unique(idx_o)
+            order = union[np.lexsort((union, -agg[union]))]
+            gap = agg[order[cfg.budget - 1]] - agg[order[cfg.budget]]
+            assert gap <= NEAR_TIE * agg.max(), f"budget keep-set differs with gap {gap}"
+            diag["near_tie"] = float(gap)
+            idx_b, w_b, keff_b = g.idx, g.w, g.keff
+    # dispatch on the same routing: bit-exact
+    counts, offsets, perm, slot_pos = oracle.dispatch(idx_b, keff_b, E)
+    assert (g.counts == counts).all() and (g.offsets == offsets).all(), "counts/offsets differ"
+    assert (g.perm == perm).all() and (g.slot_pos == slot_pos).all(), "perm/slot_pos differ"
+    # shared gate
+    if cfg.Is:
+        sg = oracle.shared_gate(W.bf16_bits(inp.ws_gvec), W.bf16_bits(inp.x))
+        np.testing.assert_allclose(g.sgate, sg, rtol=1e-5, atol=1e-6)
+    # layer output on the chosen rows
+    rows = np.arange(T, dtype=np.int32) if rows is None else rows
+    need = sorted({int(idx_b[t, j]) for t in rows for j in range(int(keff_b[t]))})
+    wg, wu, wd = _expert_dicts(inp, need)
+    kw = {}
+    if cfg.Is:
+        kw = dict(ws_gate=W.bf16_bits(inp.ws_gate), ws_up=W.bf16_bits(inp.ws_up), ws_down=W.bf16_bits(inp.ws_down),
+                  ws_gvec=W.bf16_bits(inp.ws_gvec))
+    ref = oracle.combine_rows(W.bf16_bits(inp.x), idx_b, w_b, keff_b, wg, wu, wd, I=cfg.I, rows=rows,
+                              nthreads=nthreads, **kw)
+    err = rel_l2(g.out[rows], ref)
+    diag["rel_l2"] = err
+    diag["rows"] = int(len(rows))
+    assert err <= REL_L2_TOL, f"rel-L2 {err:.3e} > {REL_L2_TOL}"
+    # rows with no kept slot and no shared expert must be exactly zero
+    if not cfg.Is:
+        empty = np.nonzero(keff_b == 0)[0]
+        assert (g.out[empty] == 0).all()
+    return diag

@@ -1,0 +1,91 @@
+"""The C ABI on a host without a GPU: the library builds, loads and exports
+every function include/moe.h declares; argument checks reject bad calls
+before any CUDA work (no compute call is made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import routed_expert_ffn_renorm_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == sorted(moe.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = moe.load_library()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (moe_\w+)", out))
+    assert set(_declared()) <= exported
+
+
+def _cfg(**kw):
+    base = dict(hidden=256, n_routed_experts=8, moe_intermediate_size=128, num_experts_per_tok=2,
+                shared_intermediate_size=0, norm_topk=True, budget=0)
+    base.update(kw)
+    return moe._Config(*[int(v) for v in base.values()])
+
+
+FAKE = ctypes.c_void_p(1 << 20)      # never dereferenced: the checks fail first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 4)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_routed_experts=0), -1), (dict(num_experts_per_tok=0), -1), (dict(num_experts_per_tok=9), -1),
+    (dict(budget=-1), -1), (dict(norm_topk=2), -1), (dict(hidden=200), -2), (dict(moe_intermediate_size=96), -2),
+    (dict(shared_intermediate_size=32), -2), (dict(n_routed_experts=2048, num_experts_per_tok=2), -2),
+    (dict(n_routed_experts=64, num_experts_per_tok=33), -2),
+])
+def test_config_checks(kw, code):
+    lib = moe.load_library()
+    c = _cfg(**kw)
+    assert lib.moe_workspace_bytes(ctypes.byref(c), 16) == 0
+    rc = lib.moe_route(ctypes.byref(c), 16, FAKE, None, None, FAKE, FAKE, None, None, None)
+    assert rc == code
+
+
+def test_pointer_checks_and_noop():
+    lib = moe.load_library()
+    c = _cfg()
+    # T = 0 is a no-op, whatever the pointers
+    assert lib.moe_forward(ctypes.byref(c), 0, None, None, None, None, None, None, 0, None) == 0
+    assert lib.moe_route(ctypes.byref(c), -1, FAKE, None, None, FAKE, FAKE, None, None, None) == -1
+    assert lib.moe_route(ctypes.byref(c), 16, MISALIGNED, None, None, FAKE, FAKE, None, None, None) == -1
+    assert lib.moe_route(ctypes.byref(c), 16, None, None, None, FAKE, FAKE, None, None, None) == -1
+    # sgate requested without a shared expert
+    assert lib.moe_route(ctypes.byref(c), 16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == -1
+    # short workspace
+    ws_need = lib.moe_workspace_bytes(ctypes.byref(c), 16)
+    assert ws_need > 0
+    assert lib.moe_budget(ctypes.byref(c), 16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws_need - 1, None) == -3
+    assert lib.moe_dispatch(ctypes.byref(c), 16, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                            ws_need - 256, None) == -3
+    w = moe._Weights(FAKE.value, FAKE.value, FAKE.value, None, None, None, None)
+    assert lib.moe_forward(ctypes.byref(c), 16, FAKE, FAKE, ctypes.byref(w), FAKE, None, FAKE, 16, None) == -3
+    # shared expert configured but its weights missing
+    cs = _cfg(shared_intermediate_size=64)
+    assert lib.moe_forward(ctypes.byref(cs), 16, FAKE, FAKE, ctypes.byref(w), FAKE, None, FAKE,
+                           1 << 30, None) == -1
+    assert lib.moe_error_string(-3) == b"workspace too small"
+
+
+def test_workspace_grows_with_tokens():
+    lib = moe.load_library()
+    c = _cfg(shared_intermediate_size=64)
+    a = lib.moe_workspace_bytes(ctypes.byref(c), 16)
+    b = lib.moe_workspace_bytes(ctypes.byref(c), 1024)
+    assert 0 < a < b and b % 256 == 0

@@ -1,0 +1,204 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle.
+
+Bit-exact for routing indices, budget drops, counts, offsets, perm and
+slot_pos; fp32-ulp close for routing weights and the shared gate; relative
+L2 <= 5e-3 on the bf16 layer output.  Small shapes compare every output
+row and span several weight tiles, several token tiles and ragged tails;
+the full-size workloads compare seeded sample rows (routing and dispatch
+always in full).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import routed_expert_ffn_renorm_b200 as moe
+from routed_expert_ffn_renorm_b200 import workloads as W
+
+from parity_util import check_layer, gpu_forward, lib_config, sample_rows, weights_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    assert torch.cuda.get_device_capability()[0] == 10, "needs an sm_100 (B200) device"
+    moe.load_library()
+
+
+def _run(cfg, device="cuda", gen_device="cpu", rows=None, **mk):
+    inp = W.make_inputs(cfg, device=gen_device, **mk)
+    if gen_device != device:
+        inp = W.MoEInputs(*(t.to(device) if t is not None else None for t in (
+            inp.x, inp.logits, inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down,
+            inp.ws_gvec)))
+    g = gpu_forward(cfg, inp)
+    return check_layer(cfg, inp, g, rows=rows), g, inp
+
+
+SMALL = [
+    W.TINY,
+    W.MoEConfig("multi_tile", T=1000, H=384, E=4, I=192, k=2, Is=128),
+    W.MoEConfig("ragged", T=37, H=256, E=16, I=64, k=3, Is=64, zipf_alpha=1.0),
+    W.MoEConfig("k_eq_E", T=20, H=128, E=4, I=64, k=4),
+    W.MoEConfig("one_expert", T=33, H=128, E=1, I=64, k=1),
+    W.MoEConfig("single_token", T=1, H=256, E=8, I=128, k=2, Is=64),
+    W.MoEConfig("no_norm", T=50, H=256, E=8, I=128, k=2, norm_topk=False, Is=64),
+    W.MoEConfig("budget_small", T=32, H=256, E=32, I=64, k=4, budget=3, zipf_alpha=1.2),
+    W.MoEConfig("budget_one", T=32, H=256, E=32, I=64, k=4, budget=1),
+    W.MoEConfig("budget_no_norm", T=40, H=256, E=32, I=64, k=4, budget=5, norm_topk=False, Is=64),
+    W.MoEConfig("budget_chunks", T=700, H=128, E=64, I=64, k=6, budget=9, zipf_alpha=0.5),
+    W.MoEConfig("max_experts", T=64, H=128, E=1024, I=64, k=8),
+    W.MoEConfig("max_topk", T=16, H=128, E=64, I=64, k=32),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_small_layers(cfg):
+    diag, g, _ = _run(cfg)
+    print(cfg.label, diag)
+
+
+def test_hot_expert_multi_tile():
+    """Every token routes to expert 3 first: one group of T rows, several token tiles."""
+    cfg = W.MoEConfig("hot", T=600, H=256, E=8, I=128, k=2, Is=64)
+    inp = W.make_inputs(cfg)
+    inp.logits[:, 3] += 50.0
+    inp = W.MoEInputs(*(t.cuda() if t is not None else None for t in (
+        inp.x, inp.logits, inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec)))
+    g = gpu_forward(cfg, inp)
+    assert g.counts[3] == cfg.T
+    print(check_layer(cfg, inp, g))
+
+
+def test_sgate_varies():
+    """A gate vector of scale 1 makes sigmoid(g.x) spread over (0, 1)."""
+    cfg = W.MoEConfig("gate", T=64, H=512, E=8, I=64, k=2, Is=128)
+    diag, g, _ = _run(cfg, std=0.5, gate_std=1.0)
+    assert g.sgate.min() < 0.2 and g.sgate.max() > 0.8
+
+
+def test_empty_tokens_after_budget_are_zero():
+    cfg = W.MoEConfig("empty", T=32, H=256, E=128, I=64, k=8, budget=4)
+    diag, g, _ = _run(cfg)
+    assert (g.keff == 0).any()
+
+
+def test_deterministic_bits():
+    cfg = W.MoEConfig("det", T=500, H=256, E=16, I=128, k=4, Is=64, budget=10, zipf_alpha=1.0)
+    inp = W.make_inputs(cfg, device="cuda")
+    a = gpu_forward(cfg, inp)
+    b = gpu_forward(cfg, inp)
+    assert (a.out_bits == b.out_bits).all() and (a.perm == b.perm).all() and (a.w == b.w).all()
+
+
+@pytest.mark.parametrize("bn", [32, 64, 128, 256])
+def test_tile_config_invariance(bn, monkeypatch):
+    """Forced token-tile sizes give bit-identical outputs (tiling never changes a K-reduction)."""
+    cfg = W.MoEConfig("inv", T=700, H=256, E=8, I=128, k=2, Is=64, zipf_alpha=1.5)
+    inp = W.make_inputs(cfg, device="cuda")
+    ref = gpu_forward(cfg, inp)
+    monkeypatch.setenv("MOE_FORCE_BN", str(bn))
+    got = gpu_forward(cfg, inp)
+    assert (got.out_bits == ref.out_bits).all()
+
+
+def test_force_bn_rejects_bad_values(monkeypatch):
+    cfg = W.TINY
+    inp = W.make_inputs(cfg, device="cuda")
+    monkeypatch.setenv("MOE_FORCE_BN", "48")
+    with pytest.raises(moe.MoEError):
+        gpu_forward(cfg, inp)
+
+
+def test_stagewise_entry_points():
+    """route -> budget -> dispatch -> expert_ffn -> combine called one by one
+    equals moe_forward bit for bit."""
+    cfg = W.MoEConfig("stages", T=96, H=256, E=16, I=128, k=4, Is=64, budget=6, zipf_alpha=1.0)
+    inp = W.make_inputs(cfg, device="cuda")
+    ref = gpu_forward(cfg, inp)
+    c = lib_config(cfg)
+    T, k, E, H = cfg.T, cfg.k, cfg.E, cfg.H
+    dev = "cuda"
+    ws = torch.zeros(moe.workspace_bytes(c, T), dtype=torch.uint8, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    sgate = torch.empty(T, dtype=torch.float32, device=dev)
+    keff = torch.empty(T, dtype=torch.int32, device=dev)
+    kept = torch.empty(E, dtype=torch.uint8, device=dev)
+    nd = torch.empty(1, dtype=torch.int32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    slot_pos = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    ybuf = torch.empty((T, k + 1, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    moe.moe_route(c, inp.logits, idx, w, x=inp.x, ws_gate_vec=inp.ws_gvec, sgate=sgate, keff=keff)
+    moe.moe_budget(c, idx, w, keff, kept, nd, ws)
+    moe.moe_dispatch(c, idx, counts, offsets, perm, slot_pos, ws, keff=keff, x=inp.x, x_perm=x_perm)
+    moe.moe_expert_ffn(c, inp.x, x_perm, offsets, perm, w, weights_of(inp), ybuf, ws, sgate=sgate)
+    moe.moe_combine(c, ybuf, out, keff=keff)
+    torch.cuda.synchronize()
+    assert moe.status_read(ws) == 0
+    assert (W.bf16_bits(out) == ref.out_bits).all()
+    total = int(offsets[E])
+    assert (perm[:total].cpu().numpy() == ref.perm).all()
+    # x_perm rows are exact copies of the routed tokens
+    xp = x_perm[:total].cpu()
+    src = inp.x.cpu()[perm[:total].cpu().long() // k]
+    assert torch.equal(xp, src)
+
+
+def test_zero_tokens_is_noop():
+    c = lib_config(W.TINY)
+    dev = "cuda"
+    ws = torch.zeros(moe.workspace_bytes(c, 1), dtype=torch.uint8, device=dev)
+    x = torch.empty((0, W.TINY.H), dtype=torch.bfloat16, device=dev)
+    inp = W.make_inputs(W.TINY, device=dev)
+    moe.moe_forward(c, x, torch.empty((0, W.TINY.E), device=dev), weights_of(inp),
+                    torch.empty((0, W.TINY.H), dtype=torch.bfloat16, device=dev), ws)
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ full sizes --
+
+@pytest.mark.parametrize("cfg,nrows", [(W.DRAFTER_16x1024, 64), (W.DRAFTER_512x512, 16),
+                                       (W.DRAFTER_512x512.with_(zipf_alpha=0.0), 12)],
+                         ids=["drafter_16x1024", "drafter_512x512_a1", "drafter_512x512_a0"])
+def test_drafter_layers(cfg, nrows):
+    rows = sample_rows(cfg.T, nrows)
+    diag, g, _ = _run(cfg, gen_device="cuda", rows=rows)
+    print(cfg.label, diag)
+
+
+@pytest.mark.parametrize("N", W.BUDGETS)
+def test_budget_layer(N):
+    cfg = W.BUDGET_S32.with_(budget=N)
+    diag, g, _ = _run(cfg, gen_device="cuda")
+    assert g.n_dropped > 0 and int(g.kept.sum()) == N
+    print(cfg.label, diag, "n_dropped", g.n_dropped)
+
+
+@pytest.fixture(scope="module")
+def large_inputs():
+    """256 experts x 2048 x 7168 (22.5 GB bf16) drawn once; logits N(0,1) for the largest T."""
+    cfg = W.LARGE_256E.with_(T=max(W.LARGE_T_SWEEP))
+    inp = W.make_inputs(cfg, device="cuda")
+    yield cfg, inp
+    del inp
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("T,alpha,nrows", [(64, 0.0, 16), (64, 1.5, 16), (512, 1.0, 12), (4096, 1.5, 8),
+                                           (16384, 0.0, 6), (16384, 1.0, 6)])
+def test_large_layer(large_inputs, T, alpha, nrows):
+    base_cfg, base = large_inputs
+    cfg = base_cfg.with_(T=T, zipf_alpha=alpha)
+    logits = base.logits[:T] + W.zipf_bias(cfg.E, alpha, "cuda")
+    inp = W.MoEInputs(base.x[:T].contiguous(), logits.contiguous(), base.w_gate, base.w_up, base.w_down)
+    g = gpu_forward(cfg, inp)
+    diag = check_layer(cfg, inp, g, rows=sample_rows(T, nrows))
+    print(cfg.label, diag, "max group", int(g.counts.max()))
