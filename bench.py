@@ -81,19 +81,25 @@ def stage_work(cfg, counts):
     down = dict(
         flops=2 * H * I * slots + 2 * H * Is * T,
         bytes=touched * H * I * 2 + sh * H * Is * 2 + (slots * I + T * Is) * 2 + (slots + sh * T) * H * 2)
+    ffn = dict(flops=gate_up["flops"] + down["flops"],
+               bytes=touched * 3 * H * I * 2 + sh * 3 * H * Is * 2 + slots * H * 2 + sh * T * H * 2
+               + (slots + sh * T) * H * 2)
     route = dict(flops=0, bytes=T * E * 4 + T * k * 8 + sh * (T * H * 2 + H * 2 + T * 4))
     budget = dict(flops=0, bytes=(T * k * 8 * 2) if cfg.budget else 0)
     dispatch = dict(flops=0, bytes=T * k * 4 * 3 + slots * H * 2 * 2)
     combine = dict(flops=0, bytes=(slots + sh * T) * H * 2 + T * H * 2)
     layer = dict(flops=gate_up["flops"] + down["flops"],
                  bytes=touched * 3 * H * I * 2 + sh * (3 * H * Is * 2 + H * 2) + 2 * T * H * 2 + T * E * 4)
-    return dict(route=route, budget=budget, dispatch=dispatch, gate_up=gate_up, down=down, combine=combine,
+    return dict(route=route, budget=budget, dispatch=dispatch, gate_up=gate_up, down=down, ffn=ffn, combine=combine,
                 layer=layer, touched=touched, slots=slots)
 
 
 def launches_per_step(cfg) -> int:
-    # route 1, budget 2, dispatch: histogram + scan + scatter + gather 4, gate/up 1, down 1, combine 1
-    return 1 + (2 if cfg.budget else 0) + 4 + 1 + 1 + 1
+    # route 1; budget 2; dispatch: one CTA-wide sort when T*k <= 8192, else
+    # histogram + scan + scatter; gather 1; expert FFN 1 (fused) or 2 (mean
+    # group >= 128 tokens); combine 1
+    ffn = 1 if (cfg.T * cfg.k + cfg.E - 1) // cfg.E < 128 else 2
+    return 1 + (2 if cfg.budget else 0) + (1 if cfg.T * cfg.k <= 8192 else 3) + 1 + ffn + 1
 
 
 def load_peaks():
@@ -105,7 +111,7 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash() -> str:  # the grouped FFN kernel's source
     h = hashlib.sha256()
     with open(os.path.join(ROOT, "routed_expert_ffn_renorm_b200", "csrc", "ffn_gemm.cu"), "rb") as f:
         h.update(f.read())
@@ -343,36 +349,44 @@ def run_ours(args, cfg):
     gvec = P(inp.ws_gvec.data_ptr()) if cfg.Is else None
     sg = p["sgate"] if cfg.Is else None
     wsb = ws.numel()
-    sp = P(stream.cuda_stream)
 
     def chk(name, rc):
         if rc != 0:
             raise moe.MoEError(name, rc, lib.moe_error_string(rc).decode())
 
-    stages = ["route", "budget", "dispatch", "gate_up", "down", "combine"]
+    stages = ["route", "budget", "dispatch", "ffn", "combine"]
+    NEV = len(stages) + 1
 
     def step(ev):
-        ev[0].record(stream)
+        sp = P(torch.cuda.current_stream(dev).cuda_stream)  # the capture stream while capturing
+        st = torch.cuda.current_stream(dev)
+        ev[0].record(st)
         chk("moe_route", lib.moe_route(pc, T, p["logits"], p["x"] if cfg.Is else None, gvec, p["idx"], p["tw"], sg,
                                        p["keff"], sp))
-        ev[1].record(stream)
+        ev[1].record(st)
         if cfg.budget:
             chk("moe_budget", lib.moe_budget(pc, T, p["idx"], p["tw"], p["keff"], p["kept"], p["nd"], p["ws"], wsb, sp))
-        ev[2].record(stream)
+        ev[2].record(st)
         chk("moe_dispatch", lib.moe_dispatch(pc, T, p["idx"], p["keff"], p["x"], p["counts"], p["offsets"], p["perm"],
                                              p["slot_pos"], p["x_perm"], p["ws"], wsb, sp))
-        ev[3].record(stream)
-        chk("moe_expert_gate_up", lib.moe_expert_gate_up(pc, T, p["x"], p["x_perm"], p["offsets"], pw, p["ws"], wsb,
-                                                         sp))
-        ev[4].record(stream)
-        chk("moe_expert_down", lib.moe_expert_down(pc, T, p["offsets"], p["perm"], p["tw"], sg, pw, p["ybuf"],
-                                                   p["ws"], wsb, sp))
-        ev[5].record(stream)
+        ev[3].record(st)
+        chk("moe_expert_ffn", lib.moe_expert_ffn(pc, T, p["x"], p["x_perm"], p["offsets"], p["perm"], p["tw"], sg, pw,
+                                                 p["ybuf"], p["ws"], wsb, sp))
+        ev[4].record(st)
         chk("moe_combine", lib.moe_combine(pc, T, p["ybuf"], p["keff"], p["out"], sp))
-        ev[6].record(stream)
+        ev[5].record(st)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        stream.wait_stream(side)
+        return g
 
     moe.status_clear(ws)
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(7)]  # noqa: E731
+    mk = lambda ext=False: [torch.cuda.Event(enable_timing=True, external=ext) for _ in range(NEV)]  # noqa: E731
     for _ in range(args.warmup):
         flush.zero_()
         step(mk())
@@ -383,8 +397,25 @@ def run_ours(args, cfg):
     counts_h = counts.cpu().tolist()
     work = stage_work(cfg, counts_h)
 
-    # ---- timed region (device-resident inputs)
+    # ---- eager launches (diagnostic): K steps back to back from the host
     evs = [mk() for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    eager_ms = sum(e[0].elapsed_time(e[NEV - 1]) for e in evs) / args.steps
+
+    # ---- timed region: the step replayed as one CUDA graph (device-resident
+    # inputs; timing events are nodes of the graph, L2 flushed between steps)
+    gev = mk(ext=True)
+    graph = capture(lambda: step(gev))
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    stage_sum = {s: 0.0 for s in stages}
+    step_sum = 0.0
     barrier(dev)
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(dev)
@@ -392,19 +423,25 @@ def run_ours(args, cfg):
     with sampler:
         for i in range(args.steps):
             flush.zero_()
-            step(evs[i])
+            graph.replay()
+            gev[NEV - 1].synchronize()
+            for j, sname in enumerate(stages):
+                stage_sum[sname] += gev[j].elapsed_time(gev[j + 1])
+            step_sum += gev[0].elapsed_time(gev[NEV - 1])
         torch.cuda.synchronize(dev)
     host_s = time.perf_counter() - t_host0
     barrier(dev)
-    per_stage = {s: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, s in enumerate(stages)}
-    step_ms = sum(e[0].elapsed_time(e[6]) for e in evs) / args.steps
-    total_ms = max_over_ranks(step_ms * args.steps, dev)
+    per_stage = {s: v / args.steps for s, v in stage_sum.items()}
+    step_ms = step_sum / args.steps
+    total_ms = max_over_ranks(step_sum, dev)
     status = moe.status_read(ws)
     if status:
         raise RuntimeError(f"device status {status} after timing")
     value = aggregate_tokens_per_s(T, args.steps, total_ms, world)
+    del graph
 
-    # ---- end to end through moe_forward with host buffers
+    # ---- end to end through moe_forward with host buffers (one graph:
+    # pinned H2D of x and logits, the layer, D2H of the output)
     e2e = None
     if not args.no_e2e:
         xh = torch.empty((T, H), dtype=torch.bfloat16, pin_memory=True)
@@ -414,35 +451,44 @@ def run_ours(args, cfg):
         lh.copy_(inp.logits)
         xd = torch.empty_like(inp.x)
         ld = torch.empty_like(inp.logits)
+        e0, e1 = mk(ext=True)[:2]
 
-        def e2e_step(e0, e1):
-            e0.record(stream)
+        def e2e_step():
+            st = torch.cuda.current_stream(dev)
+            e0.record(st)
             xd.copy_(xh, non_blocking=True)
             ld.copy_(lh, non_blocking=True)
-            moe.moe_forward(c, xd, ld, wts, out, ws, stream=stream)
+            moe.moe_forward(c, xd, ld, wts, out, ws, stream=st)
             oh.copy_(out, non_blocking=True)
-            e1.record(stream)
+            e1.record(st)
 
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        eg = capture(e2e_step)
         for _ in range(args.warmup):
             flush.zero_()
-            e2e_step(*mk()[:2])
-        ee = [mk()[:2] for _ in range(args.steps)]
+            eg.replay()
+        torch.cuda.synchronize(dev)
+        e2e_sum = 0.0
         barrier(dev)
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
             flush.zero_()
-            e2e_step(*ee[i])
+            eg.replay()
+            e1.synchronize()
+            e2e_sum += e0.elapsed_time(e1)
         torch.cuda.synchronize(dev)
         barrier(dev)
-        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), dev)
+        e2e_ms = max_over_ranks(e2e_sum, dev)
         e2e = {"value": aggregate_tokens_per_s(T, args.steps, e2e_ms, world), "unit": "tokens/s",
                "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2,
-               "ms_per_step": e2e_ms / args.steps, "api": "moe_forward"}
+               "ms_per_step": e2e_ms / args.steps, "api": "moe_forward (one CUDA graph per step with the copies)"}
         if not torch.equal(oh.to(dev), out):
             raise RuntimeError("e2e output copy mismatch")
+        del eg
 
     peaks, peak_kind = load_peaks()
-    dom = max(("gate_up", "down", "route", "dispatch", "combine", "budget"), key=lambda s: per_stage[s])
+    dom = max(stages, key=lambda s: per_stage[s])
     long_run = (total_ms * 1e-3) > 1.0
     rl = roofline(dom, work, per_stage[dom], peaks, peak_kind, long_run,
                   recorded_traffic(dom, cfg.label))
@@ -472,7 +518,9 @@ def run_ours(args, cfg):
                   "algorithmic_bytes": work["layer"]["bytes"], "algorithmic_flops": work["layer"]["flops"],
                   "GB_per_s": layer_bw, "TFLOP_per_s": layer_tf,
                   "hbm_frac": layer_bw / peaks["hbm_gbs"]},
-        "host_enqueue_s": host_s,
+        "host_s": host_s,
+        "eager_ms_per_step": eager_ms,
+        "timing": "CUDA graph replay of the stage calls; events are graph nodes; per-step sync outside the events",
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -98,8 +98,10 @@ typedef struct {
 
 /* Bytes of device workspace the calls below need for a batch of T tokens
  * (0 for an invalid config).  The workspace is caller-allocated scratch;
- * its first 256 bytes hold the status word.  Clear the status word once
- * after allocating (moe_status_clear). */
+ * its first 8 KB hold the status word and the expert FFN's scheduling
+ * counters.  Zero that block once after allocating (moe_status_clear);
+ * every kernel leaves the counters at zero, and moe_dispatch re-zeroes them.
+ * One workspace serves one stream at a time. */
 size_t moe_workspace_bytes(const moe_config_t *cfg, int32_t T);
 
 /* Route: for each token t, topk_idx[t, 0..k) = the k experts with the
@@ -142,8 +144,9 @@ int moe_dispatch(const moe_config_t *cfg, int32_t T, const int32_t *topk_idx, co
                  const moe_bf16_t *x, int32_t *counts, int32_t *offsets, int32_t *perm,
                  int32_t *slot_pos, moe_bf16_t *x_perm, void *ws, size_t ws_bytes, void *stream);
 
-/* Expert FFN over the dispatched tokens (tcgen05 grouped GEMMs), writing the
- * weighted per-slot outputs in token order:
+/* Expert FFN over the dispatched tokens (tcgen05 grouped GEMMs; both phases
+ * in one launch while the mean expert group is under 128 tokens, two
+ * launches above), writing the weighted per-slot outputs in token order:
  *   ybuf[t, j, :] = topk_w[t, j] * FFN_{topk_idx[t, j]}(x_t)   for each kept slot,
  *   ybuf[t, k, :] = sgate[t] * FFN_shared(x_t)                  when Is > 0,
  * rounded to bf16; other rows of ybuf are left untouched.
@@ -182,7 +185,8 @@ int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const f
 /* Status word: MOE_STATUS_* bits set by kernels (sticky until cleared).
  * moe_status_read enqueues a copy on `stream`, waits for the stream, and
  * returns MOE_OK with *status_out filled (host pointer).  moe_status_clear
- * enqueues a reset of the word on `stream`. */
+ * enqueues a zeroing of the workspace's first 8 KB (status word and
+ * scheduling counters) on `stream`. */
 int moe_status_read(const void *ws, int32_t *status_out, void *stream);
 int moe_status_clear(void *ws, void *stream);
 

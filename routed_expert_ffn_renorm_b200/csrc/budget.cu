@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(256) budget_partial_kernel(int T, int E, int k
                                                              const float *__restrict__ w,
                                                              float *__restrict__ part_agg,
                                                              int32_t *__restrict__ part_cnt) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int c = blockIdx.x;
     const int t0 = c * kChunk, t1 = min(T, t0 + kChunk);
     const size_t s0 = (size_t)t0 * k, s1 = (size_t)t1 * k;
@@ -53,6 +55,8 @@ __global__ void __launch_bounds__(1024) budget_select_kernel(int T, int E, int k
     __shared__ uint8_t present[kMaxExperts];
     __shared__ uint8_t keep[kMaxExperts];
     __shared__ int nu_s;
+    pdl_launch_dependents();
+    pdl_wait();
     if (threadIdx.x == 0) nu_s = 0;
     __syncthreads();
     int my_present = 0;
@@ -123,10 +127,11 @@ cudaError_t launch_budget(int T, int E, int k, int N, int norm_topk, int32_t *id
                           uint8_t *kept, int32_t *n_dropped, float *part_agg, int32_t *part_cnt,
                           cudaStream_t st) {
     const int nchunks = budget_chunks(T);
-    budget_partial_kernel<<<nchunks, 256, 0, st>>>(T, E, k, idx, w, part_agg, part_cnt);
-    budget_select_kernel<<<1, 1024, 0, st>>>(T, E, k, N, norm_topk, nchunks, idx, w, keff, kept, n_dropped,
-                                             part_agg, part_cnt);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(budget_partial_kernel, dim3(nchunks), dim3(256), 0, st, T, E, k, idx, w, part_agg,
+                               part_cnt);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(budget_select_kernel, dim3(1), dim3(1024), 0, st, T, E, k, N, norm_topk, nchunks, idx, w, keff,
+                      kept, n_dropped, part_agg, part_cnt);
 }
 
 }  // namespace moe

@@ -10,42 +10,54 @@ namespace moe {
 
 namespace {
 
-__global__ void __launch_bounds__(128) combine_kernel(int T, int k, int H, int has_shared,
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += bf16_bits_to_f32((uint16_t)(u[q] & 0xffffu));
+        acc[2 * q + 1] += bf16_bits_to_f32((uint16_t)(u[q] >> 16));
+    }
+}
+
+// One thread per (token, 16-byte column vector); the rows of a token are
+// loaded four at a time and added in slot order.
+__global__ void __launch_bounds__(256) combine_kernel(int T, int k, int vec, int has_shared,
                                                       const uint4 *__restrict__ ybuf,
                                                       const int32_t *__restrict__ keff, uint4 *__restrict__ out) {
-    const int t = blockIdx.x;
-    const int vec = H / 8;
-    const int ke = keff ? keff[t] : k;
-    const uint4 *rows = ybuf + (size_t)t * (k + 1) * vec;
-    for (int c = threadIdx.x; c < vec; c += blockDim.x) {
-        float acc[8];
+    pdl_launch_dependents();
+    pdl_wait();
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int t = (int)(gid / vec), c = (int)(gid % vec);
+    if (t >= T) return;
+    const int ke = keff ? __ldg(keff + t) : k;
+    const uint4 *rows = ybuf + (size_t)t * (k + 1) * vec + c;
+    float acc[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-        for (int j = 0; j <= k; ++j) {
-            if (j < k ? j >= ke : !has_shared) continue;
-            const uint4 v = __ldg(rows + (size_t)j * vec + c);
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int j0 = 0; j0 < ke; j0 += 4) {
+        uint4 v[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                acc[2 * q] += bf16_bits_to_f32((uint16_t)(u[q] & 0xffffu));
-                acc[2 * q + 1] += bf16_bits_to_f32((uint16_t)(u[q] >> 16));
-            }
-        }
-        uint32_t o[4];
+        for (int u = 0; u < 4; ++u) v[u] = (j0 + u < ke) ? __ldg(rows + (size_t)(j0 + u) * vec) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            o[q] = (uint32_t)f32_to_bf16_bits(acc[2 * q]) | ((uint32_t)f32_to_bf16_bits(acc[2 * q + 1]) << 16);
-        out[(size_t)t * vec + c] = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int u = 0; u < 4; ++u)
+            if (j0 + u < ke) add_bf16x8(acc, v[u]);
     }
+    if (has_shared) add_bf16x8(acc, __ldg(rows + (size_t)k * vec));
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        o[q] = (uint32_t)f32_to_bf16_bits(acc[2 * q]) | ((uint32_t)f32_to_bf16_bits(acc[2 * q + 1]) << 16);
+    out[(size_t)t * vec + c] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 }  // namespace
 
 cudaError_t launch_combine(int T, int k, int H, int has_shared, const uint16_t *ybuf, const int32_t *keff,
                            uint16_t *out, cudaStream_t st) {
-    combine_kernel<<<T, 128, 0, st>>>(T, k, H, has_shared, reinterpret_cast<const uint4 *>(ybuf), keff,
-                                      reinterpret_cast<uint4 *>(out));
-    return cudaGetLastError();
+    const int vec = H / 8;
+    const long long threads = (long long)T * vec;
+    return launch_pdl(combine_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st, T, k, vec, has_shared,
+                      reinterpret_cast<const uint4 *>(ybuf), keff, reinterpret_cast<uint4 *>(out));
 }
 
 }  // namespace moe

@@ -11,7 +11,9 @@
 //            id, 32 at a time; __match_any_sync groups lanes with the same
 //            expert, the rank inside the group is the count of lower lanes,
 //            so positions follow slot order exactly;
-//   gather   x_perm[p] = x[perm[p] / k], one 16-byte vector per thread.
+//   gather   x_perm[p] = x[perm[p] / k], four 16-byte vectors per thread.
+// Batches of up to kSmallSlots slots run hist + scan + scatter as one CTA
+// (dispatch_small_kernel) to save two launches.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -19,10 +21,37 @@ namespace moe {
 namespace {
 
 constexpr int kTokChunk = 64;
+constexpr int kSmallSlots = 8192;  // T*k up to this: the whole sort in one CTA
+
+// Exclusive prefix sum of one value per thread over a 1024-thread block.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int ws = warp_sums[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, ws, off);
+            if (lane >= off) ws += o;
+        }
+        warp_sums[lane] = ws;  // inclusive over warps
+    }
+    __syncthreads();
+    return incl - v + (wid ? warp_sums[wid - 1] : 0);
+}
 
 __global__ void __launch_bounds__(256) hist_kernel(int T, int E, int k, const int32_t *__restrict__ idx,
                                                    const int32_t *__restrict__ keff, int32_t *__restrict__ hist) {
     __shared__ int h[kMaxExperts];
+    pdl_launch_dependents();
+    pdl_wait();
     for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
     __syncthreads();
     const int t0 = blockIdx.x * kTokChunk, t1 = min(T, t0 + kTokChunk);
@@ -39,33 +68,22 @@ __global__ void __launch_bounds__(256) hist_kernel(int T, int E, int k, const in
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int32_t *__restrict__ hist,
-                                                    int32_t *__restrict__ counts, int32_t *__restrict__ offsets) {
+                                                    int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                                                    int32_t *__restrict__ sched, int32_t *__restrict__ hdone) {
     __shared__ int warp_sums[32];
+    pdl_launch_dependents();
+    pdl_wait();
     const int e = threadIdx.x;  // blockDim.x == 1024 >= E
+    if (sched != nullptr && e < 2) {  // fresh work-item counters for the grouped FFN launches
+        sched[4 + e] = 0;
+        sched[8 + e] = 0;
+    }
+    if (hdone != nullptr)
+        for (int g = e; g <= E; g += blockDim.x) hdone[g] = 0;
     int c = 0;
     if (e < E)
         for (int b = 0; b < nchunks; ++b) c += hist[(size_t)b * E + e];
-    // block-wide exclusive scan of c over e
-    const int lane = e & 31, wid = e >> 5;
-    int incl = c;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-    }
-    if (lane == 31) warp_sums[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        int ws = warp_sums[lane];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, ws, off);
-            if (lane >= off) ws += o;
-        }
-        warp_sums[lane] = ws;  // inclusive
-    }
-    __syncthreads();
-    const int excl = incl - c + (wid ? warp_sums[wid - 1] : 0);
+    const int excl = block_exclusive_scan(c, warp_sums);
     if (e < E) {
         counts[e] = c;
         offsets[e] = excl;
@@ -84,6 +102,8 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
                                                      const int32_t *__restrict__ hist, int32_t *__restrict__ perm,
                                                      int32_t *__restrict__ slot_pos) {
     __shared__ int base[kMaxExperts];
+    pdl_launch_dependents();
+    pdl_wait();
     const int lane = threadIdx.x;
     for (int e = lane; e < E; e += 32) base[e] = hist[(size_t)blockIdx.x * E + e];
     __syncwarp();
@@ -114,20 +134,106 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
     }
 }
 
-__global__ void __launch_bounds__(256) gather_kernel(int k, int H, const int32_t *__restrict__ offsets, int E,
-                                                     const int32_t *__restrict__ perm, const uint4 *__restrict__ x,
-                                                     uint4 *__restrict__ x_perm, int rows_per_block) {
-    const int total = offsets[E];
-    const int vec = H / 8;  // 16-byte vectors per row
-    const int p0 = blockIdx.x * rows_per_block;
-    for (int r = 0; r < rows_per_block; ++r) {
-        const int p = p0 + r;
-        if (p >= total) return;
-        const int t = perm[p] / k;
-        const uint4 *src = x + (size_t)t * vec;
-        uint4 *dst = x_perm + (size_t)p * vec;
-        for (int c = threadIdx.x; c < vec; c += blockDim.x) dst[c] = __ldg(src + c);
+// Whole counting sort for a small batch in one 1024-thread CTA: warps
+// 0..W-1 each own a contiguous run of slots; per-warp counts (shared
+// memory), one exclusive scan over experts, per-warp bases, then each warp
+// scatters its run in slot order with __match_any_sync ranks.
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int k, int W,
+                                                              const int32_t *__restrict__ idx,
+                                                              const int32_t *__restrict__ keff,
+                                                              int32_t *__restrict__ counts,
+                                                              int32_t *__restrict__ offsets,
+                                                              int32_t *__restrict__ perm,
+                                                              int32_t *__restrict__ slot_pos, int32_t *__restrict__ sched,
+                                                              int32_t *__restrict__ hdone) {
+    extern __shared__ int hist[];  // [W][E]
+    __shared__ int warp_sums[32];
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Tk = T * k, chunk = (Tk + W - 1) / W;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) hist[i] = 0;
+    if (sched != nullptr && threadIdx.x < 2) {
+        sched[4 + threadIdx.x] = 0;
+        sched[8 + threadIdx.x] = 0;
     }
+    if (hdone != nullptr)
+        for (int g = threadIdx.x; g <= E; g += blockDim.x) hdone[g] = 0;
+    __syncthreads();
+    const int s_begin = warp * chunk, s_end = min(Tk, s_begin + chunk);
+    if (warp < W) {
+        for (int s0 = s_begin; s0 < s_end; s0 += 32) {
+            const int s = s0 + lane;
+            int key = -1;
+            if (s < s_end) {
+                const int t = s / k, j = s - t * k;
+                const int e = idx[s];
+                if (j < (keff ? keff[t] : k) && e >= 0 && e < E) key = e;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, key);
+            if (key >= 0 && lane == __ffs(peers) - 1) hist[warp * E + key] += __popc(peers);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    const int e = threadIdx.x;
+    int c = 0;
+    if (e < E)
+        for (int w = 0; w < W; ++w) c += hist[w * E + e];
+    const int excl = block_exclusive_scan(c, warp_sums);
+    if (e < E) {
+        counts[e] = c;
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = excl + c;
+        int run = excl;
+        for (int w = 0; w < W; ++w) {
+            const int hw = hist[w * E + e];
+            hist[w * E + e] = run;
+            run += hw;
+        }
+    }
+    __syncthreads();
+    if (warp < W) {
+        int *base = hist + warp * E;
+        for (int s0 = s_begin; s0 < s_end; s0 += 32) {
+            const int s = s0 + lane;
+            int key = -1;
+            if (s < s_end) {
+                const int t = s / k, j = s - t * k;
+                const int ee = idx[s];
+                if (j < (keff ? keff[t] : k) && ee >= 0 && ee < E) key = ee;
+                else slot_pos[s] = -1;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, key);
+            if (key >= 0) {
+                const int pos = base[key] + __popc(peers & ((1u << lane) - 1u));
+                perm[pos] = s;
+                slot_pos[s] = pos;
+            }
+            __syncwarp();
+            if (key >= 0 && lane == 31 - __clz(peers)) base[key] += __popc(peers);
+            __syncwarp();
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) gather_kernel(int k, int vec4, const int32_t *__restrict__ offsets, int E,
+                                                     const int32_t *__restrict__ perm, const uint4 *__restrict__ x,
+                                                     uint4 *__restrict__ x_perm) {
+    pdl_launch_dependents();
+    pdl_wait();
+    // one thread copies 4 consecutive 16-byte vectors (64 B) of one row
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int p = (int)(gid / vec4), c = (int)(gid % vec4) * 4;
+    if (p >= __ldg(offsets + E)) return;
+    const int t = __ldg(perm + p) / k;
+    const uint4 *src = x + (size_t)t * vec4 * 4 + c;
+    uint4 *dst = x_perm + (size_t)p * vec4 * 4 + c;
+    const uint4 a = __ldg(src), b = __ldg(src + 1), d = __ldg(src + 2), e = __ldg(src + 3);
+    dst[0] = a;
+    dst[1] = b;
+    dst[2] = d;
+    dst[3] = e;
 }
 
 }  // namespace
@@ -135,22 +241,27 @@ __global__ void __launch_bounds__(256) gather_kernel(int k, int H, const int32_t
 int dispatch_chunks(int T) { return (T + kTokChunk - 1) / kTokChunk; }
 
 cudaError_t launch_dispatch(int T, int E, int k, const int32_t *idx, const int32_t *keff, int32_t *hist,
-                            int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos, cudaStream_t st) {
+                            int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
+                            int32_t *status_block, int32_t *hdone, cudaStream_t st) {
+    if ((long long)T * k <= kSmallSlots) {
+        const int W = E <= 256 ? 32 : (E <= 512 ? 16 : 8);  // per-warp counts fit in 32 KB
+        return launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), (size_t)W * E * 4, st, T, E, k, W, idx, keff,
+                          counts, offsets, perm, slot_pos, status_block, hdone);
+    }
     const int nchunks = dispatch_chunks(T);
-    hist_kernel<<<nchunks, 256, 0, st>>>(T, E, k, idx, keff, hist);
-    scan_kernel<<<1, 1024, 0, st>>>(E, nchunks, hist, counts, offsets);
-    scatter_kernel<<<nchunks, 32, 0, st>>>(T, E, k, idx, keff, hist, perm, slot_pos);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(hist_kernel, dim3(nchunks), dim3(256), 0, st, T, E, k, idx, keff, hist);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, E, nchunks, hist, counts, offsets, status_block, hdone);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(scatter_kernel, dim3(nchunks), dim3(32), 0, st, T, E, k, idx, keff, hist, perm, slot_pos);
 }
 
 cudaError_t launch_gather_rows(int T, int k, int H, const int32_t *offsets, int E, const int32_t *perm,
                                const uint16_t *x, uint16_t *x_perm, cudaStream_t st) {
-    const int rows_per_block = 4;
-    const long long max_rows = (long long)T * k;
-    const int blocks = (int)((max_rows + rows_per_block - 1) / rows_per_block);
-    gather_kernel<<<blocks, 256, 0, st>>>(k, H, offsets, E, perm, reinterpret_cast<const uint4 *>(x),
-                                          reinterpret_cast<uint4 *>(x_perm), rows_per_block);
-    return cudaGetLastError();
+    const int vec4 = H / 32;  // groups of four 16-byte vectors per row (H % 128 == 0)
+    const long long threads = (long long)T * k * vec4;
+    return launch_pdl(gather_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st, k, vec4, offsets, E,
+                      perm, reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(x_perm));
 }
 
 }  // namespace moe

@@ -1,48 +1,53 @@
 // Grouped expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM),
-// fed by TMA.  Two launches of one persistent, warp-specialised kernel:
+// fed by TMA: one persistent, warp-specialised kernel whose work items are
+// tiles of two GEMM phases,
 //
-//   gated (GEMM1):  h[p, i] = silu(W_gate[e] x_p)_i * (W_up[e] x_p)_i
-//   down  (GEMM2):  ybuf[row(p), :] = w_p * (W_down[e] h_p)
+//   gate/up (phase 0):  h[p, i] = silu(W_gate[e] x_p)_i * (W_up[e] x_p)_i
+//   down    (phase 1):  ybuf[row(p), :] = w_p * (W_down[e] h_p)
 //
 // for every dispatched row p of expert e (SpecForge PR #943,
 // "Modifications": gated expert FFN, grouped dispatch; its parameter table
 // fixes gate/up/down of H x I each), and the same for the shared expert,
 // whose rows are all T tokens in token order and whose weight is the
-// sigmoid gate.
+// sigmoid gate.  A launch runs phase 0, phase 1 or both; with both, a
+// down item of a group waits (bounded) until every gate/up item of that
+// group has stored its h rows, so the tail of one phase overlaps the start
+// of the other and the layer's FFN is one launch.
 //
 // Orientation ("swap AB").  The weights sit in the MMA M slot (128 weight
-// rows per tile) and the tokens of one expert in the N slot (16..256 per
+// rows per tile) and the tokens of one group in the N slot (16..256 per
 // tile), so a group of 3 tokens costs an N=16 MMA, not a 128-row padded
-// tile: the decode-sized batches of the drafter layers stream weights and
-// barely touch the tensor pipe, the large batches fill N = 256.
-//   gated tile: A = [64 gate rows ; 64 up rows] of the same intermediate
-//               indices, so gate and up of index i land in TMEM lanes i and
-//               64 + i and the epilogue pairs them through shared memory;
-//   down tile:  A = 128 rows of W_down (128 output columns).
+// tile: decode-sized batches stream weights and barely touch the tensor
+// pipe, large batches fill N = 256.
+//   gate/up tile: A = [64 gate rows ; 64 up rows] of the same intermediate
+//                 indices, so gate and up of index i land in TMEM lanes i and
+//                 64 + i and the epilogue pairs them through shared memory;
+//   down tile:    A = 128 rows of W_down (128 output columns).
 // Both operands are K-major bf16 in 128-byte-swizzled shared memory, loaded
 // by TMA boxes of 64 K-elements; the accumulator is fp32 in TMEM, double
 // buffered (2 x BN columns) so the epilogue of one tile overlaps the
 // mainloop of the next.
 //
-// Roles (192 threads, one CTA per SM, persistent over a static stride of
-// work items):  warp 0 -- TMA producer (one lane); warp 1 -- TMEM
-// allocation and MMA issue (one lane); warps 2..5 -- epilogue, one TMEM lane
-// quarter each.
+// Roles (192 threads, one CTA per SM, persistent): warp 0 -- TMA producer
+// (one lane); warp 1 -- TMEM allocation and MMA issue (one lane); warps
+// 2..5 -- epilogue, one TMEM lane quarter each.
 //
-// Work items are (expert, weight tile r, token tile j) ordered by expert,
-// then r, then j, so the token tiles that reuse a weight tile run side by
-// side (one HBM read, L2 hits) and the tile list is derived in-kernel from
-// the dispatch offsets -- no host sync.  The token tile's TMA box height is
-// picked per tile (16, 32, 64, 128 or 256 rows) and the MMA N is the valid
-// token count rounded up to 16.
+// Work items are handed out dynamically (a global counter) in the order
+// phase 0 [shared expert, routed experts ascending], phase 1 [routed
+// experts ascending, shared expert]; inside a group, weight tile outer and
+// token tile inner, so token tiles that reuse a weight tile run side by side
+// (one HBM read, L2 hits).  The item table is derived in-kernel from the
+// dispatch offsets -- no host sync.  The token box height (16..256 rows) is
+// picked per tile and the MMA N is the valid token count rounded up to 16.
 //
-// Every wait on an mbarrier is bounded: past the limit the kernel sets
-// MOE_STATUS_TIMEOUT in the status word, the other roles see an abort flag
-// and stop, the producer waits (bounded) for its copies in flight, the MMA
-// lane for its MMAs, and TMEM is freed before exit.
+// Every wait is bounded: past the limit the kernel sets MOE_STATUS_TIMEOUT
+// in the status word, the other roles see an abort flag and stop, the
+// producer waits (bounded) for its copies in flight, the MMA lane for its
+// MMAs, and TMEM is freed before exit.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -58,31 +63,40 @@ constexpr int kTileM = 128;                    // weight rows per tile (MMA M)
 constexpr int kABytes = kTileM * kBlockK * 2;  // 16 KB
 constexpr int kNumBox = 5;                     // token box heights 16 << i
 constexpr int kThreads = 192;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 16;
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
 constexpr int kXchgStride = 33;                // fp32 exchange row stride (bank-conflict free)
+constexpr int kQueue = 4;                      // work-item queue depth (producer -> MMA, epilogue)
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 
-struct __align__(64) GemmMaps {
-    CUtensorMap a0, a1;       // routed A (gated: W_gate, W_up as [E*I, H]; down: W_down as [E*H, I])
-    CUtensorMap s0, s1;       // shared A (gated: ws_gate, ws_up [Is, H]; down: ws_down [H, Is])
+struct PhaseMaps {
+    CUtensorMap a0, a1;       // routed A: gate/up W_gate, W_up as [E*I, H]; down W_down as [E*H, I] (a1 unused)
+    CUtensorMap s0, s1;       // shared A: gate/up ws_gate, ws_up [Is, H]; down ws_down [H, Is] (s1 unused)
     CUtensorMap b[kNumBox];   // routed activations [T*k, K], box heights 16 << i
     CUtensorMap bs[kNumBox];  // shared activations [T, K]
 };
 
-struct GemmParams {
+struct __align__(64) FfnMaps {
+    PhaseMaps ph[2];  // [0] gate/up, [1] down
+};
+
+struct FfnParams {
     int T, H, E, I, k, Is;
-    int BN;        // token tile (power of two, 16..256)
-    int R, Rs;     // weight tiles per routed / shared expert
-    int nk, nks;   // K steps routed / shared
+    int BN;             // token tile (power of two, 32..256)
     int stages;
+    int phases;         // bit 0: gate/up items, bit 1: down items
+    int R[2], Rs[2];    // weight tiles per routed / shared expert, per phase
+    int nk[2], nks[2];  // K steps routed / shared, per phase
     const int32_t *offsets;
     const int32_t *perm;
     const float *topk_w;
     const float *sgate;
-    uint16_t *out_routed;  // gated: h_perm [T*k, I]; down: ybuf [T, k+1, H]
-    uint16_t *out_shared;  // gated: h_shared [T, Is]; down: ybuf
-    int32_t *status;
+    uint16_t *h_perm;    // [T*k, I]
+    uint16_t *h_shared;  // [T, Is]
+    uint16_t *ybuf;      // [T, k+1, H]
+    int32_t *status;     // status word
+    int32_t *sched;      // [0] next work item, [1] CTAs done; zero between launches
+    int32_t *hdone;      // [E+1] finished gate/up items per group (E = shared); zero between launches
 };
 
 // ------------------------------------------------------------ PTX helpers --
@@ -193,43 +207,70 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ------------------------------------------------------------ scheduling --
 struct Item {
+    int ph;      // 0 gate/up, 1 down
     int shared;  // 1: shared expert
     int e;       // routed expert
     int r;       // weight tile
     int row0;    // first activation row of the token tile
     int nvalid;  // valid tokens in the tile (1..BN)
+    int ntt;     // token tiles of the group
 };
 
-__device__ __forceinline__ Item decode_item(int item, int routed_items, const int *item_base, const int *offs,
-                                            const GemmParams &p) {
+struct Schedule {
+    int n[2];         // items per phase (0 when the phase is not run)
+    int shared_ntt;   // token tiles of the shared expert (0 if none)
+    const int *tile_base;  // [E+1] prefix of token tiles over routed experts (shared memory)
+    const int *offs;       // [E+1] dispatch offsets (shared memory)
+};
+
+__device__ __forceinline__ Item decode_item(int item, const Schedule &sc, const FfnParams &p) {
     Item it;
-    if (item < routed_items) {
-        int lo = 0, hi = p.E - 1;  // largest e with item_base[e] <= item
+    it.ph = item < sc.n[0] ? 0 : 1;
+    if (it.ph) item -= sc.n[0];
+    const int sh_items = p.Rs[it.ph] * sc.shared_ntt;
+    const int rt_items = sc.tile_base[p.E] * p.R[it.ph];
+    // phase 0: shared first; phase 1: shared last
+    const bool is_shared = it.ph == 0 ? item < sh_items : item >= rt_items;
+    if (is_shared) {
+        const int local = it.ph == 0 ? item : item - rt_items;
+        const int j = local % sc.shared_ntt;
+        it.shared = 1;
+        it.e = p.E;
+        it.r = local / sc.shared_ntt;
+        it.row0 = j * p.BN;
+        it.nvalid = min(p.BN, p.T - j * p.BN);
+        it.ntt = sc.shared_ntt;
+    } else {
+        const int local_all = it.ph == 0 ? item - sh_items : item;
+        const int tile_item = local_all;  // routed items: tile_base[e] * R + (r * ntt + j)
+        int lo = 0, hi = p.E - 1;         // largest e with tile_base[e] * R <= tile_item
+        const int R = p.R[it.ph];
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (item_base[mid] <= item) lo = mid;
+            if (sc.tile_base[mid] * R <= tile_item) lo = mid;
             else hi = mid - 1;
         }
-        const int cnt = offs[lo + 1] - offs[lo];
+        const int cnt = sc.offs[lo + 1] - sc.offs[lo];
         const int ntt = (cnt + p.BN - 1) / p.BN;
-        const int local = item - item_base[lo];
+        const int local = tile_item - sc.tile_base[lo] * R;
         const int j = local % ntt;
         it.shared = 0;
         it.e = lo;
         it.r = local / ntt;
-        it.row0 = offs[lo] + j * p.BN;
+        it.row0 = sc.offs[lo] + j * p.BN;
         it.nvalid = min(p.BN, cnt - j * p.BN);
-    } else {
-        const int ntt = (p.T + p.BN - 1) / p.BN;
-        const int local = item - routed_items;
-        const int j = local % ntt;
-        it.shared = 1;
-        it.e = 0;
-        it.r = local / ntt;
-        it.row0 = j * p.BN;
-        it.nvalid = min(p.BN, p.T - j * p.BN);
+        it.ntt = ntt;
     }
     return it;
 }
@@ -243,28 +284,29 @@ __device__ __forceinline__ int box_index(int nvalid) {
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
 // --------------------------------------------------------------- kernel --
-template <bool kGated>
-__global__ void __launch_bounds__(kThreads, 1)
-    ffn_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnMaps maps, const FfnParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = p.stages;
     const int stage_bytes = kABytes + p.BN * 128;
     uint8_t *stages = smem;
     float *xchg = reinterpret_cast<float *>(smem + (size_t)S * stage_bytes);
-    int *item_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
-    int *offs = item_base + (p.E + 1);                                   // [E + 1]
+    int *tile_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
+    int *offs = tile_base + (p.E + 1);                                  // [E + 1]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
         (reinterpret_cast<uintptr_t>(offs + (p.E + 1)) + 7) & ~uintptr_t(7));
     uint64_t *full = bars, *empty = bars + S, *tfull = bars + 2 * S, *tempty = bars + 2 * S + 2;
     uint64_t *mma_done = bars + 2 * S + 4;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    uint64_t *qfull = bars + 2 * S + 5, *qempty = qfull + kQueue;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qempty + kQueue);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
-    int *scan_tmp = reinterpret_cast<int *>(tmem_slot + 4);  // [kThreads]
+    volatile int *epi_item = reinterpret_cast<volatile int *>(tmem_slot + 2);
+    volatile int *qitem = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kQueue]
+    int *scan_tmp = reinterpret_cast<int *>(tmem_slot + 8);                 // [kThreads]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tmem_cols = 2 * p.BN;
+    pdl_launch_dependents();
 
     // ---- setup: barriers, TMEM, tile schedule
     if (threadIdx.x == 0) {
@@ -277,16 +319,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tempty[a], 1);
         }
         mbar_init(mma_done, 1);
+        for (int q = 0; q < kQueue; ++q) {
+            mbar_init(&qfull[q], 1);
+            mbar_init(&qempty[q], 2);  // the MMA lane and the elected epilogue thread
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&maps.a0);
-        prefetch_tmap(&maps.s0);
-        if (kGated) {
-            prefetch_tmap(&maps.a1);
-            prefetch_tmap(&maps.s1);
+        for (int ph = 0; ph < 2; ++ph)
+            if ((p.phases >> ph) & 1) {
+                prefetch_tmap(&maps.ph[ph].a0);
+                prefetch_tmap(&maps.ph[ph].s0);
+            }
+        if (p.phases & 1) {
+            prefetch_tmap(&maps.ph[0].a1);
+            prefetch_tmap(&maps.ph[0].s1);
         }
     }
     if (warp == 1) {
@@ -296,7 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         tc_fence_before();
     }
-    // item_base[e] = sum_{e' < e} ceil(count(e') / BN) * R  (block scan)
+    pdl_wait();  // the dispatch outputs and activations are ready past this point
+    // tile_base[e] = sum_{e' < e} ceil(count(e') / BN)  (block scan over experts)
     {
         const int per = (p.E + kThreads - 1) / kThreads;
         const int e0 = threadIdx.x * per, e1 = min(p.E, e0 + per);
@@ -305,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int o0 = __ldg(p.offsets + e), o1 = __ldg(p.offsets + e + 1);
             offs[e] = o0;
             if (e == p.E - 1) offs[p.E] = o1;
-            local += (o1 - o0 + p.BN - 1) / p.BN * p.R;
+            local += (o1 - o0 + p.BN - 1) / p.BN;
         }
         scan_tmp[threadIdx.x] = local;
         __syncthreads();
@@ -333,15 +383,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         int run = scan_tmp[threadIdx.x];
         for (int e = e0; e < e1; ++e) {
-            item_base[e] = run;
-            run += (offs[e + 1] - offs[e] + p.BN - 1) / p.BN * p.R;
+            tile_base[e] = run;
+            run += (offs[e + 1] - offs[e] + p.BN - 1) / p.BN;
         }
-        if (e1 == p.E && e0 < e1) item_base[p.E] = run;
+        if (e1 == p.E && e0 < e1) tile_base[p.E] = run;
     }
     __syncthreads();
     tc_fence_after();
-    const int routed_items = item_base[p.E];
-    const int total_items = routed_items + (p.Is > 0 ? p.Rs * ((p.T + p.BN - 1) / p.BN) : 0);
+    Schedule sc;
+    sc.shared_ntt = p.Is > 0 ? (p.T + p.BN - 1) / p.BN : 0;
+    sc.tile_base = tile_base;
+    sc.offs = offs;
+    for (int ph = 0; ph < 2; ++ph)
+        sc.n[ph] = ((p.phases >> ph) & 1) ? p.Rs[ph] * sc.shared_ntt + tile_base[p.E] * p.R[ph] : 0;
+    const int total_items = sc.n[0] + sc.n[1];
+    const bool fused = p.phases == 3;
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
@@ -349,15 +405,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_phase = 0;
-            for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
-                const Item it = decode_item(item, routed_items, item_base, offs, p);
+            for (int li = 0;; ++li) {
+                const int slot = li % kQueue;
+                const uint32_t qph = (uint32_t)(li / kQueue) & 1u;
+                if (!mbar_wait(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
+                int item = atomicAdd(p.sched, 1);
+                if (item >= total_items) item = -1;
+                qitem[slot] = item;
+                mbar_arrive(&qfull[slot]);
+                if (item < 0) break;
+                const Item it = decode_item(item, sc, p);
+                if (fused && it.ph == 1) {
+                    // wait until every gate/up tile of the group has stored its h rows
+                    const int32_t *flag = p.hdone + (it.shared ? p.E : it.e);
+                    const int target = (it.shared ? p.Rs[0] : p.R[0]) * it.ntt;
+                    bool ready = ld_acquire(flag) >= target;
+                    const unsigned long long t0 = ready ? 0ull : globaltimer();
+                    for (uint32_t spin = 1; !ready; ++spin) {
+                        ready = ld_acquire(flag) >= target;
+                        if (!ready && (spin & 63u) == 0) {
+                            if (*abort_flag) break;
+                            if (globaltimer() - t0 > kWaitLimitNs) {
+                                *abort_flag = 1;
+                                atomicOr(p.status, MOE_STATUS_TIMEOUT);
+                                break;
+                            }
+                        }
+                    }
+                    if (!ready) break;
+                    fence_proxy_async_global();  // the TMA loads below read h written by other CTAs
+                }
+                const PhaseMaps &pm = maps.ph[it.ph];
                 const int bi = box_index(it.nvalid);
-                const CUtensorMap *ma0 = it.shared ? &maps.s0 : &maps.a0;
-                const CUtensorMap *ma1 = it.shared ? &maps.s1 : &maps.a1;
-                const CUtensorMap *mb = it.shared ? &maps.bs[bi] : &maps.b[bi];
-                const int a_row = kGated ? (it.shared ? 0 : it.e * p.I) + it.r * 64
-                                         : (it.shared ? 0 : it.e * p.H) + it.r * kTileM;
-                const int nk = it.shared ? p.nks : p.nk;
+                const CUtensorMap *ma0 = it.shared ? &pm.s0 : &pm.a0;
+                const CUtensorMap *ma1 = it.shared ? &pm.s1 : &pm.a1;
+                const CUtensorMap *mb = it.shared ? &pm.bs[bi] : &pm.b[bi];
+                const int a_row = it.ph == 0 ? (it.shared ? 0 : it.e * p.I) + it.r * 64
+                                             : (it.shared ? 0 : it.e * p.H) + it.r * kTileM;
+                const int nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
                 const uint32_t bytes = kABytes + (uint32_t)(16 << bi) * 128u;
                 bool ok = true;
                 for (int ks = 0; ks < nk; ++ks) {
@@ -367,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t *sA = stages + (size_t)stage * stage_bytes;
                     mbar_arrive_expect_tx(&full[stage], bytes);
-                    if (kGated) {
+                    if (it.ph == 0) {
                         tma_load_2d(ma0, &full[stage], sA, ks * kBlockK, a_row);
                         tma_load_2d(ma1, &full[stage], sA + kABytes / 2, ks * kBlockK, a_row);
                     } else {
@@ -390,18 +475,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
-            int stage = 0, local = 0;
+            int stage = 0;
             uint32_t phase = 0;
-            for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++local) {
-                const Item it = decode_item(item, routed_items, item_base, offs, p);
+            for (int li = 0;; ++li) {
+                const int slot = li % kQueue;
+                if (!mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) break;
+                const int item = qitem[slot];
+                mbar_arrive(&qempty[slot]);
+                if (item < 0) break;
+                const Item it = decode_item(item, sc, p);
                 const int n = (it.nvalid + 15) & ~15;
                 const uint32_t idesc = idesc_bf16(n);
-                const int acc = local & 1;
-                const uint32_t use = (uint32_t)(local >> 1);
+                const int acc = li & 1;
+                const uint32_t use = (uint32_t)(li >> 1);
                 if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag, p.status, true)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(acc * p.BN);
-                const int nk = it.shared ? p.nks : p.nk;
+                const int nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
                 bool ok = true;
                 for (int ks = 0; ks < nk; ++ks) {
                     if (!mbar_wait(&full[stage], phase, abort_flag, p.status, true)) {
@@ -430,20 +520,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================= epilogue (warps 2..5) =================
         const int q = warp & 3;  // TMEM lane quarter of this warp
         const bool elected = (warp == 2 && lane == 0);
-        int local = 0;
-        for (int item = blockIdx.x; item < total_items; item += gridDim.x, ++local) {
-            const Item it = decode_item(item, routed_items, item_base, offs, p);
-            const int acc = local & 1;
-            const uint32_t use = (uint32_t)(local >> 1);
-            if (elected) *epi_ok = mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 1 : 0;
+        for (int li = 0;; ++li) {
+            const int acc = li & 1;
+            const uint32_t use = (uint32_t)(li >> 1);
+            if (elected) {  // one thread takes the item and waits for its accumulator
+                int item = -2;
+                const int slot = li % kQueue;
+                if (mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) {
+                    item = qitem[slot];
+                    mbar_arrive(&qempty[slot]);
+                    if (item >= 0 && !mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true)) item = -2;
+                }
+                *epi_item = item;
+            }
             named_bar_sync(1, 128);
-            if (!*epi_ok) break;
+            const int item = *epi_item;
+            if (item < 0) break;
+            const Item it = decode_item(item, sc, p);
             tc_fence_after();
             const uint32_t tbase = tmem_base + (uint32_t)(acc * p.BN) + ((uint32_t)(q * 32) << 16);
             for (int c0 = 0; c0 < it.nvalid; c0 += 32) {
                 float v[32];
                 tmem_ld32(tbase + (uint32_t)c0, v);
-                if (kGated) {
+                if (it.ph == 0) {
                     if (q < 2) {  // gate rows 0..63: silu(g) to the exchange buffer
                         float *xr = xchg + (q * 32 + lane) * kXchgStride;
 #pragma unroll
@@ -453,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (q >= 2) {  // up rows 64..127: h = silu(g) * u
                         const int row = (q - 2) * 32 + lane;
                         const float *xr = xchg + row * kXchgStride;
-                        uint16_t *out = it.shared ? p.out_shared : p.out_routed;
+                        uint16_t *out = it.shared ? p.h_shared : p.h_perm;
                         const int ld = it.shared ? p.Is : p.I;
                         uint16_t *dst = out + (size_t)(it.row0 + c0) * ld + it.r * 64 + row;
 #pragma unroll
@@ -477,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mw = __ldg(p.topk_w + slot);
                         }
                     }
-                    uint16_t *out = p.out_routed + it.r * kTileM + q * 32 + lane;
+                    uint16_t *out = p.ybuf + it.r * kTileM + q * 32 + lane;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int rr = __shfl_sync(0xffffffffu, mrow, i);
@@ -487,8 +586,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_before();
+            if (fused && it.ph == 0) __threadfence();  // h rows visible before the group counter moves
             named_bar_sync(1, 128);
-            if (elected) mbar_arrive(&tempty[acc]);
+            if (elected) {
+                mbar_arrive(&tempty[acc]);
+                if (fused && it.ph == 0) atomicAdd(p.hdone + (it.shared ? p.E : it.e), 1);
+            }
         }
     }
 
@@ -497,6 +600,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols)
                      : "memory");
+    }
+    // The last CTA out resets the counters for the next launch.
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+            atomicExch(p.sched, 0);
+            atomicExch(p.sched + 1, 0);
+            if (fused)
+                for (int g = 0; g <= p.E; ++g) atomicExch(p.hdone + g, 0);
+            __threadfence();
+        }
     }
 }
 
@@ -528,16 +642,21 @@ bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, u
     return r == CUDA_SUCCESS;
 }
 
-int pick_bn(long long T, int k, int E) {
+// Token tile: at least twice the mean tokens per routed expert, and with a
+// shared expert at least min(T, 128) so its weight tiles are not re-read by
+// many narrow token tiles; 64..256.
+int pick_bn(long long T, int k, int E, int Is) {
     const long long avg = (T * k + E - 1) / E;  // mean tokens per expert
+    long long want = 2 * avg;
+    if (Is > 0) want = std::max<long long>(want, std::min<long long>(T, 128));
     int bn = 64;
-    while (bn < 256 && bn < 2 * avg) bn <<= 1;
+    while (bn < 256 && bn < want) bn <<= 1;
     return bn;
 }
 
 size_t smem_bytes_for(int BN, int E, int stages) {
     return 1024 + (size_t)stages * (kABytes + BN * 128) + 64 * kXchgStride * 4 + 2 * (size_t)(E + 1) * 4 + 8 +
-           (size_t)(2 * stages + 5) * 8 + 16 + kThreads * 4;
+           (size_t)(2 * stages + 5 + 2 * kQueue) * 8 + 32 + kThreads * 4;
 }
 
 int pick_stages(int BN, int E) {
@@ -564,115 +683,114 @@ DeviceInfo device_info() {
     return cache[dev];
 }
 
-template <bool kGated>
-int launch_one(const GemmMaps &maps, const GemmParams &p, int sms, cudaStream_t st) {
-    const size_t smem = smem_bytes_for(p.BN, p.E, p.stages);
-    if (smem > (size_t)kSmemLimit) return MOE_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(ffn_gemm_kernel<kGated>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return MOE_ERR_CUDA;
-    // upper bound on work items (the real count is known only on the device)
-    const long long slots = (long long)p.T * p.k;
-    long long items = (std::min<long long>(p.E, slots) + (slots + p.BN - 1) / p.BN) * p.R;
-    if (p.Is > 0) items += (long long)p.Rs * ((p.T + p.BN - 1) / p.BN);
-    const int grid = (int)std::max<long long>(1, std::min<long long>(sms, items));
-    ffn_gemm_kernel<kGated><<<grid, kThreads, smem, st>>>(maps, p);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
-
-}  // namespace
-
-namespace {
-
-int choose_bn(const FfnArgs &a, int *bn) {
-    *bn = pick_bn(a.T, a.k, a.E);
-    // Benchmark/test override of the token tile (config-invariance checks).
+// Benchmark/test overrides: MOE_FORCE_BN in {32, 64, 128, 256} (token tile)
+// and MOE_FORCE_STAGES in [2, 16] (pipeline depth, capped by shared memory);
+// any other value is rejected.
+int choose_tiles(const FfnArgs &a, int *bn, int *stages) {
+    *bn = pick_bn(a.T, a.k, a.E, a.Is);
     if (const char *f = getenv("MOE_FORCE_BN")) {
         char *end = nullptr;
         const long v = strtol(f, &end, 10);
         if (*f == 0 || *end != 0 || (v != 32 && v != 64 && v != 128 && v != 256)) return MOE_ERR_INVALID_ARG;
         *bn = (int)v;
     }
+    *stages = pick_stages(*bn, a.E);
+    if (const char *f = getenv("MOE_FORCE_STAGES")) {
+        char *end = nullptr;
+        const long v = strtol(f, &end, 10);
+        if (*f == 0 || *end != 0 || v < 2 || v > kMaxStages) return MOE_ERR_INVALID_ARG;
+        *stages = std::min<int>((int)v, *stages);
+    }
     return MOE_OK;
 }
 
-GemmParams base_params(const FfnArgs &a, int BN) {
-    GemmParams p{};
+}  // namespace
+
+int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
+    const DeviceInfo di = device_info();
+    if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
+    if (phases < 1 || phases > 3) return MOE_ERR_INVALID_ARG;
+    FfnParams p{};
+    if (int rc = choose_tiles(a, &p.BN, &p.stages)) return rc;
+    const int BN = p.BN;
     p.T = a.T;
     p.H = a.H;
     p.E = a.E;
     p.I = a.I;
     p.k = a.k;
     p.Is = a.Is;
-    p.BN = BN;
-    p.stages = pick_stages(BN, a.E);
+    p.phases = phases;
     p.offsets = a.offsets;
     p.perm = a.perm;
     p.topk_w = a.topk_w;
     p.sgate = a.sgate;
+    p.h_perm = a.h_perm;
+    p.h_shared = a.h_shared;
+    p.ybuf = a.ybuf;
     p.status = a.status;
-    return p;
-}
+    p.sched = a.status + (phases == 2 ? 8 : 4);
+    p.hdone = a.hdone;
+    p.R[0] = a.I / 64;
+    p.Rs[0] = a.Is / 64;
+    p.nk[0] = a.H / kBlockK;
+    p.nks[0] = a.H / kBlockK;
+    p.R[1] = a.H / kTileM;
+    p.Rs[1] = a.H / kTileM;
+    p.nk[1] = a.I / kBlockK;
+    p.nks[1] = a.Is / kBlockK;
 
-}  // namespace
-
-int ffn_launch_gate_up(const FfnArgs &a, cudaStream_t st) {
-    const DeviceInfo di = device_info();
-    if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
-    int BN = 0;
-    if (int rc = choose_bn(a, &BN)) return rc;
+    static FfnMaps zero_maps;  // unused maps stay zero
+    FfnMaps m = zero_maps;
     const uint64_t Tk = (uint64_t)a.T * a.k;
-    GemmParams p = base_params(a, BN);
-    GemmMaps m;
-    memset(&m, 0, sizeof(m));
-    bool ok = encode_2d(&m.a0, a.w_gate, (uint64_t)a.E * a.I, a.H, 64) &&
-              encode_2d(&m.a1, a.w_up, (uint64_t)a.E * a.I, a.H, 64);
-    for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&m.b[b], a.x_perm, Tk, a.H, 16 << b);
-    if (a.Is > 0) {
-        ok = ok && encode_2d(&m.s0, a.ws_gate, a.Is, a.H, 64) && encode_2d(&m.s1, a.ws_up, a.Is, a.H, 64);
-        for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&m.bs[b], a.x, a.T, a.H, 16 << b);
-    } else {
-        m.s0 = m.a0;
-        m.s1 = m.a1;
+    bool ok = true;
+    if (phases & 1) {
+        PhaseMaps &g = m.ph[0];
+        ok = ok && encode_2d(&g.a0, a.w_gate, (uint64_t)a.E * a.I, a.H, 64) &&
+             encode_2d(&g.a1, a.w_up, (uint64_t)a.E * a.I, a.H, 64);
+        for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&g.b[b], a.x_perm, Tk, a.H, 16 << b);
+        if (a.Is > 0) {
+            ok = ok && encode_2d(&g.s0, a.ws_gate, a.Is, a.H, 64) && encode_2d(&g.s1, a.ws_up, a.Is, a.H, 64);
+            for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&g.bs[b], a.x, a.T, a.H, 16 << b);
+        }
+    }
+    if (phases & 2) {
+        PhaseMaps &d = m.ph[1];
+        ok = ok && encode_2d(&d.a0, a.w_down, (uint64_t)a.E * a.H, a.I, kTileM);
+        for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&d.b[b], a.h_perm, Tk, a.I, 16 << b);
+        if (a.Is > 0) {
+            ok = ok && encode_2d(&d.s0, a.ws_down, a.H, a.Is, kTileM);
+            for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b)
+                ok = ok && encode_2d(&d.bs[b], a.h_shared, a.T, a.Is, 16 << b);
+        }
     }
     if (!ok) return MOE_ERR_CUDA;
-    p.R = a.I / 64;
-    p.Rs = a.Is / 64;
-    p.nk = a.H / kBlockK;
-    p.nks = a.H / kBlockK;
-    p.out_routed = a.h_perm;
-    p.out_shared = a.h_shared;
-    return launch_one<true>(m, p, di.sms, st);
+
+    const size_t smem = smem_bytes_for(BN, a.E, p.stages);
+    if (smem > (size_t)kSmemLimit) return MOE_ERR_UNSUPPORTED;
+    static std::atomic<int> attr_set[64];  // per device: opted in to the full shared memory
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_set[dev].store(1, std::memory_order_release);
+    }
+    // upper bound on work items (the real count is known only on the device)
+    const long long slots = (long long)a.T * a.k;
+    const long long tiles = std::min<long long>(a.E, slots) + (slots + BN - 1) / BN;
+    const long long st_tiles = a.Is > 0 ? (a.T + BN - 1) / BN : 0;
+    long long items = 0;
+    for (int ph = 0; ph < 2; ++ph)
+        if ((phases >> ph) & 1) items += tiles * p.R[ph] + st_tiles * p.Rs[ph];
+    const int grid = (int)std::max<long long>(1, std::min<long long>(di.sms, items));
+    return launch_pdl(ffn_kernel, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int ffn_launch_down(const FfnArgs &a, cudaStream_t st) {
-    const DeviceInfo di = device_info();
-    if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
-    int BN = 0;
-    if (int rc = choose_bn(a, &BN)) return rc;
-    const uint64_t Tk = (uint64_t)a.T * a.k;
-    GemmParams p = base_params(a, BN);
-    GemmMaps m;
-    memset(&m, 0, sizeof(m));
-    bool ok = encode_2d(&m.a0, a.w_down, (uint64_t)a.E * a.H, a.I, kTileM);
-    for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&m.b[b], a.h_perm, Tk, a.I, 16 << b);
-    if (a.Is > 0) {
-        ok = ok && encode_2d(&m.s0, a.ws_down, a.H, a.Is, kTileM);
-        for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b)
-            ok = ok && encode_2d(&m.bs[b], a.h_shared, a.T, a.Is, 16 << b);
-    } else {
-        m.s0 = m.a0;
-    }
-    m.a1 = m.a0;
-    m.s1 = m.s0;
-    if (!ok) return MOE_ERR_CUDA;
-    p.R = a.H / kTileM;
-    p.Rs = a.H / kTileM;
-    p.nk = a.I / kBlockK;
-    p.nks = a.Is / kBlockK;
-    p.out_routed = a.ybuf;
-    p.out_shared = a.ybuf;
-    return launch_one<false>(m, p, di.sms, st);
+int ffn_launch_both(const FfnArgs &a, cudaStream_t st) {
+    const long long avg = ((long long)a.T * a.k + a.E - 1) / a.E;
+    if (avg < 128) return ffn_launch(a, 3, st);
+    if (int rc = ffn_launch(a, 1, st)) return rc;
+    return ffn_launch(a, 2, st);
 }
 
 }  // namespace moe

@@ -11,6 +11,10 @@ using namespace moe;
 namespace {
 
 constexpr size_t kAlign = 256;
+// Head of the workspace: [0, 256) status word and work-item counters,
+// [256, 256 + 4 * (E + 1)) per-group gate/up counters of the fused FFN.
+constexpr size_t kHeadBytes = 8192;
+constexpr size_t kHdoneOffset = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
@@ -28,7 +32,7 @@ WsLayout ws_layout(const moe_config_t &c, int T) {
     };
     const size_t Tk = (size_t)T * c.num_experts_per_tok;
     const size_t E = (size_t)c.n_routed_experts;
-    L.status = take(kAlign);
+    L.status = take(kHeadBytes);
     L.idx = take(Tk * 4);
     L.w = take(Tk * 4);
     L.sgate = take((size_t)T * 4);
@@ -137,7 +141,8 @@ int moe_dispatch(const moe_config_t *cfg, int32_t T, const int32_t *topk_idx, co
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     const int E = cfg->n_routed_experts, k = cfg->num_experts_per_tok;
     cudaStream_t st = as_stream(stream);
-    rc = cuda_rc(launch_dispatch(T, E, k, topk_idx, keff, at<int32_t>(ws, L.hist), counts, offsets, perm, slot_pos, st));
+    rc = cuda_rc(launch_dispatch(T, E, k, topk_idx, keff, at<int32_t>(ws, L.hist), counts, offsets, perm, slot_pos,
+                                 at<int32_t>(ws, L.status), at<int32_t>(ws, L.status + kHdoneOffset), st));
     if (rc || !x_perm) return rc;
     return cuda_rc(launch_gather_rows(T, k, cfg->hidden, offsets, E, perm, x, x_perm, st));
 }
@@ -184,6 +189,7 @@ int ffn_args(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_
     a->h_shared = sh ? at<uint16_t>(ws, L.h_shared) : nullptr;
     a->ybuf = ybuf;
     a->status = at<int32_t>(ws, L.status);
+    a->hdone = at<int32_t>(ws, L.status + kHdoneOffset);
     return MOE_OK;
 }
 
@@ -199,7 +205,7 @@ int moe_expert_gate_up(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, 
     FfnArgs a;
     rc = ffn_args(cfg, T, x, x_perm, offsets, nullptr, nullptr, nullptr, w, nullptr, ws, ws_bytes, true, &a);
     if (rc) return rc;
-    return ffn_launch_gate_up(a, as_stream(stream));
+    return ffn_launch(a, 1, as_stream(stream));
 }
 
 int moe_expert_down(const moe_config_t *cfg, int32_t T, const int32_t *offsets, const int32_t *perm,
@@ -211,7 +217,7 @@ int moe_expert_down(const moe_config_t *cfg, int32_t T, const int32_t *offsets, 
     FfnArgs a;
     rc = ffn_args(cfg, T, nullptr, nullptr, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, false, &a);
     if (rc) return rc;
-    return ffn_launch_down(a, as_stream(stream));
+    return ffn_launch(a, 2, as_stream(stream));
 }
 
 int moe_expert_ffn(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
@@ -225,9 +231,7 @@ int moe_expert_ffn(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, cons
     if (rc) return rc;
     rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, false, &b);
     if (rc) return rc;
-    rc = ffn_launch_gate_up(a, as_stream(stream));
-    if (rc) return rc;
-    return ffn_launch_down(b, as_stream(stream));
+    return ffn_launch_both(a, as_stream(stream));
 }
 
 int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, const int32_t *keff, moe_bf16_t *out,
@@ -288,7 +292,7 @@ int moe_status_read(const void *ws, int32_t *status_out, void *stream) {
 
 int moe_status_clear(void *ws, void *stream) {
     if (!aligned(ws)) return MOE_ERR_INVALID_ARG;
-    return cuda_rc(cudaMemsetAsync(ws, 0, sizeof(int32_t), as_stream(stream)));
+    return cuda_rc(cudaMemsetAsync(ws, 0, kHeadBytes, as_stream(stream)));
 }
 
 }  // extern "C"

@@ -22,6 +22,30 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
     return *reinterpret_cast<uint16_t *>(&b);
 }
 
+// Programmatic dependent launch: every kernel of the layer lets the next one
+// launch as soon as all of its CTAs are running, and waits for its own
+// predecessor (grid completion and memory flush) before it reads anything
+// the predecessor wrote.  Set-up that touches no such data (barrier init,
+// TMEM allocation, tensor-map prefetch) runs before the wait.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------- launch wrappers --
 // Every wrapper enqueues on `st` and returns cudaGetLastError().
 
@@ -38,9 +62,11 @@ cudaError_t launch_budget(int T, int E, int k, int N, int norm_topk, int32_t *id
 
 // Dispatch: histogram, scan, stable scatter, row gather.
 int dispatch_chunks(int T);
+// `status_block`, `hdone` (may be null): the dispatch kernels also zero the
+// grouped FFN's work-item counters and per-group gate/up counters [E + 1].
 cudaError_t launch_dispatch(int T, int E, int k, const int32_t *idx, const int32_t *keff,
                             int32_t *hist, int32_t *counts, int32_t *offsets, int32_t *perm,
-                            int32_t *slot_pos, cudaStream_t st);
+                            int32_t *slot_pos, int32_t *status_block, int32_t *hdone, cudaStream_t st);
 cudaError_t launch_gather_rows(int T, int k, int H, const int32_t *offsets, int E,
                                const int32_t *perm, const uint16_t *x, uint16_t *x_perm,
                                cudaStream_t st);
@@ -57,11 +83,17 @@ struct FfnArgs {
     const float *topk_w, *sgate;
     const uint16_t *w_gate, *w_up, *w_down, *ws_gate, *ws_up, *ws_down;
     uint16_t *h_perm, *h_shared, *ybuf;
-    int32_t *status;
+    int32_t *status;  // the workspace's status block: [0] status word,
+                      // [4..5] gate/up (or fused) and [8..9] down work-item counters
+    int32_t *hdone;   // [E + 1] per-group finished gate/up tiles (fused launches)
 };
-// Each returns MOE_OK / MOE_ERR_*.  gate_up writes h_perm / h_shared; down
-// reads them and writes ybuf.
-int ffn_launch_gate_up(const FfnArgs &a, cudaStream_t st);
-int ffn_launch_down(const FfnArgs &a, cudaStream_t st);
+// One launch of the grouped FFN kernel.  phases: 1 = gate/up (writes
+// h_perm / h_shared), 2 = down (reads them, writes ybuf), 3 = both in one
+// launch.  Returns MOE_OK / MOE_ERR_*.
+int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st);
+// Both FFN phases of a layer: one fused launch while the groups are small
+// (weight streaming; the fused launch hides the tail of the gate/up phase),
+// two launches once the mean group fills a 128-token tile (tensor-bound).
+int ffn_launch_both(const FfnArgs &a, cudaStream_t st);
 
 }  // namespace moe

@@ -3,12 +3,14 @@
 // softmax router with renormalised top-k), plus the sigmoid gate of the
 // shared expert.
 //
-// One warp per token.  Lane l holds the logits of experts l, l+32, ...
+// One block per token; its first warp routes.  Lane l holds the logits of experts l, l+32, ...
 // (coalesced 128-byte loads).  Each of the k selection rounds takes a
 // lane-local best and a 5-step shuffle argmax ordered by (logit descending,
 // expert id ascending), so equal logits keep the lower id, and the winner's
-// owner lane masks it out.  The memory traffic is the logits row once; the
-// kernel is latency-bound and tiny next to the expert FFN.
+// owner lane masks it out.  The shared-expert gate is a block-wide dot
+// product with every load in flight at once.  The kernel
+// reads the logits (and x) once; it is latency-bound and small next to the
+// expert FFN.
 #include <math.h>
 
 #include "moe_internal.cuh"
@@ -21,19 +23,14 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
     return va > vb || (va == vb && ia < ib);
 }
 
-template <int V>  // logits per lane: V * 32 >= E
-__global__ void __launch_bounds__(256) route_kernel(int T, int E, int k, int norm_topk,
-                                                    const float *__restrict__ logits,
-                                                    int32_t *__restrict__ idx, float *__restrict__ w,
-                                                    int32_t *__restrict__ keff,
-                                                    const uint16_t *__restrict__ x,
-                                                    const uint16_t *__restrict__ gvec, int H,
-                                                    float *__restrict__ sgate) {
-    const int lane = threadIdx.x & 31;
-    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (t >= T) return;
-    const float *l = logits + (size_t)t * E;
+constexpr int kRouteThreads = 128;  // one token per block: warp 0 routes, all warps dot
+constexpr int kGVec = 8;             // 16-byte slices of x and g per thread per pass
 
+template <int V>  // logits per lane: V * 32 >= E
+__device__ __forceinline__ void route_token(int t, int E, int k, int norm_topk, const float *__restrict__ logits,
+                                            int32_t *__restrict__ idx, float *__restrict__ w,
+                                            int32_t *__restrict__ keff, int lane) {
+    const float *l = logits + (size_t)t * E;
     float v[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) {
@@ -96,24 +93,57 @@ __global__ void __launch_bounds__(256) route_kernel(int T, int E, int k, int nor
         w[(size_t)t * k + lane] = p;
     }
     if (keff != nullptr && lane == 0) keff[t] = k;
+}
 
-    if (sgate != nullptr) {  // sigmoid(g . x_t), 8 bf16 per 16-byte load
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
-        const uint4 *gr = reinterpret_cast<const uint4 *>(gvec);
-        float z = 0.f;
-        for (int c = lane; c < H / 8; c += 32) {
-            const uint4 a = __ldg(xr + c), b = __ldg(gr + c);
-            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+template <int V>  // logits per lane: V * 32 >= E
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int k, int norm_topk,
+                                                              const float *__restrict__ logits,
+                                                              int32_t *__restrict__ idx, float *__restrict__ w,
+                                                              int32_t *__restrict__ keff,
+                                                              const uint16_t *__restrict__ x,
+                                                              const uint16_t *__restrict__ gvec, int H,
+                                                              float *__restrict__ sgate) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int t = blockIdx.x;  // one token per block
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (wid == 0) route_token<V>(t, E, k, norm_topk, logits, idx, w, keff, lane);
+    if (sgate == nullptr) return;
+    // sigmoid(g . x_t): each thread loads up to kGVec 16-byte slices of x_t and
+    // of g, all in flight at once, then a block reduction.
+    __shared__ float part[kRouteThreads / 32];
+    const int nv = H / 8;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+    const uint4 *gr = reinterpret_cast<const uint4 *>(gvec);
+    float z = 0.f;
+    for (int c0 = threadIdx.x; c0 < nv; c0 += kRouteThreads * kGVec) {
+        uint4 a[kGVec], g[kGVec];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                z = fmaf(bf16_bits_to_f32((uint16_t)(av[q] & 0xffffu)),
-                         bf16_bits_to_f32((uint16_t)(bv[q] & 0xffffu)), z);
-                z = fmaf(bf16_bits_to_f32((uint16_t)(av[q] >> 16)), bf16_bits_to_f32((uint16_t)(bv[q] >> 16)), z);
-            }
+        for (int q = 0; q < kGVec; ++q) {
+            const int c = c0 + q * kRouteThreads;
+            a[q] = c < nv ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+            g[q] = c < nv ? __ldg(gr + c) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-        if (lane == 0) sgate[t] = 1.f / (1.f + expf(-z));
+        for (int q = 0; q < kGVec; ++q) {
+            const uint32_t av[4] = {a[q].x, a[q].y, a[q].z, a[q].w}, bv[4] = {g[q].x, g[q].y, g[q].z, g[q].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                z = fmaf(bf16_bits_to_f32((uint16_t)(av[h] & 0xffffu)), bf16_bits_to_f32((uint16_t)(bv[h] & 0xffffu)),
+                         z);
+                z = fmaf(bf16_bits_to_f32((uint16_t)(av[h] >> 16)), bf16_bits_to_f32((uint16_t)(bv[h] >> 16)), z);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if (lane == 0) part[wid] = z;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float zz = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kRouteThreads / 32; ++w2) zz += part[w2];
+        sgate[t] = 1.f / (1.f + expf(-zz));
     }
 }
 
@@ -121,10 +151,8 @@ template <int V>
 cudaError_t launch_v(int T, int E, int k, int norm_topk, const float *logits, int32_t *idx, float *w,
                      int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
                      cudaStream_t st) {
-    const int threads = 256, per_block = threads / 32;
-    route_kernel<V><<<(T + per_block - 1) / per_block, threads, 0, st>>>(T, E, k, norm_topk, logits, idx, w,
-                                                                          keff, x, gvec, H, sgate);
-    return cudaGetLastError();
+    return launch_pdl(route_kernel<V>, dim3(T), dim3(kRouteThreads), 0, st, T, E, k, norm_topk, logits, idx, w, keff,
+                      x, gvec, H, sgate);
 }
 
 }  // namespace

@@ -202,3 +202,35 @@ def test_large_layer(large_inputs, T, alpha, nrows):
     g = gpu_forward(cfg, inp)
     diag = check_layer(cfg, inp, g, rows=sample_rows(T, nrows))
     print(cfg.label, diag, "max group", int(g.counts.max()))
+
+
+@pytest.mark.parametrize("cfg", [W.MoEConfig("phases", T=300, H=256, E=8, I=192, k=2, Is=128, zipf_alpha=1.0),
+                                 W.MoEConfig("phases_noshared", T=77, H=384, E=16, I=64, k=4)],
+                         ids=lambda c: c.name)
+def test_split_phases_match_fused(cfg):
+    """moe_expert_gate_up then moe_expert_down (two launches) writes the same
+    ybuf bits as the fused one-launch moe_expert_ffn."""
+    c = lib_config(cfg)
+    T, k, E, H = cfg.T, cfg.k, cfg.E, cfg.H
+    dev = "cuda"
+    inp = W.make_inputs(cfg, device=dev)
+    ws = torch.zeros(moe.workspace_bytes(c, T), dtype=torch.uint8, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    sgate = torch.empty(T, dtype=torch.float32, device=dev) if cfg.Is else None
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    slot_pos = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    y1 = torch.zeros((T, k + 1, H), dtype=torch.bfloat16, device=dev)
+    y2 = torch.zeros((T, k + 1, H), dtype=torch.bfloat16, device=dev)
+    moe.moe_route(c, inp.logits, idx, w, x=inp.x if cfg.Is else None, ws_gate_vec=inp.ws_gvec, sgate=sgate)
+    moe.moe_dispatch(c, idx, counts, offsets, perm, slot_pos, ws, x=inp.x, x_perm=x_perm)
+    wts = weights_of(inp)
+    moe.moe_expert_ffn(c, inp.x, x_perm, offsets, perm, w, wts, y1, ws, sgate=sgate)
+    moe.moe_expert_gate_up(c, inp.x, x_perm, offsets, wts, ws)
+    moe.moe_expert_down(c, T, offsets, perm, w, wts, y2, ws, sgate=sgate)
+    torch.cuda.synchronize()
+    assert moe.status_read(ws) == 0
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
