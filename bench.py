@@ -3,11 +3,11 @@
 
 One step = the whole hot path on one batch: route -> (budget) -> dispatch ->
 expert gate/up GEMM + SwiGLU -> expert down GEMM + weighted scatter ->
-combine, called as the library's stage entry points on one stream (the same
-launches moe_forward makes), with CUDA events between stages so each
-kernel's duration is measured on its own launching stream.  Inputs are
-resident in HBM; L2 is flushed (a 256 MB write) between timed steps,
-outside the timed events.
+combine.  `value` times moe_forward (one C call) replayed as a CUDA graph
+between two events; the per-kernel breakdown replays the same launches as
+separate stage entry points with an event between stages, on the launching
+stream.  Inputs are resident in HBM; L2 is flushed (a 256 MB write) before
+every replay, outside the timed events.
 
 Prints ONE JSON line (rank 0).  `value` = tokens/s over all ranks; `e2e` =
 the same metric through moe_forward with host buffers (pinned H2D of x and
@@ -95,11 +95,11 @@ def stage_work(cfg, counts):
 
 
 def launches_per_step(cfg) -> int:
-    # route 1; budget 2; dispatch: one CTA-wide sort when T*k <= 8192, else
-    # histogram + scan + scatter; gather 1; expert FFN 1 (fused) or 2 (mean
-    # group >= 128 tokens); combine 1
+    # route 1; budget 2; dispatch: one sort+gather launch when T*k <= 8192,
+    # else histogram + scan + scatter + gather; expert FFN 1 (fused) or 2
+    # (mean group >= 128 tokens); combine 1
     ffn = 1 if (cfg.T * cfg.k + cfg.E - 1) // cfg.E < 128 else 2
-    return 1 + (2 if cfg.budget else 0) + (1 if cfg.T * cfg.k <= 8192 else 3) + 1 + ffn + 1
+    return 1 + (2 if cfg.budget else 0) + (1 if cfg.T * cfg.k <= 8192 else 4) + ffn + 1
 
 
 def load_peaks():
@@ -406,16 +406,40 @@ def run_ours(args, cfg):
     torch.cuda.synchronize(dev)
     eager_ms = sum(e[0].elapsed_time(e[NEV - 1]) for e in evs) / args.steps
 
-    # ---- timed region: the step replayed as one CUDA graph (device-resident
-    # inputs; timing events are nodes of the graph, L2 flushed between steps)
+    # ---- timed region.  Each step replays two CUDA graphs on device-resident
+    # inputs, with an L2 flush before each:
+    #   fwd:    one moe_forward call between two timing events -> `value`;
+    #   stages: the same launches as separate entry-point calls with an
+    #           event between stages -> per-kernel durations (roofline).
+    # Events are graph nodes, so host launch overhead is outside them; the
+    # per-step synchronisation and the flushes are outside the events too.
+    aux_c = moe._Aux()
+    for n_, t_ in dict(topk_idx=idx, topk_w=tw, keff=keff, expert_kept=kept, n_dropped=nd, counts=counts,
+                       offsets=offsets, perm=perm, slot_pos=slot_pos).items():
+        setattr(aux_c, n_, P(t_.data_ptr()))
+    if cfg.Is:
+        aux_c.sgate = P(sgate.data_ptr())
+
+    def fwd_step(e0, e1):
+        st = torch.cuda.current_stream(dev)
+        e0.record(st)
+        chk("moe_forward", lib.moe_forward(pc, T, p["x"], p["logits"], pw, p["out"], ctypes.byref(aux_c), p["ws"],
+                                           wsb, P(st.cuda_stream)))
+        e1.record(st)
+
+    fev = mk(ext=True)[:2]
+    fwd_graph = capture(lambda: fwd_step(*fev))
     gev = mk(ext=True)
-    graph = capture(lambda: step(gev))
+    stage_graph = capture(lambda: step(gev))
     for _ in range(args.warmup):
         flush.zero_()
-        graph.replay()
+        fwd_graph.replay()
+        flush.zero_()
+        stage_graph.replay()
     torch.cuda.synchronize(dev)
     stage_sum = {s: 0.0 for s in stages}
     step_sum = 0.0
+    staged_sum = 0.0
     barrier(dev)
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(dev)
@@ -423,11 +447,15 @@ def run_ours(args, cfg):
     with sampler:
         for i in range(args.steps):
             flush.zero_()
-            graph.replay()
+            fwd_graph.replay()
+            fev[1].synchronize()
+            step_sum += fev[0].elapsed_time(fev[1])
+            flush.zero_()
+            stage_graph.replay()
             gev[NEV - 1].synchronize()
             for j, sname in enumerate(stages):
                 stage_sum[sname] += gev[j].elapsed_time(gev[j + 1])
-            step_sum += gev[0].elapsed_time(gev[NEV - 1])
+            staged_sum += gev[0].elapsed_time(gev[NEV - 1])
         torch.cuda.synchronize(dev)
     host_s = time.perf_counter() - t_host0
     barrier(dev)
@@ -438,7 +466,7 @@ def run_ours(args, cfg):
     if status:
         raise RuntimeError(f"device status {status} after timing")
     value = aggregate_tokens_per_s(T, args.steps, total_ms, world)
-    del graph
+    del fwd_graph, stage_graph
 
     # ---- end to end through moe_forward with host buffers (one graph:
     # pinned H2D of x and logits, the layer, D2H of the output)
@@ -511,7 +539,7 @@ def run_ours(args, cfg):
         "router logits + Zipf popularity bias",
         "config": {**workload_desc(cfg), "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": rl, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches_per_step(cfg) * args.steps,
+        "gpu_launches": 2 * launches_per_step(cfg) * args.steps,
         "clocks": sampler.summary(),
         "stages_ms": per_stage,
         "layer": {"touched_experts": work["touched"], "kept_slots": work["slots"],
@@ -520,7 +548,10 @@ def run_ours(args, cfg):
                   "hbm_frac": layer_bw / peaks["hbm_gbs"]},
         "host_s": host_s,
         "eager_ms_per_step": eager_ms,
-        "timing": "CUDA graph replay of the stage calls; events are graph nodes; per-step sync outside the events",
+        "staged_ms_per_step": staged_sum / args.steps,
+        "timing": "value: CUDA-graph replay of moe_forward between two event nodes; stages_ms and roofline: a "
+                  "second graph of the stage entry points with an event node between stages; both replayed every "
+                  "step, L2 flushed before each, per-step sync outside the events",
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -12,8 +12,11 @@
 //            expert, the rank inside the group is the count of lower lanes,
 //            so positions follow slot order exactly;
 //   gather   x_perm[p] = x[perm[p] / k], four 16-byte vectors per thread.
-// Batches of up to kSmallSlots slots run hist + scan + scatter as one CTA
-// (dispatch_small_kernel) to save two launches.
+// Batches of up to kSmallSlots slots run all of it as one launch
+// (dispatch_small_kernel).
+#include <algorithm>
+#include <atomic>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -134,30 +137,39 @@ __global__ void __launch_bounds__(32) scatter_kernel(int T, int E, int k, const 
     }
 }
 
-// Whole counting sort for a small batch in one 1024-thread CTA: warps
-// 0..W-1 each own a contiguous run of slots; per-warp counts (shared
-// memory), one exclusive scan over experts, per-warp bases, then each warp
-// scatters its run in slot order with __match_any_sync ranks.
-__global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int k, int W,
+// Small batches: the whole counting sort, redundantly in every CTA of the
+// grid (it costs a few microseconds of the CTA's own time), then each CTA
+// gathers its share of x_perm rows from its own copy of perm -- one launch
+// for hist + scan + scatter + gather.  In each 1024-thread CTA, warps
+// 0..W-1 own contiguous runs of slots: per-warp counts in shared memory, one
+// exclusive scan over experts, per-warp bases, then each warp places its run
+// in slot order with __match_any_sync ranks.  CTA 0 writes counts, offsets,
+// perm and slot_pos and zeroes the FFN's scheduling counters.
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int k, int W, int vec,
                                                               const int32_t *__restrict__ idx,
                                                               const int32_t *__restrict__ keff,
+                                                              const uint4 *__restrict__ x, uint4 *__restrict__ x_perm,
                                                               int32_t *__restrict__ counts,
                                                               int32_t *__restrict__ offsets,
                                                               int32_t *__restrict__ perm,
                                                               int32_t *__restrict__ slot_pos, int32_t *__restrict__ sched,
                                                               int32_t *__restrict__ hdone) {
-    extern __shared__ int hist[];  // [W][E]
+    extern __shared__ int smem_i[];
+    int *hist = smem_i;               // [W][E]
+    int *perm_s = smem_i + W * E;     // [T*k]
     __shared__ int warp_sums[32];
+    __shared__ int total_s;
     pdl_launch_dependents();
     pdl_wait();
+    const bool writer = blockIdx.x == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Tk = T * k, chunk = (Tk + W - 1) / W;
     for (int i = threadIdx.x; i < W * E; i += blockDim.x) hist[i] = 0;
-    if (sched != nullptr && threadIdx.x < 2) {
+    if (writer && sched != nullptr && threadIdx.x < 2) {
         sched[4 + threadIdx.x] = 0;
         sched[8 + threadIdx.x] = 0;
     }
-    if (hdone != nullptr)
+    if (writer && hdone != nullptr)
         for (int g = threadIdx.x; g <= E; g += blockDim.x) hdone[g] = 0;
     __syncthreads();
     const int s_begin = warp * chunk, s_end = min(Tk, s_begin + chunk);
@@ -167,8 +179,8 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int 
             int key = -1;
             if (s < s_end) {
                 const int t = s / k, j = s - t * k;
-                const int e = idx[s];
-                if (j < (keff ? keff[t] : k) && e >= 0 && e < E) key = e;
+                const int e = __ldg(idx + s);
+                if (j < (keff ? __ldg(keff + t) : k) && e >= 0 && e < E) key = e;
             }
             const unsigned peers = __match_any_sync(0xffffffffu, key);
             if (key >= 0 && lane == __ffs(peers) - 1) hist[warp * E + key] += __popc(peers);
@@ -182,9 +194,12 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int 
         for (int w = 0; w < W; ++w) c += hist[w * E + e];
     const int excl = block_exclusive_scan(c, warp_sums);
     if (e < E) {
-        counts[e] = c;
-        offsets[e] = excl;
-        if (e == E - 1) offsets[E] = excl + c;
+        if (writer) {
+            counts[e] = c;
+            offsets[e] = excl;
+            if (e == E - 1) offsets[E] = excl + c;
+        }
+        if (e == E - 1) total_s = excl + c;
         int run = excl;
         for (int w = 0; w < W; ++w) {
             const int hw = hist[w * E + e];
@@ -200,20 +215,31 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int 
             int key = -1;
             if (s < s_end) {
                 const int t = s / k, j = s - t * k;
-                const int ee = idx[s];
-                if (j < (keff ? keff[t] : k) && ee >= 0 && ee < E) key = ee;
-                else slot_pos[s] = -1;
+                const int ee = __ldg(idx + s);
+                if (j < (keff ? __ldg(keff + t) : k) && ee >= 0 && ee < E) key = ee;
+                else if (writer) slot_pos[s] = -1;
             }
             const unsigned peers = __match_any_sync(0xffffffffu, key);
             if (key >= 0) {
                 const int pos = base[key] + __popc(peers & ((1u << lane) - 1u));
-                perm[pos] = s;
-                slot_pos[s] = pos;
+                perm_s[pos] = s;
+                if (writer) {
+                    perm[pos] = s;
+                    slot_pos[s] = pos;
+                }
             }
             __syncwarp();
             if (key >= 0 && lane == 31 - __clz(peers)) base[key] += __popc(peers);
             __syncwarp();
         }
+    }
+    if (x_perm == nullptr) return;
+    __syncthreads();
+    const int total = total_s;
+    for (int pr = blockIdx.x; pr < total; pr += gridDim.x) {
+        const uint4 *src = x + (size_t)(perm_s[pr] / k) * vec;
+        uint4 *dst = x_perm + (size_t)pr * vec;
+        for (int cc = threadIdx.x; cc < vec; cc += blockDim.x) dst[cc] = __ldg(src + cc);
     }
 }
 
@@ -240,20 +266,37 @@ __global__ void __launch_bounds__(256) gather_kernel(int k, int vec4, const int3
 
 int dispatch_chunks(int T) { return (T + kTokChunk - 1) / kTokChunk; }
 
+bool dispatch_is_small(int T, int k) { return (long long)T * k <= kSmallSlots; }
+
 cudaError_t launch_dispatch(int T, int E, int k, const int32_t *idx, const int32_t *keff, int32_t *hist,
                             int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
-                            int32_t *status_block, int32_t *hdone, cudaStream_t st) {
-    if ((long long)T * k <= kSmallSlots) {
+                            int32_t *status_block, int32_t *hdone, const uint16_t *x, uint16_t *x_perm, int H,
+                            cudaStream_t st) {
+    if (dispatch_is_small(T, k)) {
         const int W = E <= 256 ? 32 : (E <= 512 ? 16 : 8);  // per-warp counts fit in 32 KB
-        return launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), (size_t)W * E * 4, st, T, E, k, W, idx, keff,
-                          counts, offsets, perm, slot_pos, status_block, hdone);
+        const size_t smem = ((size_t)W * E + (size_t)T * k) * 4;  // <= 64 KB
+        static std::atomic<int> attr_set[64];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if (!attr_set[dev].load(std::memory_order_acquire)) {
+            const cudaError_t e = cudaFuncSetAttribute(dispatch_small_kernel,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
+            if (e != cudaSuccess) return e;
+            attr_set[dev].store(1, std::memory_order_release);
+        }
+        const int grid = x_perm ? std::max(1, std::min(device_sm_count(), T * k)) : 1;
+        return launch_pdl(dispatch_small_kernel, dim3(grid), dim3(1024), smem, st, T, E, k, W, H / 8, idx, keff,
+                          reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(x_perm), counts, offsets,
+                          perm, slot_pos, status_block, hdone);
     }
     const int nchunks = dispatch_chunks(T);
     cudaError_t e = launch_pdl(hist_kernel, dim3(nchunks), dim3(256), 0, st, T, E, k, idx, keff, hist);
     if (e != cudaSuccess) return e;
     e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, E, nchunks, hist, counts, offsets, status_block, hdone);
     if (e != cudaSuccess) return e;
-    return launch_pdl(scatter_kernel, dim3(nchunks), dim3(32), 0, st, T, E, k, idx, keff, hist, perm, slot_pos);
+    e = launch_pdl(scatter_kernel, dim3(nchunks), dim3(32), 0, st, T, E, k, idx, keff, hist, perm, slot_pos);
+    if (e != cudaSuccess || x_perm == nullptr) return e;
+    return launch_gather_rows(T, k, H, offsets, E, perm, x, x_perm, st);
 }
 
 cudaError_t launch_gather_rows(int T, int k, int H, const int32_t *offsets, int E, const int32_t *perm,

@@ -154,6 +154,20 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *ba
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+// Same, with an L2 cache-policy hint (weights are streamed once: evict first).
+__device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+        "{%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -405,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_phase = 0;
+            const uint64_t wpol = policy_evict_first();  // expert weights: read once per launch
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 const uint32_t qph = (uint32_t)(li / kQueue) & 1u;
@@ -453,10 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     uint8_t *sA = stages + (size_t)stage * stage_bytes;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     if (it.ph == 0) {
-                        tma_load_2d(ma0, &full[stage], sA, ks * kBlockK, a_row);
-                        tma_load_2d(ma1, &full[stage], sA + kABytes / 2, ks * kBlockK, a_row);
+                        tma_load_2d_hint(ma0, &full[stage], sA, ks * kBlockK, a_row, wpol);
+                        tma_load_2d_hint(ma1, &full[stage], sA + kABytes / 2, ks * kBlockK, a_row, wpol);
                     } else {
-                        tma_load_2d(ma0, &full[stage], sA, ks * kBlockK, a_row);
+                        tma_load_2d_hint(ma0, &full[stage], sA, ks * kBlockK, a_row, wpol);
                     }
                     tma_load_2d(mb, &full[stage], sA + kABytes, ks * kBlockK, it.row0);
                     issued |= 1u << stage;
@@ -785,6 +800,8 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     const int grid = (int)std::max<long long>(1, std::min<long long>(di.sms, items));
     return launch_pdl(ffn_kernel, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
+
+int device_sm_count() { return device_info().sms; }
 
 int ffn_launch_both(const FfnArgs &a, cudaStream_t st) {
     const long long avg = ((long long)a.T * a.k + a.E - 1) / a.E;

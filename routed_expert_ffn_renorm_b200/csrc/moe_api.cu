@@ -141,10 +141,9 @@ int moe_dispatch(const moe_config_t *cfg, int32_t T, const int32_t *topk_idx, co
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     const int E = cfg->n_routed_experts, k = cfg->num_experts_per_tok;
     cudaStream_t st = as_stream(stream);
-    rc = cuda_rc(launch_dispatch(T, E, k, topk_idx, keff, at<int32_t>(ws, L.hist), counts, offsets, perm, slot_pos,
-                                 at<int32_t>(ws, L.status), at<int32_t>(ws, L.status + kHdoneOffset), st));
-    if (rc || !x_perm) return rc;
-    return cuda_rc(launch_gather_rows(T, k, cfg->hidden, offsets, E, perm, x, x_perm, st));
+    return cuda_rc(launch_dispatch(T, E, k, topk_idx, keff, at<int32_t>(ws, L.hist), counts, offsets, perm, slot_pos,
+                                   at<int32_t>(ws, L.status), at<int32_t>(ws, L.status + kHdoneOffset), x, x_perm,
+                                   cfg->hidden, st));
 }
 
 }  // extern "C"

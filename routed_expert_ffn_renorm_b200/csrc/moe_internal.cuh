@@ -64,9 +64,12 @@ cudaError_t launch_budget(int T, int E, int k, int N, int norm_topk, int32_t *id
 int dispatch_chunks(int T);
 // `status_block`, `hdone` (may be null): the dispatch kernels also zero the
 // grouped FFN's work-item counters and per-group gate/up counters [E + 1].
+// x_perm (may be null): also gather x_perm[p] = x[perm[p] / k].
 cudaError_t launch_dispatch(int T, int E, int k, const int32_t *idx, const int32_t *keff,
                             int32_t *hist, int32_t *counts, int32_t *offsets, int32_t *perm,
-                            int32_t *slot_pos, int32_t *status_block, int32_t *hdone, cudaStream_t st);
+                            int32_t *slot_pos, int32_t *status_block, int32_t *hdone, const uint16_t *x,
+                            uint16_t *x_perm, int H, cudaStream_t st);
+int device_sm_count();  // SMs of the current device (cached)
 cudaError_t launch_gather_rows(int T, int k, int H, const int32_t *offsets, int E,
                                const int32_t *perm, const uint16_t *x, uint16_t *x_perm,
                                cudaStream_t st);
