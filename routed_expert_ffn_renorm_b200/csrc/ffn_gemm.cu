@@ -32,11 +32,12 @@
 // (one lane); warp 1 -- TMEM allocation and MMA issue (one lane); warps
 // 2..5 -- epilogue, one TMEM lane quarter each.
 //
-// Work items are handed out dynamically (a global counter) in the order
-// phase 0 [shared expert, routed experts ascending], phase 1 [routed
-// experts ascending, shared expert]; inside a group, weight tile outer and
-// token tile inner, so token tiles that reuse a weight tile run side by side
-// (one HBM read, L2 hits).  The item table is derived in-kernel from the
+// Work items are handed out dynamically (a global counter, claimed one item
+// ahead) in the order phase 0 [shared expert, routed experts ascending],
+// phase 1 [shared expert, routed experts ascending] -- the shared expert's
+// items are the longest, so they start first; inside a group, weight tile
+// outer and token tile inner, so token tiles that reuse a weight tile run
+// side by side (one HBM read, L2 hits).  The item table is derived in-kernel from the
 // dispatch offsets -- no host sync.  The token box height (16..256 rows) is
 // picked per tile and the MMA N is the valid token count rounded up to 16.
 //
@@ -67,6 +68,7 @@ constexpr int kMaxStages = 16;
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
 constexpr int kXchgStride = 33;                // fp32 exchange row stride (bank-conflict free)
 constexpr int kQueue = 4;                      // work-item queue depth (producer -> MMA, epilogue)
+constexpr int kReadyWords = (kMaxExperts + 1 + 31) / 32;  // one bit per group: its h rows are complete
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 
 struct PhaseMaps {
@@ -253,11 +255,9 @@ __device__ __forceinline__ Item decode_item(int item, const Schedule &sc, const 
     it.ph = item < sc.n[0] ? 0 : 1;
     if (it.ph) item -= sc.n[0];
     const int sh_items = p.Rs[it.ph] * sc.shared_ntt;
-    const int rt_items = sc.tile_base[p.E] * p.R[it.ph];
-    // phase 0: shared first; phase 1: shared last
-    const bool is_shared = it.ph == 0 ? item < sh_items : item >= rt_items;
-    if (is_shared) {
-        const int local = it.ph == 0 ? item : item - rt_items;
+    // both phases: the shared expert's items first (they are the longest)
+    if (item < sh_items) {
+        const int local = item;
         const int j = local % sc.shared_ntt;
         it.shared = 1;
         it.e = p.E;
@@ -266,8 +266,7 @@ __device__ __forceinline__ Item decode_item(int item, const Schedule &sc, const 
         it.nvalid = min(p.BN, p.T - j * p.BN);
         it.ntt = sc.shared_ntt;
     } else {
-        const int local_all = it.ph == 0 ? item - sh_items : item;
-        const int tile_item = local_all;  // routed items: tile_base[e] * R + (r * ntt + j)
+        const int tile_item = item - sh_items;  // routed items: tile_base[e] * R + (r * ntt + j)
         int lo = 0, hi = p.E - 1;         // largest e with tile_base[e] * R <= tile_item
         const int R = p.R[it.ph];
         while (lo < hi) {
@@ -317,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     volatile int *epi_item = reinterpret_cast<volatile int *>(tmem_slot + 2);
     volatile int *qitem = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kQueue]
     int *scan_tmp = reinterpret_cast<int *>(tmem_slot + 8);                 // [kThreads]
+    uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + kThreads);  // [kReadyWords], producer-private
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tmem_cols = 2 * p.BN;
@@ -338,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             mbar_init(&qempty[q], 2);  // the MMA lane and the elected epilogue thread
         }
         *abort_flag = 0;
+        for (int w = 0; w < kReadyWords; ++w) ready_bits[w] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -420,19 +421,21 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             int stage = 0;
             uint32_t phase = 0, issued = 0, last_phase = 0;
             const uint64_t wpol = policy_evict_first();  // expert weights: read once per launch
+            int next = atomicAdd(p.sched, 1);            // items are claimed one ahead
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 const uint32_t qph = (uint32_t)(li / kQueue) & 1u;
                 if (!mbar_wait(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
-                int item = atomicAdd(p.sched, 1);
-                if (item >= total_items) item = -1;
+                int item = next < total_items ? next : -1;
+                if (item >= 0) next = atomicAdd(p.sched, 1);  // its latency overlaps this item's loads
                 qitem[slot] = item;
                 mbar_arrive(&qfull[slot]);
                 if (item < 0) break;
                 const Item it = decode_item(item, sc, p);
-                if (fused && it.ph == 1) {
+                const int grp = it.shared ? p.E : it.e;
+                if (fused && it.ph == 1 && !((ready_bits[grp >> 5] >> (grp & 31)) & 1u)) {
                     // wait until every gate/up tile of the group has stored its h rows
-                    const int32_t *flag = p.hdone + (it.shared ? p.E : it.e);
+                    const int32_t *flag = p.hdone + grp;
                     const int target = (it.shared ? p.Rs[0] : p.R[0]) * it.ntt;
                     bool ready = ld_acquire(flag) >= target;
                     const unsigned long long t0 = ready ? 0ull : globaltimer();
@@ -448,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                         }
                     }
                     if (!ready) break;
+                    ready_bits[grp >> 5] |= 1u << (grp & 31);  // counts only grow within a launch
                     fence_proxy_async_global();  // the TMA loads below read h written by other CTAs
                 }
                 const PhaseMaps &pm = maps.ph[it.ph];
@@ -671,7 +675,7 @@ int pick_bn(long long T, int k, int E, int Is) {
 
 size_t smem_bytes_for(int BN, int E, int stages) {
     return 1024 + (size_t)stages * (kABytes + BN * 128) + 64 * kXchgStride * 4 + 2 * (size_t)(E + 1) * 4 + 8 +
-           (size_t)(2 * stages + 5 + 2 * kQueue) * 8 + 32 + kThreads * 4;
+           (size_t)(2 * stages + 5 + 2 * kQueue) * 8 + 32 + kThreads * 4 + kReadyWords * 4;
 }
 
 int pick_stages(int BN, int E) {
