@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int E, int nchunks, int32_t 
         sched[8 + e] = 0;
     }
     if (hdone != nullptr)
-        for (int g = e; g <= E; g += blockDim.x) hdone[g] = 0;
+        for (int g = e; g <= E + 1; g += blockDim.x) hdone[g] = 0;
     int c = 0;
     if (e < E)
         for (int b = 0; b < nchunks; ++b) c += hist[(size_t)b * E + e];
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int 
         sched[8 + threadIdx.x] = 0;
     }
     if (writer && hdone != nullptr)
-        for (int g = threadIdx.x; g <= E; g += blockDim.x) hdone[g] = 0;
+        for (int g = threadIdx.x; g <= E + 1; g += blockDim.x) hdone[g] = 0;
     __syncthreads();
     const int s_begin = warp * chunk, s_end = min(Tk, s_begin + chunk);
     if (warp < W) {

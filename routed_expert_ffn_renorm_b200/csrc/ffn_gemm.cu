@@ -98,7 +98,7 @@ struct FfnParams {
     uint16_t *ybuf;      // [T, k+1, H]
     int32_t *status;     // status word
     int32_t *sched;      // [0] next work item, [1] CTAs done; zero between launches
-    int32_t *hdone;      // [E+1] finished gate/up items per group (E = shared); zero between launches
+    int32_t *hdone;      // [E+2] finished gate/up items per group (E = shared), [E+1] in all; zero between launches
 };
 
 // ------------------------------------------------------------ PTX helpers --
@@ -422,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             uint32_t phase = 0, issued = 0, last_phase = 0;
             const uint64_t wpol = policy_evict_first();  // expert weights: read once per launch
             int next = atomicAdd(p.sched, 1);            // items are claimed one ahead
+            bool all_ready = false;                       // every gate/up item of the launch is done
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 const uint32_t qph = (uint32_t)(li / kQueue) & 1u;
@@ -433,14 +434,20 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 if (item < 0) break;
                 const Item it = decode_item(item, sc, p);
                 const int grp = it.shared ? p.E : it.e;
-                if (fused && it.ph == 1 && !((ready_bits[grp >> 5] >> (grp & 31)) & 1u)) {
+                if (fused && it.ph == 1 && !all_ready && !((ready_bits[grp >> 5] >> (grp & 31)) & 1u)) {
                     // wait until every gate/up tile of the group has stored its h rows
+                    // (or every gate/up item of the launch is done)
                     const int32_t *flag = p.hdone + grp;
                     const int target = (it.shared ? p.Rs[0] : p.R[0]) * it.ntt;
-                    bool ready = ld_acquire(flag) >= target;
+                    auto check = [&]() {
+                        const int all = ld_acquire(p.hdone + p.E + 1), mine = ld_acquire(flag);
+                        if (all >= sc.n[0]) all_ready = true;
+                        return all_ready || mine >= target;
+                    };
+                    bool ready = check();
                     const unsigned long long t0 = ready ? 0ull : globaltimer();
                     for (uint32_t spin = 1; !ready; ++spin) {
-                        ready = ld_acquire(flag) >= target;
+                        ready = check();
                         if (!ready && (spin & 63u) == 0) {
                             if (*abort_flag) break;
                             if (globaltimer() - t0 > kWaitLimitNs) {
@@ -609,7 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             named_bar_sync(1, 128);
             if (elected) {
                 mbar_arrive(&tempty[acc]);
-                if (fused && it.ph == 0) atomicAdd(p.hdone + (it.shared ? p.E : it.e), 1);
+                if (fused && it.ph == 0) {
+                    atomicAdd(p.hdone + (it.shared ? p.E : it.e), 1);
+                    atomicAdd(p.hdone + p.E + 1, 1);
+                }
             }
         }
     }
@@ -627,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             atomicExch(p.sched, 0);
             atomicExch(p.sched + 1, 0);
             if (fused)
-                for (int g = 0; g <= p.E; ++g) atomicExch(p.hdone + g, 0);
+                for (int g = 0; g <= p.E + 1; ++g) atomicExch(p.hdone + g, 0);
             __threadfence();
         }
     }

@@ -12,7 +12,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 // Head of the workspace: [0, 256) status word and work-item counters,
-// [256, 256 + 4 * (E + 1)) per-group gate/up counters of the fused FFN.
+// [256, 256 + 4 * (E + 2)) gate/up completion counters of the fused FFN.
 constexpr size_t kHeadBytes = 8192;
 constexpr size_t kHdoneOffset = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }

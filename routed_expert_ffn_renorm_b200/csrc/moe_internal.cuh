@@ -63,7 +63,7 @@ cudaError_t launch_budget(int T, int E, int k, int N, int norm_topk, int32_t *id
 // Dispatch: histogram, scan, stable scatter, row gather.
 int dispatch_chunks(int T);
 // `status_block`, `hdone` (may be null): the dispatch kernels also zero the
-// grouped FFN's work-item counters and per-group gate/up counters [E + 1].
+// grouped FFN's work-item counters and gate/up completion counters [E + 2].
 // x_perm (may be null): also gather x_perm[p] = x[perm[p] / k].
 cudaError_t launch_dispatch(int T, int E, int k, const int32_t *idx, const int32_t *keff,
                             int32_t *hist, int32_t *counts, int32_t *offsets, int32_t *perm,
@@ -88,7 +88,7 @@ struct FfnArgs {
     uint16_t *h_perm, *h_shared, *ybuf;
     int32_t *status;  // the workspace's status block: [0] status word,
                       // [4..5] gate/up (or fused) and [8..9] down work-item counters
-    int32_t *hdone;   // [E + 1] per-group finished gate/up tiles (fused launches)
+    int32_t *hdone;   // [E + 2] per-group finished gate/up tiles, then all of them (fused launches)
 };
 // One launch of the grouped FFN kernel.  phases: 1 = gate/up (writes
 // h_perm / h_shared), 2 = down (reads them, writes ybuf), 3 = both in one
