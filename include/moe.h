@@ -168,6 +168,37 @@ int moe_expert_down(const moe_config_t *cfg, int32_t T, const int32_t *offsets, 
                     const float *topk_w, const float *sgate, const moe_weights_t *w, moe_bf16_t *ybuf, void *ws,
                     size_t ws_bytes, void *stream);
 
+/* Expert FFN for callers that cannot allocate device memory.  The pages
+ * have no counterpart of this entry point; it exists for integration.
+ *
+ * Same computation, arguments and results as moe_expert_ffn, but with no
+ * workspace: the scratch it needs (the gate/up activations and the
+ * scheduling counters) lives in a fixed device array inside the library.
+ * Use it when the caller cannot allocate -- e.g. a plugin that its host
+ * framework hands only input and output buffers, or a serving loop that
+ * must not allocate (an allocation can synchronise the device) once it runs.
+ *   - Limit: 2 * (T*k*I + T*Is) bytes of activations must fit in
+ *     MOE_NOALLOC_SCRATCH_BYTES; larger batches return MOE_ERR_WORKSPACE
+ *     before anything is launched (use moe_expert_ffn for them).
+ *   - The array (MOE_NOALLOC_SCRATCH_BYTES + 8 KB) is held on every device
+ *     that loads the library until the process exits.
+ *   - The first call on a device looks the array's address up (a CUDA
+ *     runtime query); make that first call before capturing a stream into a
+ *     CUDA graph.
+ *   - All calls share the one array: calls whose work overlaps on the GPU
+ *     (e.g. on two streams at once) race and corrupt each other.  Each call
+ *     re-zeroes the counters it needs (an async memset on `stream`); nothing
+ *     else of the previous call's contents is relied on.
+ *   - The call allocates nothing: no cudaMalloc, cudaFree or allocating
+ *     library routine.
+ *   - device_status (device pointer, may be NULL) receives the kernel's
+ *     MOE_STATUS_* bits of this call.
+ * Arguments otherwise as in moe_expert_ffn (no ws/ws_bytes). */
+#define MOE_NOALLOC_SCRATCH_BYTES (8u << 20)
+int moe_expert_ffn_noalloc(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                           const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                           const moe_weights_t *w, moe_bf16_t *ybuf, int32_t *device_status, void *stream);
+
 /* Combine: out[t, :] = bf16( sum_{j < keff[t]} ybuf[t, j, :] + [Is > 0] ybuf[t, k, :] ),
  * summed in fp32 in slot order and rounded once (a token with no kept slot
  * and no shared expert gets 0).  keff == NULL means k.

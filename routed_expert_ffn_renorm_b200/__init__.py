@@ -23,7 +23,8 @@ from typing import Optional
 
 __all__ = [
     "MoEConfig", "MoEWeights", "MoEError", "load_library", "workspace_bytes", "moe_route", "moe_budget",
-    "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_forward",
+    "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn_noalloc",
+    "moe_combine", "moe_forward",
     "status_read", "status_clear",
     "EXPORTED_SYMBOLS", "MOE_STATUS_TIMEOUT",
 ]
@@ -34,8 +35,9 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_route", "moe_budget", "moe_dispatch", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_status_read", "moe_status_clear", "moe_error_string", "moe_expert_gate_up",
-    "moe_expert_down",
+    "moe_expert_down", "moe_expert_ffn_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 MOE_STATUS_TIMEOUT = 1
 
 
@@ -123,6 +125,7 @@ def load_library(build_if_stale: bool = True):
         lib.moe_combine.argtypes = [cfg, i32, P, P, P, P]
         lib.moe_expert_gate_up.argtypes = [cfg, i32, P, P, P, ctypes.POINTER(_Weights), P, sz, P]
         lib.moe_expert_down.argtypes = [cfg, i32, P, P, P, P, ctypes.POINTER(_Weights), P, P, sz, P]
+        lib.moe_expert_ffn_noalloc.argtypes = [cfg, i32, P, P, P, P, P, P, ctypes.POINTER(_Weights), P, P, P]
         lib.moe_forward.argtypes = [cfg, i32, P, P, ctypes.POINTER(_Weights), P, ctypes.POINTER(_Aux), P, sz, P]
         lib.moe_status_read.argtypes = [P, ctypes.POINTER(i32), P]
         lib.moe_status_clear.argtypes = [P, P]
@@ -217,6 +220,19 @@ def moe_expert_down(cfg: MoEConfig, T: int, offsets, perm, topk_w, weights: MoEW
     _check("moe_expert_down", load_library().moe_expert_down(
         ctypes.byref(cfg._c()), T, _ptr(offsets), _ptr(perm), _ptr(topk_w), _ptr(sgate, True), ctypes.byref(w),
         _ptr(ybuf), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_expert_ffn_noalloc(cfg: MoEConfig, x, x_perm, offsets, perm, topk_w, weights: MoEWeights, ybuf, *,
+                           sgate=None, device_status=None, stream=None):
+    """moe_expert_ffn without a workspace, for callers that cannot allocate
+    device memory: the scratch lives in a fixed 8 MiB device array inside the
+    library (batches needing more raise MoEError with code -3).  Calls whose
+    work overlaps on the GPU share that array and must not run concurrently."""
+    T = x.shape[0]
+    w = weights._c()
+    _check("moe_expert_ffn_noalloc", load_library().moe_expert_ffn_noalloc(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(perm), _ptr(topk_w), _ptr(sgate, True),
+        ctypes.byref(w), _ptr(ybuf), _ptr(device_status, True), _stream(stream)))
 
 
 def moe_combine(cfg: MoEConfig, ybuf, out, *, keff=None, stream=None):

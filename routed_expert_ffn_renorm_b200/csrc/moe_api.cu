@@ -3,6 +3,7 @@
 // moe_status_read, which waits for its own copy); every launch goes on the
 // caller's stream.
 #include <cstring>
+#include <mutex>
 
 #include "moe_internal.cuh"
 
@@ -231,6 +232,100 @@ int moe_expert_ffn(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, cons
     rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, false, &b);
     if (rc) return rc;
     return ffn_launch_both(a, as_stream(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Expert FFN without any device allocation by the caller.
+//
+// Some callers cannot allocate device memory: a plugin that a host framework
+// hands only its input and output buffers (no allocator, no way to keep a
+// workspace of its own), or a serving loop that must not allocate once it
+// is running (an allocation can synchronise the device and stall every
+// stream).  For them the FFN's scratch -- the gate/up activations h and the
+// scheduling counters -- lives in this file-scope device array instead of a
+// caller workspace.  It is sized for decode-sized batches: the routed and
+// shared h rows, 2 * (T*k*I + T*Is) bytes, must fit in kNoallocScratchBytes
+// (8 MiB), plus an 8 KiB block of counters.  Every GPU that loads the library
+// holds the array until the process exits.
+constexpr size_t kNoallocScratchBytes = MOE_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kHeadBytes + kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device (with that
+// device current) on the first call there.
+void *noalloc_scratch_ptr(int dev) {
+    static void *ptrs[64] = {};
+    static std::mutex mu;
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        ptrs[dev] = p;
+    }
+    return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_expert_ffn_noalloc(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                           const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                           const moe_weights_t *w, moe_bf16_t *ybuf, int32_t *device_status, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    const bool sh = cfg->shared_intermediate_size > 0;
+    if (!w || !aligned(offsets) || !aligned(x_perm) || !aligned(w->w_gate) || !aligned(w->w_up) || !aligned(perm) ||
+        !aligned(topk_w) || !aligned(ybuf) || !aligned(w->w_down) || !aligned_or_null(device_status))
+        return MOE_ERR_INVALID_ARG;
+    if (sh && (!aligned(x) || !aligned(w->ws_gate) || !aligned(w->ws_up) || !aligned(sgate) || !aligned(w->ws_down)))
+        return MOE_ERR_INVALID_ARG;
+    // scratch layout after the counter block: h_perm [T*k, I], then h_shared [T, Is]
+    const size_t h_perm_bytes = align_up((size_t)T * cfg->num_experts_per_tok * cfg->moe_intermediate_size * 2);
+    const size_t h_shared_bytes = align_up((size_t)T * cfg->shared_intermediate_size * 2);
+    if (h_perm_bytes + h_shared_bytes > kNoallocScratchBytes) return MOE_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    uint8_t *scratch = static_cast<uint8_t *>(noalloc_scratch_ptr(dev));
+    if (!scratch) return MOE_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    // the counters must start at zero; the array keeps whatever the last call left
+    if (cudaMemsetAsync(scratch, 0, kHeadBytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+    FfnArgs a{};
+    a.T = T;
+    a.H = cfg->hidden;
+    a.E = cfg->n_routed_experts;
+    a.I = cfg->moe_intermediate_size;
+    a.k = cfg->num_experts_per_tok;
+    a.Is = cfg->shared_intermediate_size;
+    a.x = x;
+    a.x_perm = x_perm;
+    a.offsets = offsets;
+    a.perm = perm;
+    a.topk_w = topk_w;
+    a.sgate = sgate;
+    a.w_gate = w->w_gate;
+    a.w_up = w->w_up;
+    a.w_down = w->w_down;
+    a.ws_gate = w->ws_gate;
+    a.ws_up = w->ws_up;
+    a.ws_down = w->ws_down;
+    a.status = reinterpret_cast<int32_t *>(scratch);
+    a.hdone = reinterpret_cast<int32_t *>(scratch + kHdoneOffset);
+    a.h_perm = reinterpret_cast<uint16_t *>(scratch + kHeadBytes);
+    a.h_shared = sh ? reinterpret_cast<uint16_t *>(scratch + kHeadBytes + h_perm_bytes) : nullptr;
+    a.ybuf = ybuf;
+    rc = ffn_launch_both(a, st);
+    if (rc) return rc;
+    if (device_status)  // hand the kernel's status word to the caller
+        if (cudaMemcpyAsync(device_status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    return MOE_OK;
 }
 
 int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, const int32_t *keff, moe_bf16_t *out,
