@@ -28,6 +28,22 @@
 // buffered (2 x BN columns) so the epilogue of one tile overlaps the
 // mainloop of the next.
 //
+// Shared-memory ring.  One K step needs 16 KB of weights and 128 B per
+// token row, and the token count of a tile ranges from 1 to 256, so the
+// ring is cut into 2 KB pages and each K step takes 8 + 2^b consecutive
+// pages, its token rows being one TMA box of 16 << b rows, the smallest that
+// holds the tile (a step that would straddle the end of the ring starts
+// over at page 0).  A 28-token step then holds 20 KB instead of a fixed
+// 16 KB + 32 KB slot: narrow routed tiles keep ~10 steps of weights in
+// flight, and the shared expert still gets whole 256-token tiles.  Producer
+// and MMA lane walk the same page sequence; each K step has its own barrier
+// pair ("ticket", 32 of them), and the producer reuses pages only after the
+// MMAs of the steps that held them have committed.  Both lanes are on the
+// critical path of every step, so a step carries two 64-wide K slices when
+// its token box is at most 64 rows (32 KB of weights per barrier round
+// trip), and their loops avoid divisions and out-of-line calls on the
+// common path.
+//
 // Roles (192 threads, one CTA per SM, persistent): warp 0 -- TMA producer
 // (one lane); warp 1 -- TMEM allocation and MMA issue (one lane); warps
 // 2..5 -- epilogue, one TMEM lane quarter each.
@@ -59,12 +75,16 @@ namespace moe {
 
 namespace {
 
-constexpr int kBlockK = 64;                    // K elements per stage (128 B rows)
+constexpr int kBlockK = 64;                    // K elements per step (128 B rows)
 constexpr int kTileM = 128;                    // weight rows per tile (MMA M)
 constexpr int kABytes = kTileM * kBlockK * 2;  // 16 KB
 constexpr int kNumBox = 5;                     // token box heights 16 << i
 constexpr int kThreads = 192;
-constexpr int kMaxStages = 16;
+constexpr int kPageBytes = 2048;               // ring unit: 16 token rows of 128 B
+constexpr int kAPages = kABytes / kPageBytes;  // 8 pages of weights per K step
+constexpr int kMaxStepPages = kAPages + 256 * 128 / kPageBytes;  // 24: weights + 256 token rows
+constexpr int kMaxPages = 112;
+constexpr int kTickets = 32;                   // K steps in flight at most (barrier pairs)
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
 constexpr int kXchgStride = 33;                // fp32 exchange row stride (bank-conflict free)
 constexpr int kQueue = 4;                      // work-item queue depth (producer -> MMA, epilogue)
@@ -84,8 +104,9 @@ struct __align__(64) FfnMaps {
 
 struct FfnParams {
     int T, H, E, I, k, Is;
-    int BN;             // token tile (power of two, 32..256)
-    int stages;
+    int BN;             // token tile of the routed experts (power of two, 32..256)
+    int BNs;            // token tile of the shared expert (power of two, 32..BN)
+    int pages;          // shared-memory ring size in kPageBytes pages (>= kMaxStepPages)
     int phases;         // bit 0: gate/up items, bit 1: down items
     int R[2], Rs[2];    // weight tiles per routed / shared expert, per phase
     int nk[2], nks[2];  // K steps routed / shared, per phase
@@ -148,6 +169,11 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
             }
         }
     }
+}
+// The common case (already complete) inline; the bounded spin out of line.
+__device__ __forceinline__ bool mbar_wait_fast(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                               int32_t *status, bool watch_abort) {
+    return mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort_flag, status, watch_abort);
 }
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y) {
     asm volatile(
@@ -262,8 +288,8 @@ __device__ __forceinline__ Item decode_item(int item, const Schedule &sc, const 
         it.shared = 1;
         it.e = p.E;
         it.r = local / sc.shared_ntt;
-        it.row0 = j * p.BN;
-        it.nvalid = min(p.BN, p.T - j * p.BN);
+        it.row0 = j * p.BNs;
+        it.nvalid = min(p.BNs, p.T - j * p.BNs);
         it.ntt = sc.shared_ntt;
     } else {
         const int tile_item = item - sh_items;  // routed items: tile_base[e] * R + (r * ntt + j)
@@ -288,10 +314,46 @@ __device__ __forceinline__ Item decode_item(int item, const Schedule &sc, const 
     return it;
 }
 
-__device__ __forceinline__ int box_index(int nvalid) {
+// Next K step of `need` pages.  `vhead` counts pages without wrapping,
+// `off` is its position in the ring (vhead mod P, kept without a division).
+// A step never straddles the ring end: the pages left before the end are
+// skipped and belong to this step.  Returns the step's first ring page.  The
+// producer and the MMA lane call this on the same sequence of steps.
+__device__ __forceinline__ uint32_t ring_alloc(uint32_t &vhead, uint32_t &off, uint32_t need, uint32_t P) {
+    if (off + need > P) {
+        vhead += P - off;
+        off = 0;
+    }
+    const uint32_t first = off;
+    vhead += need;
+    off += need;
+    return first;
+}
+
+__device__ __forceinline__ int box_index(int nvalid) {  // smallest box of 16 << b rows holding the tile
     int b = 0;
     while ((16 << b) < nvalid) ++b;
     return b;
+}
+
+// Ring steps of an item.  A sub-step is one 64-wide K slice: 16 KB of
+// weights followed by one token box of 16 << bi rows (sub_pages pages).  A
+// ring step carries ns sub-steps -- two while the token box is at most 64
+// rows, so the per-step work of the producer and MMA lanes is spent once per
+// 32 KB of weights -- and never more than kMaxStepPages pages.
+struct StepShape {
+    int bi;              // token box index
+    uint32_t sub_pages;  // pages per sub-step
+    int ns;              // sub-steps per ring step (the item's last step may hold fewer)
+    int nk;              // 64-wide K slices of the item
+};
+__device__ __forceinline__ StepShape step_shape(const Item &it, const FfnParams &p) {
+    StepShape sh;
+    sh.bi = box_index(it.nvalid);
+    sh.sub_pages = kAPages + (1u << sh.bi);
+    sh.ns = 2 * sh.sub_pages <= (uint32_t)kMaxStepPages ? 2 : 1;
+    sh.nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
+    return sh;
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
@@ -300,23 +362,23 @@ __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g));
 __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnMaps maps, const FfnParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int S = p.stages;
-    const int stage_bytes = kABytes + p.BN * 128;
-    uint8_t *stages = smem;
-    float *xchg = reinterpret_cast<float *>(smem + (size_t)S * stage_bytes);
+    const uint32_t P = (uint32_t)p.pages;
+    uint8_t *ring = smem;
+    float *xchg = reinterpret_cast<float *>(smem + (size_t)P * kPageBytes);
     int *tile_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
     int *offs = tile_base + (p.E + 1);                                  // [E + 1]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
         (reinterpret_cast<uintptr_t>(offs + (p.E + 1)) + 7) & ~uintptr_t(7));
-    uint64_t *full = bars, *empty = bars + S, *tfull = bars + 2 * S, *tempty = bars + 2 * S + 2;
-    uint64_t *mma_done = bars + 2 * S + 4;
-    uint64_t *qfull = bars + 2 * S + 5, *qempty = qfull + kQueue;
+    uint64_t *full = bars, *empty = bars + kTickets, *tfull = bars + 2 * kTickets, *tempty = tfull + 2;
+    uint64_t *mma_done = tfull + 4;
+    uint64_t *qfull = tfull + 5, *qempty = qfull + kQueue;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qempty + kQueue);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_item = reinterpret_cast<volatile int *>(tmem_slot + 2);
     volatile int *qitem = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kQueue]
     int *scan_tmp = reinterpret_cast<int *>(tmem_slot + 8);                 // [kThreads]
     uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + kThreads);  // [kReadyWords], producer-private
+    uint32_t *ticket_start = ready_bits + kReadyWords;  // [kTickets] first ring page (virtual) of each step; producer-private
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tmem_cols = 2 * p.BN;
@@ -324,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
 
     // ---- setup: barriers, TMEM, tile schedule
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < kTickets; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -406,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     __syncthreads();
     tc_fence_after();
     Schedule sc;
-    sc.shared_ntt = p.Is > 0 ? (p.T + p.BN - 1) / p.BN : 0;
+    sc.shared_ntt = p.Is > 0 ? (p.T + p.BNs - 1) / p.BNs : 0;
     sc.tile_base = tile_base;
     sc.offs = offs;
     for (int ph = 0; ph < 2; ++ph)
@@ -418,8 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     if (warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0, issued = 0, last_phase = 0;
+            uint32_t vhead = 0, off = 0;       // ring pages handed out (virtual: never wraps) / its ring position
+            uint32_t issued = 0, retired = 0;  // K steps issued / whose MMAs have released their pages
+            uint32_t oldest = 0;               // first page (virtual) of step `retired` while one is in flight
             const uint64_t wpol = policy_evict_first();  // expert weights: read once per launch
             int next = atomicAdd(p.sched, 1);            // items are claimed one ahead
             bool all_ready = false;                       // every gate/up item of the launch is done
@@ -462,47 +525,57 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     fence_proxy_async_global();  // the TMA loads below read h written by other CTAs
                 }
                 const PhaseMaps &pm = maps.ph[it.ph];
-                const int bi = box_index(it.nvalid);
                 const CUtensorMap *ma0 = it.shared ? &pm.s0 : &pm.a0;
                 const CUtensorMap *ma1 = it.shared ? &pm.s1 : &pm.a1;
-                const CUtensorMap *mb = it.shared ? &pm.bs[bi] : &pm.b[bi];
+                const StepShape sh = step_shape(it, p);
+                const CUtensorMap *mb = it.shared ? &pm.bs[sh.bi] : &pm.b[sh.bi];
                 const int a_row = it.ph == 0 ? (it.shared ? 0 : it.e * p.I) + it.r * 64
                                              : (it.shared ? 0 : it.e * p.H) + it.r * kTileM;
-                const int nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
-                const uint32_t bytes = kABytes + (uint32_t)(16 << bi) * 128u;
                 bool ok = true;
-                for (int ks = 0; ks < nk; ++ks) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, true)) {
-                        ok = false;
-                        break;
+                for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
+                    const int nsub = min(sh.ns, sh.nk - k0);
+                    const uint32_t need = (uint32_t)nsub * sh.sub_pages;
+                    const uint32_t first = ring_alloc(vhead, off, need, P);
+                    // Free a ticket and the pages of this step: retire the oldest steps
+                    // until the steps in flight and this one lie within P consecutive
+                    // (virtual) pages -- then no two of them share a physical page.
+                    while (issued != retired && (vhead - oldest > P || issued - retired >= (uint32_t)kTickets)) {
+                        if (!mbar_wait_fast(&empty[retired % kTickets], (retired / kTickets) & 1u, abort_flag,
+                                            p.status, true)) {
+                            ok = false;
+                            break;
+                        }
+                        ++retired;
+                        oldest = ticket_start[retired % kTickets];  // read only while retired != issued
                     }
-                    uint8_t *sA = stages + (size_t)stage * stage_bytes;
-                    mbar_arrive_expect_tx(&full[stage], bytes);
-                    if (it.ph == 0) {
-                        tma_load_2d_hint(ma0, &full[stage], sA, ks * kBlockK, a_row, wpol);
-                        tma_load_2d_hint(ma1, &full[stage], sA + kABytes / 2, ks * kBlockK, a_row, wpol);
-                    } else {
-                        tma_load_2d_hint(ma0, &full[stage], sA, ks * kBlockK, a_row, wpol);
+                    if (!ok) break;
+                    const uint32_t tk = issued % kTickets;
+                    if (issued == retired) oldest = vhead - need;
+                    ticket_start[tk] = vhead - need;
+                    mbar_arrive_expect_tx(&full[tk], need * kPageBytes);
+                    for (int j = 0; j < nsub; ++j) {
+                        uint8_t *sA = ring + (size_t)(first + j * sh.sub_pages) * kPageBytes;
+                        const int kx = (k0 + j) * kBlockK;
+                        if (it.ph == 0) {
+                            tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
+                            tma_load_2d_hint(ma1, &full[tk], sA + kABytes / 2, kx, a_row, wpol);
+                        } else {
+                            tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
+                        }
+                        tma_load_2d(mb, &full[tk], sA + kABytes, kx, it.row0);
                     }
-                    tma_load_2d(mb, &full[stage], sA + kABytes, ks * kBlockK, it.row0);
-                    issued |= 1u << stage;
-                    last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    ++issued;
                 }
                 if (!ok) break;
             }
             // wait for every copy still in flight before the CTA may exit
-            for (int s = 0; s < S; ++s)
-                if ((issued >> s) & 1u) mbar_wait(&full[s], (last_phase >> s) & 1u, abort_flag, p.status, false);
+            for (uint32_t j = retired; j < issued; ++j)
+                mbar_wait(&full[j % kTickets], (j / kTickets) & 1u, abort_flag, p.status, false);
         }
     } else if (warp == 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
+            uint32_t vhead = 0, off = 0, step = 0;  // the producer's page sequence, replayed
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 if (!mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) break;
@@ -510,31 +583,32 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 mbar_arrive(&qempty[slot]);
                 if (item < 0) break;
                 const Item it = decode_item(item, sc, p);
-                const int n = (it.nvalid + 15) & ~15;
-                const uint32_t idesc = idesc_bf16(n);
+                const StepShape sh = step_shape(it, p);
+                const uint32_t idesc = idesc_bf16((it.nvalid + 15) & ~15);
                 const int acc = li & 1;
                 const uint32_t use = (uint32_t)(li >> 1);
                 if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag, p.status, true)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(acc * p.BN);
-                const int nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
                 bool ok = true;
-                for (int ks = 0; ks < nk; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag, p.status, true)) {
+                for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
+                    const int nsub = min(sh.ns, sh.nk - k0);
+                    const uint32_t first = ring_alloc(vhead, off, (uint32_t)nsub * sh.sub_pages, P);
+                    const uint32_t tk = step % kTickets;
+                    if (!mbar_wait_fast(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sA = smem_u32(stages + (size_t)stage * stage_bytes);
-                    const uint64_t da = sw128_desc(sA), db = sw128_desc(sA + kABytes);
+                    for (int j = 0; j < nsub; ++j) {
+                        const uint32_t sA = smem_u32(ring + (size_t)(first + j * sh.sub_pages) * kPageBytes);
+                        const uint64_t da = sw128_desc(sA), db = sw128_desc(sA + kABytes);
 #pragma unroll
-                    for (int kk = 0; kk < kBlockK / 16; ++kk)  // +32 bytes per K16 step
-                        umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
-                    umma_commit(&empty[stage]);
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1u;
+                        for (int kk = 0; kk < kBlockK / 16; ++kk)  // +32 bytes per K16 step
+                            umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (k0 | j | kk) != 0);
                     }
+                    umma_commit(&empty[tk]);
+                    ++step;
                 }
                 if (!ok) break;
                 umma_commit(&tfull[acc]);
@@ -671,27 +745,32 @@ bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, u
     return r == CUDA_SUCCESS;
 }
 
-// Token tile: at least twice the mean tokens per routed expert, and with a
-// shared expert at least min(T, 128) so its weight tiles are not re-read by
-// many narrow token tiles; 64..256.
-int pick_bn(long long T, int k, int E, int Is) {
-    const long long avg = (T * k + E - 1) / E;  // mean tokens per expert
-    long long want = 2 * avg;
-    if (Is > 0) want = std::max<long long>(want, std::min<long long>(T, 128));
-    int bn = 64;
-    while (bn < 256 && bn < want) bn <<= 1;
-    return bn;
+// Token tile of the routed experts: the largest MMA N.  A tile's
+// shared-memory cost follows its real token count (the paged ring), so a
+// wide tile costs nothing for small groups and saves re-reading a weight
+// tile for every 128 tokens of large ones.
+int pick_bn() { return 256; }
+
+// Token tile of the shared expert, which sees all T tokens.  One 256-token
+// tile streams each weight tile once, but its items then run about twice as
+// long as the routed ones; when the gate/up phase has few items per SM that
+// unbalances the launch, and two 128-token tiles (the second one's weights
+// from L2) finish sooner.  The item estimate counts every expert as active.
+int pick_bns(const FfnArgs &a, int bn, int sms) {
+    if (a.Is == 0 || a.T <= 128) return bn;
+    const long long est = std::min<long long>(a.E, (long long)a.T * a.k) * (a.I / 64);
+    return est >= 4LL * sms ? bn : std::min(bn, 128);
 }
 
-size_t smem_bytes_for(int BN, int E, int stages) {
-    return 1024 + (size_t)stages * (kABytes + BN * 128) + 64 * kXchgStride * 4 + 2 * (size_t)(E + 1) * 4 + 8 +
-           (size_t)(2 * stages + 5 + 2 * kQueue) * 8 + 32 + kThreads * 4 + kReadyWords * 4;
+size_t smem_bytes_for(int E, int pages) {
+    return 1024 + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 + 2 * (size_t)(E + 1) * 4 + 8 +
+           (size_t)(2 * kTickets + 5 + 2 * kQueue) * 8 + 32 + kThreads * 4 + kReadyWords * 4 + kTickets * 4;
 }
 
-int pick_stages(int BN, int E) {
-    int s = kMaxStages;
-    while (s > 2 && smem_bytes_for(BN, E, s) > (size_t)kSmemLimit) --s;
-    return s;
+int pick_pages(int E) {
+    const size_t fixed = smem_bytes_for(E, 0);
+    if (fixed >= (size_t)kSmemLimit) return 0;
+    return (int)std::min<size_t>(kMaxPages, ((size_t)kSmemLimit - fixed) / kPageBytes);
 }
 
 struct DeviceInfo {
@@ -712,25 +791,34 @@ DeviceInfo device_info() {
     return cache[dev];
 }
 
-// Benchmark/test overrides: MOE_FORCE_BN in {32, 64, 128, 256} (token tile)
-// and MOE_FORCE_STAGES in [2, 16] (pipeline depth, capped by shared memory);
-// any other value is rejected.
-int choose_tiles(const FfnArgs &a, int *bn, int *stages) {
-    *bn = pick_bn(a.T, a.k, a.E, a.Is);
-    if (const char *f = getenv("MOE_FORCE_BN")) {
-        char *end = nullptr;
-        const long v = strtol(f, &end, 10);
-        if (*f == 0 || *end != 0 || (v != 32 && v != 64 && v != 128 && v != 256)) return MOE_ERR_INVALID_ARG;
-        *bn = (int)v;
-    }
-    *stages = pick_stages(*bn, a.E);
-    if (const char *f = getenv("MOE_FORCE_STAGES")) {
-        char *end = nullptr;
-        const long v = strtol(f, &end, 10);
-        if (*f == 0 || *end != 0 || v < 2 || v > kMaxStages) return MOE_ERR_INVALID_ARG;
-        *stages = std::min<int>((int)v, *stages);
-    }
+// Benchmark/test overrides: MOE_FORCE_BN and MOE_FORCE_BNS in {32, 64, 128,
+// 256} (routed / shared token tile, BNS <= BN) and MOE_FORCE_PAGES in
+// [24, 112] (ring size in 2 KB pages, capped by shared memory; 24 holds one
+// widest K step); any other value is rejected.
+int parse_tile(const char *f, int *out) {
+    char *end = nullptr;
+    const long v = strtol(f, &end, 10);
+    if (*f == 0 || *end != 0 || (v != 32 && v != 64 && v != 128 && v != 256)) return MOE_ERR_INVALID_ARG;
+    *out = (int)v;
     return MOE_OK;
+}
+
+int choose_tiles(const FfnArgs &a, int sms, int *bn, int *bns, int *pages) {
+    *bn = pick_bn();
+    if (const char *f = getenv("MOE_FORCE_BN"))
+        if (int rc = parse_tile(f, bn)) return rc;
+    *bns = pick_bns(a, *bn, sms);
+    if (const char *f = getenv("MOE_FORCE_BNS"))
+        if (int rc = parse_tile(f, bns)) return rc;
+    if (*bns > *bn) return MOE_ERR_INVALID_ARG;
+    *pages = pick_pages(a.E);
+    if (const char *f = getenv("MOE_FORCE_PAGES")) {
+        char *end = nullptr;
+        const long v = strtol(f, &end, 10);
+        if (*f == 0 || *end != 0 || v < kMaxStepPages || v > kMaxPages) return MOE_ERR_INVALID_ARG;
+        *pages = std::min<int>((int)v, *pages);
+    }
+    return *pages >= kMaxStepPages ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -740,7 +828,7 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
     if (phases < 1 || phases > 3) return MOE_ERR_INVALID_ARG;
     FfnParams p{};
-    if (int rc = choose_tiles(a, &p.BN, &p.stages)) return rc;
+    if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
     const int BN = p.BN;
     p.T = a.T;
     p.H = a.H;
@@ -794,7 +882,7 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     }
     if (!ok) return MOE_ERR_CUDA;
 
-    const size_t smem = smem_bytes_for(BN, a.E, p.stages);
+    const size_t smem = smem_bytes_for(a.E, p.pages);
     if (smem > (size_t)kSmemLimit) return MOE_ERR_UNSUPPORTED;
     static std::atomic<int> attr_set[64];  // per device: opted in to the full shared memory
     int dev = 0;
@@ -807,7 +895,7 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     // upper bound on work items (the real count is known only on the device)
     const long long slots = (long long)a.T * a.k;
     const long long tiles = std::min<long long>(a.E, slots) + (slots + BN - 1) / BN;
-    const long long st_tiles = a.Is > 0 ? (a.T + BN - 1) / BN : 0;
+    const long long st_tiles = a.Is > 0 ? (a.T + p.BNs - 1) / p.BNs : 0;
     long long items = 0;
     for (int ph = 0; ph < 2; ++ph)
         if ((phases >> ph) & 1) items += tiles * p.R[ph] + st_tiles * p.Rs[ph];

@@ -94,21 +94,40 @@ def test_deterministic_bits():
     assert (a.out_bits == b.out_bits).all() and (a.perm == b.perm).all() and (a.w == b.w).all()
 
 
-@pytest.mark.parametrize("bn", [32, 64, 128, 256])
-def test_tile_config_invariance(bn, monkeypatch):
-    """Forced token-tile sizes give bit-identical outputs (tiling never changes a K-reduction)."""
+@pytest.mark.parametrize("bn,bns", [(32, None), (64, None), (128, None), (256, None), (256, 32), (256, 128),
+                                    (128, 64)])
+def test_tile_config_invariance(bn, bns, monkeypatch):
+    """Forced token-tile sizes (routed / shared) give bit-identical outputs
+    (tiling never changes a K-reduction)."""
     cfg = W.MoEConfig("inv", T=700, H=256, E=8, I=128, k=2, Is=64, zipf_alpha=1.5)
     inp = W.make_inputs(cfg, device="cuda")
     ref = gpu_forward(cfg, inp)
     monkeypatch.setenv("MOE_FORCE_BN", str(bn))
+    if bns is not None:
+        monkeypatch.setenv("MOE_FORCE_BNS", str(bns))
     got = gpu_forward(cfg, inp)
     assert (got.out_bits == ref.out_bits).all()
 
 
-def test_force_bn_rejects_bad_values(monkeypatch):
+@pytest.mark.parametrize("pages", [24, 25, 33, 57])
+def test_ring_size_invariance(pages, monkeypatch):
+    """Small shared-memory rings (24 pages hold one 256-token K step) force
+    wrap-around skips and retire waits at every step; the output bits stay put."""
+    cfg = W.MoEConfig("ring", T=300, H=512, E=8, I=128, k=2, Is=128, zipf_alpha=1.2)
+    inp = W.make_inputs(cfg, device="cuda")
+    ref = gpu_forward(cfg, inp)
+    monkeypatch.setenv("MOE_FORCE_PAGES", str(pages))
+    got = gpu_forward(cfg, inp)
+    assert (got.out_bits == ref.out_bits).all()
+
+
+@pytest.mark.parametrize("env", [{"MOE_FORCE_BN": "48"}, {"MOE_FORCE_BNS": "512"}, {"MOE_FORCE_PAGES": "23"},
+                                 {"MOE_FORCE_PAGES": "x"}, {"MOE_FORCE_BN": "64", "MOE_FORCE_BNS": "128"}])
+def test_force_overrides_reject_bad_values(env, monkeypatch):
     cfg = W.TINY
     inp = W.make_inputs(cfg, device="cuda")
-    monkeypatch.setenv("MOE_FORCE_BN", "48")
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
     with pytest.raises(moe.MoEError):
         gpu_forward(cfg, inp)
 
