@@ -22,7 +22,11 @@
 //   gate/up tile: A = [64 gate rows ; 64 up rows] of the same intermediate
 //                 indices, so gate and up of index i land in TMEM lanes i and
 //                 64 + i and the epilogue pairs them through shared memory;
-//   down tile:    A = 128 rows of W_down (128 output columns).
+//   down tile:    A = 128 rows of W_down (128 output columns); when the
+//                 down phase has many items, a group of at most BN/2 tokens
+//                 takes two such tiles per item, into two accumulators side
+//                 by side, so the token box is read once for both and there
+//                 are half as many short items.
 // Both operands are K-major bf16 in 128-byte-swizzled shared memory, loaded
 // by TMA boxes of 64 K-elements; the accumulator is fp32 in TMEM, double
 // buffered (2 x BN columns) so the epilogue of one tile overlaps the
@@ -267,51 +271,154 @@ struct Item {
     int row0;    // first activation row of the token tile
     int nvalid;  // valid tokens in the tile (1..BN)
     int ntt;     // token tiles of the group
+    int m;       // weight tiles r .. r+m-1 in this item (2: a down item of a group of <= BN/2 tokens)
+};
+
+struct ItemSlot {  // one work-item queue entry: the item number and its decoded form
+    int item;        // -1: no more items
+    Item it;
 };
 
 struct Schedule {
-    int n[2];         // items per phase (0 when the phase is not run)
-    int shared_ntt;   // token tiles of the shared expert (0 if none)
+    int n[2];              // items per phase (0 when the phase is not run)
+    int sh0, sh1;          // of which the shared expert's, per phase (they come first)
+    int shared_ntt;        // token tiles of the shared expert (0 if none)
+    int merge;             // down items of small groups take two weight tiles
+    int shared_merge;      // the shared expert's down items take two weight tiles
     const int *tile_base;  // [E+1] prefix of token tiles over routed experts (shared memory)
+    const int *dbase;      // [E+1] prefix of down items over routed experts when merging (shared memory)
     const int *offs;       // [E+1] dispatch offsets (shared memory)
 };
 
+// Down items of a group with `cnt` tokens.  When the down phase has plenty of
+// items (`merge`: at least kMergePerCta per CTA), a group that fits half a
+// token tile takes two weight tiles per item (two accumulators side by side
+// in TMEM, one token box read for both): half the items, each twice as long.
+// With few items the shorter ones balance the launch better.  Without
+// merging a group has ntt * R1 down items (token tiles x weight tiles).
+constexpr int kMergePerCta = 8;
+__device__ __forceinline__ bool down_merged(int cnt, int BN, bool merge) {
+    return merge && cnt > 0 && cnt <= (BN >> 1);
+}
+__device__ __forceinline__ int merged_down_items(int cnt, int BN, int R1) {
+    return down_merged(cnt, BN, true) ? (R1 + 1) >> 1 : ((cnt + BN - 1) / BN) * R1;
+}
+
+// Work item -> (phase, group, weight tile(s), token tile).  Phase 0 items of a
+// group: weight tile outer, token tile inner; phase 1 the same, or pairs of
+// weight tiles for a merged group.
 __device__ __forceinline__ Item decode_item(int item, const Schedule &sc, const FfnParams &p) {
     Item it;
+    it.m = 1;
     it.ph = item < sc.n[0] ? 0 : 1;
     if (it.ph) item -= sc.n[0];
-    const int sh_items = p.Rs[it.ph] * sc.shared_ntt;
-    // both phases: the shared expert's items first (they are the longest)
-    if (item < sh_items) {
-        const int local = item;
-        const int j = local % sc.shared_ntt;
+    const int sh_items = it.ph ? sc.sh1 : sc.sh0;
+    if (item < sh_items) {  // the shared expert's items first (they are the longest)
         it.shared = 1;
         it.e = p.E;
-        it.r = local / sc.shared_ntt;
-        it.row0 = j * p.BNs;
-        it.nvalid = min(p.BNs, p.T - j * p.BNs);
         it.ntt = sc.shared_ntt;
-    } else {
-        const int tile_item = item - sh_items;  // routed items: tile_base[e] * R + (r * ntt + j)
-        int lo = 0, hi = p.E - 1;         // largest e with tile_base[e] * R <= tile_item
-        const int R = p.R[it.ph];
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (sc.tile_base[mid] * R <= tile_item) lo = mid;
-            else hi = mid - 1;
+        if (it.ph == 1 && sc.shared_merge) {
+            it.r = 2 * item;
+            it.m = min(2, p.Rs[1] - it.r);
+            it.row0 = 0;
+            it.nvalid = p.T;
+        } else {
+            const int j = item % sc.shared_ntt;
+            it.r = item / sc.shared_ntt;
+            it.row0 = j * p.BNs;
+            it.nvalid = min(p.BNs, p.T - j * p.BNs);
         }
-        const int cnt = sc.offs[lo + 1] - sc.offs[lo];
-        const int ntt = (cnt + p.BN - 1) / p.BN;
-        const int local = tile_item - sc.tile_base[lo] * R;
+        return it;
+    }
+    item -= sh_items;
+    // largest e whose first item is <= item: tile_base[e] * R (phase 0, or phase 1
+    // unmerged), dbase[e] (phase 1 merged)
+    const bool by_dbase = it.ph == 1 && sc.merge;
+    const int R = p.R[it.ph];
+    const int *base = by_dbase ? sc.dbase : sc.tile_base;
+    const int scale = by_dbase ? 1 : R;
+    int lo = 0, hi = p.E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (base[mid] * scale <= item) lo = mid;
+        else hi = mid - 1;
+    }
+    const int cnt = sc.offs[lo + 1] - sc.offs[lo];
+    const int ntt = (cnt + p.BN - 1) / p.BN;
+    const int local = item - base[lo] * scale;
+    it.shared = 0;
+    it.e = lo;
+    it.ntt = ntt;
+    if (it.ph == 1 && down_merged(cnt, p.BN, sc.merge)) {
+        it.r = 2 * local;
+        it.m = min(2, p.R[1] - it.r);
+        it.row0 = sc.offs[lo];
+        it.nvalid = cnt;
+    } else {
         const int j = local % ntt;
-        it.shared = 0;
-        it.e = lo;
         it.r = local / ntt;
         it.row0 = sc.offs[lo] + j * p.BN;
         it.nvalid = min(p.BN, cnt - j * p.BN);
-        it.ntt = ntt;
     }
     return it;
+}
+
+// Exclusive block scan over the experts of two counts at once:
+// a[e] = sum_{e' < e} f(e').x, b[e] likewise with .y; a[E], b[E] = the totals.
+// Every thread of the block calls it.
+template <class F>
+__device__ __forceinline__ void expert_scan2(int E, int *a, int *b, int2 *scan_tmp, F f) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = (E + kThreads - 1) / kThreads;
+    const int e0 = threadIdx.x * per, e1 = min(E, e0 + per);
+    int2 local = make_int2(0, 0);
+    for (int e = e0; e < e1; ++e) {
+        const int2 v = f(e);
+        local.x += v.x;
+        local.y += v.y;
+    }
+    scan_tmp[threadIdx.x] = local;
+    __syncthreads();
+    if (warp == 0) {  // kThreads partials, kThreads / 32 per lane
+        int2 v[kThreads / 32];
+        int2 sum = make_int2(0, 0);
+#pragma unroll
+        for (int q = 0; q < kThreads / 32; ++q) {
+            v[q] = scan_tmp[lane * (kThreads / 32) + q];
+            sum.x += v[q].x;
+            sum.y += v[q].y;
+        }
+        int2 incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, incl.x, o), y = __shfl_up_sync(0xffffffffu, incl.y, o);
+            if (lane >= o) {
+                incl.x += x;
+                incl.y += y;
+            }
+        }
+        int2 run = make_int2(incl.x - sum.x, incl.y - sum.y);
+#pragma unroll
+        for (int q = 0; q < kThreads / 32; ++q) {
+            scan_tmp[lane * (kThreads / 32) + q] = run;
+            run.x += v[q].x;
+            run.y += v[q].y;
+        }
+    }
+    __syncthreads();
+    int2 run = scan_tmp[threadIdx.x];
+    for (int e = e0; e < e1; ++e) {
+        a[e] = run.x;
+        b[e] = run.y;
+        const int2 v = f(e);
+        run.x += v.x;
+        run.y += v.y;
+    }
+    if (e1 == E && e0 < e1) {
+        a[E] = run.x;
+        b[E] = run.y;
+    }
+    __syncthreads();
 }
 
 // Next K step of `need` pages.  `vhead` counts pages without wrapping,
@@ -337,10 +444,10 @@ __device__ __forceinline__ int box_index(int nvalid) {  // smallest box of 16 <<
 }
 
 // Ring steps of an item.  A sub-step is one 64-wide K slice: 16 KB of
-// weights followed by one token box of 16 << bi rows (sub_pages pages).  A
-// ring step carries ns sub-steps -- two while the token box is at most 64
-// rows, so the per-step work of the producer and MMA lanes is spent once per
-// 32 KB of weights -- and never more than kMaxStepPages pages.
+// weights per weight tile of the item (m of them) followed by one token box
+// of 16 << bi rows (sub_pages pages).  A ring step carries ns sub-steps --
+// two while that is at most kMaxStepPages, so the per-step work of the
+// producer and MMA lanes is spent once per 32 KB of weights.
 struct StepShape {
     int bi;              // token box index
     uint32_t sub_pages;  // pages per sub-step
@@ -350,13 +457,30 @@ struct StepShape {
 __device__ __forceinline__ StepShape step_shape(const Item &it, const FfnParams &p) {
     StepShape sh;
     sh.bi = box_index(it.nvalid);
-    sh.sub_pages = kAPages + (1u << sh.bi);
+    sh.sub_pages = (uint32_t)it.m * kAPages + (1u << sh.bi);
     sh.ns = 2 * sh.sub_pages <= (uint32_t)kMaxStepPages ? 2 : 1;
     sh.nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
     return sh;
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+
+// Down item, token n of the tile: its ybuf row (t*(k+1) + j, or t*(k+1) + k for
+// the shared expert) and the weight applied to it.
+__device__ __forceinline__ void down_dest(const Item &it, int n, const FfnParams &p, int &mrow, float &mw) {
+    mrow = 0;
+    mw = 0.f;
+    if (n >= it.nvalid) return;
+    if (it.shared) {
+        const int t = it.row0 + n;
+        mrow = t * (p.k + 1) + p.k;
+        mw = __ldg(p.sgate + t);
+    } else {
+        const int slot = __ldg(p.perm + it.row0 + n);
+        mrow = slot + slot / p.k;  // t*(k+1) + j
+        mw = __ldg(p.topk_w + slot);
+    }
+}
 
 // --------------------------------------------------------------- kernel --
 __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnMaps maps, const FfnParams p) {
@@ -366,7 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     uint8_t *ring = smem;
     float *xchg = reinterpret_cast<float *>(smem + (size_t)P * kPageBytes);
     int *tile_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
-    int *offs = tile_base + (p.E + 1);                                  // [E + 1]
+    int *dbase = tile_base + (p.E + 1);                                 // [E + 1]
+    int *offs = dbase + (p.E + 1);                                      // [E + 1]
     uint64_t *bars = reinterpret_cast<uint64_t *>(
         (reinterpret_cast<uintptr_t>(offs + (p.E + 1)) + 7) & ~uintptr_t(7));
     uint64_t *full = bars, *empty = bars + kTickets, *tfull = bars + 2 * kTickets, *tempty = tfull + 2;
@@ -374,10 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     uint64_t *qfull = tfull + 5, *qempty = qfull + kQueue;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qempty + kQueue);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_item = reinterpret_cast<volatile int *>(tmem_slot + 2);
-    volatile int *qitem = reinterpret_cast<volatile int *>(tmem_slot + 4);  // [kQueue]
-    int *scan_tmp = reinterpret_cast<int *>(tmem_slot + 8);                 // [kThreads]
-    uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + kThreads);  // [kReadyWords], producer-private
+    volatile int *epi_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // elected -> epilogue: 0 go, -1 stop
+    ItemSlot *qdesc = reinterpret_cast<ItemSlot *>(tmem_slot + 4);  // [kQueue], written by the producer
+    ItemSlot *epi_desc = qdesc + kQueue;                             // the epilogue's current item
+    int *scan_tmp = reinterpret_cast<int *>(                          // [2 * kThreads] (int2 partials)
+        (reinterpret_cast<uintptr_t>(epi_desc + 1) + 7) & ~uintptr_t(7));
+    uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + 2 * kThreads);  // [kReadyWords], producer-private
     uint32_t *ticket_start = ready_bits + kReadyWords;  // [kTickets] first ring page (virtual) of each step; producer-private
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -423,56 +550,31 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         tc_fence_before();
     }
     pdl_wait();  // the dispatch outputs and activations are ready past this point
-    // tile_base[e] = sum_{e' < e} ceil(count(e') / BN)  (block scan over experts)
-    {
-        const int per = (p.E + kThreads - 1) / kThreads;
-        const int e0 = threadIdx.x * per, e1 = min(p.E, e0 + per);
-        int local = 0;
-        for (int e = e0; e < e1; ++e) {
-            const int o0 = __ldg(p.offsets + e), o1 = __ldg(p.offsets + e + 1);
-            offs[e] = o0;
-            if (e == p.E - 1) offs[p.E] = o1;
-            local += (o1 - o0 + p.BN - 1) / p.BN;
-        }
-        scan_tmp[threadIdx.x] = local;
-        __syncthreads();
-        if (warp == 0) {  // 192 partials, 6 per lane
-            int v[kThreads / 32];
-            int sum = 0;
-#pragma unroll
-            for (int q = 0; q < kThreads / 32; ++q) {
-                v[q] = scan_tmp[lane * (kThreads / 32) + q];
-                sum += v[q];
-            }
-            int incl = sum;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int o = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += o;
-            }
-            int run = incl - sum;
-#pragma unroll
-            for (int q = 0; q < kThreads / 32; ++q) {
-                scan_tmp[lane * (kThreads / 32) + q] = run;
-                run += v[q];
-            }
-        }
-        __syncthreads();
-        int run = scan_tmp[threadIdx.x];
-        for (int e = e0; e < e1; ++e) {
-            tile_base[e] = run;
-            run += (offs[e + 1] - offs[e] + p.BN - 1) / p.BN;
-        }
-        if (e1 == p.E && e0 < e1) tile_base[p.E] = run;
-    }
+    // dispatch offsets to shared memory, then the per-expert prefix sums of token
+    // tiles and of down items
+    for (int e = threadIdx.x; e <= p.E; e += kThreads) offs[e] = __ldg(p.offsets + e);
     __syncthreads();
-    tc_fence_after();
     Schedule sc;
     sc.shared_ntt = p.Is > 0 ? (p.T + p.BNs - 1) / p.BNs : 0;
+    {
+        const int BN = p.BN, R1 = p.R[1];
+        const int *o = offs;
+        expert_scan2(p.E, tile_base, dbase, reinterpret_cast<int2 *>(scan_tmp), [=](int e) {
+            const int cnt = o[e + 1] - o[e];
+            return make_int2((cnt + BN - 1) / BN, merged_down_items(cnt, BN, R1));
+        });
+        // every CTA takes the same decision from the same offsets
+        sc.merge = (tile_base[p.E] * R1 + p.Rs[1] * sc.shared_ntt) >= kMergePerCta * (int)gridDim.x;
+    }
+    tc_fence_after();
+    sc.shared_merge = p.Is > 0 && sc.shared_ntt == 1 && down_merged(p.T, p.BN, sc.merge);
     sc.tile_base = tile_base;
+    sc.dbase = dbase;
     sc.offs = offs;
-    for (int ph = 0; ph < 2; ++ph)
-        sc.n[ph] = ((p.phases >> ph) & 1) ? p.Rs[ph] * sc.shared_ntt + tile_base[p.E] * p.R[ph] : 0;
+    sc.sh0 = p.Rs[0] * sc.shared_ntt;
+    sc.sh1 = sc.shared_merge ? (p.Rs[1] + 1) >> 1 : p.Rs[1] * sc.shared_ntt;
+    sc.n[0] = (p.phases & 1) ? sc.sh0 + tile_base[p.E] * p.R[0] : 0;
+    sc.n[1] = (p.phases & 2) ? sc.sh1 + (sc.merge ? dbase[p.E] : tile_base[p.E] * p.R[1]) : 0;
     const int total_items = sc.n[0] + sc.n[1];
     const bool fused = p.phases == 3;
     const uint32_t tmem_base = *tmem_slot;
@@ -492,10 +594,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 if (!mbar_wait(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
                 int item = next < total_items ? next : -1;
                 if (item >= 0) next = atomicAdd(p.sched, 1);  // its latency overlaps this item's loads
-                qitem[slot] = item;
+                Item it{};
+                if (item >= 0) it = decode_item(item, sc, p);  // decoded once, for all three roles
+                qdesc[slot].item = item;
+                qdesc[slot].it = it;
                 mbar_arrive(&qfull[slot]);
                 if (item < 0) break;
-                const Item it = decode_item(item, sc, p);
                 const int grp = it.shared ? p.E : it.e;
                 if (fused && it.ph == 1 && !all_ready && !((ready_bits[grp >> 5] >> (grp & 31)) & 1u)) {
                     // wait until every gate/up tile of the group has stored its h rows
@@ -561,8 +665,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                             tma_load_2d_hint(ma1, &full[tk], sA + kABytes / 2, kx, a_row, wpol);
                         } else {
                             tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
+                            if (it.m == 2) tma_load_2d_hint(ma0, &full[tk], sA + kABytes, kx, a_row + kTileM, wpol);
                         }
-                        tma_load_2d(mb, &full[tk], sA + kABytes, kx, it.row0);
+                        tma_load_2d(mb, &full[tk], sA + it.m * kABytes, kx, it.row0);
                     }
                     ++issued;
                 }
@@ -576,20 +681,21 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         // ================= MMA issuer =================
         if (lane == 0) {
             uint32_t vhead = 0, off = 0, step = 0;  // the producer's page sequence, replayed
+            const uint64_t desc0 = sw128_desc(smem_u32(ring));  // ring page 0; other pages by addition
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 if (!mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) break;
-                const int item = qitem[slot];
+                const int item = qdesc[slot].item;
+                const Item it = qdesc[slot].it;
                 mbar_arrive(&qempty[slot]);
                 if (item < 0) break;
-                const Item it = decode_item(item, sc, p);
                 const StepShape sh = step_shape(it, p);
                 const uint32_t idesc = idesc_bf16((it.nvalid + 15) & ~15);
                 const int acc = li & 1;
                 const uint32_t use = (uint32_t)(li >> 1);
                 if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag, p.status, true)) break;
                 tc_fence_after();
-                const uint32_t d = tmem_base + (uint32_t)(acc * p.BN);
+                const uint32_t d = tmem_base + (uint32_t)(acc * p.BN), d1 = d + (uint32_t)(p.BN >> 1);
                 bool ok = true;
                 for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
                     const int nsub = min(sh.ns, sh.nk - k0);
@@ -601,11 +707,21 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     }
                     tc_fence_after();
                     for (int j = 0; j < nsub; ++j) {
-                        const uint32_t sA = smem_u32(ring + (size_t)(first + j * sh.sub_pages) * kPageBytes);
-                        const uint64_t da = sw128_desc(sA), db = sw128_desc(sA + kABytes);
+                        // descriptor start addresses count 16-byte units
+                        const uint64_t da = desc0 + (first + j * sh.sub_pages) * (kPageBytes / 16);
+                        if (it.m == 1) {
+                            const uint64_t db = da + kABytes / 16;
 #pragma unroll
-                        for (int kk = 0; kk < kBlockK / 16; ++kk)  // +32 bytes per K16 step
-                            umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (k0 | j | kk) != 0);
+                            for (int kk = 0; kk < kBlockK / 16; ++kk)  // +32 bytes per K16 step
+                                umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (k0 | j | kk) != 0);
+                        } else {  // weight tile 1 -> accumulator columns BN/2 ..
+                            const uint64_t db = da + 2 * kABytes / 16;
+#pragma unroll
+                            for (int kk = 0; kk < kBlockK / 16; ++kk) {
+                                umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (k0 | j | kk) != 0);
+                                umma_bf16(d1, da + kABytes / 16 + 2 * kk, db + 2 * kk, idesc, (k0 | j | kk) != 0);
+                            }
+                        }
                     }
                     umma_commit(&empty[tk]);
                     ++step;
@@ -623,26 +739,32 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         for (int li = 0;; ++li) {
             const int acc = li & 1;
             const uint32_t use = (uint32_t)(li >> 1);
-            if (elected) {  // one thread takes the item and waits for its accumulator
-                int item = -2;
+            if (elected) {  // one thread takes the item; its accumulator is awaited below
                 const int slot = li % kQueue;
                 if (mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) {
-                    item = qitem[slot];
+                    *epi_desc = qdesc[slot];
                     mbar_arrive(&qempty[slot]);
-                    if (item >= 0 && !mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true)) item = -2;
+                } else {
+                    epi_desc->item = -2;
                 }
-                *epi_item = item;
             }
             named_bar_sync(1, 128);
-            const int item = *epi_item;
-            if (item < 0) break;
-            const Item it = decode_item(item, sc, p);
+            if (epi_desc->item < 0) break;
+            const Item it = epi_desc->it;
+            // down items: destination row and weight of token `lane`, loaded while the
+            // item's MMAs still run
+            int mrow0 = 0;
+            float mw0 = 0.f;
+            if (it.ph == 1) down_dest(it, lane, p, mrow0, mw0);
+            if (elected) *epi_flag = mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 0 : -1;
+            named_bar_sync(1, 128);
+            if (*epi_flag) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + (uint32_t)(acc * p.BN) + ((uint32_t)(q * 32) << 16);
             for (int c0 = 0; c0 < it.nvalid; c0 += 32) {
-                float v[32];
-                tmem_ld32(tbase + (uint32_t)c0, v);
                 if (it.ph == 0) {
+                    float v[32];
+                    tmem_ld32(tbase + (uint32_t)c0, v);
                     if (q < 2) {  // gate rows 0..63: silu(g) to the exchange buffer
                         float *xr = xchg + (q * 32 + lane) * kXchgStride;
 #pragma unroll
@@ -662,35 +784,30 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     named_bar_sync(1, 128);
                 } else {
                     // per-token destination row of ybuf and weight, token c0 + lane
-                    int mrow = 0;
-                    float mw = 0.f;
-                    const int n = c0 + lane;
-                    if (n < it.nvalid) {
-                        if (it.shared) {
-                            const int t = it.row0 + n;
-                            mrow = t * (p.k + 1) + p.k;
-                            mw = __ldg(p.sgate + t);
-                        } else {
-                            const int slot = __ldg(p.perm + it.row0 + n);
-                            mrow = slot + slot / p.k;  // t*(k+1) + j
-                            mw = __ldg(p.topk_w + slot);
-                        }
-                    }
-                    uint16_t *out = p.ybuf + it.r * kTileM + q * 32 + lane;
+                    int mrow = mrow0;
+                    float mw = mw0;
+                    if (c0 > 0) down_dest(it, c0 + lane, p, mrow, mw);
+                    for (int t = 0; t < it.m; ++t) {  // weight tile r + t: accumulator columns t * BN/2
+                        float v[32];
+                        tmem_ld32(tbase + (uint32_t)(t * (p.BN >> 1) + c0), v);
+                        uint16_t *out = p.ybuf + (it.r + t) * kTileM + q * 32 + lane;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int rr = __shfl_sync(0xffffffffu, mrow, i);
-                        const float ww = __shfl_sync(0xffffffffu, mw, i);
-                        if (c0 + i < it.nvalid) out[(size_t)rr * p.H] = f32_to_bf16_bits(v[i] * ww);
+                        for (int i = 0; i < 32; ++i) {
+                            const int rr = __shfl_sync(0xffffffffu, mrow, i);
+                            const float ww = __shfl_sync(0xffffffffu, mw, i);
+                            if (c0 + i < it.nvalid) out[(size_t)rr * p.H] = f32_to_bf16_bits(v[i] * ww);
+                        }
                     }
                 }
             }
             tc_fence_before();
-            if (fused && it.ph == 0) __threadfence();  // h rows visible before the group counter moves
             named_bar_sync(1, 128);
             if (elected) {
                 mbar_arrive(&tempty[acc]);
                 if (fused && it.ph == 0) {
+                    // the CTA's h rows (ordered before this by the barrier) become visible
+                    // device-wide before the group counter moves
+                    __threadfence();
                     atomicAdd(p.hdone + (it.shared ? p.E : it.e), 1);
                     atomicAdd(p.hdone + p.E + 1, 1);
                 }
@@ -763,8 +880,9 @@ int pick_bns(const FfnArgs &a, int bn, int sms) {
 }
 
 size_t smem_bytes_for(int E, int pages) {
-    return 1024 + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 + 2 * (size_t)(E + 1) * 4 + 8 +
-           (size_t)(2 * kTickets + 5 + 2 * kQueue) * 8 + 32 + kThreads * 4 + kReadyWords * 4 + kTickets * 4;
+    return 1024 + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 + 3 * (size_t)(E + 1) * 4 + 8 +
+           (size_t)(2 * kTickets + 5 + 2 * kQueue) * 8 + 16 + (kQueue + 1) * sizeof(ItemSlot) + 8 + 2 * kThreads * 4 +
+           kReadyWords * 4 + kTickets * 4;
 }
 
 int pick_pages(int E) {

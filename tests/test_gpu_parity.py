@@ -61,6 +61,33 @@ def test_small_layers(cfg):
     print(cfg.label, diag)
 
 
+# Enough down items (>= 8 per SM) that small groups take two weight tiles per
+# down item; H = 1920 gives an odd number of 128-row output tiles (a last
+# item with one tile), and T = 96 lets the shared expert's down items pair up.
+MERGED = [
+    W.MoEConfig("merged_odd_tiles", T=256, H=1920, E=128, I=128, k=4, Is=128, zipf_alpha=0.5),
+    W.MoEConfig("merged_shared", T=96, H=1920, E=128, I=128, k=4, Is=128),
+]
+
+
+@pytest.mark.parametrize("cfg", MERGED, ids=lambda c: c.name)
+def test_merged_down_items(cfg):
+    diag, g, _ = _run(cfg)
+    print(cfg.label, diag)
+
+
+@pytest.mark.parametrize("bn", [32, 64])
+def test_merged_down_items_bits(bn, monkeypatch):
+    """Narrower token tiles pair fewer groups (only those of <= BN/2 tokens); the
+    output bits do not move."""
+    cfg = MERGED[0]
+    inp = W.make_inputs(cfg, device="cuda")
+    ref = gpu_forward(cfg, inp)
+    monkeypatch.setenv("MOE_FORCE_BN", str(bn))
+    got = gpu_forward(cfg, inp)
+    assert (got.out_bits == ref.out_bits).all()
+
+
 def test_hot_expert_multi_tile():
     """Every token routes to expert 3 first: one group of T rows, several token tiles."""
     cfg = W.MoEConfig("hot", T=600, H=256, E=8, I=128, k=2, Is=64)
