@@ -3,7 +3,10 @@
 // N, keeping the experts with the highest aggregate gate weight, dropping
 // the rest from every token and renormalising what survives.
 //
-// Kernel 1 (one block per chunk of kChunk tokens): thread e sums, in token
+// Batches of up to kSmallSlots slots: one block does all of it in shared
+// memory (budget_block, front.cuh), the aggregates summed in exactly
+// token-then-slot order.  Larger batches take two kernels:
+// kernel 1 (one block per chunk of kChunk tokens): thread e sums, in token
 // then slot order, the weights routed to expert e inside the chunk, and
 // counts the slots; chunk partials go to the workspace.
 // Kernel 2 (one block): agg[e] = chunk partials summed in chunk order, the
@@ -11,15 +14,59 @@
 // number of union experts ahead of it in (agg descending, id ascending),
 // the first N are kept; then one thread per token compacts its slots in
 // order and renormalises when it lost one.
-// Both kernels are deterministic: every sum has a fixed order.  For T up to
-// kChunk tokens the aggregate is summed in exactly token-then-slot order.
-#include "moe_internal.cuh"
+// Every sum has a fixed order, so the result is deterministic; the
+// two-kernel path rounds the aggregates chunk by chunk.
+#include <atomic>
+
+#include "front.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kChunk = 256;  // tokens per partial-sum chunk
+constexpr int kChunk = 256;        // tokens per partial-sum chunk
+constexpr int kSmallSlots = 8192;  // T*k up to this: one block in shared memory
+
+// Shared memory of budget_small_kernel.
+size_t budget_small_smem(int T, int E, int k) {
+    const size_t Tk = (size_t)T * k;
+    return Tk * 12 + (size_t)T * 4 + (size_t)sort_warps(E) * E * 4 + (size_t)(E + 1) * 4 + (size_t)E * 6 + 16;
+}
+
+__global__ void __launch_bounds__(1024) budget_small_kernel(int T, int E, int k, int N, int norm_topk,
+                                                            int32_t *__restrict__ idx, float *__restrict__ w,
+                                                            int32_t *__restrict__ keff, uint8_t *__restrict__ kept,
+                                                            int32_t *__restrict__ n_dropped) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int Tk = T * k, W = sort_warps(E);
+    int32_t *idx_s = reinterpret_cast<int32_t *>(sm);
+    float *w_s = reinterpret_cast<float *>(idx_s + Tk);
+    int *sorted = reinterpret_cast<int *>(w_s + Tk);
+    int32_t *keff_s = sorted + Tk;
+    int *hist = keff_s + T;
+    int *off = hist + W * E;
+    float *agg = reinterpret_cast<float *>(off + E + 1);
+    uint8_t *pres = reinterpret_cast<uint8_t *>(agg + E);
+    uint8_t *keep = pres + E;
+    __shared__ int warp_sums[32];
+    __shared__ int nu_s, nd_s;
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int s = threadIdx.x; s < Tk; s += blockDim.x) {
+        idx_s[s] = idx[s];
+        w_s[s] = w[s];
+    }
+    __syncthreads();
+    budget_block(T, E, k, N, norm_topk, idx_s, w_s, keff_s, keep, &nd_s, hist, off, sorted, agg, pres, warp_sums,
+                 &nu_s);
+    for (int s = threadIdx.x; s < Tk; s += blockDim.x) {
+        idx[s] = idx_s[s];
+        w[s] = w_s[s];
+    }
+    for (int t = threadIdx.x; t < T; t += blockDim.x) keff[t] = keff_s[t];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) kept[e] = keep[e];
+    if (threadIdx.x == 0) *n_dropped = nd_s;
+}
 
 __global__ void __launch_bounds__(256) budget_partial_kernel(int T, int E, int k, const int32_t *__restrict__ idx,
                                                              const float *__restrict__ w,
@@ -126,6 +173,19 @@ int budget_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 cudaError_t launch_budget(int T, int E, int k, int N, int norm_topk, int32_t *idx, float *w, int32_t *keff,
                           uint8_t *kept, int32_t *n_dropped, float *part_agg, int32_t *part_cnt,
                           cudaStream_t st) {
+    if ((long long)T * k <= kSmallSlots) {
+        static std::atomic<int> attr_set[64];  // per device: opted in to more than 48 KB
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if (!attr_set[dev].load(std::memory_order_acquire)) {
+            const cudaError_t e = cudaFuncSetAttribute(budget_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)budget_small_smem(kSmallSlots, kMaxExperts, 1));
+            if (e != cudaSuccess) return e;
+            attr_set[dev].store(1, std::memory_order_release);
+        }
+        return launch_pdl(budget_small_kernel, dim3(1), dim3(1024), budget_small_smem(T, E, k), st, T, E, k, N,
+                          norm_topk, idx, w, keff, kept, n_dropped);
+    }
     const int nchunks = budget_chunks(T);
     cudaError_t e = launch_pdl(budget_partial_kernel, dim3(nchunks), dim3(256), 0, st, T, E, k, idx, w, part_agg,
                                part_cnt);

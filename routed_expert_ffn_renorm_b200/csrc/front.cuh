@@ -1,0 +1,361 @@
+// Device building blocks of the layer's front end -- routing, the shared
+// expert's gate, the stable sort of slots by expert and the expert budget --
+// shared by the stand-alone stage kernels (router.cu, budget.cu) and the
+// fused small-batch front-end kernel (front.cu), so that every path
+// computes the same bits.
+#pragma once
+
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------- routing --
+// Softmax over the E logits of a token, top-k by logit with the kept
+// probabilities renormalised (SpecForge PR #943, "Modifications": softmax
+// router with renormalised top-k).  One warp per token: lane l holds the
+// logits of experts l, l+32, ... (coalesced loads).  Each of the k selection
+// rounds takes a lane-local best and a 5-step shuffle argmax ordered by
+// (logit descending, expert id ascending), so equal logits keep the lower
+// id; the winner's owner lane masks it out.  The logits come from global
+// memory (kGlobal, read-only path) or from shared memory; idx / w may point
+// to global or shared memory; keff (may be null) receives k.
+__device__ __forceinline__ bool route_better(float va, int ia, float vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+template <int V, bool kGlobal = true>  // logits per lane: V * 32 >= E
+__device__ __forceinline__ void route_token(int t, int E, int k, int norm_topk, const float *__restrict__ logits,
+                                            int32_t *idx, float *w, int32_t *keff, int lane) {
+    const float *l = logits + (size_t)t * E;
+    float v[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? (kGlobal ? __ldg(l + e) : l[e]) : -INFINITY;
+    }
+    // softmax denominator: max, then sum of exp(l - max) over all E
+    float m = v[0];
+#pragma unroll
+    for (int i = 1; i < V; ++i) m = fmaxf(m, v[i]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+        if (lane + 32 * i < E) s += expf(v[i] - m);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+
+    // k selection rounds; lane j keeps the j-th winner
+    uint32_t taken = 0;
+    int my_idx = -1;
+    float my_logit = -INFINITY;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u) && route_better(v[i], e, bv, bi)) {
+                bv = v[i];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (route_better(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == j) {
+            my_idx = bi;
+            my_logit = bv;
+        }
+    }
+    // probabilities of the kept experts; renormalise with the sum taken in
+    // slot order
+    float p = (lane < k) ? expf(my_logit - m) / s : 0.f;
+    if (norm_topk) {
+        float ps = 0.f;
+        for (int j = 0; j < k; ++j) ps += __shfl_sync(0xffffffffu, p, j);
+        p = p / ps;
+    }
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = my_idx;
+        w[(size_t)t * k + lane] = p;
+    }
+    if (keff != nullptr && lane == 0) keff[t] = k;
+}
+
+// One token per thread, for E <= kLaneRouteMaxE: the same decisions as
+// route_token, with every sum taken in expert order (max, then
+// sum_e exp(l_e - max), then k rounds of first-maximum selection over the
+// untaken experts, then the renormalising sum in slot order).  A warp routes
+// 32 tokens at once with no shuffles.  `l` is the token's row of logits
+// (global memory when kGlobal, else shared memory).
+constexpr int kLaneRouteMaxE = 64;
+
+template <bool kGlobal>
+__device__ __forceinline__ void route_token_lane(int t, int E, int k, int norm_topk, const float *l, int32_t *idx,
+                                                 float *w) {
+    auto L = [&](int e) { return kGlobal ? __ldg(l + e) : l[e]; };
+    float m = L(0);
+    for (int e = 1; e < E; ++e) {
+        const float v = L(e);
+        if (v > m) m = v;
+    }
+    float s = 0.f;
+    for (int e = 0; e < E; ++e) s += expf(L(e) - m);
+    uint64_t taken = 0;
+    float ps = 0.f;
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        float bv = 0.f;
+        for (int e = 0; e < E; ++e) {
+            if ((taken >> e) & 1ull) continue;
+            const float v = L(e);
+            if (best < 0 || v > bv) {  // strict: equal logits keep the lower id
+                best = e;
+                bv = v;
+            }
+        }
+        taken |= 1ull << best;
+        const float p = expf(bv - m) / s;
+        idx[(size_t)t * k + j] = best;
+        w[(size_t)t * k + j] = p;
+        ps += p;
+    }
+    if (norm_topk)
+        for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = w[(size_t)t * k + j] / ps;
+}
+
+// ------------------------------------------------------------ shared gate --
+// sigmoid(g . x_t) (SpecForge PR #943, "Modifications": sigmoid-gated
+// shared expert), computed by a group of kGateThreads threads: each loads up
+// to kGateVec 16-byte slices of x_t and of g, all in flight at once, then a
+// warp reduction and the kGateThreads / 32 warp partials in order.  `tid`
+// is the thread's index in the group, `part` the group's kGateThreads / 32
+// floats of shared memory, `bar` a named barrier id the group owns.  The
+// result is valid in group thread 0.
+constexpr int kGateThreads = 128;
+constexpr int kGateVec = 8;
+
+__device__ __forceinline__ float shared_gate_group(int t, const uint16_t *__restrict__ x,
+                                                   const uint16_t *__restrict__ gvec, int H, float *part, int bar,
+                                                   int tid) {
+    const int lane = tid & 31, wid = tid >> 5;
+    const int nv = H / 8;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+    const uint4 *gr = reinterpret_cast<const uint4 *>(gvec);
+    float z = 0.f;
+    for (int c0 = tid; c0 < nv; c0 += kGateThreads * kGateVec) {
+        uint4 a[kGateVec], g[kGateVec];
+#pragma unroll
+        for (int q = 0; q < kGateVec; ++q) {
+            const int c = c0 + q * kGateThreads;
+            a[q] = c < nv ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+            g[q] = c < nv ? __ldg(gr + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int q = 0; q < kGateVec; ++q) {
+            const uint32_t av[4] = {a[q].x, a[q].y, a[q].z, a[q].w}, bv[4] = {g[q].x, g[q].y, g[q].z, g[q].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                z = fmaf(bf16_bits_to_f32((uint16_t)(av[h] & 0xffffu)), bf16_bits_to_f32((uint16_t)(bv[h] & 0xffffu)),
+                         z);
+                z = fmaf(bf16_bits_to_f32((uint16_t)(av[h] >> 16)), bf16_bits_to_f32((uint16_t)(bv[h] >> 16)), z);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if (lane == 0) part[wid] = z;
+    asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(kGateThreads) : "memory");
+    float r = 0.f;
+    if (tid == 0) {
+        float zz = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kGateThreads / 32; ++w2) zz += part[w2];
+        r = 1.f / (1.f + expf(-zz));
+    }
+    asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(kGateThreads) : "memory");  // part reusable afterwards
+    return r;
+}
+
+// ------------------------------------------------- block sort by expert --
+// Exclusive prefix sum of one value per thread over a 1024-thread block.
+__device__ __forceinline__ int block_exclusive_scan_1024(int v, int *warp_sums) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int ws = warp_sums[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, ws, off);
+            if (lane >= off) ws += o;
+        }
+        warp_sums[lane] = ws;  // inclusive over warps
+    }
+    __syncthreads();
+    const int r = incl - v + (wid ? warp_sums[wid - 1] : 0);
+    __syncthreads();  // warp_sums reusable afterwards
+    return r;
+}
+
+// Per-warp count columns for a block sort over E experts: [W][E] ints fit in 32 KB.
+__host__ __device__ inline int sort_warps(int E) { return E <= 256 ? 32 : (E <= 512 ? 16 : 8); }
+
+// Stable counting sort of the slots 0..n-1 by expert inside one 1024-thread
+// block: key(s) is the slot's expert in [0, E), or -1 to leave it out.  W
+// warps each take a contiguous chunk of slots; __match_any_sync groups the
+// lanes with the same expert, and a lane's position inside its group is the
+// number of lower lanes, so the order inside an expert is ascending slot id.
+// Out (shared memory): sorted[pos] = slot, off[e] = first position of expert
+// e, off[E] = number of sorted slots.  hist: W * E ints; warp_sums: 32 ints.
+template <class Key>
+__device__ __forceinline__ void block_sort_by_expert(int n, int E, int W, Key key, int *hist, int *off, int *sorted,
+                                                     int *warp_sums) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = (n + W - 1) / W;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int s_begin = warp * chunk, s_end = min(n, s_begin + chunk);
+    if (warp < W) {
+        for (int s0 = s_begin; s0 < s_end; s0 += 32) {
+            const int s = s0 + lane;
+            const int kk = s < s_end ? key(s) : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, kk);
+            if (kk >= 0 && lane == __ffs(peers) - 1) hist[warp * E + kk] += __popc(peers);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    const int e = threadIdx.x;  // blockDim.x == 1024 >= E
+    int c = 0;
+    if (e < E)
+        for (int w = 0; w < W; ++w) c += hist[w * E + e];
+    const int excl = block_exclusive_scan_1024(c, warp_sums);
+    if (e < E) {
+        off[e] = excl;
+        if (e == E - 1) off[E] = excl + c;
+        int run = excl;
+        for (int w = 0; w < W; ++w) {
+            const int hw = hist[w * E + e];
+            hist[w * E + e] = run;
+            run += hw;
+        }
+    }
+    __syncthreads();
+    if (warp < W) {
+        int *base = hist + warp * E;
+        for (int s0 = s_begin; s0 < s_end; s0 += 32) {
+            const int s = s0 + lane;
+            const int kk = s < s_end ? key(s) : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, kk);
+            if (kk >= 0) sorted[base[kk] + __popc(peers & ((1u << lane) - 1u))] = s;
+            __syncwarp();
+            if (kk >= 0 && lane == 31 - __clz(peers)) base[kk] += __popc(peers);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------- budget --
+// Expert budget (colibri issue_budget.md, "EXPERT_BUDGET", section "How it
+// works", steps 1-5) inside one 1024-thread block, on a routing held in
+// shared memory (idx_s, w_s: T * k slots, every slot valid).
+//   step 1: agg[e] = the weights routed to e summed in token-then-slot order
+//           (the slots are sorted by expert first, so each expert's thread
+//           sums exactly that sequence);
+//   step 2-3: the union is every expert with a slot; each union expert's
+//           rank is the number of union experts ahead of it in (agg
+//           descending, id ascending); the first N are kept;
+//   step 4: each token's kept slots move to the front in order, the others
+//           become (-1, 0); a token that lost some but not all renormalises;
+//   step 5: n_dropped = union size - N.
+// A budget of 0, or a union of at most N experts, changes nothing (keff = k,
+// kept = the union).  Out (shared memory): idx_s / w_s compacted, keff_s[T],
+// keep[E], *nd_s.  Scratch: hist (W * E), off (E + 1), sorted (T * k), agg
+// (E), pres (E), warp_sums (32), nu_s.
+__device__ __forceinline__ void budget_block(int T, int E, int k, int N, int norm_topk, int32_t *idx_s, float *w_s,
+                                             int32_t *keff_s, uint8_t *keep, int *nd_s, int *hist, int *off,
+                                             int *sorted, float *agg, uint8_t *pres, int *warp_sums, int *nu_s) {
+    const int Tk = T * k;
+    if (threadIdx.x == 0) *nu_s = 0;
+    block_sort_by_expert(
+        Tk, E, sort_warps(E),
+        [=](int s) {
+            const int x = idx_s[s];
+            return (x >= 0 && x < E) ? x : -1;
+        },
+        hist, off, sorted, warp_sums);
+    const int e = threadIdx.x;
+    int my_present = 0;
+    if (e < E) {
+        float a = 0.f;
+        for (int p = off[e]; p < off[e + 1]; ++p) a += w_s[sorted[p]];
+        agg[e] = a;
+        pres[e] = off[e + 1] > off[e];
+        my_present = pres[e];
+    }
+    if (my_present) atomicAdd(nu_s, 1);  // integer: order-independent
+    __syncthreads();
+    const int nu = *nu_s;
+    const bool active = N > 0 && nu > N;
+    if (e < E) {
+        uint8_t kp = pres[e];
+        if (active && kp) {
+            const float a = agg[e];
+            int rank = 0;
+            for (int o = 0; o < E; ++o) rank += pres[o] && (agg[o] > a || (agg[o] == a && o < e));
+            kp = rank < N;
+        }
+        keep[e] = kp;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+        int32_t *ti = idx_s + (size_t)t * k;
+        float *tw = w_s + (size_t)t * k;
+        int c = k;
+        if (active) {
+            c = 0;
+            for (int j = 0; j < k; ++j) {
+                const int ej = ti[j];
+                if (ej >= 0 && ej < E && keep[ej]) {
+                    const float wj = tw[j];
+                    ti[c] = ej;
+                    tw[c] = wj;
+                    ++c;
+                }
+            }
+            for (int j = c; j < k; ++j) {
+                ti[j] = -1;
+                tw[j] = 0.f;
+            }
+            if (norm_topk && c > 0 && c < k) {
+                float s = 0.f;
+                for (int j = 0; j < c; ++j) s += tw[j];
+                for (int j = 0; j < c; ++j) tw[j] = tw[j] / s;
+            }
+        }
+        keff_s[t] = c;
+    }
+    if (threadIdx.x == 0) *nd_s = active ? nu - N : 0;
+    __syncthreads();
+}
+
+}  // namespace moe

@@ -74,6 +74,18 @@ cudaError_t launch_gather_rows(int T, int k, int H, const int32_t *offsets, int 
                                const int32_t *perm, const uint16_t *x, uint16_t *x_perm,
                                cudaStream_t st);
 
+// Fused small-batch front end: route -> budget (N > 0) -> dispatch -> row
+// gather + shared gate in one launch, for T*k <= kFrontMaxSlots and
+// T*E <= kFrontMaxLogits.  Same outputs, bit for bit, as launch_route,
+// launch_budget and launch_dispatch in sequence.
+constexpr int kFrontMaxSlots = 8192;
+constexpr int kFrontMaxLogits = 16384;
+bool front_fits(int T, int E, int k);
+cudaError_t launch_front(int T, int E, int k, int N, int norm_topk, int H, const float *logits, const uint16_t *x,
+                         const uint16_t *gvec, int32_t *idx, float *w, float *sgate, int32_t *keff, uint8_t *kept,
+                         int32_t *n_dropped, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
+                         uint16_t *x_perm, int32_t *status_block, int32_t *hdone, cudaStream_t st);
+
 // Combine.
 cudaError_t launch_combine(int T, int k, int H, int has_shared, const uint16_t *ybuf,
                            const int32_t *keff, uint16_t *out, cudaStream_t st);

@@ -159,10 +159,24 @@ def test_force_overrides_reject_bad_values(env, monkeypatch):
         gpu_forward(cfg, inp)
 
 
-def test_stagewise_entry_points():
+# moe_forward takes the fused front-end launch when a budget is set, T*k <= 8192
+# and T*E <= 16384, the separate route / budget / dispatch launches otherwise;
+# both must match the stage entry points bit for bit.
+STAGEWISE = [
+    W.MoEConfig("stages", T=96, H=256, E=16, I=128, k=4, Is=64, budget=6, zipf_alpha=1.0),  # front
+    W.MoEConfig("stages_nobudget", T=200, H=256, E=32, I=64, k=3, Is=64),  # separate
+    W.MoEConfig("stages_budget_idle", T=40, H=128, E=16, I=64, k=2, budget=16),  # front, union <= N
+    W.MoEConfig("stages_no_norm", T=64, H=128, E=64, I=64, k=6, budget=5, norm_topk=False, zipf_alpha=0.8),  # front
+    W.MoEConfig("stages_e1024", T=16, H=128, E=1024, I=64, k=8, budget=20),  # front, largest E
+    W.MoEConfig("stages_slots_max", T=1024, H=128, E=16, I=64, k=8, Is=64, budget=9),  # front, T*k = 8192
+    W.MoEConfig("stages_big_logits", T=700, H=128, E=64, I=64, k=6, budget=9, zipf_alpha=0.5),  # separate
+]
+
+
+@pytest.mark.parametrize("cfg", STAGEWISE, ids=lambda c: c.name)
+def test_stagewise_entry_points(cfg):
     """route -> budget -> dispatch -> expert_ffn -> combine called one by one
-    equals moe_forward bit for bit."""
-    cfg = W.MoEConfig("stages", T=96, H=256, E=16, I=128, k=4, Is=64, budget=6, zipf_alpha=1.0)
+    equals moe_forward bit for bit, every auxiliary output included."""
     inp = W.make_inputs(cfg, device="cuda")
     ref = gpu_forward(cfg, inp)
     c = lib_config(cfg)
@@ -171,10 +185,10 @@ def test_stagewise_entry_points():
     ws = torch.zeros(moe.workspace_bytes(c, T), dtype=torch.uint8, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    sgate = torch.empty(T, dtype=torch.float32, device=dev)
+    sgate = torch.empty(T, dtype=torch.float32, device=dev) if cfg.Is else None
     keff = torch.empty(T, dtype=torch.int32, device=dev)
-    kept = torch.empty(E, dtype=torch.uint8, device=dev)
-    nd = torch.empty(1, dtype=torch.int32, device=dev)
+    kept = torch.zeros(E, dtype=torch.uint8, device=dev)
+    nd = torch.zeros(1, dtype=torch.int32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(T * k, dtype=torch.int32, device=dev)
@@ -182,20 +196,45 @@ def test_stagewise_entry_points():
     x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
     ybuf = torch.empty((T, k + 1, H), dtype=torch.bfloat16, device=dev)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    moe.moe_route(c, inp.logits, idx, w, x=inp.x, ws_gate_vec=inp.ws_gvec, sgate=sgate, keff=keff)
-    moe.moe_budget(c, idx, w, keff, kept, nd, ws)
+    moe.moe_route(c, inp.logits, idx, w, x=inp.x if cfg.Is else None, ws_gate_vec=inp.ws_gvec if cfg.Is else None,
+                  sgate=sgate, keff=keff)
+    if cfg.budget:
+        moe.moe_budget(c, idx, w, keff, kept, nd, ws)
     moe.moe_dispatch(c, idx, counts, offsets, perm, slot_pos, ws, keff=keff, x=inp.x, x_perm=x_perm)
     moe.moe_expert_ffn(c, inp.x, x_perm, offsets, perm, w, weights_of(inp), ybuf, ws, sgate=sgate)
     moe.moe_combine(c, ybuf, out, keff=keff)
     torch.cuda.synchronize()
     assert moe.status_read(ws) == 0
-    assert (W.bf16_bits(out) == ref.out_bits).all()
+    assert (idx.cpu().numpy() == ref.idx).all()
+    assert (w.cpu().numpy().view(np.uint32) == ref.w.view(np.uint32)).all()
+    assert (keff.cpu().numpy() == ref.keff).all()
+    if cfg.budget:
+        assert (kept.cpu().numpy() == ref.kept).all() and int(nd.item()) == ref.n_dropped
+    if cfg.Is:
+        assert (sgate.cpu().numpy().view(np.uint32) == ref.sgate.view(np.uint32)).all()
+    assert (counts.cpu().numpy() == ref.counts).all() and (offsets.cpu().numpy() == ref.offsets).all()
     total = int(offsets[E])
     assert (perm[:total].cpu().numpy() == ref.perm).all()
+    assert (slot_pos.cpu().numpy() == ref.slot_pos).all()
+    assert (W.bf16_bits(out) == ref.out_bits).all()
     # x_perm rows are exact copies of the routed tokens
     xp = x_perm[:total].cpu()
     src = inp.x.cpu()[perm[:total].cpu().long() // k]
     assert torch.equal(xp, src)
+
+
+def test_budget_is_exact_sequential_sum():
+    """Up to 8192 slots the budget sums each expert's weights in exactly token-then-slot
+    order, so the kept set equals the oracle's with no near-tie allowance."""
+    import oracle
+    for cfg in (W.MoEConfig("bex", T=700, H=128, E=64, I=64, k=6, budget=9, zipf_alpha=0.5),
+                W.MoEConfig("bex2", T=1000, H=128, E=128, I=64, k=8, budget=40, zipf_alpha=0.3)):
+        inp = W.make_inputs(cfg, device="cuda")
+        g = gpu_forward(cfg, inp)
+        idx_o, w_o = oracle.route(inp.logits.cpu().numpy(), cfg.k, cfg.norm_topk)
+        idx_b, w_b, keff_b, kept_b, nd_b = oracle.budget(idx_o, w_o, cfg.E, cfg.budget, cfg.norm_topk)
+        assert (g.kept == kept_b).all() and g.n_dropped == nd_b
+        assert (g.idx == idx_b).all() and (g.keff == keff_b).all()
 
 
 def test_zero_tokens_is_noop():
