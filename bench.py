@@ -94,12 +94,22 @@ def stage_work(cfg, counts):
                 layer=layer, touched=touched, slots=slots)
 
 
-def launches_per_step(cfg) -> int:
-    # route 1; budget 2; dispatch: one sort+gather launch when T*k <= 8192,
-    # else histogram + scan + scatter + gather; expert FFN 1 (fused) or 2
-    # (mean group >= 128 tokens); combine 1
-    ffn = 1 if (cfg.T * cfg.k + cfg.E - 1) // cfg.E < 128 else 2
-    return 1 + (2 if cfg.budget else 0) + (1 if cfg.T * cfg.k <= 8192 else 4) + ffn + 1
+def launches_forward(cfg) -> int:
+    """Our kernel launches in one moe_forward call."""
+    Tk = cfg.T * cfg.k
+    ffn = 1 if (Tk + cfg.E - 1) // cfg.E < 128 else 2  # fused, or gate/up + down once the mean group >= 128
+    if cfg.budget and Tk <= 8192 and cfg.T * cfg.E <= 16384:
+        return 1 + ffn + 1  # fused front end (route + budget + dispatch + gather), FFN, combine
+    return launches_stages(cfg)
+
+
+def launches_stages(cfg) -> int:
+    """Our kernel launches of the stage entry points called one by one."""
+    Tk = cfg.T * cfg.k
+    ffn = 1 if (Tk + cfg.E - 1) // cfg.E < 128 else 2
+    budget = (1 if Tk <= 8192 else 2) if cfg.budget else 0  # one block, or partial sums + select
+    dispatch = 1 if Tk <= 8192 else 4  # sort + gather, or histogram + scan + scatter + gather
+    return 1 + budget + dispatch + ffn + 1
 
 
 def load_peaks():
@@ -539,7 +549,7 @@ def run_ours(args, cfg):
         "router logits + Zipf popularity bias",
         "config": {**workload_desc(cfg), "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": rl, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": 2 * launches_per_step(cfg) * args.steps,
+        "gpu_launches": (launches_forward(cfg) + launches_stages(cfg)) * args.steps,
         "clocks": sampler.summary(),
         "stages_ms": per_stage,
         "layer": {"touched_experts": work["touched"], "kept_slots": work["slots"],

@@ -3,11 +3,11 @@
 // softmax router with renormalised top-k), plus the sigmoid gate of the
 // shared expert.
 //
-// One block per token: its four warps compute the shared-expert gate
-// (shared_gate_group, front.cuh) and the routing is done by its first warp
-// (route_token), or, for E <= 64, by the first warp of every 32nd block, one
-// token per lane (route_token_lane).  The kernel reads the logits (and x)
-// once; it is latency-bound and small next to the expert FFN.
+// route_kernel<V>: one block per token; its first warp routes (route_token,
+// front.cuh) and its four warps compute the shared-expert gate
+// (shared_gate_group).  route_lane_kernel (E <= 64): separate blocks route
+// 32 tokens lane by lane and compute the gates.  Both read the logits (and
+// x) once; they are latency-bound and small next to the expert FFN.
 #include "front.cuh"
 
 namespace moe {
@@ -35,9 +35,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int 
     if (threadIdx.x == 0) sgate[t] = g;
 }
 
-// E <= kLaneRouteMaxE: block b routes tokens b .. b+31 lane by lane when b is a
-// multiple of 32 (route_token_lane), and every block computes its token's
-// shared gate.
+// E <= kLaneRouteMaxE: the first ceil(T / 32) blocks route 32 tokens each, one
+// token per lane of their first warp (route_token_lane), from the tokens'
+// logits staged in shared memory; the remaining T blocks (with a shared
+// expert) compute one token's shared gate each.  Routing and gate blocks run
+// side by side instead of one after the other.
 __global__ void __launch_bounds__(kRouteThreads) route_lane_kernel(int T, int E, int k, int norm_topk,
                                                                    const float *__restrict__ logits,
                                                                    int32_t *__restrict__ idx, float *__restrict__ w,
@@ -46,17 +48,25 @@ __global__ void __launch_bounds__(kRouteThreads) route_lane_kernel(int T, int E,
                                                                    const uint16_t *__restrict__ gvec, int H,
                                                                    float *__restrict__ sgate) {
     __shared__ float part[kGateThreads / 32];
+    __shared__ float lg[32 * (kLaneRouteMaxE + 1)];  // 32 rows of logits, odd stride: no bank conflicts
     pdl_launch_dependents();
     pdl_wait();
-    if ((blockIdx.x & 31) == 0 && threadIdx.x < 32) {
-        const int t = blockIdx.x + threadIdx.x;
-        if (t < T) {
-            route_token_lane<true>(t, E, k, norm_topk, logits + (size_t)t * E, idx, w);
-            if (keff != nullptr) keff[t] = k;
+    const int nrt = (T + 31) / 32;  // routing blocks
+    if ((int)blockIdx.x < nrt) {
+        if (threadIdx.x >= 32) return;
+        const int lane = threadIdx.x, t0 = blockIdx.x * 32, n = min(32, T - t0), ls = E | 1;
+        for (int i = lane; i < n * E; i += 32) {  // coalesced copy of the 32 tokens' rows
+            const int r = i / E;
+            lg[r * ls + (i - r * E)] = __ldg(logits + (size_t)t0 * E + i);
         }
+        __syncwarp();
+        if (lane < n) {
+            route_token_lane<false>(t0 + lane, E, k, norm_topk, lg + lane * ls, idx, w);
+            if (keff != nullptr) keff[t0 + lane] = k;
+        }
+        return;
     }
-    if (sgate == nullptr) return;
-    const int t = blockIdx.x;
+    const int t = blockIdx.x - nrt;
     const float g = shared_gate_group(t, x, gvec, H, part, 1, threadIdx.x);
     if (threadIdx.x == 0) sgate[t] = g;
 }
@@ -75,8 +85,8 @@ cudaError_t launch_route(int T, int E, int k, int norm_topk, const float *logits
                          int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
                          cudaStream_t st) {
     if (E <= kLaneRouteMaxE)
-        return launch_pdl(route_lane_kernel, dim3(T), dim3(kRouteThreads), 0, st, T, E, k, norm_topk, logits, idx, w,
-                          keff, x, gvec, H, sgate);
+        return launch_pdl(route_lane_kernel, dim3((T + 31) / 32 + (sgate != nullptr ? T : 0)), dim3(kRouteThreads), 0,
+                          st, T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate);
     if (E <= 128) return launch_v<4>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
     if (E <= 256) return launch_v<8>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
     if (E <= 512) return launch_v<16>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
