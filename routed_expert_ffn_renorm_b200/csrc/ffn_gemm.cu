@@ -145,25 +145,37 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// kCl: acquire at cluster scope (barriers that the other CTA of a pair arrives on).
+template <bool kCl = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
+    if constexpr (kCl)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
     return ok != 0;
 }
 // Bounded wait.  Returns false when the limit passes (status + abort flag
 // set) or, if watch_abort, when another role has aborted.
+template <bool kCl = false>
 __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
                                        bool watch_abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kCl>(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait<kCl>(bar, parity)) return true;
         if ((it & 63u) == 0) {
             if (watch_abort && *abort_flag) return false;
             if (globaltimer() - t0 > kWaitLimitNs) {
@@ -175,9 +187,10 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
     }
 }
 // The common case (already complete) inline; the bounded spin out of line.
+template <bool kCl = false>
 __device__ __forceinline__ bool mbar_wait_fast(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                int32_t *status, bool watch_abort) {
-    return mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort_flag, status, watch_abort);
+    return mbar_try_wait<kCl>(bar, parity) || mbar_wait<kCl>(bar, parity, abort_flag, status, watch_abort);
 }
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y) {
     asm volatile(
@@ -220,9 +233,10 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     d |= (uint64_t)2 << 61;                    // 128-byte swizzle
     return d;
 }
-// kind::f16 instruction descriptor: fp32 D, bf16 A and B, both K-major, M = 128.
-__device__ __forceinline__ uint32_t idesc_bf16(int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+// kind::f16 instruction descriptor: fp32 D, bf16 A and B, both K-major, M = 128
+// (or 256 for a CTA pair).
+__device__ __forceinline__ uint32_t idesc_bf16(int n, int m = kTileM) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -251,6 +265,64 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---- CTA pair (cluster of 2, cta_group::2) ----
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// TMA load of one CTA of the pair whose completion is counted on the mbarrier
+// of CTA 0 (the mbarrier's own-CTA address with the peer bit cleared).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cta0, void *dst, int x, int y,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cta0), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on the mbarrier at this offset in both CTAs of the pair once the pair's MMAs complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 __device__ __forceinline__ int ld_acquire(const int32_t *p) {
@@ -448,15 +520,20 @@ __device__ __forceinline__ int box_index(int nvalid) {  // smallest box of 16 <<
 // of 16 << bi rows (sub_pages pages).  A ring step carries ns sub-steps --
 // two while that is at most kMaxStepPages, so the per-step work of the
 // producer and MMA lanes is spent once per 32 KB of weights.
+// A CTA pair splits a tile's MMA N (the valid tokens rounded up to 16) in two
+// halves, one per CTA.
+__device__ __forceinline__ int pair_half(int nvalid) { return ((nvalid + 15) & ~15) >> 1; }
+
 struct StepShape {
     int bi;              // token box index
     uint32_t sub_pages;  // pages per sub-step
     int ns;              // sub-steps per ring step (the item's last step may hold fewer)
     int nk;              // 64-wide K slices of the item
 };
+template <bool kPair = false>
 __device__ __forceinline__ StepShape step_shape(const Item &it, const FfnParams &p) {
     StepShape sh;
-    sh.bi = box_index(it.nvalid);
+    sh.bi = box_index(kPair ? pair_half(it.nvalid) : it.nvalid);
     sh.sub_pages = (uint32_t)it.m * kAPages + (1u << sh.bi);
     sh.ns = 2 * sh.sub_pages <= (uint32_t)kMaxStepPages ? 2 : 1;
     sh.nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
@@ -483,6 +560,7 @@ __device__ __forceinline__ void down_dest(const Item &it, int n, const FfnParams
 }
 
 // --------------------------------------------------------------- kernel --
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnMaps maps, const FfnParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -509,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tmem_cols = 2 * p.BN;
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;  // 0: the pair's MMA issuer
     pdl_launch_dependents();
 
     // ---- setup: barriers, TMEM, tile schedule
@@ -519,12 +598,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 1);
+            mbar_init(&tempty[a], kPair ? 2 : 1);  // pair: both CTAs' epilogues
         }
         mbar_init(mma_done, 1);
         for (int q = 0; q < kQueue; ++q) {
             mbar_init(&qfull[q], 1);
-            mbar_init(&qempty[q], 2);  // the MMA lane and the elected epilogue thread
+            // the MMA lane and the elected epilogue thread (pair: and the other CTA's
+            // producer and epilogue)
+            mbar_init(&qempty[q], kPair ? 4 : 2);
         }
         *abort_flag = 0;
         for (int w = 0; w < kReadyWords; ++w) ready_bits[w] = 0;
@@ -543,12 +624,22 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         }
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(tmem_cols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (kPair) {  // both CTAs' warp 1, same address: one allocation mirrored in the pair
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_slot)),
+                         "r"(tmem_cols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_slot)),
+                         "r"(tmem_cols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
         tc_fence_before();
     }
+    if constexpr (kPair) cluster_sync();  // both CTAs' barriers initialised before any cross-CTA arrive
     pdl_wait();  // the dispatch outputs and activations are ready past this point
     // dispatch offsets to shared memory, then the per-expert prefix sums of token
     // tiles and of down items
@@ -564,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             return make_int2((cnt + BN - 1) / BN, merged_down_items(cnt, BN, R1));
         });
         // every CTA takes the same decision from the same offsets
-        sc.merge = (tile_base[p.E] * R1 + p.Rs[1] * sc.shared_ntt) >= kMergePerCta * (int)gridDim.x;
+        sc.merge = !kPair && (tile_base[p.E] * R1 + p.Rs[1] * sc.shared_ntt) >= kMergePerCta * (int)gridDim.x;
     }
     tc_fence_after();
     sc.shared_merge = p.Is > 0 && sc.shared_ntt == 1 && down_merged(p.T, p.BN, sc.merge);
@@ -586,19 +677,35 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             uint32_t issued = 0, retired = 0;  // K steps issued / whose MMAs have released their pages
             uint32_t oldest = 0;               // first page (virtual) of step `retired` while one is in flight
             const uint64_t wpol = policy_evict_first();  // expert weights: read once per launch
-            int next = atomicAdd(p.sched, 1);            // items are claimed one ahead
+            const uint64_t bpol = policy_evict_normal();  // token rows (pair loads take a policy)
+            int next = (!kPair || rank == 0) ? atomicAdd(p.sched, 1) : 0;  // items are claimed one ahead
             bool all_ready = false;                       // every gate/up item of the launch is done
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 const uint32_t qph = (uint32_t)(li / kQueue) & 1u;
-                if (!mbar_wait(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
-                int item = next < total_items ? next : -1;
-                if (item >= 0) next = atomicAdd(p.sched, 1);  // its latency overlaps this item's loads
+                int item;
                 Item it{};
-                if (item >= 0) it = decode_item(item, sc, p);  // decoded once, for all three roles
-                qdesc[slot].item = item;
-                qdesc[slot].it = it;
-                mbar_arrive(&qfull[slot]);
+                if (!kPair || rank == 0) {
+                    if (!mbar_wait<kPair>(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
+                    item = next < total_items ? next : -1;
+                    if (item >= 0) next = atomicAdd(p.sched, 1);  // its latency overlaps this item's loads
+                    if (item >= 0) it = decode_item(item, sc, p);  // decoded once, for all roles
+                    qdesc[slot].item = item;
+                    qdesc[slot].it = it;
+                    if constexpr (kPair) {  // the same entry in the other CTA's queue, then its qfull
+                        const uint32_t *src = reinterpret_cast<const uint32_t *>(&qdesc[slot]);
+                        const uint32_t dst = mapa(smem_u32(&qdesc[slot]), 1);
+#pragma unroll
+                        for (int w = 0; w < (int)(sizeof(ItemSlot) / 4); ++w) st_cluster_u32(dst + 4 * w, src[w]);
+                        mbar_arrive_cluster(mapa(smem_u32(&qfull[slot]), 1));
+                    }
+                    mbar_arrive(&qfull[slot]);
+                } else {  // the other CTA of a pair takes the item CTA 0 published
+                    if (!mbar_wait<true>(&qfull[slot], qph, abort_flag, p.status, true)) break;
+                    item = qdesc[slot].item;
+                    it = qdesc[slot].it;
+                    mbar_arrive_cluster(mapa(smem_u32(&qempty[slot]), 0));
+                }
                 if (item < 0) break;
                 const int grp = it.shared ? p.E : it.e;
                 if (fused && it.ph == 1 && !all_ready && !((ready_bits[grp >> 5] >> (grp & 31)) & 1u)) {
@@ -631,10 +738,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 const PhaseMaps &pm = maps.ph[it.ph];
                 const CUtensorMap *ma0 = it.shared ? &pm.s0 : &pm.a0;
                 const CUtensorMap *ma1 = it.shared ? &pm.s1 : &pm.a1;
-                const StepShape sh = step_shape(it, p);
+                const StepShape sh = step_shape<kPair>(it, p);
                 const CUtensorMap *mb = it.shared ? &pm.bs[sh.bi] : &pm.b[sh.bi];
-                const int a_row = it.ph == 0 ? (it.shared ? 0 : it.e * p.I) + it.r * 64
-                                             : (it.shared ? 0 : it.e * p.H) + it.r * kTileM;
+                // pair: this CTA's weight tile of the two, and its half of the token rows
+                const int rt = kPair ? 2 * it.r + (int)rank : it.r;
+                const int a_row = it.ph == 0 ? (it.shared ? 0 : it.e * p.I) + rt * 64
+                                             : (it.shared ? 0 : it.e * p.H) + rt * kTileM;
+                const int b_row = it.row0 + (kPair ? (int)rank * pair_half(it.nvalid) : 0);
                 bool ok = true;
                 for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
                     const int nsub = min(sh.ns, sh.nk - k0);
@@ -644,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     // until the steps in flight and this one lie within P consecutive
                     // (virtual) pages -- then no two of them share a physical page.
                     while (issued != retired && (vhead - oldest > P || issued - retired >= (uint32_t)kTickets)) {
-                        if (!mbar_wait_fast(&empty[retired % kTickets], (retired / kTickets) & 1u, abort_flag,
+                        if (!mbar_wait_fast<kPair>(&empty[retired % kTickets], (retired / kTickets) & 1u, abort_flag,
                                             p.status, true)) {
                             ok = false;
                             break;
@@ -656,30 +766,54 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     const uint32_t tk = issued % kTickets;
                     if (issued == retired) oldest = vhead - need;
                     ticket_start[tk] = vhead - need;
-                    mbar_arrive_expect_tx(&full[tk], need * kPageBytes);
-                    for (int j = 0; j < nsub; ++j) {
-                        uint8_t *sA = ring + (size_t)(first + j * sh.sub_pages) * kPageBytes;
-                        const int kx = (k0 + j) * kBlockK;
-                        if (it.ph == 0) {
-                            tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
-                            tma_load_2d_hint(ma1, &full[tk], sA + kABytes / 2, kx, a_row, wpol);
-                        } else {
-                            tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
-                            if (it.m == 2) tma_load_2d_hint(ma0, &full[tk], sA + kABytes, kx, a_row + kTileM, wpol);
+                    if constexpr (kPair) {
+                        // both CTAs' loads complete on CTA 0's barrier, armed there with both halves
+                        if (rank == 0) mbar_arrive_expect_tx(&full[tk], 2 * need * kPageBytes);
+                        const uint32_t bar0 = mapa(smem_u32(&full[tk]), 0);
+                        for (int j = 0; j < nsub; ++j) {
+                            uint8_t *sA = ring + (size_t)(first + j * sh.sub_pages) * kPageBytes;
+                            const int kx = (k0 + j) * kBlockK;
+                            if (it.ph == 0) {
+                                tma_load_2d_pair(ma0, bar0, sA, kx, a_row, wpol);
+                                tma_load_2d_pair(ma1, bar0, sA + kABytes / 2, kx, a_row, wpol);
+                            } else {
+                                tma_load_2d_pair(ma0, bar0, sA, kx, a_row, wpol);
+                            }
+                            tma_load_2d_pair(mb, bar0, sA + kABytes, kx, b_row, bpol);
                         }
-                        tma_load_2d(mb, &full[tk], sA + it.m * kABytes, kx, it.row0);
+                    } else {
+                        mbar_arrive_expect_tx(&full[tk], need * kPageBytes);
+                        for (int j = 0; j < nsub; ++j) {
+                            uint8_t *sA = ring + (size_t)(first + j * sh.sub_pages) * kPageBytes;
+                            const int kx = (k0 + j) * kBlockK;
+                            if (it.ph == 0) {
+                                tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
+                                tma_load_2d_hint(ma1, &full[tk], sA + kABytes / 2, kx, a_row, wpol);
+                            } else {
+                                tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
+                                if (it.m == 2)
+                                    tma_load_2d_hint(ma0, &full[tk], sA + kABytes, kx, a_row + kTileM, wpol);
+                            }
+                            tma_load_2d(mb, &full[tk], sA + it.m * kABytes, kx, it.row0);
+                        }
                     }
                     ++issued;
                 }
                 if (!ok) break;
             }
-            // wait for every copy still in flight before the CTA may exit
-            for (uint32_t j = retired; j < issued; ++j)
-                mbar_wait(&full[j % kTickets], (j / kTickets) & 1u, abort_flag, p.status, false);
+            // wait for every copy still in flight before the CTA may exit (pair: the
+            // copies complete on CTA 0's barrier; the MMAs that consumed them release
+            // this CTA's pages)
+            for (uint32_t j = retired; j < issued; ++j) {
+                if constexpr (kPair)
+                    mbar_wait<true>(&empty[j % kTickets], (j / kTickets) & 1u, abort_flag, p.status, false);
+                else
+                    mbar_wait(&full[j % kTickets], (j / kTickets) & 1u, abort_flag, p.status, false);
+            }
         }
     } else if (warp == 1) {
         // ================= MMA issuer =================
-        if (lane == 0) {
+        if (lane == 0 && (!kPair || rank == 0)) {  // a pair's MMAs are issued by CTA 0
             uint32_t vhead = 0, off = 0, step = 0;  // the producer's page sequence, replayed
             const uint64_t desc0 = sw128_desc(smem_u32(ring));  // ring page 0; other pages by addition
             for (int li = 0;; ++li) {
@@ -689,11 +823,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 const Item it = qdesc[slot].it;
                 mbar_arrive(&qempty[slot]);
                 if (item < 0) break;
-                const StepShape sh = step_shape(it, p);
-                const uint32_t idesc = idesc_bf16((it.nvalid + 15) & ~15);
+                const StepShape sh = step_shape<kPair>(it, p);
+                const uint32_t idesc = idesc_bf16((it.nvalid + 15) & ~15, kPair ? 2 * kTileM : kTileM);
                 const int acc = li & 1;
                 const uint32_t use = (uint32_t)(li >> 1);
-                if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag, p.status, true)) break;
+                if (!mbar_wait<kPair>(&tempty[acc], (use & 1u) ^ 1u, abort_flag, p.status, true)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(acc * p.BN), d1 = d + (uint32_t)(p.BN >> 1);
                 bool ok = true;
@@ -701,7 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     const int nsub = min(sh.ns, sh.nk - k0);
                     const uint32_t first = ring_alloc(vhead, off, (uint32_t)nsub * sh.sub_pages, P);
                     const uint32_t tk = step % kTickets;
-                    if (!mbar_wait_fast(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true)) {
+                    if (!mbar_wait_fast<kPair>(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true)) {
                         ok = false;
                         break;
                     }
@@ -709,7 +843,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     for (int j = 0; j < nsub; ++j) {
                         // descriptor start addresses count 16-byte units
                         const uint64_t da = desc0 + (first + j * sh.sub_pages) * (kPageBytes / 16);
-                        if (it.m == 1) {
+                        if constexpr (kPair) {  // M = 256: each CTA's 128 weight rows, N split over the two
+                            const uint64_t db = da + kABytes / 16;
+#pragma unroll
+                            for (int kk = 0; kk < kBlockK / 16; ++kk)
+                                umma_bf16_pair(d, da + 2 * kk, db + 2 * kk, idesc, (k0 | j | kk) != 0);
+                        } else if (it.m == 1) {
                             const uint64_t db = da + kABytes / 16;
 #pragma unroll
                             for (int kk = 0; kk < kBlockK / 16; ++kk)  // +32 bytes per K16 step
@@ -723,13 +862,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                             }
                         }
                     }
-                    umma_commit(&empty[tk]);
+                    if constexpr (kPair) umma_commit_pair(&empty[tk]);  // frees the pages in both CTAs
+                    else umma_commit(&empty[tk]);
                     ++step;
                 }
                 if (!ok) break;
-                umma_commit(&tfull[acc]);
+                if constexpr (kPair) umma_commit_pair(&tfull[acc]);  // both CTAs' epilogues
+                else umma_commit(&tfull[acc]);
             }
-            umma_commit(mma_done);  // completes once every MMA above has
+            if constexpr (kPair) umma_commit_pair_local(mma_done);  // completes once every MMA above has
+            else umma_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.status, false);
         }
     } else {
@@ -741,9 +883,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             const uint32_t use = (uint32_t)(li >> 1);
             if (elected) {  // one thread takes the item; its accumulator is awaited below
                 const int slot = li % kQueue;
-                if (mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) {
+                if (mbar_wait<kPair>(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) {
                     *epi_desc = qdesc[slot];
-                    mbar_arrive(&qempty[slot]);
+                    if (kPair && rank != 0) mbar_arrive_cluster(mapa(smem_u32(&qempty[slot]), 0));
+                    else mbar_arrive(&qempty[slot]);
                 } else {
                     epi_desc->item = -2;
                 }
@@ -756,11 +899,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             int mrow0 = 0;
             float mw0 = 0.f;
             if (it.ph == 1) down_dest(it, lane, p, mrow0, mw0);
-            if (elected) *epi_flag = mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 0 : -1;
+            if (elected) *epi_flag = mbar_wait<kPair>(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 0 : -1;
             named_bar_sync(1, 128);
             if (*epi_flag) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + (uint32_t)(acc * p.BN) + ((uint32_t)(q * 32) << 16);
+            const int rt = kPair ? 2 * it.r + (int)rank : it.r;  // pair: this CTA's weight tile
             for (int c0 = 0; c0 < it.nvalid; c0 += 32) {
                 if (it.ph == 0) {
                     float v[32];
@@ -776,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                         const float *xr = xchg + row * kXchgStride;
                         uint16_t *out = it.shared ? p.h_shared : p.h_perm;
                         const int ld = it.shared ? p.Is : p.I;
-                        uint16_t *dst = out + (size_t)(it.row0 + c0) * ld + it.r * 64 + row;
+                        uint16_t *dst = out + (size_t)(it.row0 + c0) * ld + rt * 64 + row;
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (c0 + i < it.nvalid) dst[(size_t)i * ld] = f32_to_bf16_bits(xr[i] * v[i]);
@@ -790,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     for (int t = 0; t < it.m; ++t) {  // weight tile r + t: accumulator columns t * BN/2
                         float v[32];
                         tmem_ld32(tbase + (uint32_t)(t * (p.BN >> 1) + c0), v);
-                        uint16_t *out = p.ybuf + (it.r + t) * kTileM + q * 32 + lane;
+                        uint16_t *out = p.ybuf + (rt + t) * kTileM + q * 32 + lane;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
                             const int rr = __shfl_sync(0xffffffffu, mrow, i);
@@ -803,7 +947,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             tc_fence_before();
             named_bar_sync(1, 128);
             if (elected) {
-                mbar_arrive(&tempty[acc]);
+                if (kPair && rank != 0) mbar_arrive_cluster(mapa(smem_u32(&tempty[acc]), 0));
+                else mbar_arrive(&tempty[acc]);
                 if (fused && it.ph == 0) {
                     // the CTA's h rows (ordered before this by the barrier) become visible
                     // device-wide before the group counter moves
@@ -816,10 +961,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     }
 
     __syncthreads();
+    if constexpr (kPair) cluster_sync();  // the other CTA is done with the shared TMEM allocation and our barriers
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols)
-                     : "memory");
+        if constexpr (kPair)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols)
+                         : "memory");
     }
     // The last CTA out resets the counters for the next launch.
     if (threadIdx.x == 0) {
@@ -941,12 +1091,52 @@ int choose_tiles(const FfnArgs &a, int sms, int *bn, int *bns, int *pages) {
 
 }  // namespace
 
+// CTA pairs (cta_group::2) for a single-phase launch whose groups fill wide
+// token tiles: the mean group has at least 128 tokens (the regime where a
+// 256-token tile's operand bytes, not the weight stream, limit the tensor
+// pipe), and every weight-tile count of the phase is even.  MOE_FORCE_PAIR
+// = 0 / 1 overrides the first condition (tests and benchmarking only).
+int choose_pair(const FfnArgs &a, int phases, int sms, bool *pair) {
+    *pair = false;
+    bool want = phases != 3 && ((long long)a.T * a.k + a.E - 1) / a.E >= 128;
+    if (const char *f = getenv("MOE_FORCE_PAIR")) {
+        if (f[0] != '0' && f[0] != '1') return MOE_ERR_INVALID_ARG;
+        if (f[1] != 0) return MOE_ERR_INVALID_ARG;
+        want = f[0] == '1' && phases != 3;
+    }
+    const bool even = ((phases & 1) == 0 || ((a.I / 64) % 2 == 0 && (a.Is / 64) % 2 == 0)) &&
+                      ((phases & 2) == 0 || (a.H / kTileM) % 2 == 0);
+    *pair = want && even && sms >= 2;
+    return MOE_OK;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     const DeviceInfo di = device_info();
     if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
     if (phases < 1 || phases > 3) return MOE_ERR_INVALID_ARG;
     FfnParams p{};
     if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
+    bool pair = false;
+    if (int rc = choose_pair(a, phases, di.sms, &pair)) return rc;
     const int BN = p.BN;
     p.T = a.T;
     p.H = a.H;
@@ -965,12 +1155,13 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     p.status = a.status;
     p.sched = a.status + (phases == 2 ? 8 : 4);
     p.hdone = a.hdone;
-    p.R[0] = a.I / 64;
-    p.Rs[0] = a.Is / 64;
+    const int per = pair ? 2 : 1;  // weight tiles per item (a pair covers two)
+    p.R[0] = a.I / 64 / per;
+    p.Rs[0] = a.Is / 64 / per;
     p.nk[0] = a.H / kBlockK;
     p.nks[0] = a.H / kBlockK;
-    p.R[1] = a.H / kTileM;
-    p.Rs[1] = a.H / kTileM;
+    p.R[1] = a.H / kTileM / per;
+    p.Rs[1] = a.H / kTileM / per;
     p.nk[1] = a.I / kBlockK;
     p.nks[1] = a.Is / kBlockK;
 
@@ -1006,7 +1197,10 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
     if (!attr_set[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
+        if (cudaFuncSetAttribute(ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+                cudaSuccess)
             return MOE_ERR_CUDA;
         attr_set[dev].store(1, std::memory_order_release);
     }
@@ -1017,8 +1211,14 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     long long items = 0;
     for (int ph = 0; ph < 2; ++ph)
         if ((phases >> ph) & 1) items += tiles * p.R[ph] + st_tiles * p.Rs[ph];
+    if (pair) {  // clusters of two CTAs: an even grid
+        const int grid = 2 * (int)std::max<long long>(1, std::min<long long>(di.sms / 2, items));
+        return launch_pair(ffn_kernel<true>, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess ? MOE_OK
+                                                                                                          : MOE_ERR_CUDA;
+    }
     const int grid = (int)std::max<long long>(1, std::min<long long>(di.sms, items));
-    return launch_pdl(ffn_kernel, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_pdl(ffn_kernel<false>, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess ? MOE_OK
+                                                                                                   : MOE_ERR_CUDA;
 }
 
 int device_sm_count() { return device_info().sms; }

@@ -88,6 +88,41 @@ def test_merged_down_items_bits(bn, monkeypatch):
     assert (got.out_bits == ref.out_bits).all()
 
 
+# CTA pairs (cta_group::2): layers whose mean group has >= 128 tokens run the
+# FFN as two launches of CTA pairs; every weight-tile count here is even.
+PAIRED = [
+    W.MoEConfig("pair_shared", T=600, H=512, E=8, I=256, k=2, Is=256),
+    W.MoEConfig("pair_ragged", T=333, H=256, E=4, I=128, k=3, Is=128, zipf_alpha=1.0),
+]
+
+
+@pytest.mark.parametrize("cfg", PAIRED, ids=lambda c: c.name)
+def test_cta_pair_layers(cfg):
+    diag, g, _ = _run(cfg)
+    print(cfg.label, diag)
+
+
+@pytest.mark.parametrize("cfg", PAIRED, ids=lambda c: c.name)
+def test_cta_pair_bits_equal_single_cta(cfg, monkeypatch):
+    """The pair's M = 256 MMAs accumulate every output element in the same K
+    order as the single-CTA path: identical bits."""
+    inp = W.make_inputs(cfg, device="cuda")
+    monkeypatch.setenv("MOE_FORCE_PAIR", "1")
+    a = gpu_forward(cfg, inp)
+    monkeypatch.setenv("MOE_FORCE_PAIR", "0")
+    b = gpu_forward(cfg, inp)
+    assert a.status == 0 and b.status == 0
+    assert (a.out_bits == b.out_bits).all()
+
+
+def test_force_pair_rejects_bad_values(monkeypatch):
+    cfg = PAIRED[0]
+    inp = W.make_inputs(cfg, device="cuda")
+    monkeypatch.setenv("MOE_FORCE_PAIR", "2")
+    with pytest.raises(moe.MoEError):
+        gpu_forward(cfg, inp)
+
+
 def test_hot_expert_multi_tile():
     """Every token routes to expert 3 first: one group of T rows, several token tiles."""
     cfg = W.MoEConfig("hot", T=600, H=256, E=8, I=128, k=2, Is=64)
