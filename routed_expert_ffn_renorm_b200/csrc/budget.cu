@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(1024) budget_small_kernel(int T, int E, int k,
     uint8_t *pres = reinterpret_cast<uint8_t *>(agg + E);
     uint8_t *keep = pres + E;
     __shared__ int warp_sums[32];
-    __shared__ int nu_s, nd_s;
+    __shared__ int nd_s;
     pdl_launch_dependents();
     pdl_wait();
     for (int s = threadIdx.x; s < Tk; s += blockDim.x) {
@@ -57,8 +57,7 @@ __global__ void __launch_bounds__(1024) budget_small_kernel(int T, int E, int k,
         w_s[s] = w[s];
     }
     __syncthreads();
-    budget_block(T, E, k, N, norm_topk, idx_s, w_s, keff_s, keep, &nd_s, hist, off, sorted, agg, pres, warp_sums,
-                 &nu_s);
+    budget_block(T, E, k, N, norm_topk, idx_s, w_s, keff_s, keep, &nd_s, hist, off, sorted, agg, pres, warp_sums);
     for (int s = threadIdx.x; s < Tk; s += blockDim.x) {
         idx[s] = idx_s[s];
         w[s] = w_s[s];

@@ -122,7 +122,7 @@ struct FfnParams {
     uint16_t *h_shared;  // [T, Is]
     uint16_t *ybuf;      // [T, k+1, H]
     int32_t *status;     // status word
-    int32_t *sched;      // [0] next work item, [1] CTAs done; zero between launches
+    int32_t *sched;      // [0] items claimed past the first grid's worth, [1] CTAs done; zero between launches
     int32_t *hdone;      // [E+2] finished gate/up items per group (E = shared), [E+1] in all; zero between launches
 };
 
@@ -678,7 +678,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             uint32_t oldest = 0;               // first page (virtual) of step `retired` while one is in flight
             const uint64_t wpol = policy_evict_first();  // expert weights: read once per launch
             const uint64_t bpol = policy_evict_normal();  // token rows (pair loads take a policy)
-            int next = (!kPair || rank == 0) ? atomicAdd(p.sched, 1) : 0;  // items are claimed one ahead
+            // items are claimed one ahead: a CTA (pair) takes item blockIdx (cluster
+            // index) first, then from the counter, past the first grid's worth
+            const int claimers = kPair ? (int)gridDim.x / 2 : (int)gridDim.x;
+            int next = kPair ? (int)blockIdx.x / 2 : (int)blockIdx.x;
             bool all_ready = false;                       // every gate/up item of the launch is done
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
@@ -688,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 if (!kPair || rank == 0) {
                     if (!mbar_wait<kPair>(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
                     item = next < total_items ? next : -1;
-                    if (item >= 0) next = atomicAdd(p.sched, 1);  // its latency overlaps this item's loads
+                    if (item >= 0) next = claimers + atomicAdd(p.sched, 1);  // latency overlaps this item's loads
                     if (item >= 0) it = decode_item(item, sc, p);  // decoded once, for all roles
                     qdesc[slot].item = item;
                     qdesc[slot].it = it;
@@ -971,16 +974,22 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols)
                          : "memory");
     }
-    // The last CTA out resets the counters for the next launch.
+    // The last CTA out resets the counters for the next launch, all its threads
+    // sharing the group counters (a serial loop of E + 2 atomics would hold the
+    // grid open for microseconds).
     if (threadIdx.x == 0) {
         __threadfence();
-        if (atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+        *epi_flag = atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (*epi_flag) {
+        if (threadIdx.x == 0) {
             atomicExch(p.sched, 0);
             atomicExch(p.sched + 1, 0);
-            if (fused)
-                for (int g = 0; g <= p.E + 1; ++g) atomicExch(p.hdone + g, 0);
-            __threadfence();
         }
+        if (fused)
+            for (int g = threadIdx.x; g <= p.E + 1; g += kThreads) atomicExch(p.hdone + g, 0);
+        __threadfence();
     }
 }
 

@@ -6,9 +6,9 @@
 // routes all T tokens itself from there (route_token_lane, one token per
 // thread, for E <= 64; route_token, one warp per token, above),
 // applies the budget (budget_block) and sorts the kept slots by expert
-// (block_sort_by_expert) -- the same device code, in the same order, as the
-// stand-alone route / budget / dispatch kernels, so the results are the same
-// bits.  CTA 0 writes the routing, budget and dispatch outputs; all CTAs
+// (block_sort_by_expert, or regroup_kept from the budget's own sort) -- the
+// same device code, or the same order, as the stand-alone route / budget /
+// dispatch kernels, so the results are the same bits.  CTA 0 writes the routing, budget and dispatch outputs; all CTAs
 // then share the rest: x_perm rows in CTA-strided order and the shared
 // gate sigmoid(g . x_t) for tokens in CTA-strided order (a 128-thread group
 // per token, as in the route kernel).  Redundant routing costs each CTA one
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_small_kernel(const Fro
     uint8_t *pres = reinterpret_cast<uint8_t *>(agg + E);
     uint8_t *keep = pres + E;
     __shared__ int warp_sums[32];
-    __shared__ int nu_s, nd_s;
+    __shared__ int nd_s;
     __shared__ float part[kFrontGroups][kGateThreads / 32];
     pdl_launch_dependents();
     pdl_wait();
@@ -107,18 +107,20 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_small_kernel(const Fro
     }
     __syncthreads();
     // budget (a union of at most N experts, or N == 0, leaves everything as it is)
-    if (a.N > 0)
+    // and dispatch: kept slots by expert, slot order inside one
+    if (a.N > 0) {
         budget_block(T, E, k, a.N, a.norm_topk, idx_s, w_s, keff_s, keep, &nd_s, hist, off, sorted, agg, pres,
-                     warp_sums, &nu_s);
-    // dispatch: kept slots by expert, slot order inside one
-    block_sort_by_expert(
-        Tk, E, W,
-        [=](int s) {
-            const int t = s / k, j = s - t * k;
-            const int e = idx_s[s];
-            return (j < keff_s[t] && e >= 0 && e < E) ? e : -1;
-        },
-        hist, off, sorted, warp_sums);
+                     warp_sums);
+        regroup_kept(E, k, idx_s, keff_s, keep, off, sorted, hist, warp_sums);
+    } else {
+        block_sort_by_expert(
+            Tk, E, sort_warps_for(Tk, E),
+            [=](int s) {
+                const int e = idx_s[s];
+                return (e >= 0 && e < E) ? e : -1;
+            },
+            hist, off, sorted, warp_sums);
+    }
     const int total = off[E];
     if (writer) {
         for (int s = threadIdx.x; s < Tk; s += kFrontThreads) {

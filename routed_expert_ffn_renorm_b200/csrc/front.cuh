@@ -16,13 +16,20 @@ namespace moe {
 // probabilities renormalised (SpecForge PR #943, "Modifications": softmax
 // router with renormalised top-k).  One warp per token: lane l holds the
 // logits of experts l, l+32, ... (coalesced loads).  Each of the k selection
-// rounds takes a lane-local best and a 5-step shuffle argmax ordered by
-// (logit descending, expert id ascending), so equal logits keep the lower
-// id; the winner's owner lane masks it out.  The logits come from global
+// rounds takes a lane-local best, then two warp reductions: the largest
+// logit (as an order-preserving integer key, -0 read as +0) and the lowest
+// expert id holding it, so equal logits keep the lower id; the winner's
+// owner lane masks it out.  The logits come from global
 // memory (kGlobal, read-only path) or from shared memory; idx / w may point
 // to global or shared memory; keff (may be null) receives k.
 __device__ __forceinline__ bool route_better(float va, int ia, float vb, int ib) {
     return va > vb || (va == vb && ia < ib);
+}
+// Unsigned key with the order of the float (for non-NaN values); -0 and +0 map
+// to the same key, as they compare equal.
+__device__ __forceinline__ uint32_t float_order_key(float v) {
+    const uint32_t b = v == 0.f ? 0u : __float_as_uint(v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
 template <int V, bool kGlobal = true>  // logits per lane: V * 32 >= E
@@ -63,15 +70,11 @@ __device__ __forceinline__ void route_token(int t, int E, int k, int norm_topk, 
                 bi = e;
             }
         }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (route_better(ov, oi, bv, bi)) {
-                bv = ov;
-                bi = oi;
-            }
-        }
+        // the warp's best: the largest key, then the lowest id among lanes holding it
+        const uint32_t key = bi == 0x7fffffff ? 0u : float_order_key(bv);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0xffffffffu);
+        bv = __shfl_sync(0xffffffffu, bv, bi & 31);  // the owner lane's value (== per key)
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
         if (lane == j) {
             my_idx = bi;
@@ -217,6 +220,9 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int *warp_sums) 
 
 // Per-warp count columns for a block sort over E experts: [W][E] ints fit in 32 KB.
 __host__ __device__ inline int sort_warps(int E) { return E <= 256 ? 32 : (E <= 512 ? 16 : 8); }
+// Warps a sort of n slots uses: one 32-slot pass each where sort_warps allows
+// (fewer count columns to zero and scan for small n).
+__device__ __forceinline__ int sort_warps_for(int n, int E) { return max(1, min(sort_warps(E), (n + 31) >> 5)); }
 
 // Stable counting sort of the slots 0..n-1 by expert inside one 1024-thread
 // block: key(s) is the slot's expert in [0, E), or -1 to leave it out.  W
@@ -225,6 +231,7 @@ __host__ __device__ inline int sort_warps(int E) { return E <= 256 ? 32 : (E <= 
 // number of lower lanes, so the order inside an expert is ascending slot id.
 // Out (shared memory): sorted[pos] = slot, off[e] = first position of expert
 // e, off[E] = number of sorted slots.  hist: W * E ints; warp_sums: 32 ints.
+// The result does not depend on W.
 template <class Key>
 __device__ __forceinline__ void block_sort_by_expert(int n, int E, int W, Key key, int *hist, int *off, int *sorted,
                                                      int *warp_sums) {
@@ -246,6 +253,7 @@ __device__ __forceinline__ void block_sort_by_expert(int n, int E, int W, Key ke
     const int e = threadIdx.x;  // blockDim.x == 1024 >= E
     int c = 0;
     if (e < E)
+#pragma unroll 8
         for (int w = 0; w < W; ++w) c += hist[w * E + e];
     const int excl = block_exclusive_scan_1024(c, warp_sums);
     if (e < E) {
@@ -289,43 +297,50 @@ __device__ __forceinline__ void block_sort_by_expert(int n, int E, int W, Key ke
 //   step 5: n_dropped = union size - N.
 // A budget of 0, or a union of at most N experts, changes nothing (keff = k,
 // kept = the union).  Out (shared memory): idx_s / w_s compacted, keff_s[T],
-// keep[E], *nd_s.  Scratch: hist (W * E), off (E + 1), sorted (T * k), agg
-// (E), pres (E), warp_sums (32), nu_s.
+// keep[E], *nd_s; off / sorted keep the sort of all slots by expert.
+// Scratch: hist (sort_warps(E) * E), off (E + 1), sorted (T * k), agg (E),
+// pres (E), warp_sums (32).  The ranks are counted by up to blockDim / E
+// threads per expert, each over a range of the others (integer sums: the
+// result does not depend on the split).
 __device__ __forceinline__ void budget_block(int T, int E, int k, int N, int norm_topk, int32_t *idx_s, float *w_s,
                                              int32_t *keff_s, uint8_t *keep, int *nd_s, int *hist, int *off,
-                                             int *sorted, float *agg, uint8_t *pres, int *warp_sums, int *nu_s) {
+                                             int *sorted, float *agg, uint8_t *pres, int *warp_sums) {
     const int Tk = T * k;
-    if (threadIdx.x == 0) *nu_s = 0;
     block_sort_by_expert(
-        Tk, E, sort_warps(E),
+        Tk, E, sort_warps_for(Tk, E),
         [=](int s) {
             const int x = idx_s[s];
             return (x >= 0 && x < E) ? x : -1;
         },
         hist, off, sorted, warp_sums);
     const int e = threadIdx.x;
+    int *rank = hist;  // free once the sort is done
     int my_present = 0;
     if (e < E) {
         float a = 0.f;
         for (int p = off[e]; p < off[e + 1]; ++p) a += w_s[sorted[p]];
         agg[e] = a;
-        pres[e] = off[e + 1] > off[e];
-        my_present = pres[e];
+        my_present = off[e + 1] > off[e];
+        pres[e] = (uint8_t)my_present;
+        rank[e] = 0;
     }
-    if (my_present) atomicAdd(nu_s, 1);  // integer: order-independent
-    __syncthreads();
-    const int nu = *nu_s;
-    const bool active = N > 0 && nu > N;
-    if (e < E) {
-        uint8_t kp = pres[e];
-        if (active && kp) {
-            const float a = agg[e];
-            int rank = 0;
-            for (int o = 0; o < E; ++o) rank += pres[o] && (agg[o] > a || (agg[o] == a && o < e));
-            kp = rank < N;
+    const int nu = __syncthreads_count(my_present);
+    const bool active = N > 0 && nu > N;  // the same in every thread
+    if (active) {
+        const int parts = max(1, min(E, (int)blockDim.x / E));
+        if ((int)threadIdx.x < parts * E) {
+            const int re = threadIdx.x % E, part = threadIdx.x / E;
+            if (pres[re]) {
+                const float a = agg[re];
+                int r = 0;
+                const int o1 = (part + 1) * E / parts;
+                for (int o = part * E / parts; o < o1; ++o) r += pres[o] && (agg[o] > a || (agg[o] == a && o < re));
+                if (r) atomicAdd(rank + re, r);
+            }
         }
-        keep[e] = kp;
+        __syncthreads();
     }
+    if (e < E) keep[e] = pres[e] && (!active || rank[e] < N);
     __syncthreads();
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
         int32_t *ti = idx_s + (size_t)t * k;
@@ -355,6 +370,55 @@ __device__ __forceinline__ void budget_block(int T, int E, int k, int N, int nor
         keff_s[t] = c;
     }
     if (threadIdx.x == 0) *nd_s = active ? nu - N : 0;
+    __syncthreads();
+}
+
+// The dispatch order from the budget's own sort.  budget_block leaves off /
+// sorted holding every slot by expert, ascending slot id inside an expert --
+// that is, ascending token, as a token holds an expert at most once.  A kept
+// expert keeps its slots in that token order, each renamed to the slot the
+// expert now holds in its token's compacted list; a dropped expert's slots
+// go.  That is the order block_sort_by_expert gives the kept slots, here
+// without a second sort.  Positions only move down, and each pass reads its
+// 1024 positions before any is written.  Scratch: hist (E + 1 ints),
+// warp_sums (32).
+__device__ __forceinline__ void regroup_kept(int E, int k, const int32_t *idx_s, const int32_t *keff_s,
+                                             const uint8_t *keep, int *off, int *sorted, int *hist, int *warp_sums) {
+    const int e = threadIdx.x;
+    const int cnt = (e < E && keep[e]) ? off[e + 1] - off[e] : 0;
+    const int nofs = block_exclusive_scan_1024(cnt, warp_sums);
+    if (e < E) {
+        hist[e] = nofs;
+        if (e == E - 1) hist[E] = nofs + cnt;
+    }
+    __syncthreads();
+    const int total = off[E];
+    for (int p0 = 0; p0 < total; p0 += blockDim.x) {
+        const int p = p0 + threadIdx.x;
+        int np = -1, ns = 0;
+        if (p < total) {
+            int lo = 0, hi = E - 1;  // the expert whose range holds p
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (off[mid] <= p)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            if (keep[lo]) {
+                const int t = sorted[p] / k;
+                const int32_t *ti = idx_s + (size_t)t * k;
+                int j = 0;
+                while (j < keff_s[t] - 1 && ti[j] != lo) ++j;
+                np = hist[lo] + (p - off[lo]);
+                ns = t * k + j;
+            }
+        }
+        __syncthreads();
+        if (np >= 0) sorted[np] = ns;
+        __syncthreads();
+    }
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = hist[i];
     __syncthreads();
 }
 
