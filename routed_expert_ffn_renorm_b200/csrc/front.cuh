@@ -14,76 +14,104 @@ namespace moe {
 // ---------------------------------------------------------------- routing --
 // Softmax over the E logits of a token, top-k by logit with the kept
 // probabilities renormalised (SpecForge PR #943, "Modifications": softmax
-// router with renormalised top-k).  One warp per token: lane l holds the
-// logits of experts l, l+32, ... (coalesced loads).  Each of the k selection
-// rounds takes a lane-local best, then two warp reductions: the largest
-// logit (as an order-preserving integer key, -0 read as +0) and the lowest
-// expert id holding it, so equal logits keep the lower id; the winner's
-// owner lane masks it out.  The logits come from global
-// memory (kGlobal, read-only path) or from shared memory; idx / w may point
-// to global or shared memory; keff (may be null) receives k.
-__device__ __forceinline__ bool route_better(float va, int ia, float vb, int ib) {
-    return va > vb || (va == vb && ia < ib);
-}
-// Unsigned key with the order of the float (for non-NaN values); -0 and +0 map
-// to the same key, as they compare equal.
+// router with renormalised top-k).  One warp per token; each lane holds V
+// logits as order-preserving integer keys (-0 and +0 share one; a taken or
+// absent expert holds 0, below every logit's key).  For E > 128 a multiple
+// of 4, with 16-byte aligned rows (kVec), lane l holds experts 128c + 4l + q
+// (one 16-byte load per c), else experts l + 32i; either way a lane's slots
+// run in ascending expert order.  Each of the k selection rounds takes the lane's
+// best key (a tree over its V keys; equal keys keep the lower slot, so the
+// lower expert), then two warp reductions: the largest key, and the lowest
+// expert id among the lanes holding it -- so equal logits keep the lower id.
+// The winner's lane clears its key; lane j keeps the j-th winner and its key.
+// The logits come from global memory (kGlobal, read-only path) or from
+// shared memory; idx / w may point to global or shared memory; keff (may be
+// null) receives k.
 __device__ __forceinline__ uint32_t float_order_key(float v) {
     const uint32_t b = v == 0.f ? 0u : __float_as_uint(v);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+__device__ __forceinline__ float order_key_float(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
 
-template <int V, bool kGlobal = true>  // logits per lane: V * 32 >= E
-__device__ __forceinline__ void route_token(int t, int E, int k, int norm_topk, const float *__restrict__ logits,
-                                            int32_t *idx, float *w, int32_t *keff, int lane) {
+template <int V, bool kGlobal, bool kVec>
+__device__ __forceinline__ void route_token_impl(int t, int E, int k, int norm_topk, const float *__restrict__ logits,
+                                                 int32_t *idx, float *w, int32_t *keff, int lane) {
     const float *l = logits + (size_t)t * E;
+    // expert of slot i of this lane
+    auto expert = [&](int i) { return kVec ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i; };
     float v[V];
+    uint32_t key[V];
+    if constexpr (kVec) {
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = (e < E) ? (kGlobal ? __ldg(l + e) : l[e]) : -INFINITY;
+        for (int c = 0; c < V / 4; ++c) {
+            const int e0 = 128 * c + 4 * lane;  // E % 4 == 0: all four present or none
+            float4 q = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            if (e0 < E) q = kGlobal ? __ldg(reinterpret_cast<const float4 *>(l + e0)) : *reinterpret_cast<const float4 *>(l + e0);
+            v[4 * c] = q.x;
+            v[4 * c + 1] = q.y;
+            v[4 * c + 2] = q.z;
+            v[4 * c + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int e = expert(i);
+            v[i] = e < E ? (kGlobal ? __ldg(l + e) : l[e]) : -INFINITY;
+        }
     }
-    // softmax denominator: max, then sum of exp(l - max) over all E
-    float m = v[0];
 #pragma unroll
-    for (int i = 1; i < V; ++i) m = fmaxf(m, v[i]);
+    for (int i = 0; i < V; ++i) key[i] = expert(i) < E ? float_order_key(v[i]) : 0u;
+    // softmax denominator: the largest logit, then sum of exp(l - max) over all E
+    uint32_t km = key[0];
 #pragma unroll
-    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    for (int i = 1; i < V; ++i) km = max(km, key[i]);
+    const float m = order_key_float(__reduce_max_sync(0xffffffffu, km));
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < V; ++i)
-        if (lane + 32 * i < E) s += expf(v[i] - m);
+        if (expert(i) < E) s += expf(v[i] - m);
 #pragma unroll
     for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
 
     // k selection rounds; lane j keeps the j-th winner
-    uint32_t taken = 0;
     int my_idx = -1;
-    float my_logit = -INFINITY;
+    uint32_t my_key = 0u;
     for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
+        uint32_t tk[V];
+        int ti[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && !((taken >> i) & 1u) && route_better(v[i], e, bv, bi)) {
-                bv = v[i];
-                bi = e;
-            }
+            tk[i] = key[i];
+            ti[i] = i;
         }
-        // the warp's best: the largest key, then the lowest id among lanes holding it
-        const uint32_t key = bi == 0x7fffffff ? 0u : float_order_key(bv);
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-        bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0xffffffffu);
-        bv = __shfl_sync(0xffffffffu, bv, bi & 31);  // the owner lane's value (== per key)
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+#pragma unroll
+        for (int d = 1; d < V; d *= 2)
+#pragma unroll
+            for (int i = 0; i + d < V; i += 2 * d)
+                if (tk[i + d] > tk[i]) {  // strict: the lower slot keeps a tie
+                    tk[i] = tk[i + d];
+                    ti[i] = ti[i + d];
+                }
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, tk[0]);
+        const int win = (int)__reduce_min_sync(0xffffffffu, tk[0] == kmax ? (uint32_t)expert(ti[0]) : 0xffffffffu);
+        const int owner = kVec ? (win & 127) >> 2 : win & 31;
+        const int wslot = kVec ? 4 * (win >> 7) + (win & 3) : win >> 5;
+        if (owner == lane) {
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                if (i == wslot) key[i] = 0u;
+        }
         if (lane == j) {
-            my_idx = bi;
-            my_logit = bv;
+            my_idx = win;
+            my_key = kmax;
         }
     }
-    // probabilities of the kept experts; renormalise with the sum taken in
-    // slot order
-    float p = (lane < k) ? expf(my_logit - m) / s : 0.f;
+    // probabilities of the kept experts (the logit back from its key: exact up
+    // to the sign of a zero, which exp does not see); renormalise with the sum
+    // taken in slot order
+    float p = (lane < k) ? expf(order_key_float(my_key) - m) / s : 0.f;
     if (norm_topk) {
         float ps = 0.f;
         for (int j = 0; j < k; ++j) ps += __shfl_sync(0xffffffffu, p, j);
@@ -94,6 +122,16 @@ __device__ __forceinline__ void route_token(int t, int E, int k, int norm_topk, 
         w[(size_t)t * k + lane] = p;
     }
     if (keff != nullptr && lane == 0) keff[t] = k;
+}
+
+template <int V, bool kGlobal = true>  // logits per lane: V * 32 >= E, V a power of two >= 4
+__device__ __forceinline__ void route_token(int t, int E, int k, int norm_topk, const float *__restrict__ logits,
+                                            int32_t *idx, float *w, int32_t *keff, int lane) {
+    static_assert(V >= 4 && (V & (V - 1)) == 0, "V: a power of two >= 4");
+    if (V >= 8 && (E & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0)  // measured: no gain at V = 4
+        route_token_impl<V, kGlobal, true>(t, E, k, norm_topk, logits, idx, w, keff, lane);
+    else
+        route_token_impl<V, kGlobal, false>(t, E, k, norm_topk, logits, idx, w, keff, lane);
 }
 
 // One token per thread, for E <= kLaneRouteMaxE: the same decisions as

@@ -4,8 +4,8 @@
 // shared expert.
 //
 // route_kernel<V>: one block per token; its first warp routes (route_token,
-// front.cuh) and its four warps compute the shared-expert gate
-// (shared_gate_group).  route_lane_kernel (E <= 64): separate blocks route
+// front.cuh) while the next four compute the shared-expert gate
+// (shared_gate_group), side by side.  route_lane_kernel (E <= 64): separate blocks route
 // 32 tokens lane by lane and compute the gates.  Both read the logits (and
 // x) once; they are latency-bound and small next to the expert FFN.
 #include "front.cuh"
@@ -14,7 +14,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kRouteThreads = kGateThreads;  // one token per block: warp 0 routes, all warps dot
+constexpr int kRouteThreads = 32 + kGateThreads;  // one token per block: warp 0 routes, warps 1.. dot
 
 template <int V>  // logits per lane: V * 32 >= E
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int k, int norm_topk,
@@ -29,10 +29,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int 
     pdl_wait();
     const int t = blockIdx.x;  // one token per block
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    if (wid == 0) route_token<V>(t, E, k, norm_topk, logits, idx, w, keff, lane);
+    if (wid == 0) {
+        route_token<V>(t, E, k, norm_topk, logits, idx, w, keff, lane);
+        return;
+    }
     if (sgate == nullptr) return;
-    const float g = shared_gate_group(t, x, gvec, H, part, 1, threadIdx.x);
-    if (threadIdx.x == 0) sgate[t] = g;
+    const int tid = threadIdx.x - 32;
+    const float g = shared_gate_group(t, x, gvec, H, part, 1, tid);
+    if (tid == 0) sgate[t] = g;
 }
 
 // E <= kLaneRouteMaxE: the first ceil(T / 32) blocks route 32 tokens each, one
@@ -40,7 +44,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int 
 // logits staged in shared memory; the remaining T blocks (with a shared
 // expert) compute one token's shared gate each.  Routing and gate blocks run
 // side by side instead of one after the other.
-__global__ void __launch_bounds__(kRouteThreads) route_lane_kernel(int T, int E, int k, int norm_topk,
+__global__ void __launch_bounds__(kGateThreads) route_lane_kernel(int T, int E, int k, int norm_topk,
                                                                    const float *__restrict__ logits,
                                                                    int32_t *__restrict__ idx, float *__restrict__ w,
                                                                    int32_t *__restrict__ keff,
@@ -85,7 +89,7 @@ cudaError_t launch_route(int T, int E, int k, int norm_topk, const float *logits
                          int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
                          cudaStream_t st) {
     if (E <= kLaneRouteMaxE)
-        return launch_pdl(route_lane_kernel, dim3((T + 31) / 32 + (sgate != nullptr ? T : 0)), dim3(kRouteThreads), 0,
+        return launch_pdl(route_lane_kernel, dim3((T + 31) / 32 + (sgate != nullptr ? T : 0)), dim3(kGateThreads), 0,
                           st, T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate);
     if (E <= 128) return launch_v<4>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
     if (E <= 256) return launch_v<8>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
