@@ -87,6 +87,7 @@ constexpr int kThreads = 192;
 constexpr int kPageBytes = 2048;               // ring unit: 16 token rows of 128 B
 constexpr int kAPages = kABytes / kPageBytes;  // 8 pages of weights per K step
 constexpr int kMaxStepPages = kAPages + 256 * 128 / kPageBytes;  // 24: weights + 256 token rows
+constexpr int kTwoSlicePages = 32;  // two K slices per ring step up to here, when the ring holds 4 slices
 constexpr int kMaxPages = 112;
 constexpr int kTickets = 32;                   // K steps in flight at most (barrier pairs)
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
@@ -518,8 +519,12 @@ __device__ __forceinline__ int box_index(int nvalid) {  // smallest box of 16 <<
 // Ring steps of an item.  A sub-step is one 64-wide K slice: 16 KB of
 // weights per weight tile of the item (m of them) followed by one token box
 // of 16 << bi rows (sub_pages pages).  A ring step carries ns sub-steps --
-// two while that is at most kMaxStepPages, so the per-step work of the
-// producer and MMA lanes is spent once per 32 KB of weights.
+// two while they take at most kMaxStepPages pages, or at most kTwoSlicePages
+// with room for two such steps in the ring -- so the per-step work of the
+// producer and MMA lanes (a barrier round trip each, some hundreds of cycles)
+// is spent once per 32 KB of weights.  Measured: wide tiles (a 256-token
+// tile of a CTA pair, 16 pages a slice) ran their K loop 15% faster with two
+// slices per step.
 // A CTA pair splits a tile's MMA N (the valid tokens rounded up to 16) in two
 // halves, one per CTA.
 __device__ __forceinline__ int pair_half(int nvalid) { return ((nvalid + 15) & ~15) >> 1; }
@@ -535,7 +540,8 @@ __device__ __forceinline__ StepShape step_shape(const Item &it, const FfnParams 
     StepShape sh;
     sh.bi = box_index(kPair ? pair_half(it.nvalid) : it.nvalid);
     sh.sub_pages = (uint32_t)it.m * kAPages + (1u << sh.bi);
-    sh.ns = 2 * sh.sub_pages <= (uint32_t)kMaxStepPages ? 2 : 1;
+    const uint32_t two = 2 * sh.sub_pages;
+    sh.ns = (two <= (uint32_t)kMaxStepPages || (two <= (uint32_t)kTwoSlicePages && 2 * two <= (uint32_t)p.pages)) ? 2 : 1;
     sh.nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
     return sh;
 }
@@ -676,7 +682,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             uint32_t vhead = 0, off = 0;       // ring pages handed out (virtual: never wraps) / its ring position
             uint32_t issued = 0, retired = 0;  // K steps issued / whose MMAs have released their pages
             uint32_t oldest = 0;               // first page (virtual) of step `retired` while one is in flight
-            const uint64_t wpol = policy_evict_first();  // expert weights: read once per launch
+            // expert weights: evict-first where a weight tile is read once (a group of
+            // one token tile).  A routed group of several token tiles reads each weight
+            // tile once per token tile, so its loads keep the normal policy and the
+            // repeats hit L2 (a 32-expert, 512-tokens-per-expert gate/up read 2.4
+            // instead of 3.7 GB from DRAM).
+            const uint64_t wpol = policy_evict_first();
             const uint64_t bpol = policy_evict_normal();  // token rows (pair loads take a policy)
             // items are claimed one ahead: a CTA (pair) takes item blockIdx (cluster
             // index) first, then from the counter, past the first grid's worth
@@ -748,6 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 const int a_row = it.ph == 0 ? (it.shared ? 0 : it.e * p.I) + rt * 64
                                              : (it.shared ? 0 : it.e * p.H) + rt * kTileM;
                 const int b_row = it.row0 + (kPair ? (int)rank * pair_half(it.nvalid) : 0);
+                const uint64_t apol = (it.ntt > 1 && !it.shared) ? bpol : wpol;
                 bool ok = true;
                 for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
                     const int nsub = min(sh.ns, sh.nk - k0);
@@ -777,10 +789,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                             uint8_t *sA = ring + (size_t)(first + j * sh.sub_pages) * kPageBytes;
                             const int kx = (k0 + j) * kBlockK;
                             if (it.ph == 0) {
-                                tma_load_2d_pair(ma0, bar0, sA, kx, a_row, wpol);
-                                tma_load_2d_pair(ma1, bar0, sA + kABytes / 2, kx, a_row, wpol);
+                                tma_load_2d_pair(ma0, bar0, sA, kx, a_row, apol);
+                                tma_load_2d_pair(ma1, bar0, sA + kABytes / 2, kx, a_row, apol);
                             } else {
-                                tma_load_2d_pair(ma0, bar0, sA, kx, a_row, wpol);
+                                tma_load_2d_pair(ma0, bar0, sA, kx, a_row, apol);
                             }
                             tma_load_2d_pair(mb, bar0, sA + kABytes, kx, b_row, bpol);
                         }
@@ -790,12 +802,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                             uint8_t *sA = ring + (size_t)(first + j * sh.sub_pages) * kPageBytes;
                             const int kx = (k0 + j) * kBlockK;
                             if (it.ph == 0) {
-                                tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
-                                tma_load_2d_hint(ma1, &full[tk], sA + kABytes / 2, kx, a_row, wpol);
+                                tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, apol);
+                                tma_load_2d_hint(ma1, &full[tk], sA + kABytes / 2, kx, a_row, apol);
                             } else {
-                                tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, wpol);
+                                tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, apol);
                                 if (it.m == 2)
-                                    tma_load_2d_hint(ma0, &full[tk], sA + kABytes, kx, a_row + kTileM, wpol);
+                                    tma_load_2d_hint(ma0, &full[tk], sA + kABytes, kx, a_row + kTileM, apol);
                             }
                             tma_load_2d(mb, &full[tk], sA + it.m * kABytes, kx, it.row0);
                         }
