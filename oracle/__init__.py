@@ -13,7 +13,8 @@ Each function follows a passage of the pages:
     softmax router with renormalised top-k, sigmoid-gated shared expert,
     grouped dispatch; its FFN parameter table fixes the gated FFN's shape.
   * colibri issue_budget.md (EXPERT_BUDGET), "How it works" steps 1-5 and
-    "Safety": the batch-union expert budget.
+    "Safety": the batch-union expert budget; "Relationship to existing
+    features": the per-position top-p trim (TOPP) that runs before it.
 """
 from __future__ import annotations
 
@@ -53,11 +54,12 @@ def _load():
     lib.oracle_ffn_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
     lib.oracle_route.argtypes = [i32, i32, i32, i32, P, P, P]
     lib.oracle_budget.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P]
+    lib.oracle_topp.argtypes = [i32, i32, i32, ctypes.c_float, P, P, P]
     lib.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, P, P, P]
     lib.oracle_expert_rows.argtypes = [i32, i32, P, P, P, i32, P, P, i32]
     lib.oracle_shared_gate_row.restype = ctypes.c_double
     lib.oracle_shared_gate_row.argtypes = [i32, P, P]
-    lib.oracle_forward.argtypes = [i32] * 8 + [P] * 9 + [i32, P, P] + [P] * 9 + [i32]  # pointer arrays pass as P
+    lib.oracle_forward.argtypes = [i32] * 8 + [ctypes.c_float] + [P] * 9 + [i32, P, P] + [P] * 9 + [i32]
     lib.oracle_combine_rows.argtypes = [i32] * 5 + [P] * 4 + [P] * 3 + [P] * 4 + [i32, P, P, i32]
     lib.oracle_max_threads.restype = ctypes.c_int
     _lib = lib
@@ -98,8 +100,22 @@ def route(logits: np.ndarray, k: int, norm_topk: bool = True):
     return idx, w
 
 
+def topp(idx: np.ndarray, w: np.ndarray, p: float, norm_topk: bool = True):
+    """Per-token top-p trim of the router output (copies; inputs untouched):
+    the shortest prefix of each token's slots whose weights reach p.
+
+    Returns (idx, w, keff [T])."""
+    idx = np.array(idx, np.int32, copy=True, order="C")
+    w = np.array(w, np.float32, copy=True, order="C")
+    T, k = idx.shape
+    keff = np.empty(max(T, 1), np.int32)
+    _check(_load().oracle_topp(T, k, int(bool(norm_topk)), float(p), _ptr(idx), _ptr(w), _ptr(keff)), "topp")
+    return idx, w, keff[:T]
+
+
 def budget(idx: np.ndarray, w: np.ndarray, E: int, N: int, norm_topk: bool = True):
     """EXPERT_BUDGET cap over the batch union (copies; inputs untouched).
+    Slots with idx -1 (a top-p trim's tail) take no part.
 
     Returns (idx, w, keff [T], kept [E] uint8, n_dropped)."""
     idx = np.array(idx, np.int32, copy=True, order="C")
@@ -183,8 +199,8 @@ def _expert_ptrs(w, E):
 
 
 def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, budget: int = 0,
-            ws_gate=None, ws_up=None, ws_down=None, ws_gvec=None, rows=None, nthreads: int = 1,
-            I: int = None) -> ForwardResult:
+            topp: float = 0.0, ws_gate=None, ws_up=None, ws_down=None, ws_gvec=None, rows=None,
+            nthreads: int = 1, I: int = None) -> ForwardResult:
     """The whole layer. x and all weights are bf16 bit patterns (uint16).
 
     x [T,H]; logits [T,E] f32; w_gate, w_up [E,I,H] and w_down [E,H,I] as full
@@ -220,7 +236,7 @@ def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, 
     perm = np.full(max(T * k, 1), -1, np.int32)
     slot_pos = np.empty(max(T * k, 1), np.int32)
     rc = _load().oracle_forward(
-        T, H, E, I, k, Is, int(bool(norm_topk)), budget,
+        T, H, E, I, k, Is, int(bool(norm_topk)), budget, float(topp),
         _ptr(x), _ptr(logits), pg, pu, pd,
         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec),
         n_rows, _ptr(rows), _ptr(out),

@@ -15,7 +15,10 @@
  *           gate, up and down projections).
  *  [BUDGET] colibri issue_budget.md "EXPERT_BUDGET", section "How it works"
  *           (steps 1-5 of the batch-union cap) and section "Safety"
- *           (dropped experts omitted, the rest renormalised; off by default).
+ *           (dropped experts omitted, the rest renormalised; off by default);
+ *           section "Relationship to existing features" (TOPP trims each
+ *           position to its top-p mass within its top-K, before the budget
+ *           caps the union; the trimmed state is keff < K, as the budget's).
  *
  * Precision.  Routing weights, the budget's aggregate weights and every
  * quantity that decides an integer (which expert is kept) are computed in
@@ -31,6 +34,9 @@
  *  - budget ties: equal aggregate weight -> the lower expert id is kept;
  *  - budget aggregate: summed over tokens ascending, then slots ascending;
  *  - only tokens that lost a slot are renormalised;
+ *  - top-p: the shortest prefix of a token's slots whose weights (after the
+ *    norm_topk renormalisation, summed in slot order) reach topp; topp <= 0
+ *    or >= 1 is off;
  *  - dispatch order inside an expert: slot id t*k+j ascending;
  *  - the shared-expert gate is a per-token scalar sigmoid(g . x_t).
  */
@@ -107,15 +113,55 @@ int oracle_route(int32_t T, int32_t E, int32_t k, int32_t norm_topk,
 }
 
 /* ---------------------------------------------------------------------- */
+/* Top-p trim ([BUDGET] "Relationship to existing features": TOPP trims     */
+/* within one position's top-K; the two compose, TOPP first).              */
+/* ---------------------------------------------------------------------- */
+/* For each token t of the router output (slots in descending-logit order,
+ * weights after the norm_topk renormalisation):
+ *   1. slot 0 is kept; slot j > 0 is kept while the weights of slots
+ *      0..j-1, added in slot order in fp32, are still below topp -- the
+ *      shortest prefix whose mass reaches topp;
+ *   2. the dropped tail becomes (idx -1, w 0) and keff[t] = kept slots;
+ *   3. if norm_topk and a slot was dropped, the kept weights are divided by
+ *      their sum (slot order, fp32), as the budget renormalises.
+ * topp <= 0 (the default) or topp >= 1: no change, keff[t] = k. */
+int oracle_topp(int32_t T, int32_t k, int32_t norm_topk, float topp, int32_t *idx, float *w, int32_t *keff)
+{
+    if (T < 0 || k < 1 || topp != topp) return ORACLE_EINVAL;
+    for (int32_t t = 0; t < T; ++t) {
+        int32_t *ti = idx + (size_t)t * k;
+        float *tw = w + (size_t)t * k;
+        int32_t c = k;
+        if (topp > 0.0f && topp < 1.0f) {
+            float mass = 0.0f; /* weights of the slots before j */
+            for (int32_t j = 0; j < k; ++j) {
+                if (j > 0 && mass >= topp) { c = j; break; }
+                mass += tw[j];
+            }
+            for (int32_t j = c; j < k; ++j) { ti[j] = -1; tw[j] = 0.0f; }
+            if (norm_topk && c < k) {
+                float s = 0.0f;
+                for (int32_t j = 0; j < c; ++j) s += tw[j];
+                for (int32_t j = 0; j < c; ++j) tw[j] = tw[j] / s;
+            }
+        }
+        keff[t] = c;
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------- */
 /* Budget ([BUDGET] "How it works", steps 1-5; "Safety").                  */
 /* ---------------------------------------------------------------------- */
-/* Input: the router output idx/w [T, k] (every token holds k slots).
+/* Input: the router output idx/w [T, k], possibly trimmed by top-p (a
+ * token's valid slots first, then idx = -1).
  * Output, in place: idx/w with each token's surviving slots first (original
  * order kept), the tail filled with idx = -1, w = 0; keff[t] = surviving
  * slots; kept[e] = 1 for experts of the (possibly capped) batch union;
  * *n_dropped = number of distinct experts dropped.
  * N <= 0, or a union no larger than N, changes nothing ("default off";
- * the cap applies only when the union exceeds the budget). */
+ * the cap applies only when the union exceeds the budget): keff[t] = the
+ * token's valid slots. */
 typedef struct { float agg; int32_t id; } agg_entry;
 
 static int agg_cmp(const void *a, const void *b)
@@ -130,12 +176,17 @@ int oracle_budget(int32_t T, int32_t E, int32_t k, int32_t N, int32_t norm_topk,
                   int32_t *idx, float *w, int32_t *keff, uint8_t *kept, int32_t *n_dropped)
 {
     if (T < 0 || E < 1 || k < 1 || k > E || N < 0) return ORACLE_EINVAL;
-    /* the batch union uniq[0..nu) */
+    /* the batch union uniq[0..nu) over the valid slots */
     memset(kept, 0, (size_t)E);
-    for (size_t s = 0; s < (size_t)T * k; ++s) kept[idx[s]] = 1;
+    for (size_t s = 0; s < (size_t)T * k; ++s)
+        if (idx[s] >= 0) kept[idx[s]] = 1;
     int32_t nu = 0;
     for (int32_t e = 0; e < E; ++e) nu += kept[e];
-    for (int32_t t = 0; t < T; ++t) keff[t] = k;
+    for (int32_t t = 0; t < T; ++t) {
+        int32_t v = 0;
+        for (int32_t j = 0; j < k; ++j) v += idx[(size_t)t * k + j] >= 0;
+        keff[t] = v;
+    }
     *n_dropped = 0;
     if (N == 0 || nu <= N) return ORACLE_OK;
 
@@ -145,7 +196,7 @@ int oracle_budget(int32_t T, int32_t E, int32_t k, int32_t N, int32_t norm_topk,
     if (!agg || !order) { free(agg); free(order); return ORACLE_ENOMEM; }
     for (int32_t t = 0; t < T; ++t)
         for (int32_t j = 0; j < k; ++j)
-            agg[idx[(size_t)t * k + j]] += w[(size_t)t * k + j];
+            if (idx[(size_t)t * k + j] >= 0) agg[idx[(size_t)t * k + j]] += w[(size_t)t * k + j];
     /* step 2: sort the union by aggregate weight, descending */
     int32_t n = 0;
     for (int32_t e = 0; e < E; ++e)
@@ -154,15 +205,16 @@ int oracle_budget(int32_t T, int32_t E, int32_t k, int32_t N, int32_t norm_topk,
     /* step 3: keep the first N, mark the rest dropped */
     memset(kept, 0, (size_t)E);
     for (int32_t r = 0; r < N; ++r) kept[order[r].id] = 1;
-    /* step 4: remove dropped experts from each token's list, renormalise */
+    /* step 4: remove dropped experts from each token's list, renormalise the
+     * tokens that lost a slot (keff[t] holds the valid slots before) */
     for (int32_t t = 0; t < T; ++t) {
         int32_t *ti = idx + (size_t)t * k;
         float *tw = w + (size_t)t * k;
         int32_t c = 0;
         for (int32_t j = 0; j < k; ++j)
-            if (kept[ti[j]]) { ti[c] = ti[j]; tw[c] = tw[j]; ++c; }
+            if (ti[j] >= 0 && kept[ti[j]]) { ti[c] = ti[j]; tw[c] = tw[j]; ++c; }
         for (int32_t j = c; j < k; ++j) { ti[j] = -1; tw[j] = 0.0f; }
-        if (norm_topk && c > 0 && c < k) {
+        if (norm_topk && c > 0 && c < keff[t]) {
             float s = 0.0f;
             for (int32_t j = 0; j < c; ++j) s += tw[j];
             for (int32_t j = 0; j < c; ++j) tw[j] = tw[j] / s;
@@ -343,11 +395,11 @@ int oracle_combine_rows(int32_t T, int32_t H, int32_t I, int32_t k, int32_t Is,
 }
 
 /* ---------------------------------------------------------------------- */
-/* Whole layer: route -> budget -> dispatch over all T tokens (the budget  */
-/* couples tokens), then FFN + combine for the listed rows.                */
+/* Whole layer: route -> top-p -> budget -> dispatch over all T tokens    */
+/* (the budget couples tokens), then FFN + combine for the listed rows.    */
 /* ---------------------------------------------------------------------- */
 int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_t Is,
-                   int32_t norm_topk, int32_t budget,
+                   int32_t norm_topk, int32_t budget, float topp,
                    const uint16_t *x, const float *logits,
                    const uint16_t *const *w_gate, const uint16_t *const *w_up,
                    const uint16_t *const *w_down,
@@ -361,6 +413,8 @@ int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_
     if (T < 0 || H < 1 || E < 1 || I < 1 || k < 1 || k > E || Is < 0 || budget < 0 || n_rows < 0)
         return ORACLE_EINVAL;
     int rc = oracle_route(T, E, k, norm_topk, logits, idx, w);
+    if (rc) return rc;
+    rc = oracle_topp(T, k, norm_topk, topp, idx, w, keff);
     if (rc) return rc;
     rc = oracle_budget(T, E, k, budget, norm_topk, idx, w, keff, kept, n_dropped);
     if (rc) return rc;

@@ -38,8 +38,15 @@ MUTANTS = {
                                   "agg[idx[(size_t)t * k + j]] += 1.0f;"),
     "budget_tie_higher_id": ("return (x->id < y->id) ? -1 : (x->id > y->id); /* equal -> lower id first */",
                              "return (x->id > y->id) ? -1 : (x->id < y->id);"),
-    "budget_no_renorm": ("if (norm_topk && c > 0 && c < k) {", "if (norm_topk && c > 0 && c < 0) {"),
-    "budget_renorm_all": ("if (norm_topk && c > 0 && c < k) {", "if (norm_topk && c > 0 && c <= k) {"),
+    "budget_no_renorm": ("if (norm_topk && c > 0 && c < keff[t]) {", "if (norm_topk && c > 0 && c < 0) {"),
+    "budget_renorm_all": ("if (norm_topk && c > 0 && c < keff[t]) {", "if (norm_topk && c > 0 && c <= k) {"),
+    "budget_renorm_by_k": ("if (norm_topk && c > 0 && c < keff[t]) {", "if (norm_topk && c > 0 && c < k) {"),
+    "topp_strict": ("if (j > 0 && mass >= topp) { c = j; break; }", "if (j > 0 && mass > topp) { c = j; break; }"),
+    "topp_drops_crossing_slot": ("                if (j > 0 && mass >= topp) { c = j; break; }\n                mass += tw[j];",
+                                 "                mass += tw[j];\n                if (j > 0 && mass >= topp) { c = j; break; }"),
+    "topp_no_renorm": ("if (norm_topk && c < k) {", "if (norm_topk && c < 0) {"),
+    "forward_skips_topp": ("rc = oracle_topp(T, k, norm_topk, topp, idx, w, keff);",
+                           "rc = oracle_topp(T, k, norm_topk, 0.0f, idx, w, keff);"),
     "budget_off_by_one": ("if (N == 0 || nu <= N) return ORACLE_OK;", "if (N == 0 || nu <= N + 1) return ORACLE_OK;"),
     "dispatch_tokens_descending": ("        for (int32_t t = 0; t < T; ++t)\n            for (int32_t j = 0; j < keff[t]; ++j)\n                if (idx[(size_t)t * k + j] == e) {",
                                    "        for (int32_t t = T - 1; t >= 0; --t)\n            for (int32_t j = 0; j < keff[t]; ++j)\n                if (idx[(size_t)t * k + j] == e) {"),
@@ -60,6 +67,10 @@ PINS = [
     ("test_budget_brute_force_keeps_heaviest_subset", dict(seed=0)),
     ("test_budget_invariants", dict(norm=True)),
     ("test_budget_drops_can_empty_tokens", {}),
+    ("test_topp_worked_example", {}),
+    ("test_topp_invariants", dict(norm=True)),
+    ("test_topp_then_budget_composition", {}),
+    ("test_forward_routes_topp_then_budget", dict(N=4, p=0.8)),
     ("test_dispatch_matches_stable_sort", dict(T=33, E=16, k=4, N=5)),
     ("test_ffn_closed_form_unit_vectors", {}),
     ("test_ffn_single_expert_is_plain_swiglu_mlp", {}),

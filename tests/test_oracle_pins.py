@@ -142,6 +142,88 @@ def test_budget_worked_example(oracle_mod):
     assert perm.tolist() == d["perm"] and slot_pos.tolist() == d["slot_pos"]
 
 
+# ----------------------------------------------------------------- top-p --
+
+def test_topp_worked_example(oracle_mod):
+    g = _gold("topp_worked_example.json")
+    idx = np.array(g["idx"], np.int32)
+    w = np.array(g["w"], np.float32)
+    for case in g["cases"]:
+        for norm, key in ((True, "expect_norm"), (False, "expect_no_norm")):
+            if key not in case:
+                continue
+            ex = case[key]
+            i2, w2, keff = oracle_mod.topp(idx, w, case["topp"], norm_topk=norm)
+            assert i2.tolist() == ex["idx"], (case["topp"], norm)
+            assert w2.tolist() == ex["w"], (case["topp"], norm)
+            assert keff.tolist() == ex["keff"], (case["topp"], norm)
+    b = g["with_budget"]
+    i2, w2, keff = oracle_mod.topp(idx, w, b["topp"], norm_topk=True)
+    i3, w3, keff3, kept, nd = oracle_mod.budget(i2, w2, g["E"], b["N"], norm_topk=True)
+    ex = b["expect"]
+    assert i3.tolist() == ex["idx"] and w3.tolist() == ex["w"] and keff3.tolist() == ex["keff"]
+    assert kept.tolist() == ex["kept"] and nd == ex["n_dropped"]
+
+
+@pytest.mark.parametrize("norm", [True, False])
+def test_topp_invariants(oracle_mod, norm):
+    T, E, k = 64, 64, 8
+    rng = np.random.default_rng(11)
+    idx, w = oracle_mod.route((rng.standard_normal((T, E)) * 1.5).astype(np.float32), k, norm_topk=norm)
+    for p in (0.0, 1.0, 1.5, -0.25):  # off: unchanged, bit for bit
+        i2, w2, keff = oracle_mod.topp(idx, w, p, norm_topk=norm)
+        assert (i2 == idx).all() and (w2.view(np.uint32) == w.view(np.uint32)).all() and (keff == k).all()
+    for p in (1e-6, 0.3, 0.5, 0.8, 0.95):
+        i2, w2, keff = oracle_mod.topp(idx, w, p, norm_topk=norm)
+        for t in range(T):
+            c = int(keff[t])
+            assert 1 <= c <= k
+            # the mass before the last kept slot is below p, the kept mass reaches p (fp32, slot order)
+            mass = [np.float32(0.0)]
+            for j in range(k):
+                mass.append(np.float32(mass[-1] + w[t, j]))
+            assert c == 1 or mass[c - 1] < np.float32(p)
+            assert c == k or mass[c] >= np.float32(p)
+            assert i2[t, :c].tolist() == idx[t, :c].tolist()
+            assert (i2[t, c:] == -1).all() and (w2[t, c:] == 0).all()
+            if c == k or not norm:
+                assert (w2[t, :c].view(np.uint32) == w[t, :c].view(np.uint32)).all()
+            else:
+                s = np.float32(0.0)
+                for j in range(c):
+                    s = np.float32(s + w[t, j])
+                assert (w2[t, :c] == (w[t, :c] / s).astype(np.float32)).all()
+        if p == 1e-6:
+            assert (keff == 1).all()
+            if norm:
+                assert (w2[:, 0] == 1.0).all()
+
+
+def test_topp_then_budget_composition(oracle_mod):
+    """The budget after a top-p trim: trimmed slots take no part, and a token
+    the budget leaves whole keeps its post-trim weights bit for bit."""
+    T, E, k = 40, 48, 6
+    rng = np.random.default_rng(17)
+    idx, w = oracle_mod.route((rng.standard_normal((T, E)) - 0.8 * np.log1p(np.arange(E))).astype(np.float32), k)
+    i1, w1, keff1 = oracle_mod.topp(idx, w, 0.7)
+    union = sorted(set(i1[i1 >= 0].tolist()))
+    i_off, w_off, keff_off, kept_off, nd_off = oracle_mod.budget(i1, w1, E, 0)
+    assert (i_off == i1).all() and (w_off.view(np.uint32) == w1.view(np.uint32)).all()
+    assert keff_off.tolist() == keff1.tolist() and nd_off == 0
+    assert sorted(np.nonzero(kept_off)[0].tolist()) == union
+    N = len(union) // 2
+    i2, w2, keff2, kept, nd = oracle_mod.budget(i1, w1, E, N)
+    assert nd == len(union) - N and int(kept.sum()) == N
+    whole = 0
+    for t in range(T):
+        surv = [j for j in range(keff1[t]) if kept[i1[t, j]]]
+        assert keff2[t] == len(surv) and i2[t, :len(surv)].tolist() == [int(i1[t, j]) for j in surv]
+        if len(surv) == keff1[t]:
+            whole += 1
+            assert (w2[t, :keff1[t]].view(np.uint32) == w1[t, :keff1[t]].view(np.uint32)).all()
+    assert whole > 0
+
+
 def _route_for_budget(oracle_mod, T, E, k, seed, alpha=0.0):
     rng = np.random.default_rng(seed)
     logits = rng.standard_normal((T, E)).astype(np.float32)
@@ -300,6 +382,30 @@ def test_forward_dense_masked_loop(oracle_mod, N, norm):
         s = torch.sigmoid(torch.dot(inp.ws_gvec.double(), x[t]))
         out[t] += s * F.linear(F.silu(F.linear(x[t], inp.ws_gate.double())) * F.linear(x[t], inp.ws_up.double()),
                                inp.ws_down.double())
+    np.testing.assert_allclose(r.out, out.numpy(), rtol=1e-9, atol=1e-13)
+
+
+@pytest.mark.parametrize("N,p", [(0, 0.6), (4, 0.8), (3, 0.0)])
+def test_forward_routes_topp_then_budget(oracle_mod, N, p):
+    """forward() applies the top-p trim before the budget, and its dense
+    output follows the resulting routing."""
+    cfg = W.MoEConfig("dense", T=12, H=64, E=6, I=32, k=3, norm_topk=True, budget=N, zipf_alpha=0.5)
+    inp = W.make_inputs(cfg, std=0.2)
+    r = oracle_mod.forward(bits(inp.x), inp.logits.numpy(), bits(inp.w_gate), bits(inp.w_up), bits(inp.w_down),
+                           k=3, budget=N, topp=p)
+    idx, w = oracle_mod.route(inp.logits.numpy(), 3)
+    i1, w1, _ = oracle_mod.topp(idx, w, p)
+    i2, w2, keff, kept, nd = oracle_mod.budget(i1, w1, cfg.E, N)
+    assert (r.idx == i2).all() and (r.w.view(np.uint32) == w2.view(np.uint32)).all()
+    assert (r.keff == keff).all() and r.n_dropped == nd
+    x = inp.x.double()
+    out = torch.zeros((cfg.T, cfg.H), dtype=torch.float64)
+    for t in range(cfg.T):
+        for j in range(int(keff[t])):
+            e = int(i2[t, j])
+            y = F.linear(F.silu(F.linear(x[t], inp.w_gate[e].double())) * F.linear(x[t], inp.w_up[e].double()),
+                         inp.w_down[e].double())
+            out[t] += float(w2[t, j]) * y
     np.testing.assert_allclose(r.out, out.numpy(), rtol=1e-9, atol=1e-13)
 
 
