@@ -54,13 +54,16 @@ def workload_from_args(args):
         kw["zipf_alpha"] = args.alpha
     if args.budget is not None:
         kw["budget"] = args.budget
+    if args.topp is not None:
+        kw["topp"] = args.topp
     return cfg.with_(**kw) if kw else cfg
 
 
 def workload_desc(cfg) -> dict:
     d = {"workload": cfg.label, "tokens": cfg.T, "hidden": cfg.H, "n_routed_experts": cfg.E,
          "moe_intermediate_size": cfg.I, "num_experts_per_tok": cfg.k, "shared_intermediate_size": cfg.Is,
-         "norm_topk": cfg.norm_topk, "budget": cfg.budget, "zipf_alpha": cfg.zipf_alpha, "seed": cfg.seed,
+         "norm_topk": cfg.norm_topk, "budget": cfg.budget, "topp": cfg.topp, "zipf_alpha": cfg.zipf_alpha,
+         "seed": cfg.seed,
          "l2": "flushed between timed steps (256 MB write, outside the timed events)"}
     return d
 
@@ -272,7 +275,7 @@ def oracle_rows_per_s(cfg, inp_host, target_s: float, max_rows: int):
 
     def run(nrows):
         t0 = time.perf_counter()
-        oracle.forward(x, logits, wg, wu, wd, k=cfg.k, norm_topk=cfg.norm_topk, budget=cfg.budget,
+        oracle.forward(x, logits, wg, wu, wd, k=cfg.k, norm_topk=cfg.norm_topk, budget=cfg.budget, topp=cfg.topp,
                        rows=order[:nrows], nthreads=nthreads, I=cfg.I, **shared)
         return time.perf_counter() - t0
 
@@ -328,7 +331,7 @@ def run_ours(args, cfg):
     lib = moe.load_library()
 
     inp = W.make_inputs(cfg, device=dev)
-    c = moe.MoEConfig(cfg.H, cfg.E, cfg.I, cfg.k, cfg.Is, cfg.norm_topk, cfg.budget)
+    c = moe.MoEConfig(cfg.H, cfg.E, cfg.I, cfg.k, cfg.Is, cfg.norm_topk, cfg.budget, cfg.topp)
     T, k, E, H = cfg.T, cfg.k, cfg.E, cfg.H
     ws = torch.zeros(moe.workspace_bytes(c, T), dtype=torch.uint8, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
@@ -589,7 +592,7 @@ def run_reference(args, cfg):
     rows = sample_order(cfg.T)[:nrows]
 
     def one():
-        oracle.forward(x, logits, wg, wu, wd, k=cfg.k, norm_topk=cfg.norm_topk, budget=cfg.budget, rows=rows,
+        oracle.forward(x, logits, wg, wu, wd, k=cfg.k, norm_topk=cfg.norm_topk, budget=cfg.budget, topp=cfg.topp, rows=rows,
                        nthreads=thr, I=cfg.I, **shared)
 
     for _ in range(args.warmup):
@@ -621,6 +624,7 @@ def main(argv=None):
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--topp", type=float, default=None, help="per-token top-p trim (0 = off)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

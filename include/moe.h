@@ -5,6 +5,8 @@
  *   route    softmax over the E router logits of each token, the k largest
  *            logits kept, their probabilities renormalised to sum 1 when
  *            norm_topk is set;
+ *   top-p    optional per-token trim: each token keeps the shortest prefix
+ *            of its k slots whose weights reach topp (renormalised);
  *   budget   optional cap N on the number of distinct experts the whole
  *            batch uses: when the batch union holds more than N experts,
  *            only the N with the highest aggregate gate weight survive and
@@ -22,7 +24,9 @@
  *     its FFN parameter table (3*H*I parameters per expert).
  *   colibri issue_budget.md, "EXPERT_BUDGET", section "How it works", steps
  *     1-5 (the budget) and section "Safety" (off by default, dropped experts
- *     omitted and the rest renormalised).
+ *     omitted and the rest renormalised); section "Relationship to existing
+ *     features" (TOPP trims each position's top-K to its top-p mass, and
+ *     composes with the budget, TOPP first).
  *
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers owned by the caller, 16-byte
@@ -37,7 +41,7 @@
  *     launched when an argument check fails.
  *   - Limits: 1 <= E <= 1024; 1 <= k <= min(E, 32); H % 128 == 0;
  *     I % 64 == 0; Is % 64 == 0 (Is = 0: no shared expert); budget >= 0;
- *     0 <= T and T * (k + 1) * H < 2^31.
+ *     topp finite and >= 0; 0 <= T and T * (k + 1) * H < 2^31.
  */
 #ifndef MOE_B200_MOE_H
 #define MOE_B200_MOE_H
@@ -69,6 +73,7 @@ typedef struct {
     int32_t shared_intermediate_size; /* Is; 0 = no shared expert */
     int32_t norm_topk;                /* 1: renormalise the kept weights to sum 1 */
     int32_t budget;                   /* N (EXPERT_BUDGET); 0 = off */
+    float topp;                       /* per-token top-p mass (TOPP); 0 (or >= 1) = off */
 } moe_config_t;
 
 typedef struct {
@@ -107,9 +112,13 @@ size_t moe_workspace_bytes(const moe_config_t *cfg, int32_t T);
 /* Route: for each token t, topk_idx[t, 0..k) = the k experts with the
  * largest logits (descending; equal logits: lower expert id first),
  * topk_w[t, j] = softmax(logits[t])[topk_idx[t, j]], divided by the sum of
- * the k kept probabilities when cfg->norm_topk.  When sgate != NULL (needs
- * Is > 0, x and ws_gate_vec), sgate[t] = sigmoid(ws_gate_vec . x_t).  When
- * keff != NULL, keff[t] = k.
+ * the k kept probabilities when cfg->norm_topk.  With 0 < cfg->topp < 1 the
+ * top-p trim follows: slot 0 stays, slot j > 0 stays while the weights of
+ * slots 0..j-1 (added in slot order, fp32) are below topp; the rest become
+ * (idx -1, w 0), and with norm_topk the kept weights are divided by their
+ * sum (slot order).  When sgate != NULL (needs Is > 0, x and ws_gate_vec),
+ * sgate[t] = sigmoid(ws_gate_vec . x_t).  keff[t] = the kept slots (k
+ * without the trim); keff may be NULL only when the trim is off.
  *   logits [T, E] f32; x [T, H]; ws_gate_vec [H]; topk_idx [T, k] i32;
  *   topk_w [T, k] f32; sgate [T] f32; keff [T] i32. */
 int moe_route(const moe_config_t *cfg, int32_t T, const float *logits, const moe_bf16_t *x,
@@ -117,14 +126,15 @@ int moe_route(const moe_config_t *cfg, int32_t T, const float *logits, const moe
               int32_t *keff, void *stream);
 
 /* Budget (EXPERT_BUDGET, colibri issue_budget.md "How it works"): works in
- * place on the router output topk_idx/topk_w [T, k].  Let U be the set of
- * experts any token routes to.  When cfg->budget > 0 and |U| > budget:
- * agg[e] = sum of the weights routed to e (tokens, then slots, ascending);
- * the budget experts first in (agg descending, id ascending) are kept;
- * every token's kept slots move to the front in their original order, the
- * tail becomes (idx -1, w 0), keff[t] = kept slots, and a token that lost a
- * slot has its kept weights divided by their sum when cfg->norm_topk.
- * Otherwise topk_idx/topk_w are unchanged and keff[t] = k.
+ * place on the router output topk_idx/topk_w [T, k]; slots with idx -1 (a
+ * top-p trim's tail) take no part.  Let U be the set of experts any token
+ * routes to.  When cfg->budget > 0 and |U| > budget: agg[e] = sum of the
+ * weights routed to e (tokens, then slots, ascending); the budget experts
+ * first in (agg descending, id ascending) are kept; every token's kept slots
+ * move to the front in their original order, the tail becomes (idx -1, w 0),
+ * keff[t] = kept slots, and a token that lost a slot has its kept weights
+ * divided by their sum when cfg->norm_topk.  Otherwise topk_idx/topk_w are
+ * unchanged and keff[t] = the token's valid slots (k without a trim).
  * expert_kept[e] = 1 for experts of the final union; *n_dropped = |U| -
  * budget or 0.  keff [T] i32; expert_kept [E] u8; n_dropped [1] i32 (all
  * device).  Uses the workspace. */

@@ -50,7 +50,7 @@ class MoEError(RuntimeError):
 class _Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "hidden", "n_routed_experts", "moe_intermediate_size", "num_experts_per_tok",
-        "shared_intermediate_size", "norm_topk", "budget")]
+        "shared_intermediate_size", "norm_topk", "budget")] + [("topp", ctypes.c_float)]
 
 
 class _Weights(ctypes.Structure):
@@ -74,10 +74,11 @@ class MoEConfig:
     shared_intermediate_size: int = 0
     norm_topk: bool = True
     budget: int = 0
+    topp: float = 0.0  # per-token top-p trim; 0 (or >= 1) = off
 
     def _c(self) -> _Config:
         return _Config(self.hidden, self.n_routed_experts, self.moe_intermediate_size, self.num_experts_per_tok,
-                       self.shared_intermediate_size, int(bool(self.norm_topk)), self.budget)
+                       self.shared_intermediate_size, int(bool(self.norm_topk)), self.budget, float(self.topp))
 
 
 @dataclass

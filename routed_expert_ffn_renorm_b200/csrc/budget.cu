@@ -13,7 +13,8 @@
 // union is every expert with a routed slot, each union expert's rank is the
 // number of union experts ahead of it in (agg descending, id ascending),
 // the first N are kept; then one thread per token compacts its slots in
-// order and renormalises when it lost one.
+// order and renormalises when it lost one.  Slots with idx -1 (dropped by a
+// top-p trim) take no part; keff counts a token's valid slots.
 // Every sum has a fixed order, so the result is deterministic; the
 // two-kernel path rounds the aggregates chunk by chunk.
 #include <atomic>
@@ -138,8 +139,11 @@ __global__ void __launch_bounds__(1024) budget_select_kernel(int T, int E, int k
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
         int32_t *ti = idx + (size_t)t * k;
         float *tw = w + (size_t)t * k;
-        int c = 0;
+        int valid = 0;  // slots a top-p trim left (all k without one)
+        for (int j = 0; j < k; ++j) valid += ti[j] >= 0;
+        int c = valid;
         if (active) {
+            c = 0;
             for (int j = 0; j < k; ++j) {
                 const int e = ti[j];
                 if (e >= 0 && e < E && keep[e]) {
@@ -153,13 +157,11 @@ __global__ void __launch_bounds__(1024) budget_select_kernel(int T, int E, int k
                 ti[j] = -1;
                 tw[j] = 0.f;
             }
-            if (norm_topk && c > 0 && c < k) {
+            if (norm_topk && c > 0 && c < valid) {
                 float s = 0.f;
                 for (int j = 0; j < c; ++j) s += tw[j];
                 for (int j = 0; j < c; ++j) tw[j] = tw[j] / s;
             }
-        } else {
-            c = k;
         }
         keff[t] = c;
     }

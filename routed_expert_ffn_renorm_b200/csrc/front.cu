@@ -28,6 +28,7 @@ constexpr int kFrontGroups = kFrontThreads / kGateThreads;  // shared-gate group
 
 struct FrontArgs {
     int T, E, k, N, norm_topk, H;
+    float topp;
     const float *logits;
     const uint16_t *x, *gvec;
     int32_t *idx;
@@ -95,14 +96,12 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_small_kernel(const Fro
     }
     __syncthreads();
     if (lane_route) {
-        for (int t = threadIdx.x; t < T; t += kFrontThreads) {
-            route_token_lane<false>(t, E, k, a.norm_topk, logit_s + (size_t)t * ls, idx_s, w_s);
-            keff_s[t] = k;
-        }
+        for (int t = threadIdx.x; t < T; t += kFrontThreads)
+            keff_s[t] = route_token_lane<false>(t, E, k, a.norm_topk, a.topp, logit_s + (size_t)t * ls, idx_s, w_s);
     } else {
         for (int t = warp; t < T; t += kFrontThreads / 32) {
-            route_token<V, false>(t, E, k, a.norm_topk, logit_s, idx_s, w_s, nullptr, lane);
-            if (lane == 0) keff_s[t] = k;
+            const int c = route_token<V, false>(t, E, k, a.norm_topk, a.topp, logit_s, idx_s, w_s, nullptr, lane);
+            if (lane == 0) keff_s[t] = c;
         }
     }
     __syncthreads();
@@ -204,11 +203,12 @@ bool front_fits(int T, int E, int k) {
            front_smem(T, E, k) <= (size_t)kFrontSmemMax;
 }
 
-cudaError_t launch_front(int T, int E, int k, int N, int norm_topk, int H, const float *logits, const uint16_t *x,
+cudaError_t launch_front(int T, int E, int k, int N, int norm_topk, float topp, int H, const float *logits,
+                         const uint16_t *x,
                          const uint16_t *gvec, int32_t *idx, float *w, float *sgate, int32_t *keff, uint8_t *kept,
                          int32_t *n_dropped, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
                          uint16_t *x_perm, int32_t *status_block, int32_t *hdone, cudaStream_t st) {
-    FrontArgs a{T, E, k, N, norm_topk, H, logits, x, gvec, idx, w, sgate, keff, kept, n_dropped,
+    FrontArgs a{T, E, k, N, norm_topk, H, topp, logits, x, gvec, idx, w, sgate, keff, kept, n_dropped,
                 counts, offsets, perm, slot_pos, x_perm, status_block, hdone};
     if (E <= 128) return launch_v<4>(a, st);  // E <= 64 routes lane by lane
     if (E <= 256) return launch_v<8>(a, st);

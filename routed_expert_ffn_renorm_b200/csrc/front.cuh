@@ -26,7 +26,14 @@ namespace moe {
 // The winner's lane clears its key; lane j keeps the j-th winner and its key.
 // The logits come from global memory (kGlobal, read-only path) or from
 // shared memory; idx / w may point to global or shared memory; keff (may be
-// null) receives k.
+// null) receives the kept slot count, which the function also returns.
+//
+// Top-p trim (colibri issue_budget.md, "Relationship to existing features":
+// TOPP trims a position's top-K to its top-p mass, before the budget), for
+// 0 < topp < 1: slot 0 stays; slot j > 0 stays while the weights of slots
+// 0..j-1 (after the norm_topk renormalisation), added in slot order, are
+// below topp.  The dropped tail becomes (idx -1, w 0), and with norm_topk
+// the kept weights are divided by their sum in slot order.
 __device__ __forceinline__ uint32_t float_order_key(float v) {
     const uint32_t b = v == 0.f ? 0u : __float_as_uint(v);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
@@ -36,8 +43,9 @@ __device__ __forceinline__ float order_key_float(uint32_t key) {
 }
 
 template <int V, bool kGlobal, bool kVec>
-__device__ __forceinline__ void route_token_impl(int t, int E, int k, int norm_topk, const float *__restrict__ logits,
-                                                 int32_t *idx, float *w, int32_t *keff, int lane) {
+__device__ __forceinline__ int route_token_impl(int t, int E, int k, int norm_topk, float topp,
+                                                const float *__restrict__ logits, int32_t *idx, float *w,
+                                                int32_t *keff, int lane) {
     const float *l = logits + (size_t)t * E;
     // expert of slot i of this lane
     auto expert = [&](int i) { return kVec ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i; };
@@ -117,34 +125,53 @@ __device__ __forceinline__ void route_token_impl(int t, int E, int k, int norm_t
         for (int j = 0; j < k; ++j) ps += __shfl_sync(0xffffffffu, p, j);
         p = p / ps;
     }
-    if (lane < k) {
-        idx[(size_t)t * k + lane] = my_idx;
-        w[(size_t)t * k + lane] = p;
+    int c = k;  // kept slots
+    if (topp > 0.f && topp < 1.f) {
+        float mass = 0.f;  // the same in every lane
+        for (int j = 0; j < k; ++j) {
+            const float pj = __shfl_sync(0xffffffffu, p, j);
+            if (j > 0 && mass >= topp) {
+                c = j;
+                break;
+            }
+            mass += pj;
+        }
+        if (norm_topk && c < k) {
+            float s2 = 0.f;
+            for (int j = 0; j < c; ++j) s2 += __shfl_sync(0xffffffffu, p, j);
+            p = p / s2;
+        }
     }
-    if (keff != nullptr && lane == 0) keff[t] = k;
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = lane < c ? my_idx : -1;
+        w[(size_t)t * k + lane] = lane < c ? p : 0.f;
+    }
+    if (keff != nullptr && lane == 0) keff[t] = c;
+    return c;
 }
 
 template <int V, bool kGlobal = true>  // logits per lane: V * 32 >= E, V a power of two >= 4
-__device__ __forceinline__ void route_token(int t, int E, int k, int norm_topk, const float *__restrict__ logits,
-                                            int32_t *idx, float *w, int32_t *keff, int lane) {
+__device__ __forceinline__ int route_token(int t, int E, int k, int norm_topk, float topp,
+                                           const float *__restrict__ logits, int32_t *idx, float *w, int32_t *keff,
+                                           int lane) {
     static_assert(V >= 4 && (V & (V - 1)) == 0, "V: a power of two >= 4");
     if (V >= 8 && (E & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0)  // measured: no gain at V = 4
-        route_token_impl<V, kGlobal, true>(t, E, k, norm_topk, logits, idx, w, keff, lane);
-    else
-        route_token_impl<V, kGlobal, false>(t, E, k, norm_topk, logits, idx, w, keff, lane);
+        return route_token_impl<V, kGlobal, true>(t, E, k, norm_topk, topp, logits, idx, w, keff, lane);
+    return route_token_impl<V, kGlobal, false>(t, E, k, norm_topk, topp, logits, idx, w, keff, lane);
 }
 
 // One token per thread, for E <= kLaneRouteMaxE: the same decisions as
 // route_token, with every sum taken in expert order (max, then
 // sum_e exp(l_e - max), then k rounds of first-maximum selection over the
-// untaken experts, then the renormalising sum in slot order).  A warp routes
-// 32 tokens at once with no shuffles.  `l` is the token's row of logits
-// (global memory when kGlobal, else shared memory).
+// untaken experts, then the renormalising sum in slot order, then the top-p
+// trim).  A warp routes 32 tokens at once with no shuffles.  `l` is the
+// token's row of logits (global memory when kGlobal, else shared memory).
+// Returns the kept slot count.
 constexpr int kLaneRouteMaxE = 64;
 
 template <bool kGlobal>
-__device__ __forceinline__ void route_token_lane(int t, int E, int k, int norm_topk, const float *l, int32_t *idx,
-                                                 float *w) {
+__device__ __forceinline__ int route_token_lane(int t, int E, int k, int norm_topk, float topp, const float *l,
+                                                int32_t *idx, float *w) {
     auto L = [&](int e) { return kGlobal ? __ldg(l + e) : l[e]; };
     float m = L(0);
     for (int e = 1; e < E; ++e) {
@@ -174,6 +201,28 @@ __device__ __forceinline__ void route_token_lane(int t, int E, int k, int norm_t
     }
     if (norm_topk)
         for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = w[(size_t)t * k + j] / ps;
+    int c = k;  // kept slots
+    if (topp > 0.f && topp < 1.f) {
+        float *tw = w + (size_t)t * k;
+        float mass = 0.f;
+        for (int j = 0; j < k; ++j) {
+            if (j > 0 && mass >= topp) {
+                c = j;
+                break;
+            }
+            mass += tw[j];
+        }
+        if (norm_topk && c < k) {
+            float s2 = 0.f;
+            for (int j = 0; j < c; ++j) s2 += tw[j];
+            for (int j = 0; j < c; ++j) tw[j] = tw[j] / s2;
+        }
+        for (int j = c; j < k; ++j) {
+            idx[(size_t)t * k + j] = -1;
+            tw[j] = 0.f;
+        }
+    }
+    return c;
 }
 
 // ------------------------------------------------------------ shared gate --
@@ -323,7 +372,8 @@ __device__ __forceinline__ void block_sort_by_expert(int n, int E, int W, Key ke
 // ---------------------------------------------------------------- budget --
 // Expert budget (colibri issue_budget.md, "EXPERT_BUDGET", section "How it
 // works", steps 1-5) inside one 1024-thread block, on a routing held in
-// shared memory (idx_s, w_s: T * k slots, every slot valid).
+// shared memory (idx_s, w_s: T * k slots; a token's valid slots first, then
+// idx -1 where a top-p trim dropped them).
 //   step 1: agg[e] = the weights routed to e summed in token-then-slot order
 //           (the slots are sorted by expert first, so each expert's thread
 //           sums exactly that sequence);
@@ -331,10 +381,11 @@ __device__ __forceinline__ void block_sort_by_expert(int n, int E, int W, Key ke
 //           rank is the number of union experts ahead of it in (agg
 //           descending, id ascending); the first N are kept;
 //   step 4: each token's kept slots move to the front in order, the others
-//           become (-1, 0); a token that lost some but not all renormalises;
+//           become (-1, 0); a token that lost some but not all of its valid
+//           slots renormalises;
 //   step 5: n_dropped = union size - N.
-// A budget of 0, or a union of at most N experts, changes nothing (keff = k,
-// kept = the union).  Out (shared memory): idx_s / w_s compacted, keff_s[T],
+// A budget of 0, or a union of at most N experts, changes nothing (keff =
+// the token's valid slots, kept = the union).  Out (shared memory): idx_s / w_s compacted, keff_s[T],
 // keep[E], *nd_s; off / sorted keep the sort of all slots by expert.
 // Scratch: hist (sort_warps(E) * E), off (E + 1), sorted (T * k), agg (E),
 // pres (E), warp_sums (32).  The ranks are counted by up to blockDim / E
@@ -383,7 +434,9 @@ __device__ __forceinline__ void budget_block(int T, int E, int k, int N, int nor
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
         int32_t *ti = idx_s + (size_t)t * k;
         float *tw = w_s + (size_t)t * k;
-        int c = k;
+        int valid = 0;
+        for (int j = 0; j < k; ++j) valid += ti[j] >= 0;
+        int c = valid;
         if (active) {
             c = 0;
             for (int j = 0; j < k; ++j) {
@@ -399,7 +452,7 @@ __device__ __forceinline__ void budget_block(int T, int E, int k, int N, int nor
                 ti[j] = -1;
                 tw[j] = 0.f;
             }
-            if (norm_topk && c > 0 && c < k) {
+            if (norm_topk && c > 0 && c < valid) {
                 float s = 0.f;
                 for (int j = 0; j < c; ++j) s += tw[j];
                 for (int j = 0; j < c; ++j) tw[j] = tw[j] / s;

@@ -55,11 +55,15 @@ WsLayout ws_layout(const moe_config_t &c, int T) {
     return L;
 }
 
+// The top-p trim is on for 0 < topp < 1 (0, the default, and 1 or more leave the routing as it is).
+bool topp_on(const moe_config_t *c) { return c->topp > 0.f && c->topp < 1.f; }
+
 int check_config(const moe_config_t *c, int32_t T) {
     if (!c || T < 0) return MOE_ERR_INVALID_ARG;
     const int E = c->n_routed_experts, k = c->num_experts_per_tok;
     if (E < 1 || k < 1 || k > E || c->budget < 0 || c->shared_intermediate_size < 0 || c->hidden < 1 ||
-        c->moe_intermediate_size < 1 || (c->norm_topk != 0 && c->norm_topk != 1))
+        c->moe_intermediate_size < 1 || (c->norm_topk != 0 && c->norm_topk != 1) || !(c->topp >= 0.f) ||
+        c->topp > 3.4e38f)  // NaN, negative or infinite top-p
         return MOE_ERR_INVALID_ARG;
     if (E > kMaxExperts || k > kMaxTopK || c->hidden % 128 != 0 || c->moe_intermediate_size % 64 != 0 ||
         c->shared_intermediate_size % 64 != 0)
@@ -109,10 +113,12 @@ int moe_route(const moe_config_t *cfg, int32_t T, const float *logits, const moe
     if (T == 0) return MOE_OK;
     if (!aligned(logits) || !aligned(topk_idx) || !aligned(topk_w) || !aligned_or_null(keff))
         return MOE_ERR_INVALID_ARG;
+    if (topp_on(cfg) && keff == nullptr) return MOE_ERR_INVALID_ARG;  // the trimmed counts must go somewhere
     if (sgate && (cfg->shared_intermediate_size == 0 || !aligned(x) || !aligned(ws_gate_vec) || !aligned(sgate)))
         return MOE_ERR_INVALID_ARG;
-    return cuda_rc(launch_route(T, cfg->n_routed_experts, cfg->num_experts_per_tok, cfg->norm_topk, logits,
-                                topk_idx, topk_w, keff, x, ws_gate_vec, cfg->hidden, sgate, as_stream(stream)));
+    return cuda_rc(launch_route(T, cfg->n_routed_experts, cfg->num_experts_per_tok, cfg->norm_topk, cfg->topp,
+                                logits, topk_idx, topk_w, keff, x, ws_gate_vec, cfg->hidden, sgate,
+                                as_stream(stream)));
 }
 
 int moe_budget(const moe_config_t *cfg, int32_t T, int32_t *topk_idx, float *topk_w, int32_t *keff,
@@ -368,7 +374,7 @@ int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const f
     // instead of four.  (Without a budget the separate route and dispatch
     // launches measured faster for the drafter layers.)
     if (cfg->budget > 0 && front_fits(T, E, k)) {
-        rc = cuda_rc(launch_front(T, E, k, cfg->budget, cfg->norm_topk, cfg->hidden, logits, x,
+        rc = cuda_rc(launch_front(T, E, k, cfg->budget, cfg->norm_topk, cfg->topp, cfg->hidden, logits, x,
                                   sh ? w->ws_gate_vec : nullptr, idx, tw, sgate, keff, kept, ndrop, counts, offsets,
                                   perm, slot_pos, x_perm, at<int32_t>(ws, L.status),
                                   at<int32_t>(ws, L.status + kHdoneOffset), as_stream(stream)));

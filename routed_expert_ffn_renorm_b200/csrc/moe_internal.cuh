@@ -50,7 +50,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Every wrapper enqueues on `st` and returns cudaGetLastError().
 
 // Route (one warp per token).
-cudaError_t launch_route(int T, int E, int k, int norm_topk, const float *logits, int32_t *idx,
+cudaError_t launch_route(int T, int E, int k, int norm_topk, float topp, const float *logits, int32_t *idx,
                          float *w, int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H,
                          float *sgate, cudaStream_t st);
 
@@ -81,7 +81,8 @@ cudaError_t launch_gather_rows(int T, int k, int H, const int32_t *offsets, int 
 constexpr int kFrontMaxSlots = 8192;
 constexpr int kFrontMaxLogits = 16384;
 bool front_fits(int T, int E, int k);
-cudaError_t launch_front(int T, int E, int k, int N, int norm_topk, int H, const float *logits, const uint16_t *x,
+cudaError_t launch_front(int T, int E, int k, int N, int norm_topk, float topp, int H, const float *logits,
+                         const uint16_t *x,
                          const uint16_t *gvec, int32_t *idx, float *w, float *sgate, int32_t *keff, uint8_t *kept,
                          int32_t *n_dropped, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
                          uint16_t *x_perm, int32_t *status_block, int32_t *hdone, cudaStream_t st);

@@ -1,7 +1,8 @@
 // Router: softmax over the E logits of a token, top-k by logit with the
 // kept probabilities renormalised (SpecForge PR #943, "Modifications":
-// softmax router with renormalised top-k), plus the sigmoid gate of the
-// shared expert.
+// softmax router with renormalised top-k), the optional per-token top-p trim
+// (colibri issue_budget.md, "Relationship to existing features"), plus the
+// sigmoid gate of the shared expert.
 //
 // route_kernel<V>: one block per token; its first warp routes (route_token,
 // front.cuh) while the next four compute the shared-expert gate
@@ -17,7 +18,7 @@ namespace {
 constexpr int kRouteThreads = 32 + kGateThreads;  // one token per block: warp 0 routes, warps 1.. dot
 
 template <int V>  // logits per lane: V * 32 >= E
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int k, int norm_topk,
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int k, int norm_topk, float topp,
                                                               const float *__restrict__ logits,
                                                               int32_t *__restrict__ idx, float *__restrict__ w,
                                                               int32_t *__restrict__ keff,
@@ -30,7 +31,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int 
     const int t = blockIdx.x;  // one token per block
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     if (wid == 0) {
-        route_token<V>(t, E, k, norm_topk, logits, idx, w, keff, lane);
+        route_token<V>(t, E, k, norm_topk, topp, logits, idx, w, keff, lane);
         return;
     }
     if (sgate == nullptr) return;
@@ -44,7 +45,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int 
 // logits staged in shared memory; the remaining T blocks (with a shared
 // expert) compute one token's shared gate each.  Routing and gate blocks run
 // side by side instead of one after the other.
-__global__ void __launch_bounds__(kGateThreads) route_lane_kernel(int T, int E, int k, int norm_topk,
+__global__ void __launch_bounds__(kGateThreads) route_lane_kernel(int T, int E, int k, int norm_topk, float topp,
                                                                    const float *__restrict__ logits,
                                                                    int32_t *__restrict__ idx, float *__restrict__ w,
                                                                    int32_t *__restrict__ keff,
@@ -65,8 +66,8 @@ __global__ void __launch_bounds__(kGateThreads) route_lane_kernel(int T, int E, 
         }
         __syncwarp();
         if (lane < n) {
-            route_token_lane<false>(t0 + lane, E, k, norm_topk, lg + lane * ls, idx, w);
-            if (keff != nullptr) keff[t0 + lane] = k;
+            const int c = route_token_lane<false>(t0 + lane, E, k, norm_topk, topp, lg + lane * ls, idx, w);
+            if (keff != nullptr) keff[t0 + lane] = c;
         }
         return;
     }
@@ -76,25 +77,25 @@ __global__ void __launch_bounds__(kGateThreads) route_lane_kernel(int T, int E, 
 }
 
 template <int V>
-cudaError_t launch_v(int T, int E, int k, int norm_topk, const float *logits, int32_t *idx, float *w,
+cudaError_t launch_v(int T, int E, int k, int norm_topk, float topp, const float *logits, int32_t *idx, float *w,
                      int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
                      cudaStream_t st) {
-    return launch_pdl(route_kernel<V>, dim3(T), dim3(kRouteThreads), 0, st, T, E, k, norm_topk, logits, idx, w, keff,
-                      x, gvec, H, sgate);
+    return launch_pdl(route_kernel<V>, dim3(T), dim3(kRouteThreads), 0, st, T, E, k, norm_topk, topp, logits, idx, w,
+                      keff, x, gvec, H, sgate);
 }
 
 }  // namespace
 
-cudaError_t launch_route(int T, int E, int k, int norm_topk, const float *logits, int32_t *idx, float *w,
+cudaError_t launch_route(int T, int E, int k, int norm_topk, float topp, const float *logits, int32_t *idx, float *w,
                          int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
                          cudaStream_t st) {
     if (E <= kLaneRouteMaxE)
         return launch_pdl(route_lane_kernel, dim3((T + 31) / 32 + (sgate != nullptr ? T : 0)), dim3(kGateThreads), 0,
-                          st, T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate);
-    if (E <= 128) return launch_v<4>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
-    if (E <= 256) return launch_v<8>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
-    if (E <= 512) return launch_v<16>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
-    return launch_v<32>(T, E, k, norm_topk, logits, idx, w, keff, x, gvec, H, sgate, st);
+                          st, T, E, k, norm_topk, topp, logits, idx, w, keff, x, gvec, H, sgate);
+    if (E <= 128) return launch_v<4>(T, E, k, norm_topk, topp, logits, idx, w, keff, x, gvec, H, sgate, st);
+    if (E <= 256) return launch_v<8>(T, E, k, norm_topk, topp, logits, idx, w, keff, x, gvec, H, sgate, st);
+    if (E <= 512) return launch_v<16>(T, E, k, norm_topk, topp, logits, idx, w, keff, x, gvec, H, sgate, st);
+    return launch_v<32>(T, E, k, norm_topk, topp, logits, idx, w, keff, x, gvec, H, sgate, st);
 }
 
 }  // namespace moe

@@ -40,6 +40,7 @@ class MoEConfig:
     norm_topk: bool = True
     budget: int = 0   # EXPERT_BUDGET (0 = off)
     zipf_alpha: float = 0.0
+    topp: float = 0.0  # per-token top-p trim (0 = off)
     seed: int = 0
 
     def with_(self, **kw) -> "MoEConfig":
@@ -54,6 +55,8 @@ class MoEConfig:
             s += f"_N{self.budget}"
         if self.zipf_alpha:
             s += f"_a{self.zipf_alpha:g}"
+        if self.topp:
+            s += f"_p{self.topp:g}"
         return s
 
 

@@ -10,6 +10,11 @@ Comparison rules (the tolerance is the one stated for the layer output):
     oracle's aggregate gap between the last kept and first dropped expert
     must be <= 1e-5 of the largest aggregate; the downstream comparison then
     runs the oracle on the GPU's post-budget routing.
+  * top-p near-ties: when the GPU keeps a different number of slots of a
+    token, the oracle's prefix mass at some slot of that token must be
+    within 1e-5 of topp (the trim decided on ulp-different weights), and
+    the kept slots must still be a prefix of the oracle's top-k; the
+    downstream comparison then uses the GPU's routing.
 """
 from __future__ import annotations
 
@@ -29,7 +34,18 @@ NEAR_TIE = 1e-5
 
 
 def lib_config(cfg: W.MoEConfig) -> moe.MoEConfig:
-    return moe.MoEConfig(cfg.H, cfg.E, cfg.I, cfg.k, cfg.Is, cfg.norm_topk, cfg.budget)
+    return moe.MoEConfig(cfg.H, cfg.E, cfg.I, cfg.k, cfg.Is, cfg.norm_topk, cfg.budget, cfg.topp)
+
+
+def topp_margin(w: np.ndarray, p: float, t: int) -> float:
+    """Smallest |prefix mass - p| over the decisions of token t (fp32, slot order)."""
+    mass = np.float32(0.0)
+    m = np.inf
+    for j in range(w.shape[1]):
+        if j > 0:
+            m = min(m, abs(float(mass) - p))
+        mass = np.float32(mass + w[t, j])
+    return m
 
 
 def weights_of(inp: W.MoEInputs) -> moe.MoEWeights:
@@ -116,25 +132,41 @@ def check_layer(cfg: W.MoEConfig, inp: W.MoEInputs, g: GpuResult, rows: Optional
     # route (bit-exact indices, fp32 weights within ulps)
     idx_o, w_o = oracle.route(logits, k, cfg.norm_topk)
     diag = {}
-    if cfg.budget == 0:
-        assert (g.idx == idx_o).all(), "routing indices differ"
-        np.testing.assert_allclose(g.w, w_o, rtol=W_RTOL, atol=1e-7)
-        assert (g.keff == k).all()
-        idx_b, w_b, keff_b = idx_o, w_o, np.full(T, k, np.int32)
+    # the top-p trim on the oracle's routing
+    if cfg.topp:
+        idx_p, w_p, keff_p = oracle.topp(idx_o, w_o, cfg.topp, cfg.norm_topk)
     else:
-        # the budget on the oracle's own routing
-        idx_b, w_b, keff_b, kept_b, nd_b = oracle.budget(idx_o, w_o, E, cfg.budget, cfg.norm_topk)
-        if (kept_b == g.kept).all():
+        idx_p, w_p, keff_p = idx_o, w_o, np.full(T, k, np.int32)
+    if cfg.budget == 0:
+        if (g.idx == idx_p).all() and (g.keff == keff_p).all():
+            np.testing.assert_allclose(g.w, w_p, rtol=W_RTOL, atol=1e-7)
+            idx_b, w_b, keff_b = idx_p, w_p, keff_p
+        else:
+            assert cfg.topp, "routing indices differ"
+            bad = np.nonzero((g.keff != keff_p) | (g.idx != idx_p).any(1))[0]
+            for t in bad:
+                c = int(g.keff[t])
+                assert (g.idx[t, :c] == idx_o[t, :c]).all() and (g.idx[t, c:] == -1).all(), "not a top-k prefix"
+                m = topp_margin(w_o, cfg.topp, int(t))
+                assert m <= NEAR_TIE, f"top-p kept count differs with margin {m}"
+            diag["topp_near"] = int(len(bad))
+            idx_b, w_b, keff_b = g.idx, g.w, g.keff
+    else:
+        # the budget on the oracle's own (trimmed) routing
+        idx_b, w_b, keff_b, kept_b, nd_b = oracle.budget(idx_p, w_p, E, cfg.budget, cfg.norm_topk)
+        if (kept_b == g.kept).all() and (g.idx == idx_b).all() and (g.keff == keff_b).all():
             assert g.n_dropped == nd_b
-            assert (g.idx == idx_b).all() and (g.keff == keff_b).all()
             np.testing.assert_allclose(g.w, w_b, rtol=W_RTOL, atol=1e-7)
         else:
+            valid = idx_p >= 0
             agg = np.zeros(E)
-            np.add.at(agg, idx_o.ravel(), w_o.ravel().astype(np.float64))
-            union = np.unique(idx_o)
+            np.add.at(agg, idx_p[valid], w_p[valid].astype(np.float64))
+            union = np.unique(idx_p[valid])
             order = union[np.lexsort((union, -agg[union]))]
-            gap = agg[order[cfg.budget - 1]] - agg[order[cfg.budget]]
-            assert gap <= NEAR_TIE * agg.max(), f"budget keep-set differs with gap {gap}"
+            gap = agg[order[cfg.budget - 1]] - agg[order[cfg.budget]] if len(union) > cfg.budget else np.inf
+            near_budget = gap <= NEAR_TIE * agg.max()
+            near_topp = bool(cfg.topp) and min(topp_margin(w_o, cfg.topp, t) for t in range(T)) <= NEAR_TIE
+            assert near_budget or near_topp, f"budget keep-set differs with gap {gap}"
             diag["near_tie"] = float(gap)
             idx_b, w_b, keff_b = g.idx, g.w, g.keff
     # dispatch on the same routing: bit-exact

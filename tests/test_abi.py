@@ -35,9 +35,9 @@ def test_library_exports_every_declared_symbol():
 
 def _cfg(**kw):
     base = dict(hidden=256, n_routed_experts=8, moe_intermediate_size=128, num_experts_per_tok=2,
-                shared_intermediate_size=0, norm_topk=True, budget=0)
+                shared_intermediate_size=0, norm_topk=True, budget=0, topp=0.0)
     base.update(kw)
-    return moe._Config(*[int(v) for v in base.values()])
+    return moe._Config(*[float(v) if n == "topp" else int(v) for n, v in base.items()])
 
 
 FAKE = ctypes.c_void_p(1 << 20)      # never dereferenced: the checks fail first
@@ -49,6 +49,7 @@ MISALIGNED = ctypes.c_void_p((1 << 20) + 4)
     (dict(budget=-1), -1), (dict(norm_topk=2), -1), (dict(hidden=200), -2), (dict(moe_intermediate_size=96), -2),
     (dict(shared_intermediate_size=32), -2), (dict(n_routed_experts=2048, num_experts_per_tok=2), -2),
     (dict(n_routed_experts=64, num_experts_per_tok=33), -2),
+    (dict(topp=float("nan")), -1), (dict(topp=-0.5), -1), (dict(topp=float("inf")), -1),
 ])
 def test_config_checks(kw, code):
     lib = moe.load_library()
@@ -68,6 +69,9 @@ def test_pointer_checks_and_noop():
     assert lib.moe_route(ctypes.byref(c), 16, None, None, None, FAKE, FAKE, None, None, None) == -1
     # sgate requested without a shared expert
     assert lib.moe_route(ctypes.byref(c), 16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == -1
+    # a top-p trim needs somewhere to put the kept counts
+    cp = _cfg(topp=0.5)
+    assert lib.moe_route(ctypes.byref(cp), 16, FAKE, None, None, FAKE, FAKE, None, None, None) == -1
     # short workspace
     ws_need = lib.moe_workspace_bytes(ctypes.byref(c), 16)
     assert ws_need > 0

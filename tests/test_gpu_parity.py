@@ -52,6 +52,16 @@ SMALL = [
     W.MoEConfig("budget_chunks", T=700, H=128, E=64, I=64, k=6, budget=9, zipf_alpha=0.5),
     W.MoEConfig("max_experts", T=64, H=128, E=1024, I=64, k=8),
     W.MoEConfig("max_topk", T=16, H=128, E=64, I=64, k=32),
+    # per-token top-p trim: lane router (E <= 64), warp router, 16-byte lane loads (E > 128), no norm,
+    # with the budget (fused front end, one-block and chunked budgets)
+    W.MoEConfig("topp_lane", T=64, H=256, E=32, I=64, k=6, Is=64, topp=0.7),
+    W.MoEConfig("topp_warp", T=50, H=256, E=128, I=64, k=8, topp=0.5, zipf_alpha=0.5),
+    W.MoEConfig("topp_vec", T=40, H=128, E=256, I=64, k=8, topp=0.85),
+    W.MoEConfig("topp_no_norm", T=48, H=256, E=16, I=64, k=4, norm_topk=False, topp=0.3),
+    W.MoEConfig("topp_budget", T=32, H=256, E=128, I=64, k=8, budget=12, topp=0.8, zipf_alpha=1.2),
+    W.MoEConfig("topp_budget_block", T=700, H=128, E=64, I=64, k=6, budget=9, topp=0.6, zipf_alpha=0.5),
+    W.MoEConfig("topp_budget_chunks", T=1500, H=128, E=64, I=64, k=6, budget=9, topp=0.6, zipf_alpha=0.5),
+    W.MoEConfig("topp_tiny_p", T=33, H=128, E=16, I=64, k=4, Is=64, topp=1e-6),
 ]
 
 
@@ -205,6 +215,10 @@ STAGEWISE = [
     W.MoEConfig("stages_e1024", T=16, H=128, E=1024, I=64, k=8, budget=20),  # front, largest E
     W.MoEConfig("stages_slots_max", T=1024, H=128, E=16, I=64, k=8, Is=64, budget=9),  # front, T*k = 8192
     W.MoEConfig("stages_big_logits", T=700, H=128, E=64, I=64, k=6, budget=9, zipf_alpha=0.5),  # separate
+    W.MoEConfig("stages_topp", T=96, H=256, E=16, I=128, k=4, Is=64, budget=6, topp=0.6, zipf_alpha=1.0),  # front
+    W.MoEConfig("stages_topp_warp", T=64, H=128, E=128, I=64, k=8, budget=12, topp=0.8),  # front, warp router
+    W.MoEConfig("stages_topp_nobudget", T=200, H=256, E=32, I=64, k=3, Is=64, topp=0.5),  # separate
+    W.MoEConfig("stages_topp_chunks", T=1500, H=128, E=64, I=64, k=6, budget=9, topp=0.7),  # separate, chunked
 ]
 
 
