@@ -10,7 +10,8 @@ it, and the two share no source.
 
 Each function follows a passage of the pages:
   * SpecForge PR #943 (Qwen3.8-27B DSpark MoE drafter), "Modifications":
-    softmax router with renormalised top-k, sigmoid-gated shared expert,
+    the router projection and softmax router with renormalised top-k,
+    sigmoid-gated shared expert,
     grouped dispatch; its FFN parameter table fixes the gated FFN's shape.
   * colibri issue_budget.md (EXPERT_BUDGET), "How it works" steps 1-5 and
     "Safety": the batch-union expert budget; "Relationship to existing
@@ -53,6 +54,7 @@ def _load():
     lib.oracle_ffn_params.restype = ctypes.c_int64
     lib.oracle_ffn_params.argtypes = [ctypes.c_int64, ctypes.c_int64]
     lib.oracle_route.argtypes = [i32, i32, i32, i32, P, P, P]
+    lib.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P]
     lib.oracle_budget.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P]
     lib.oracle_topp.argtypes = [i32, i32, i32, ctypes.c_float, P, P, P]
     lib.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, P, P, P]
@@ -86,6 +88,18 @@ def max_threads() -> int:
 def ffn_params(H: int, I: int) -> int:
     """Parameters of one gated expert FFN (gate, up, down projections)."""
     return int(_load().oracle_ffn_params(H, I))
+
+
+def router_logits(x: np.ndarray, w_router: np.ndarray) -> np.ndarray:
+    """logits = x . W_r^T (fp64 accumulation, rounded once to fp32).
+    x [T, H], w_router [E, H]: bf16 bit patterns.  Returns [T, E] float32."""
+    x = _c(x, np.uint16)
+    wr = _c(w_router, np.uint16)
+    T, H = x.shape
+    E = wr.shape[0]
+    out = np.empty((max(T, 1), E), np.float32)
+    _check(_load().oracle_router_logits(T, H, E, _ptr(x), _ptr(wr), _ptr(out)), "router_logits")
+    return out[:T]
 
 
 def route(logits: np.ndarray, k: int, norm_topk: bool = True):

@@ -66,6 +66,26 @@ static double bf16_to_f64(uint16_t v)
 int64_t oracle_ffn_params(int64_t H, int64_t I) { return 3 * H * I; }
 
 /* ---------------------------------------------------------------------- */
+/* Router projection ([SF943] "Modifications": the softmax router whose     */
+/* logits the route step takes; a bias-free linear map of the hidden state, */
+/* the plain reading of a router over n_routed_experts).                   */
+/* ---------------------------------------------------------------------- */
+/* logits[t, e] = sum_h x[t, h] * W_r[e, h], accumulated in fp64 and rounded
+ * once to fp32.  x [T, H] and W_r [E, H] are bf16 bit patterns. */
+int oracle_router_logits(int32_t T, int32_t H, int32_t E, const uint16_t *x, const uint16_t *wr, float *logits)
+{
+    if (T < 0 || H < 1 || E < 1) return ORACLE_EINVAL;
+    for (int32_t t = 0; t < T; ++t)
+        for (int32_t e = 0; e < E; ++e) {
+            double a = 0.0;
+            for (int32_t h = 0; h < H; ++h)
+                a += bf16_to_f64(x[(size_t)t * H + h]) * bf16_to_f64(wr[(size_t)e * H + h]);
+            logits[(size_t)t * E + e] = (float)a;
+        }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------- */
 /* Route ([SF943] "Modifications": softmax router, renormalised top-k).    */
 /* ---------------------------------------------------------------------- */
 /* For each token t:

@@ -41,6 +41,10 @@ MUTANTS = {
     "budget_no_renorm": ("if (norm_topk && c > 0 && c < keff[t]) {", "if (norm_topk && c > 0 && c < 0) {"),
     "budget_renorm_all": ("if (norm_topk && c > 0 && c < keff[t]) {", "if (norm_topk && c > 0 && c <= k) {"),
     "budget_renorm_by_k": ("if (norm_topk && c > 0 && c < keff[t]) {", "if (norm_topk && c > 0 && c < k) {"),
+    "router_transposed": ("a += bf16_to_f64(x[(size_t)t * H + h]) * bf16_to_f64(wr[(size_t)e * H + h]);",
+                          "a += bf16_to_f64(x[(size_t)t * H + h]) * bf16_to_f64(wr[((size_t)h * E + e) % ((size_t)E * H)]);"),
+    "router_skips_first": ("for (int32_t h = 0; h < H; ++h)\n                a += bf16_to_f64(x",
+                           "for (int32_t h = 1; h < H; ++h)\n                a += bf16_to_f64(x"),
     "topp_strict": ("if (j > 0 && mass >= topp) { c = j; break; }", "if (j > 0 && mass > topp) { c = j; break; }"),
     "topp_drops_crossing_slot": ("                if (j > 0 && mass >= topp) { c = j; break; }\n                mass += tw[j];",
                                  "                mass += tw[j];\n                if (j > 0 && mass >= topp) { c = j; break; }"),
@@ -58,6 +62,7 @@ MUTANTS = {
 # every pin test with the arguments it is run with
 PINS = [
     ("test_param_counts_match_drafter_table", {}),
+    ("test_router_logits_unit_vectors_and_torch", {}),
     ("test_route_closed_form_worked_example", {}),
     ("test_route_ties_take_lower_id", {}),
     ("test_route_brute_force_topk", dict(E=8, k=3)),

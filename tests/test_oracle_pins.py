@@ -59,6 +59,21 @@ def test_param_counts_match_drafter_table(oracle_mod):
 
 # ----------------------------------------------------------------- route --
 
+def test_router_logits_unit_vectors_and_torch(oracle_mod):
+    """x = unit vector e_h picks column h of W_r exactly; random inputs match
+    torch's fp64 linear map rounded to fp32."""
+    H, E = 48, 7
+    wr = _bf(np.random.default_rng(2).standard_normal((E, H)))
+    eye = _bf(np.eye(H))
+    lg = oracle_mod.router_logits(bits(eye), bits(wr))
+    assert (lg == wr.float().numpy().T).all()
+    x = _bf(np.random.default_rng(3).standard_normal((9, H)))
+    ref = F.linear(x.double(), wr.double()).float().numpy()
+    np.testing.assert_allclose(oracle_mod.router_logits(bits(x), bits(wr)), ref, rtol=1e-6, atol=1e-7)
+    # the bias-free map is linear: doubling x (exact in bf16) doubles the logits exactly
+    assert (oracle_mod.router_logits(bits(x * 2), bits(wr)) == 2 * oracle_mod.router_logits(bits(x), bits(wr))).all()
+
+
 def test_route_closed_form_worked_example(oracle_mod):
     # logits ln(1..4): softmax = (1,2,3,4)/10; top-2 = experts 3, 2;
     # renormalised weights 4/7, 3/7.
