@@ -2,6 +2,7 @@
  * moe.h -- C ABI of the B200 (sm_100a) routed Mixture-of-Experts FFN forward.
  *
  * The layer, for a batch of T tokens x_t (hidden size H):
+ *   logits   optionally the router projection logits_t = W_r x_t, else given;
  *   route    softmax over the E router logits of each token, the k largest
  *            logits kept, their probabilities renormalised to sum 1 when
  *            norm_topk is set;
@@ -84,6 +85,7 @@ typedef struct {
     const moe_bf16_t *ws_up;       /* [Is, H] shared up projection, NULL if Is = 0 */
     const moe_bf16_t *ws_down;     /* [H, Is] shared down projection, NULL if Is = 0 */
     const moe_bf16_t *ws_gate_vec; /* [H] shared-expert gate vector g, NULL if Is = 0 */
+    const moe_bf16_t *w_router;    /* [E, H] router projection; read by moe_forward only when its logits are NULL */
 } moe_weights_t;
 
 /* Optional device outputs of moe_forward; any NULL member is kept inside
@@ -99,6 +101,7 @@ typedef struct {
     int32_t *offsets;      /* [E+1]  */
     int32_t *perm;         /* [T*k]  first offsets[E] entries valid */
     int32_t *slot_pos;     /* [T*k]  */
+    float *logits;         /* [T, E] the router projection's logits (when moe_forward computed them) */
 } moe_aux_t;
 
 /* Bytes of device workspace the calls below need for a batch of T tokens
@@ -108,6 +111,16 @@ typedef struct {
  * every kernel leaves the counters at zero, and moe_dispatch re-zeroes them.
  * One workspace serves one stream at a time. */
 size_t moe_workspace_bytes(const moe_config_t *cfg, int32_t T);
+
+/* Router projection: logits[t, e] = sum_h x[t, h] * w_router[e, h], bf16
+ * operands on the tensor cores with fp32 accumulation, fp32 out (SpecForge
+ * PR #943, "Modifications": the softmax router's logits; a bias-free linear
+ * map).  Small batches split the H sum over CTAs and add the fp32 partials in
+ * a fixed order, so the result is the same bits on every run.
+ *   x [T, H]; w_router [E, H]; logits [T, E] f32.  Uses the workspace (its
+ *   head must be zeroed once, as for every call below). */
+int moe_router_logits(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                      float *logits, void *ws, size_t ws_bytes, void *stream);
 
 /* Route: for each token t, topk_idx[t, 0..k) = the k experts with the
  * largest logits (descending; equal logits: lower expert id first),
@@ -216,9 +229,11 @@ int moe_expert_ffn_noalloc(const moe_config_t *cfg, int32_t T, const moe_bf16_t 
 int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, const int32_t *keff,
                 moe_bf16_t *out, void *stream);
 
-/* The whole layer: route -> budget (if cfg->budget > 0) -> dispatch ->
- * expert FFN -> combine, enqueued on one stream with no host sync.
- * x [T, H]; logits [T, E] f32; out [T, H]; aux may be NULL. */
+/* The whole layer: [router projection] -> route -> [top-p] -> [budget] ->
+ * dispatch -> expert FFN -> combine, enqueued on one stream with no host
+ * sync.  x [T, H]; logits [T, E] f32, or NULL to compute them from
+ * w->w_router (moe_router_logits; then aux->logits, if set, receives them);
+ * out [T, H]; aux may be NULL. */
 int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
                 const moe_weights_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
                 size_t ws_bytes, void *stream);

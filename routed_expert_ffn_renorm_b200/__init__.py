@@ -22,7 +22,8 @@ from dataclasses import dataclass
 from typing import Optional
 
 __all__ = [
-    "MoEConfig", "MoEWeights", "MoEError", "load_library", "workspace_bytes", "moe_route", "moe_budget",
+    "MoEConfig", "MoEWeights", "MoEError", "load_library", "workspace_bytes", "moe_router_logits", "moe_route",
+    "moe_budget",
     "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn_noalloc",
     "moe_combine", "moe_forward",
     "status_read", "status_clear",
@@ -35,7 +36,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_route", "moe_budget", "moe_dispatch", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_status_read", "moe_status_clear", "moe_error_string", "moe_expert_gate_up",
-    "moe_expert_down", "moe_expert_ffn_noalloc",
+    "moe_expert_down", "moe_expert_ffn_noalloc", "moe_router_logits",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 MOE_STATUS_TIMEOUT = 1
@@ -55,13 +56,13 @@ class _Config(ctypes.Structure):
 
 class _Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
-        "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec")]
+        "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec", "w_router")]
 
 
 class _Aux(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "topk_idx", "topk_w", "sgate", "keff", "expert_kept", "n_dropped", "counts", "offsets", "perm",
-        "slot_pos")]
+        "slot_pos", "logits")]
 
 
 @dataclass(frozen=True)
@@ -84,7 +85,8 @@ class MoEConfig:
 @dataclass
 class MoEWeights:
     """Device bf16 weights: w_gate, w_up [E, I, H]; w_down [E, H, I];
-    optional shared expert ws_gate, ws_up [Is, H], ws_down [H, Is], ws_gate_vec [H]."""
+    optional shared expert ws_gate, ws_up [Is, H], ws_down [H, Is], ws_gate_vec [H];
+    optional router projection w_router [E, H] (used when moe_forward gets no logits)."""
     w_gate: "torch.Tensor"
     w_up: "torch.Tensor"
     w_down: "torch.Tensor"
@@ -92,10 +94,11 @@ class MoEWeights:
     ws_up: Optional["torch.Tensor"] = None
     ws_down: Optional["torch.Tensor"] = None
     ws_gate_vec: Optional["torch.Tensor"] = None
+    w_router: Optional["torch.Tensor"] = None
 
     def _c(self) -> _Weights:
         return _Weights(*(_ptr(getattr(self, n), allow_none=True) for n in (
-            "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec")))
+            "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec", "w_router")))
 
 
 _lib = None
@@ -120,6 +123,7 @@ def load_library(build_if_stale: bool = True):
         lib.moe_workspace_bytes.restype = sz
         lib.moe_workspace_bytes.argtypes = [cfg, i32]
         lib.moe_route.argtypes = [cfg, i32, P, P, P, P, P, P, P, P]
+        lib.moe_router_logits.argtypes = [cfg, i32, P, P, P, P, sz, P]
         lib.moe_budget.argtypes = [cfg, i32, P, P, P, P, P, P, sz, P]
         lib.moe_dispatch.argtypes = [cfg, i32, P, P, P, P, P, P, P, P, P, sz, P]
         lib.moe_expert_ffn.argtypes = [cfg, i32, P, P, P, P, P, P, ctypes.POINTER(_Weights), P, P, sz, P]
@@ -171,6 +175,14 @@ def workspace_bytes(cfg: MoEConfig, T: int) -> int:
     if n == 0:
         raise MoEError("moe_workspace_bytes", -1, "invalid configuration")
     return int(n)
+
+
+def moe_router_logits(cfg: MoEConfig, x, w_router, logits, ws, stream=None):
+    """logits [T, E] f32 = x [T, H] . w_router [E, H]^T on the tensor cores."""
+    T = x.shape[0]
+    _check("moe_router_logits", load_library().moe_router_logits(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(w_router), _ptr(logits), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def moe_route(cfg: MoEConfig, logits, topk_idx, topk_w, *, x=None, ws_gate_vec=None, sgate=None, keff=None,
@@ -244,9 +256,11 @@ def moe_combine(cfg: MoEConfig, ybuf, out, *, keff=None, stream=None):
 
 def moe_forward(cfg: MoEConfig, x, logits, weights: MoEWeights, out, ws, *, aux: Optional[dict] = None,
                 stream=None):
-    """The whole layer on the current stream.  ``aux`` may map moe_aux_t
-    member names (topk_idx, topk_w, sgate, keff, expert_kept, n_dropped,
-    counts, offsets, perm, slot_pos) to device tensors to receive them."""
+    """The whole layer on the current stream.  ``logits`` may be None when
+    ``weights.w_router`` is set: the router projection computes them.
+    ``aux`` may map moe_aux_t member names (topk_idx, topk_w, sgate, keff,
+    expert_kept, n_dropped, counts, offsets, perm, slot_pos, logits) to
+    device tensors to receive them."""
     T = x.shape[0]
     w = weights._c()
     a = _Aux()
@@ -254,8 +268,8 @@ def moe_forward(cfg: MoEConfig, x, logits, weights: MoEWeights, out, ws, *, aux:
         for name, t in aux.items():
             setattr(a, name, _ptr(t))
     _check("moe_forward", load_library().moe_forward(
-        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(logits), ctypes.byref(w), _ptr(out), ctypes.byref(a), _ptr(ws),
-        ws.numel() * ws.element_size(), _stream(stream)))
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(logits, True), ctypes.byref(w), _ptr(out), ctypes.byref(a),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def status_read(ws, stream=None) -> int:

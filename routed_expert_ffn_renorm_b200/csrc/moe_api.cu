@@ -13,14 +13,18 @@ namespace {
 
 constexpr size_t kAlign = 256;
 // Head of the workspace: [0, 256) status word and work-item counters,
-// [256, 256 + 4 * (E + 2)) gate/up completion counters of the fused FFN.
+// [256, 256 + 4 * (E + 2)) gate/up completion counters of the fused FFN,
+// [4608, 8192) the router projection's K-split counters.
 constexpr size_t kHeadBytes = 8192;
 constexpr size_t kHdoneOffset = 256;
+constexpr size_t kRpCntOffset = 4608;
+static_assert(kRpCntOffset >= kHdoneOffset + 4 * (kMaxExperts + 2), "counter regions overlap");
+static_assert(kRpCntOffset + 4 * kRpMaxCounters <= kHeadBytes, "projection counters exceed the head");
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
     size_t status, idx, w, sgate, keff, kept, ndrop, counts, offsets, perm, slot_pos, hist, bagg, bcnt;
-    size_t x_perm, h_perm, h_shared, ybuf, total;
+    size_t x_perm, h_perm, h_shared, ybuf, logits, rpart, total;
 };
 
 WsLayout ws_layout(const moe_config_t &c, int T) {
@@ -51,6 +55,8 @@ WsLayout ws_layout(const moe_config_t &c, int T) {
     L.h_perm = take(Tk * c.moe_intermediate_size * 2);
     L.h_shared = take((size_t)T * c.shared_intermediate_size * 2);
     L.ybuf = take((size_t)T * (c.num_experts_per_tok + 1) * c.hidden * 2);
+    L.logits = take((size_t)T * E * 4);
+    L.rpart = take(rp_partial_bytes(T, (int)E, c.hidden));
     L.total = off;
     return L;
 }
@@ -344,18 +350,39 @@ int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, cons
                                   keff, out, as_stream(stream)));
 }
 
+int moe_router_logits(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *w_router,
+                      float *logits, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    if (!aligned(x) || !aligned(w_router) || !aligned(logits) || !aligned(ws)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    return cuda_rc(launch_router_proj(T, cfg->n_routed_experts, cfg->hidden, x, w_router, logits,
+                                      at<float>(ws, L.rpart), at<int32_t>(ws, L.status + kRpCntOffset),
+                                      at<int32_t>(ws, L.status), as_stream(stream)));
+}
+
 int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits, const moe_weights_t *w,
                 moe_bf16_t *out, const moe_aux_t *aux, void *ws, size_t ws_bytes, void *stream) {
     int rc = check_config(cfg, T);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
     const bool sh = cfg->shared_intermediate_size > 0;
-    if (!aligned(x) || !aligned(logits) || !aligned(out) || !aligned(ws) || !w) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x) || !aligned_or_null(logits) || !aligned(out) || !aligned(ws) || !w) return MOE_ERR_INVALID_ARG;
+    if (!logits && !aligned(w->w_router)) return MOE_ERR_INVALID_ARG;  // no logits: the projection makes them
     if (sh && !aligned(w->ws_gate_vec)) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(*cfg, T);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     moe_aux_t a{};
     if (aux) a = *aux;
+    if (a.logits && !aligned(a.logits)) return MOE_ERR_INVALID_ARG;
+    if (!logits) {  // router projection first
+        float *lg = a.logits ? a.logits : at<float>(ws, L.logits);
+        rc = moe_router_logits(cfg, T, x, w->w_router, lg, ws, ws_bytes, stream);
+        if (rc) return rc;
+        logits = lg;
+    }
     int32_t *idx = a.topk_idx ? a.topk_idx : at<int32_t>(ws, L.idx);
     float *tw = a.topk_w ? a.topk_w : at<float>(ws, L.w);
     float *sgate = sh ? (a.sgate ? a.sgate : at<float>(ws, L.sgate)) : nullptr;

@@ -9,6 +9,9 @@ Recipe (the same for every workload):
     W_down, shared gate vector -- all from one torch.Generator seeded with
     ``seed`` on the chosen device;
   * x and every weight ~ N(0, 0.02) drawn in fp32, rounded once to bf16;
+  * with a router projection (``router=True``), W_r [E, H] ~ N(0, 1 / (std
+    sqrt(H))) drawn last, so that x . W_r^T is about N(0, 1) like the
+    given logits;
   * router logits ~ N(0, 1) in fp32, plus a per-expert popularity bias
     -alpha * ln(e + 1) (Zipf popularity 1/(e+1)^alpha; alpha = 0 is uniform
     routing).  The skew knob follows the "--skew-alpha" Zipf router bias of
@@ -22,6 +25,7 @@ SpecForge PR #943 (7-token DSpark blocks x 32 requests = 224 tokens,
 """
 from __future__ import annotations
 
+import math
 from dataclasses import dataclass, replace
 from typing import Optional
 
@@ -84,6 +88,7 @@ class MoEInputs:
     ws_up: Optional[torch.Tensor] = None     # [Is, H] bf16
     ws_down: Optional[torch.Tensor] = None   # [H, Is] bf16
     ws_gvec: Optional[torch.Tensor] = None   # [H] bf16
+    w_router: Optional[torch.Tensor] = None  # [E, H] bf16 (router projection)
 
 
 def zipf_bias(E: int, alpha: float, device="cpu") -> torch.Tensor:
@@ -97,7 +102,7 @@ def _normal_bf16(shape, std, gen, device):
 
 
 def make_inputs(cfg: MoEConfig, device="cpu", seed: Optional[int] = None, std: float = 0.02,
-                gate_std: Optional[float] = None) -> MoEInputs:
+                gate_std: Optional[float] = None, router: bool = False) -> MoEInputs:
     """Draw one seeded input set for ``cfg`` on ``device``.
 
     Large expert tensors are drawn one expert at a time so that the fp32
@@ -125,6 +130,8 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed: Optional[int] = None, std: f
         inp.ws_up = _normal_bf16((cfg.Is, H), std, gen, device)
         inp.ws_down = _normal_bf16((H, cfg.Is), std, gen, device)
         inp.ws_gvec = _normal_bf16((H,), std if gate_std is None else gate_std, gen, device)
+    if router:
+        inp.w_router = _normal_bf16((E, H), 1.0 / (std * math.sqrt(H)), gen, device)
     return inp
 
 

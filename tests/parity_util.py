@@ -49,7 +49,17 @@ def topp_margin(w: np.ndarray, p: float, t: int) -> float:
 
 
 def weights_of(inp: W.MoEInputs) -> moe.MoEWeights:
-    return moe.MoEWeights(inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec)
+    return moe.MoEWeights(inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec,
+                          inp.w_router)
+
+
+def logits_bound(x_bits: np.ndarray, wr_bits: np.ndarray) -> np.ndarray:
+    """Per-logit error bound of an fp32 accumulation: 1e-5 * sum_h |x_h w_h| (+ 1e-6)."""
+    x = x_bits.view(np.uint16).astype(np.uint32) << 16
+    w = wr_bits.view(np.uint16).astype(np.uint32) << 16
+    xf = np.abs(x.view(np.float32).astype(np.float64))
+    wf = np.abs(w.view(np.float32).astype(np.float64))
+    return 1e-5 * (xf @ wf.T) + 1e-6
 
 
 @dataclass

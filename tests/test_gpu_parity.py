@@ -16,7 +16,8 @@ import torch
 import routed_expert_ffn_renorm_b200 as moe
 from routed_expert_ffn_renorm_b200 import workloads as W
 
-from parity_util import check_layer, gpu_forward, lib_config, sample_rows, weights_of
+import oracle
+from parity_util import check_layer, gpu_forward, lib_config, logits_bound, sample_rows, weights_of
 
 pytestmark = pytest.mark.gpu
 
@@ -270,6 +271,63 @@ def test_stagewise_entry_points(cfg):
     xp = x_perm[:total].cpu()
     src = inp.x.cpu()[perm[:total].cpu().long() // k]
     assert torch.equal(xp, src)
+
+
+# ------------------------------------------------------ router projection --
+PROJ = [
+    W.MoEConfig("proj_tiny", T=16, H=256, E=8, I=128, k=2),                 # one split, one tile
+    W.MoEConfig("proj_split", T=40, H=1024, E=24, I=64, k=4, Is=64),        # K split over CTAs
+    W.MoEConfig("proj_wide", T=300, H=512, E=200, I=64, k=6, topp=0.8),     # 3 x 2 tiles, ragged E, split
+    W.MoEConfig("proj_many_tiles", T=2000, H=256, E=64, I=64, k=2),         # 16 tiles, no split
+    W.MoEConfig("proj_e1000", T=7, H=384, E=1000, I=64, k=8, budget=30),    # 8 expert tiles, budget front end
+    W.MoEConfig("proj_drafter", T=224, H=5120, E=16, I=1024, k=2, Is=2048),  # the drafter layer's shape
+]
+
+
+@pytest.mark.parametrize("cfg", PROJ, ids=lambda c: c.name)
+def test_router_projection(cfg):
+    """moe_router_logits against the oracle's fp64 projection (fp32 error
+    bound per logit), the same bits twice, and moe_forward without logits
+    equal, bit for bit, to moe_forward on those logits; the layer then
+    matches the oracle run on the GPU's logits."""
+    inp = W.make_inputs(cfg, device="cuda", router=True)
+    c = lib_config(cfg)
+    ws = torch.zeros(moe.workspace_bytes(c, cfg.T), dtype=torch.uint8, device="cuda")
+    lg = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device="cuda")
+    moe.moe_router_logits(c, inp.x, inp.w_router, lg, ws)
+    lg2 = torch.full_like(lg, float("nan"))
+    moe.moe_router_logits(c, inp.x, inp.w_router, lg2, ws)
+    torch.cuda.synchronize()
+    assert moe.status_read(ws) == 0
+    g = lg.cpu().numpy()
+    assert (g.view(np.uint32) == lg2.cpu().numpy().view(np.uint32)).all(), "projection not deterministic"
+    xb, wb = W.bf16_bits(inp.x), W.bf16_bits(inp.w_router)
+    ref = oracle.router_logits(xb, wb)
+    assert (np.abs(g.astype(np.float64) - ref) <= logits_bound(xb, wb)).all(), \
+        f"max logit error {np.abs(g - ref).max():.3e}"
+    # the layer with the projection inside moe_forward
+    inp_l = W.MoEInputs(inp.x, lg, inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down,
+                        inp.ws_gvec)
+    ref_run = gpu_forward(cfg, inp_l)
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    aux_lg = torch.full_like(lg, float("nan"))
+    ws2 = torch.zeros(moe.workspace_bytes(c, cfg.T), dtype=torch.uint8, device="cuda")
+    moe.moe_forward(c, inp.x, None, weights_of(inp), out, ws2, aux={"logits": aux_lg})
+    torch.cuda.synchronize()
+    assert moe.status_read(ws2) == 0
+    assert (aux_lg.cpu().numpy().view(np.uint32) == g.view(np.uint32)).all()
+    assert (W.bf16_bits(out) == ref_run.out_bits).all()
+    check_layer(cfg, inp_l, ref_run, rows=sample_rows(cfg.T, 48))
+
+
+def test_forward_without_logits_needs_router_weights():
+    cfg = W.MoEConfig("noproj", T=8, H=256, E=8, I=128, k=2)
+    inp = W.make_inputs(cfg, device="cuda")
+    c = lib_config(cfg)
+    ws = torch.zeros(moe.workspace_bytes(c, cfg.T), dtype=torch.uint8, device="cuda")
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError):
+        moe.moe_forward(c, inp.x, None, weights_of(inp), out, ws)
 
 
 def test_budget_is_exact_sequential_sum():
