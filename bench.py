@@ -56,13 +56,16 @@ def workload_from_args(args):
         kw["budget"] = args.budget
     if args.topp is not None:
         kw["topp"] = args.topp
+    if args.router_proj:
+        kw["router_proj"] = True
     return cfg.with_(**kw) if kw else cfg
 
 
 def workload_desc(cfg) -> dict:
     d = {"workload": cfg.label, "tokens": cfg.T, "hidden": cfg.H, "n_routed_experts": cfg.E,
          "moe_intermediate_size": cfg.I, "num_experts_per_tok": cfg.k, "shared_intermediate_size": cfg.Is,
-         "norm_topk": cfg.norm_topk, "budget": cfg.budget, "topp": cfg.topp, "zipf_alpha": cfg.zipf_alpha,
+         "norm_topk": cfg.norm_topk, "budget": cfg.budget, "topp": cfg.topp, "router_proj": cfg.router_proj,
+         "zipf_alpha": cfg.zipf_alpha,
          "seed": cfg.seed,
          "l2": "flushed between timed steps (256 MB write, outside the timed events)"}
     return d
@@ -88,13 +91,16 @@ def stage_work(cfg, counts):
                bytes=touched * 3 * H * I * 2 + sh * 3 * H * Is * 2 + slots * H * 2 + sh * T * H * 2
                + (slots + sh * T) * H * 2)
     route = dict(flops=0, bytes=T * E * 4 + T * k * 8 + sh * (T * H * 2 + H * 2 + T * 4))
+    proj = cfg.router_proj
+    router_proj = dict(flops=2 * T * E * H if proj else 0, bytes=(T * H * 2 + E * H * 2 + T * E * 4) if proj else 0)
     budget = dict(flops=0, bytes=(T * k * 8 * 2) if cfg.budget else 0)
     dispatch = dict(flops=0, bytes=T * k * 4 * 3 + slots * H * 2 * 2)
     combine = dict(flops=0, bytes=(slots + sh * T) * H * 2 + T * H * 2)
-    layer = dict(flops=gate_up["flops"] + down["flops"],
-                 bytes=touched * 3 * H * I * 2 + sh * (3 * H * Is * 2 + H * 2) + 2 * T * H * 2 + T * E * 4)
-    return dict(route=route, budget=budget, dispatch=dispatch, gate_up=gate_up, down=down, ffn=ffn, combine=combine,
-                layer=layer, touched=touched, slots=slots)
+    layer = dict(flops=gate_up["flops"] + down["flops"] + router_proj["flops"],
+                 bytes=touched * 3 * H * I * 2 + sh * (3 * H * Is * 2 + H * 2) + 2 * T * H * 2
+                 + (E * H * 2 if proj else T * E * 4))
+    return dict(router_proj=router_proj, route=route, budget=budget, dispatch=dispatch, gate_up=gate_up, down=down,
+                ffn=ffn, combine=combine, layer=layer, touched=touched, slots=slots)
 
 
 def launches_forward(cfg) -> int:
@@ -102,7 +108,7 @@ def launches_forward(cfg) -> int:
     Tk = cfg.T * cfg.k
     ffn = 1 if (Tk + cfg.E - 1) // cfg.E < 128 else 2  # fused, or gate/up + down once the mean group >= 128
     if cfg.budget and Tk <= 8192 and cfg.T * cfg.E <= 16384:
-        return 1 + ffn + 1  # fused front end (route + budget + dispatch + gather), FFN, combine
+        return int(cfg.router_proj) + 1 + ffn + 1  # [projection], fused front end, FFN, combine
     return launches_stages(cfg)
 
 
@@ -112,7 +118,7 @@ def launches_stages(cfg) -> int:
     ffn = 1 if (Tk + cfg.E - 1) // cfg.E < 128 else 2
     budget = (1 if Tk <= 8192 else 2) if cfg.budget else 0  # one block, or partial sums + select
     dispatch = 1 if Tk <= 8192 else 4  # sort + gather, or histogram + scan + scatter + gather
-    return 1 + budget + dispatch + ffn + 1
+    return int(cfg.router_proj) + 1 + budget + dispatch + ffn + 1
 
 
 def load_peaks():
@@ -294,7 +300,10 @@ def host_inputs(cfg, inp, max_rows: int):
     import oracle
     from routed_expert_ffn_renorm_b200 import workloads as W
     x = W.bf16_bits(inp.x)
-    logits = inp.logits.float().cpu().numpy()
+    if cfg.router_proj:  # the projection's logits, computed once before the timed oracle runs
+        logits = oracle.router_logits(x, W.bf16_bits(inp.w_router))
+    else:
+        logits = inp.logits.float().cpu().numpy()
     if 3 * cfg.E * cfg.H * cfg.I * 2 <= (2 << 30):
         wg, wu, wd = W.bf16_bits(inp.w_gate), W.bf16_bits(inp.w_up), W.bf16_bits(inp.w_down)
     else:
@@ -353,7 +362,8 @@ def run_ours(args, cfg):
     # prebuilt C arguments: the timed loop makes plain C calls
     P = ctypes.c_void_p
     pc = ctypes.byref(c._c())
-    wts = moe.MoEWeights(inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec)
+    wts = moe.MoEWeights(inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec,
+                         inp.w_router)
     pw = ctypes.byref(wts._c())
     p = {n: P(t.data_ptr()) for n, t in dict(idx=idx, tw=tw, sgate=sgate, keff=keff, kept=kept, nd=nd,
                                                 counts=counts, offsets=offsets, perm=perm, slot_pos=slot_pos,
@@ -367,27 +377,32 @@ def run_ours(args, cfg):
         if rc != 0:
             raise moe.MoEError(name, rc, lib.moe_error_string(rc).decode())
 
-    stages = ["route", "budget", "dispatch", "ffn", "combine"]
+    stages = (["router_proj"] if cfg.router_proj else []) + ["route", "budget", "dispatch", "ffn", "combine"]
     NEV = len(stages) + 1
+    pr = int(cfg.router_proj)  # event index shift
+    wr = P(inp.w_router.data_ptr()) if cfg.router_proj else None
 
     def step(ev):
         sp = P(torch.cuda.current_stream(dev).cuda_stream)  # the capture stream while capturing
         st = torch.cuda.current_stream(dev)
         ev[0].record(st)
+        if cfg.router_proj:  # the logits buffer then holds the projection's logits
+            chk("moe_router_logits", lib.moe_router_logits(pc, T, p["x"], wr, p["logits"], p["ws"], wsb, sp))
+            ev[1].record(st)
         chk("moe_route", lib.moe_route(pc, T, p["logits"], p["x"] if cfg.Is else None, gvec, p["idx"], p["tw"], sg,
                                        p["keff"], sp))
-        ev[1].record(st)
+        ev[pr + 1].record(st)
         if cfg.budget:
             chk("moe_budget", lib.moe_budget(pc, T, p["idx"], p["tw"], p["keff"], p["kept"], p["nd"], p["ws"], wsb, sp))
-        ev[2].record(st)
+        ev[pr + 2].record(st)
         chk("moe_dispatch", lib.moe_dispatch(pc, T, p["idx"], p["keff"], p["x"], p["counts"], p["offsets"], p["perm"],
                                              p["slot_pos"], p["x_perm"], p["ws"], wsb, sp))
-        ev[3].record(st)
+        ev[pr + 3].record(st)
         chk("moe_expert_ffn", lib.moe_expert_ffn(pc, T, p["x"], p["x_perm"], p["offsets"], p["perm"], p["tw"], sg, pw,
                                                  p["ybuf"], p["ws"], wsb, sp))
-        ev[4].record(st)
+        ev[pr + 4].record(st)
         chk("moe_combine", lib.moe_combine(pc, T, p["ybuf"], p["keff"], p["out"], sp))
-        ev[5].record(st)
+        ev[pr + 5].record(st)
 
     def capture(fn):
         g = torch.cuda.CUDAGraph()
@@ -436,7 +451,8 @@ def run_ours(args, cfg):
     def fwd_step(e0, e1):
         st = torch.cuda.current_stream(dev)
         e0.record(st)
-        chk("moe_forward", lib.moe_forward(pc, T, p["x"], p["logits"], pw, p["out"], ctypes.byref(aux_c), p["ws"],
+        chk("moe_forward", lib.moe_forward(pc, T, p["x"], None if cfg.router_proj else p["logits"], pw, p["out"],
+                                           ctypes.byref(aux_c), p["ws"],
                                            wsb, P(st.cuda_stream)))
         e1.record(st)
 
@@ -498,8 +514,9 @@ def run_ours(args, cfg):
             st = torch.cuda.current_stream(dev)
             e0.record(st)
             xd.copy_(xh, non_blocking=True)
-            ld.copy_(lh, non_blocking=True)
-            moe.moe_forward(c, xd, ld, wts, out, ws, stream=st)
+            if not cfg.router_proj:  # else the layer computes its logits from x
+                ld.copy_(lh, non_blocking=True)
+            moe.moe_forward(c, xd, None if cfg.router_proj else ld, wts, out, ws, stream=st)
             oh.copy_(out, non_blocking=True)
             e1.record(st)
 
@@ -522,7 +539,7 @@ def run_ours(args, cfg):
         barrier(dev)
         e2e_ms = max_over_ranks(e2e_sum, dev)
         e2e = {"value": aggregate_tokens_per_s(T, args.steps, e2e_ms, world), "unit": "tokens/s",
-               "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2,
+               "h2d_bytes_per_step": T * H * 2 + (0 if cfg.router_proj else T * E * 4), "d2h_bytes_per_step": T * H * 2,
                "ms_per_step": e2e_ms / args.steps, "api": "moe_forward (one CUDA graph per step with the copies)"}
         if not torch.equal(oh.to(dev), out):
             raise RuntimeError("e2e output copy mismatch")
@@ -557,6 +574,8 @@ def run_ours(args, cfg):
         "gpu_launches": (launches_forward(cfg) + launches_stages(cfg)) * args.steps,
         "clocks": sampler.summary(),
         "stages_ms": per_stage,
+        **({"router_proj_roofline": roofline("router_proj", work, per_stage["router_proj"], peaks, peak_kind,
+                                             long_run, None)} if cfg.router_proj else {}),
         "layer": {"touched_experts": work["touched"], "kept_slots": work["slots"],
                   "algorithmic_bytes": work["layer"]["bytes"], "algorithmic_flops": work["layer"]["flops"],
                   "GB_per_s": layer_bw, "TFLOP_per_s": layer_tf,
@@ -625,6 +644,8 @@ def main(argv=None):
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--topp", type=float, default=None, help="per-token top-p trim (0 = off)")
+    ap.add_argument("--router-proj", action="store_true",
+                    help="compute the logits with the router projection x . W_r^T inside the layer")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -13,13 +13,9 @@ namespace {
 
 constexpr size_t kAlign = 256;
 // Head of the workspace: [0, 256) status word and work-item counters,
-// [256, 256 + 4 * (E + 2)) gate/up completion counters of the fused FFN,
-// [4608, 8192) the router projection's K-split counters.
+// [256, 256 + 4 * (E + 2)) gate/up completion counters of the fused FFN.
 constexpr size_t kHeadBytes = 8192;
 constexpr size_t kHdoneOffset = 256;
-constexpr size_t kRpCntOffset = 4608;
-static_assert(kRpCntOffset >= kHdoneOffset + 4 * (kMaxExperts + 2), "counter regions overlap");
-static_assert(kRpCntOffset + 4 * kRpMaxCounters <= kHeadBytes, "projection counters exceed the head");
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
@@ -359,8 +355,7 @@ int moe_router_logits(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, c
     const WsLayout L = ws_layout(*cfg, T);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     return cuda_rc(launch_router_proj(T, cfg->n_routed_experts, cfg->hidden, x, w_router, logits,
-                                      at<float>(ws, L.rpart), at<int32_t>(ws, L.status + kRpCntOffset),
-                                      at<int32_t>(ws, L.status), as_stream(stream)));
+                                      at<float>(ws, L.rpart), at<int32_t>(ws, L.status), as_stream(stream)));
 }
 
 int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits, const moe_weights_t *w,

@@ -88,12 +88,10 @@ cudaError_t launch_front(int T, int E, int k, int N, int norm_topk, float topp, 
                          uint16_t *x_perm, int32_t *status_block, int32_t *hdone, cudaStream_t st);
 
 // Router projection logits = x . W_r^T on the tensor cores (router_proj.cu).
-// `part` holds rp_partial_bytes(T, E, H) bytes of K-split partials; `cnt` is
-// kRpMaxCounters zeroed ints (the kernel leaves them zero).
-constexpr int kRpMaxCounters = 896;
+// `part` holds rp_partial_bytes(T, E, H) bytes of K-split partials.
 size_t rp_partial_bytes(int T, int E, int H);
 cudaError_t launch_router_proj(int T, int E, int H, const uint16_t *x, const uint16_t *w_router, float *logits,
-                               float *part, int32_t *cnt, int32_t *status, cudaStream_t st);
+                               float *part, int32_t *status, cudaStream_t st);
 
 // Combine.
 cudaError_t launch_combine(int T, int k, int H, int has_shared, const uint16_t *ybuf,

@@ -13,9 +13,9 @@
 //
 // Small batches have few tiles and a long K (H / 64 slices), so a tile's K
 // range is split over several CTAs: each split stores its fp32 partial in
-// the workspace, and the last split of the tile to finish (an atomic count)
-// adds the partials in split order -- a fixed order, so the logits are the
-// same bits on every run -- and resets the count for the next launch.
+// the workspace, and a second, element-parallel kernel adds the partials in
+// split order -- a fixed order, so the logits are the same bits on every
+// run.
 //
 // Roles (192 threads): warp 0 -- TMA producer (one lane); warp 1 -- TMEM
 // allocation and MMA issue (one lane); warps 2..5 -- epilogue, one TMEM lane
@@ -32,13 +32,15 @@ namespace {
 using namespace tc;
 
 constexpr int kRpThreads = 192;
-constexpr int kRpStages = 6;                      // ring stages of one K slice each
+constexpr int kRpStages = 3;                      // ring stages of up to two K slices each
+constexpr int kRpSlices = 2;                      // K slices per stage: one barrier round trip per two
 constexpr int kRpBN = 128;                        // widest token tile (MMA N)
 constexpr int kRpABytes = 128 * 64 * 2;           // 16 KB: 128 rows of W_r x 64 K
-constexpr int kRpStageBytes = kRpABytes + kRpBN * 128;  // + BN token rows x 64 K
+constexpr int kRpSubBytes = kRpABytes + kRpBN * 128;    // one slice: + BN token rows x 64 K
+constexpr int kRpStageBytes = kRpSlices * kRpSubBytes;  // 64 KB
 constexpr int kRpMinSlices = 4;                   // K slices per split at least
+constexpr int kRpMaxSplits = 16;                  // K splits at most
 constexpr int kRpMaxSms = 160;                    // no device has more SMs (workspace sizing)
-constexpr int kRpMaxTiles = kRpMaxCounters;       // tiles whose splits the workspace head can count
 
 struct __align__(64) RpMaps {
     CUtensorMap a;  // W_r [E, H], box 64 x 128
@@ -51,7 +53,6 @@ struct RpParams {
     int wt, items;        // expert tiles, work items (token tiles x expert tiles x splits)
     float *logits;        // [T, E]
     float *part;          // [S, T, E] partials (S > 1)
-    int32_t *cnt;         // [token tiles x expert tiles] finished splits, zero between launches
     int32_t *status;
 };
 
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(kRpThreads, 1) router_proj_kernel(const __grid
     uint64_t *mma_done = tempty + 2;       // every MMA of the CTA has completed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *last_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);
+    volatile int *epi_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // elected -> epilogue: 0 go, -1 stop
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t tmem_cols = 2 * kRpBN;  // two accumulators of up to 128 columns
     pdl_launch_dependents();
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kRpThreads, 1) router_proj_kernel(const __grid
     if (warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
-            const uint32_t bytes = kRpABytes + (uint32_t)p.BN * 128;
+            const uint32_t sub_bytes = kRpABytes + (uint32_t)p.BN * 128;
             int st = 0;
             uint32_t ph = 0;
             uint32_t issued = 0;
@@ -123,16 +124,19 @@ __global__ void __launch_bounds__(kRpThreads, 1) router_proj_kernel(const __grid
                 int j, r, s;
                 decode(item, j, r, s);
                 const int k0 = s * p.kper, k1 = min(p.nk, k0 + p.kper);
-                for (int k = k0; k < k1; ++k) {
+                for (int k = k0; k < k1; k += kRpSlices) {
+                    const int n = min(kRpSlices, k1 - k);
                     if (issued >= (uint32_t)kRpStages &&
                         !mbar_wait_fast(&empty[st], ph ^ 1u, abort_flag, p.status, true)) {
                         ok = false;
                         break;
                     }
                     uint8_t *dst = ring + (size_t)st * kRpStageBytes;
-                    mbar_arrive_expect_tx(&full[st], bytes);
-                    tma_load_2d(&maps.a, &full[st], dst, k * 64, r * 128);
-                    tma_load_2d(&maps.b, &full[st], dst + kRpABytes, k * 64, j * p.BN);
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)n * sub_bytes);
+                    for (int u = 0; u < n; ++u) {
+                        tma_load_2d(&maps.a, &full[st], dst + u * kRpSubBytes, (k + u) * 64, r * 128);
+                        tma_load_2d(&maps.b, &full[st], dst + u * kRpSubBytes + kRpABytes, (k + u) * 64, j * p.BN);
+                    }
                     ++issued;
                     if (++st == kRpStages) {
                         st = 0;
@@ -162,17 +166,20 @@ __global__ void __launch_bounds__(kRpThreads, 1) router_proj_kernel(const __grid
                 if (!mbar_wait_fast(&tempty[acc], (use & 1u) ^ 1u, abort_flag, p.status, true)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(acc * kRpBN);
-                for (int k = k0; k < k1; ++k) {
+                for (int k = k0; k < k1; k += kRpSlices) {
+                    const int n = min(kRpSlices, k1 - k);
                     if (!mbar_wait_fast(&full[st], ph, abort_flag, p.status, true)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t da = desc0 + (uint64_t)st * (kRpStageBytes / 16);
-                    const uint64_t db = da + kRpABytes / 16;
+                    for (int u = 0; u < n; ++u) {
+                        const uint64_t da = desc0 + (uint64_t)(st * kRpStageBytes + u * kRpSubBytes) / 16;
+                        const uint64_t db = da + kRpABytes / 16;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // K16 steps: +32 bytes each
-                        umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (k > k0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)  // K16 steps: +32 bytes each
+                            umma_bf16(d, da + 2 * kk, db + 2 * kk, idesc, (k + u > k0 || kk > 0) ? 1u : 0u);
+                    }
                     umma_commit(&empty[st]);
                     if (++st == kRpStages) {
                         st = 0;
@@ -189,16 +196,15 @@ __global__ void __launch_bounds__(kRpThreads, 1) router_proj_kernel(const __grid
         // ================= epilogue (warps 2..5) =================
         const int q = warp & 3;  // TMEM lane quarter of this warp: experts r*128 + 32q ..
         const bool elected = (warp == 2 && lane == 0);
-        const int et = threadIdx.x - 64;  // 0..127 over the epilogue warps
         int li = 0;
         for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++li) {
             int j, r, s;
             decode(item, j, r, s);
             const int acc = li & 1;
             const uint32_t use = (uint32_t)(li >> 1);
-            if (elected) *last_flag = mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 0 : -1;
+            if (elected) *epi_flag = mbar_wait(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 0 : -1;
             named_bar_sync(1, 128);
-            if (*last_flag) break;
+            if (*epi_flag) break;
             tc_fence_after();
             float *dst = p.S > 1 ? p.part + (size_t)s * p.T * p.E : p.logits;
             const int e = r * 128 + q * 32 + lane;
@@ -216,30 +222,6 @@ __global__ void __launch_bounds__(kRpThreads, 1) router_proj_kernel(const __grid
             tc_fence_before();
             named_bar_sync(1, 128);
             if (elected) mbar_arrive(&tempty[acc]);
-            if (p.S > 1) {
-                // the tile's last split to finish adds the partials in split order
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (elected) {
-                    const int tile = j * p.wt + r;
-                    *last_flag = atomicAdd(p.cnt + tile, 1) == p.S - 1;
-                }
-                named_bar_sync(1, 128);
-                if (*last_flag) {
-                    __threadfence();
-                    const int tn = min(p.BN, p.T - j * p.BN), en = min(128, p.E - r * 128);
-                    for (int idx = et; idx < tn * en; idx += 128) {
-                        const int t = j * p.BN + idx / en, ee = r * 128 + idx % en;
-                        const size_t off = (size_t)t * p.E + ee;
-                        float a = 0.f;
-                        for (int ss = 0; ss < p.S; ++ss) a += __ldcg(p.part + (size_t)ss * p.T * p.E + off);
-                        p.logits[off] = a;
-                    }
-                    if (elected) atomicExch(p.cnt + j * p.wt + r, 0);
-                }
-                named_bar_sync(1, 128);
-                if (elected) *last_flag = 0;
-            }
         }
     }
 
@@ -251,19 +233,35 @@ __global__ void __launch_bounds__(kRpThreads, 1) router_proj_kernel(const __grid
     }
 }
 
+// logits = the S split partials of every element added in split order.
+__global__ void __launch_bounds__(256) router_proj_reduce_kernel(long long n, int S, const float *__restrict__ part,
+                                                                 float *__restrict__ logits) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float v[kRpMaxSplits];  // every partial in flight at once
+#pragma unroll
+    for (int s = 0; s < kRpMaxSplits; ++s) v[s] = s < S ? __ldg(part + s * n + i) : 0.f;
+    float a = v[0];
+#pragma unroll
+    for (int s = 1; s < kRpMaxSplits; ++s)
+        if (s < S) a += v[s];
+    logits[i] = a;
+}
+
 }  // namespace
 
 // Token tile and K splits of a projection of T tokens over E experts with H
 // hidden units on `sms` SMs: BN = the tokens rounded up to 16, at most 128;
-// a tile's K range is split while there are fewer tiles than SMs, each split
-// keeping at least kRpMinSlices slices, and only while the tile counters fit
-// the workspace head.
+// a tile's K range is split (into at most kRpMaxSplits) while there are fewer
+// tiles than SMs, each split keeping at least kRpMinSlices slices.
 void rp_shape(int T, int E, int H, int sms, int *BN, int *S, int *kper) {
     *BN = std::min(kRpBN, std::max(16, (T + 15) / 16 * 16));
     const int tt = (T + *BN - 1) / *BN, wt = (E + 127) / 128, nk = H / 64;
     const int tiles = tt * wt;
     int s = 1;
-    if (tiles < sms && tiles <= kRpMaxTiles) s = std::max(1, std::min(nk / kRpMinSlices, sms / tiles));
+    if (tiles < sms) s = std::max(1, std::min(std::min(nk / kRpMinSlices, sms / tiles), kRpMaxSplits));
     *kper = (nk + s - 1) / s;
     *S = (nk + *kper - 1) / *kper;  // no empty split
 }
@@ -275,7 +273,7 @@ size_t rp_partial_bytes(int T, int E, int H) {
 }
 
 cudaError_t launch_router_proj(int T, int E, int H, const uint16_t *x, const uint16_t *w_router, float *logits,
-                               float *part, int32_t *cnt, int32_t *status, cudaStream_t st) {
+                               float *part, int32_t *status, cudaStream_t st) {
     const int sms = device_sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
     int BN, S, kper;
@@ -294,7 +292,6 @@ cudaError_t launch_router_proj(int T, int E, int H, const uint16_t *x, const uin
     p.items = ((T + BN - 1) / BN) * p.wt * S;
     p.logits = logits;
     p.part = part;
-    p.cnt = cnt;
     p.status = status;
     static std::atomic<int> attr_set[64];  // per device: opted in to the ring's shared memory
     int dev = 0;
@@ -306,7 +303,11 @@ cudaError_t launch_router_proj(int T, int E, int H, const uint16_t *x, const uin
         attr_set[dev].store(1, std::memory_order_release);
     }
     const int grid = std::max(1, std::min(sms, p.items));
-    return launch_pdl(router_proj_kernel, dim3(grid), dim3(kRpThreads), rp_smem(), st, m, p);
+    cudaError_t e = launch_pdl(router_proj_kernel, dim3(grid), dim3(kRpThreads), rp_smem(), st, m, p);
+    if (e != cudaSuccess || S == 1) return e;
+    const long long n = (long long)T * E;
+    return launch_pdl(router_proj_reduce_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, n, S,
+                      static_cast<const float *>(part), logits);
 }
 
 }  // namespace moe

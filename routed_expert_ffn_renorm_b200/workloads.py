@@ -45,6 +45,7 @@ class MoEConfig:
     budget: int = 0   # EXPERT_BUDGET (0 = off)
     zipf_alpha: float = 0.0
     topp: float = 0.0  # per-token top-p trim (0 = off)
+    router_proj: bool = False  # logits from the router projection x . W_r^T instead of given
     seed: int = 0
 
     def with_(self, **kw) -> "MoEConfig":
@@ -61,6 +62,8 @@ class MoEConfig:
             s += f"_a{self.zipf_alpha:g}"
         if self.topp:
             s += f"_p{self.topp:g}"
+        if self.router_proj:
+            s += "_proj"
         return s
 
 
@@ -130,7 +133,7 @@ def make_inputs(cfg: MoEConfig, device="cpu", seed: Optional[int] = None, std: f
         inp.ws_up = _normal_bf16((cfg.Is, H), std, gen, device)
         inp.ws_down = _normal_bf16((H, cfg.Is), std, gen, device)
         inp.ws_gvec = _normal_bf16((H,), std if gate_std is None else gate_std, gen, device)
-    if router:
+    if router or cfg.router_proj:
         inp.w_router = _normal_bf16((E, H), 1.0 / (std * math.sqrt(H)), gen, device)
     return inp
 
