@@ -273,7 +273,8 @@ cudaError_t launch_dispatch(int T, int E, int k, const int32_t *idx, const int32
                             int32_t *status_block, int32_t *hdone, const uint16_t *x, uint16_t *x_perm, int H,
                             cudaStream_t st) {
     if (dispatch_is_small(T, k)) {
-        const int W = E <= 256 ? 32 : (E <= 512 ? 16 : 8);  // per-warp counts fit in 32 KB
+        // per-warp counts fit in 32 KB; no more warps than 32-slot passes (fewer columns to scan)
+        const int W = std::min(E <= 256 ? 32 : (E <= 512 ? 16 : 8), std::max(1, (T * k + 31) / 32));
         const size_t smem = ((size_t)W * E + (size_t)T * k) * 4;  // <= 64 KB
         static std::atomic<int> attr_set[64];
         int dev = 0;

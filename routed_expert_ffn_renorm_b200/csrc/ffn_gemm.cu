@@ -483,8 +483,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             const uint64_t bpol = policy_evict_normal();  // token rows (pair loads take a policy)
             // items are claimed one ahead: a CTA (pair) takes item blockIdx (cluster
             // index) first, then from the counter, past the first grid's worth
+            // (the counter's value is only added to when the next claim is made, so the
+            // atomic's round trip -- long at launch, when every CTA claims at once -- never
+            // stalls this lane's in-order issue)
             const int claimers = kPair ? (int)gridDim.x / 2 : (int)gridDim.x;
-            int next = kPair ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+            int pending = -1;  // counter value of the claim in flight; -1: the first, static item
             bool all_ready = false;                       // every gate/up item of the launch is done
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
@@ -493,8 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 Item it{};
                 if (!kPair || rank == 0) {
                     if (!mbar_wait<kPair>(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
-                    item = next < total_items ? next : -1;
-                    if (item >= 0) next = claimers + atomicAdd(p.sched, 1);  // latency overlaps this item's loads
+                    item = pending < 0 ? (kPair ? (int)blockIdx.x / 2 : (int)blockIdx.x) : claimers + pending;
+                    if (item >= total_items) item = -1;
+                    if (item >= 0) pending = atomicAdd(p.sched, 1);  // latency overlaps this item's loads
                     if (item >= 0) it = decode_item(item, sc, p);  // decoded once, for all roles
                     qdesc[slot].item = item;
                     qdesc[slot].it = it;

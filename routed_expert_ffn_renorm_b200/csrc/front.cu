@@ -4,7 +4,7 @@
 //
 // Every CTA copies the T x E logits to shared memory in one coalesced pass and
 // routes all T tokens itself from there (route_token_lane, one token per
-// thread, for E <= 64; route_token, one warp per token, above),
+// thread, for 32 < E <= 64; route_token, one warp per token, otherwise),
 // applies the budget (budget_block) and sorts the kept slots by expert
 // (block_sort_by_expert, or regroup_kept from the budget's own sort) -- the
 // same device code, or the same order, as the stand-alone route / budget /
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_small_kernel(const Fro
     const int T = a.T, E = a.E, k = a.k, Tk = T * k, W = sort_warps(E);
     // logit rows: stride E for warp routing, an odd stride for lane routing (a
     // warp then reads 32 rows at once without bank conflicts)
-    const bool lane_route = E <= kLaneRouteMaxE;
+    const bool lane_route = lane_routed(E);
     const int ls = lane_route ? (E | 1) : E;
     float *logit_s = reinterpret_cast<float *>(sm);  // [T * ls]
     int32_t *idx_s = reinterpret_cast<int32_t *>(logit_s + (size_t)T * (E + 1));

@@ -160,14 +160,18 @@ __device__ __forceinline__ int route_token(int t, int E, int k, int norm_topk, f
     return route_token_impl<V, kGlobal, false>(t, E, k, norm_topk, topp, logits, idx, w, keff, lane);
 }
 
-// One token per thread, for E <= kLaneRouteMaxE: the same decisions as
+// One token per thread, for 32 < E <= kLaneRouteMaxE: the same decisions as
 // route_token, with every sum taken in expert order (max, then
 // sum_e exp(l_e - max), then k rounds of first-maximum selection over the
 // untaken experts, then the renormalising sum in slot order, then the top-p
 // trim).  A warp routes 32 tokens at once with no shuffles.  `l` is the
 // token's row of logits (global memory when kGlobal, else shared memory).
-// Returns the kept slot count.
+// Returns the kept slot count.  Used for 32 < E <= 64: at most 32 experts one
+// logit per lane of the warp router is faster (measured, the 16-expert drafter
+// layer), above 64 the warp router is.
+constexpr int kLaneRouteMinE = 33;
 constexpr int kLaneRouteMaxE = 64;
+__host__ __device__ inline bool lane_routed(int E) { return E >= kLaneRouteMinE && E <= kLaneRouteMaxE; }
 
 template <bool kGlobal>
 __device__ __forceinline__ int route_token_lane(int t, int E, int k, int norm_topk, float topp, const float *l,

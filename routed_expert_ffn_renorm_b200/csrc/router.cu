@@ -6,8 +6,8 @@
 //
 // route_kernel<V>: one block per token; its first warp routes (route_token,
 // front.cuh) while the next four compute the shared-expert gate
-// (shared_gate_group), side by side.  route_lane_kernel (E <= 64): separate blocks route
-// 32 tokens lane by lane and compute the gates.  Both read the logits (and
+// (shared_gate_group), side by side.  route_lane_kernel (32 < E <= 64):
+// separate blocks route 32 tokens lane by lane and compute the gates.  Both read the logits (and
 // x) once; they are latency-bound and small next to the expert FFN.
 #include "front.cuh"
 
@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int 
     if (tid == 0) sgate[t] = g;
 }
 
-// E <= kLaneRouteMaxE: the first ceil(T / 32) blocks route 32 tokens each, one
+// 32 < E <= kLaneRouteMaxE: the first ceil(T / 32) blocks route 32 tokens each, one
 // token per lane of their first warp (route_token_lane), from the tokens'
 // logits staged in shared memory; the remaining T blocks (with a shared
 // expert) compute one token's shared gate each.  Routing and gate blocks run
@@ -89,7 +89,7 @@ cudaError_t launch_v(int T, int E, int k, int norm_topk, float topp, const float
 cudaError_t launch_route(int T, int E, int k, int norm_topk, float topp, const float *logits, int32_t *idx, float *w,
                          int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,
                          cudaStream_t st) {
-    if (E <= kLaneRouteMaxE)
+    if (lane_routed(E))
         return launch_pdl(route_lane_kernel, dim3((T + 31) / 32 + (sgate != nullptr ? T : 0)), dim3(kGateThreads), 0,
                           st, T, E, k, norm_topk, topp, logits, idx, w, keff, x, gvec, H, sgate);
     if (E <= 128) return launch_v<4>(T, E, k, norm_topk, topp, logits, idx, w, keff, x, gvec, H, sgate, st);

@@ -53,9 +53,9 @@ SMALL = [
     W.MoEConfig("budget_chunks", T=700, H=128, E=64, I=64, k=6, budget=9, zipf_alpha=0.5),
     W.MoEConfig("max_experts", T=64, H=128, E=1024, I=64, k=8),
     W.MoEConfig("max_topk", T=16, H=128, E=64, I=64, k=32),
-    # per-token top-p trim: lane router (E <= 64), warp router, 16-byte lane loads (E > 128), no norm,
+    # per-token top-p trim: lane router (32 < E <= 64), warp router, 16-byte lane loads (E > 128), no norm,
     # with the budget (fused front end, one-block and chunked budgets)
-    W.MoEConfig("topp_lane", T=64, H=256, E=32, I=64, k=6, Is=64, topp=0.7),
+    W.MoEConfig("topp_lane", T=64, H=256, E=48, I=64, k=6, Is=64, topp=0.7),
     W.MoEConfig("topp_warp", T=50, H=256, E=128, I=64, k=8, topp=0.5, zipf_alpha=0.5),
     W.MoEConfig("topp_vec", T=40, H=128, E=256, I=64, k=8, topp=0.85),
     W.MoEConfig("topp_no_norm", T=48, H=256, E=16, I=64, k=4, norm_topk=False, topp=0.3),
