@@ -20,7 +20,9 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 v) {
 }
 
 // One thread per (token, 16-byte column vector); the rows of a token are
-// loaded four at a time and added in slot order.
+// added in slot order.  The first four slot rows and the shared row are
+// loaded together with keff (every row of ybuf is in bounds; rows past keff
+// are loaded but not added), so the common case takes one memory round trip.
 __global__ void __launch_bounds__(256) combine_kernel(int T, int k, int vec, int has_shared,
                                                       const uint4 *__restrict__ ybuf,
                                                       const int32_t *__restrict__ keff, uint4 *__restrict__ out) {
@@ -29,20 +31,26 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int k, int vec, int
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const int t = (int)(gid / vec), c = (int)(gid % vec);
     if (t >= T) return;
-    const int ke = keff ? __ldg(keff + t) : k;
     const uint4 *rows = ybuf + (size_t)t * (k + 1) * vec + c;
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = u < k ? __ldg(rows + (size_t)u * vec) : make_uint4(0, 0, 0, 0);
+    const uint4 vs = has_shared ? __ldg(rows + (size_t)k * vec) : make_uint4(0, 0, 0, 0);
+    const int ke = keff ? __ldg(keff + t) : k;
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j0 = 0; j0 < ke; j0 += 4) {
-        uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        if (u < ke) add_bf16x8(acc, v[u]);
+    for (int j0 = 4; j0 < ke; j0 += 4) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) v[u] = (j0 + u < ke) ? __ldg(rows + (size_t)(j0 + u) * vec) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             if (j0 + u < ke) add_bf16x8(acc, v[u]);
     }
-    if (has_shared) add_bf16x8(acc, __ldg(rows + (size_t)k * vec));
+    if (has_shared) add_bf16x8(acc, vs);
     uint32_t o[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q)

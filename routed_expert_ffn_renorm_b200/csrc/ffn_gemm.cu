@@ -44,9 +44,9 @@
 // pair ("ticket", 32 of them), and the producer reuses pages only after the
 // MMAs of the steps that held them have committed.  Both lanes are on the
 // critical path of every step, so a step carries two 64-wide K slices when
-// its token box is at most 64 rows (32 KB of weights per barrier round
-// trip), and their loops avoid divisions and out-of-line calls on the
-// common path.
+// they fit 24 pages, or 32 pages with room for two such steps in the ring
+// (32 KB of weights per barrier round trip), and their loops avoid divisions
+// and out-of-line calls on the common path.
 //
 // Roles (192 threads, one CTA per SM, persistent): warp 0 -- TMA producer
 // (one lane); warp 1 -- TMEM allocation and MMA issue (one lane); warps
