@@ -269,10 +269,12 @@ def sample_order(T: int):
     return np.random.default_rng(0).permutation(T).astype(np.int32)
 
 
-def oracle_rows_per_s(cfg, inp_host, target_s: float, max_rows: int):
+def oracle_rows_per_s(cfg, inp_host, target_s: float, max_rows: int, repeat: bool = False):
     """Time the oracle on a bounded sample of rows (the first n of
     sample_order).  Routing, budget and dispatch run over the whole batch; the
-    FFN and combine over the sample.  Returns (rows/s, rows, seconds, threads)."""
+    FFN and combine over the sample.  With `repeat`, a batch whose every row
+    fits well inside target_s is run again until about target_s has passed.
+    Returns (rows/s, rows, passes, seconds, threads)."""
     import oracle
     x, logits, wg, wu, wd, shared = inp_host
     nthreads = oracle.max_threads()
@@ -290,7 +292,11 @@ def oracle_rows_per_s(cfg, inp_host, target_s: float, max_rows: int):
     n2 = int(min(max_rows, max(n, n * target_s / max(dt, 1e-6))))
     if n2 > n:
         n, dt = n2, run(n2)
-    return n / dt, n, dt, nthreads
+    passes = 1
+    if repeat and n == max_rows and 2 * dt < target_s:
+        passes = int(target_s / max(dt, 1e-6))
+        dt = sum(run(n) for _ in range(passes))
+    return n * passes / dt, n, passes, dt, nthreads
 
 
 def host_inputs(cfg, inp, max_rows: int):
@@ -559,10 +565,10 @@ def run_ours(args, cfg):
     if rank == 0 and world == 1 and not args.no_cpu:
         mr = cpu_max_rows(cfg)
         hi = host_inputs(cfg, inp, mr)
-        rps, nrows, secs, thr = oracle_rows_per_s(cfg, hi, args.cpu_seconds, mr)
+        rps, nrows, passes, secs, thr = oracle_rows_per_s(cfg, hi, args.cpu_seconds, mr, repeat=True)
         cpu = {"value": rps, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                "sample": f"{nrows} of {T} tokens of {cfg.label}: routing, budget and dispatch over all {T} tokens, "
-                         f"expert FFN + combine (fp64 accumulate) for the sample; {secs:.1f} s"}
+                         f"expert FFN + combine (fp64 accumulate) for the sample; {passes} pass(es), {secs:.1f} s"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -605,7 +611,7 @@ def run_reference(args, cfg):
     mr = cpu_max_rows(cfg)
     hi = host_inputs(cfg, inp, mr)
     per_step = min(5.0, 150.0 / max(args.steps + args.warmup, 1))  # whole run within a few minutes
-    rps, nrows, secs, thr = oracle_rows_per_s(cfg, hi, per_step, mr)
+    rps, nrows, _, secs, thr = oracle_rows_per_s(cfg, hi, per_step, mr)
     import oracle
     x, logits, wg, wu, wd, shared = hi
     rows = sample_order(cfg.T)[:nrows]
