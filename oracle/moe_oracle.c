@@ -28,7 +28,7 @@
  * Activations and weights arrive as bf16 bit patterns and are widened
  * exactly.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent or leave a step open:
  *  - top-k ties: equal logits -> the lower expert id ranks first;
  *  - slot order inside a token: descending logit;
  *  - budget ties: equal aggregate weight -> the lower expert id is kept;
