@@ -16,6 +16,10 @@ Each function follows a passage of the pages:
   * colibri issue_budget.md (EXPERT_BUDGET), "How it works" steps 1-5 and
     "Safety": the batch-union expert budget; "Relationship to existing
     features": the per-position top-p trim (TOPP) that runs before it.
+  * ``quant_oracle.c``: the block-scaled FP8 (MXFP8) and NVFP4 expert-weight
+    formats that DeepGEMM fork PR #5 and DeepGEMM PR #381 name for expert
+    weights, with their published definitions (E4M3, E2M1, UE8M0 codecs,
+    block quantisers and dequantisers).
 """
 from __future__ import annotations
 
@@ -28,6 +32,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
+_SRCS = (_SRC, os.path.join(_HERE, "quant_oracle.c"))
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 _lib = None
@@ -35,9 +40,9 @@ _lib = None
 
 def build(force: bool = False) -> str:
     """Compile liboracle.so next to its source (gcc, OpenMP)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(os.path.getmtime(f) for f in _SRCS):
         tmp = _LIB + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", _SRC, "-o", tmp, "-lm"]
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", *_SRCS, "-o", tmp, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB)
     return _LIB
@@ -64,6 +69,15 @@ def _load():
     lib.oracle_forward.argtypes = [i32] * 8 + [ctypes.c_float] + [P] * 9 + [i32, P, P] + [P] * 9 + [i32]
     lib.oracle_combine_rows.argtypes = [i32] * 5 + [P] * 4 + [P] * 3 + [P] * 4 + [i32, P, P, i32]
     lib.oracle_max_threads.restype = ctypes.c_int
+    i64 = ctypes.c_int64
+    for name in ("oracle_e4m3_decode", "oracle_e4m3_encode", "oracle_e2m1_decode", "oracle_e2m1_encode",
+                 "oracle_ue8m0_decode"):
+        getattr(lib, name).argtypes = [i64, P, P]
+        getattr(lib, name).restype = None
+    lib.oracle_mxfp8_quantize.argtypes = [i64, i64, P, P, P]
+    lib.oracle_mxfp8_dequantize.argtypes = [i64, i64, P, P, P]
+    lib.oracle_nvfp4_quantize.argtypes = [i64, i64, P, P, P, P]
+    lib.oracle_nvfp4_dequantize.argtypes = [i64, i64, P, P, ctypes.c_float, P]
     _lib = lib
     return lib
 
@@ -295,3 +309,109 @@ def combine_rows(x, idx, w, keff, w_gate, w_up, w_down, *, I: int, ws_gate=None,
                                        rows.shape[0], _ptr(rows), _ptr(out), nthreads), "combine_rows")
     return out[: rows.shape[0]]
 
+
+
+# ------------------------------------------------ block-scaled weights --
+def _codec(name, a, in_dtype, out_dtype):
+    a = _c(a, in_dtype)
+    out = np.empty(a.shape, out_dtype)
+    getattr(_load(), name)(a.size, _ptr(a), _ptr(out))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 codes (uint8) -> their values (float64; NaN for 0x7F, 0xFF)."""
+    return _codec("oracle_e4m3_decode", codes, np.uint8, np.float64)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Values -> the nearest E4M3 codes (ties to even, saturating at 448)."""
+    return _codec("oracle_e4m3_encode", x, np.float64, np.uint8)
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """E2M1 codes (low nibble of each uint8) -> their values (float64)."""
+    return _codec("oracle_e2m1_decode", codes, np.uint8, np.float64)
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """Values -> the nearest E2M1 codes (ties to even, saturating at 6)."""
+    return _codec("oracle_e2m1_encode", x, np.float64, np.uint8)
+
+
+def ue8m0_decode(codes) -> np.ndarray:
+    """UE8M0 scale codes -> 2^(c - 127) (NaN for 255)."""
+    return _codec("oracle_ue8m0_decode", codes, np.uint8, np.float64)
+
+
+def mxfp8_quantize(w):
+    """bf16 bit patterns [rows, K] (K % 32 == 0) -> (E4M3 codes [rows, K],
+    UE8M0 scales [rows, K / 32]); blocks run along the last axis."""
+    w = _c(w, np.uint16)
+    rows, K = w.reshape(-1, w.shape[-1]).shape
+    codes = np.empty(w.shape, np.uint8)
+    scales = np.empty(w.shape[:-1] + (K // 32,), np.uint8)
+    _check(_load().oracle_mxfp8_quantize(rows, K, _ptr(w), _ptr(codes), _ptr(scales)), "mxfp8_quantize")
+    return codes, scales
+
+
+def mxfp8_dequantize(codes, scales) -> np.ndarray:
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    K = codes.shape[-1]
+    out = np.empty(codes.shape, np.float64)
+    _check(_load().oracle_mxfp8_dequantize(codes.size // K, K, _ptr(codes), _ptr(scales), _ptr(out)),
+           "mxfp8_dequantize")
+    return out
+
+
+def nvfp4_quantize(w):
+    """bf16 bit patterns [rows, K] (K % 16 == 0), one matrix -> (packed E2M1
+    codes [rows, K / 2], E4M3 block scales [rows, K / 16], fp32 matrix scale)."""
+    w = _c(w, np.uint16)
+    rows, K = w.reshape(-1, w.shape[-1]).shape
+    codes = np.empty(w.shape[:-1] + (K // 2,), np.uint8)
+    scales = np.empty(w.shape[:-1] + (K // 16,), np.uint8)
+    st = np.zeros(1, np.float32)
+    _check(_load().oracle_nvfp4_quantize(rows, K, _ptr(w), _ptr(codes), _ptr(scales), _ptr(st)),
+           "nvfp4_quantize")
+    return codes, scales, float(st[0])
+
+
+def nvfp4_dequantize(codes, scales, tensor_scale: float) -> np.ndarray:
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    K = codes.shape[-1] * 2
+    out = np.empty(codes.shape[:-1] + (K,), np.float64)
+    _check(_load().oracle_nvfp4_dequantize(codes.size * 2 // K, K, _ptr(codes), _ptr(scales),
+                                           float(np.float32(tensor_scale)), _ptr(out)), "nvfp4_dequantize")
+    return out
+
+
+def f64_to_bf16_exact(v) -> np.ndarray:
+    """float64 values that bf16 holds exactly -> bf16 bit patterns; raises
+    when one is not exact (the dequantised MXFP8 weights always are in the
+    exponent range of these layers)."""
+    v = np.asarray(v, np.float64)
+    f = v.astype(np.float32)
+    bits = f.view(np.uint32)
+    if not np.array_equal(f.astype(np.float64), v, equal_nan=True) or np.any(bits & 0xFFFF):
+        raise ValueError("value not representable in bf16")
+    return (bits >> 16).astype(np.uint16)
+
+
+def mxfp8_weights(w):
+    """An expert matrix (bf16 bits, reduction axis last) stored as MXFP8:
+    the bf16 bit patterns of its dequantised values, which the MMA then
+    consumes unchanged."""
+    codes, scales = mxfp8_quantize(w)
+    return f64_to_bf16_exact(mxfp8_dequantize(codes, scales))
+
+
+def forward_mxfp8(x, logits, w_gate, w_up, w_down, *, ws_gate=None, ws_up=None, ws_down=None, **kw):
+    """The layer with MXFP8 expert weights (routed and shared; the shared
+    gate vector stays bf16): each matrix quantised along its reduction axis,
+    dequantised exactly, then the bf16 layer definition."""
+    shared = {}
+    if ws_gate is not None:
+        shared = dict(ws_gate=mxfp8_weights(ws_gate), ws_up=mxfp8_weights(ws_up), ws_down=mxfp8_weights(ws_down))
+    return forward(x, logits, mxfp8_weights(w_gate), mxfp8_weights(w_up), mxfp8_weights(w_down),
+                   **shared, **kw)

@@ -93,7 +93,8 @@ def _load_mutant(name, tmp):
     path_so = os.path.join(tmp, f"lib{name}.so")
     with open(path_c, "w") as f:
         f.write(src.replace(old, new))
-    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fopenmp", path_c, "-o", path_so, "-lm"],
+    quant_c = os.path.join(ROOT, "oracle", "quant_oracle.c")  # the rest of the oracle library, unchanged
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fopenmp", path_c, quant_c, "-o", path_so, "-lm"],
                    check=True)
     # a fresh copy of the oracle wrapper module bound to the mutant library
     spec = importlib.util.spec_from_file_location(f"oracle_mutant_{name}", os.path.join(ROOT, "oracle", "__init__.py"))
