@@ -66,8 +66,8 @@ def _load():
     lib.oracle_expert_rows.argtypes = [i32, i32, P, P, P, i32, P, P, i32]
     lib.oracle_shared_gate_row.restype = ctypes.c_double
     lib.oracle_shared_gate_row.argtypes = [i32, P, P]
-    lib.oracle_forward.argtypes = [i32] * 8 + [ctypes.c_float] + [P] * 9 + [i32, P, P] + [P] * 9 + [i32]
-    lib.oracle_combine_rows.argtypes = [i32] * 5 + [P] * 4 + [P] * 3 + [P] * 4 + [i32, P, P, i32]
+    lib.oracle_forward.argtypes = [i32] * 8 + [ctypes.c_float] + [P] * 11 + [i32, P, P] + [P] * 9 + [i32]
+    lib.oracle_combine_rows.argtypes = [i32] * 5 + [P] * 4 + [P] * 3 + [P] * 6 + [i32, P, P, i32]
     lib.oracle_max_threads.restype = ctypes.c_int
     i64 = ctypes.c_int64
     for name in ("oracle_e4m3_decode", "oracle_e4m3_encode", "oracle_e2m1_decode", "oracle_e2m1_encode",
@@ -226,16 +226,34 @@ def _expert_ptrs(w, E):
     return arr, keep
 
 
+def _scale_ptrs(scales, shared_scales, E):
+    """Per-projection output factors: scales [E, 3] (gate, up, down) and
+    shared_scales [3], float64; None passes NULL (no factor)."""
+    keep = []
+    ps = pss = None
+    if scales is not None:
+        a = _c(scales, np.float64).reshape(E, 3)
+        keep.append(a)
+        ps = _ptr(a)
+    if shared_scales is not None:
+        b = _c(shared_scales, np.float64).reshape(3)
+        keep.append(b)
+        pss = _ptr(b)
+    return ps, pss, keep
+
+
 def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, budget: int = 0,
             topp: float = 0.0, ws_gate=None, ws_up=None, ws_down=None, ws_gvec=None, rows=None,
-            nthreads: int = 1, I: int = None) -> ForwardResult:
+            nthreads: int = 1, I: int = None, scales=None, shared_scales=None) -> ForwardResult:
     """The whole layer. x and all weights are bf16 bit patterns (uint16).
 
     x [T,H]; logits [T,E] f32; w_gate, w_up [E,I,H] and w_down [E,H,I] as full
     arrays, or as dicts {expert: [I,H] / [H,I] array} holding only the experts
     the requested rows route to (then pass I);
     shared (optional): ws_gate, ws_up [Is,H], ws_down [H,Is], ws_gvec [H].
-    rows: token ids whose output to compute (default: all)."""
+    rows: token ids whose output to compute (default: all);
+    scales [E, 3], shared_scales [3]: factors on each projection's output
+    (gate, up, down), the fp32 matrix scales of block-scaled weights."""
     x = _c(x, np.uint16)
     logits = _c(logits, np.float32)
     T, H = x.shape
@@ -263,10 +281,11 @@ def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, 
     offsets = np.empty(E + 1, np.int32)
     perm = np.full(max(T * k, 1), -1, np.int32)
     slot_pos = np.empty(max(T * k, 1), np.int32)
+    ps, pss, _keep = _scale_ptrs(scales, shared_scales, E)
     rc = _load().oracle_forward(
         T, H, E, I, k, Is, int(bool(norm_topk)), budget, float(topp),
         _ptr(x), _ptr(logits), pg, pu, pd,
-        _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec),
+        _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec), ps, pss,
         n_rows, _ptr(rows), _ptr(out),
         _ptr(idx), _ptr(w), _ptr(keff), _ptr(kept), _ptr(nd),
         _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(slot_pos), nthreads)
@@ -277,7 +296,7 @@ def forward(x, logits, w_gate, w_up, w_down, *, k: int, norm_topk: bool = True, 
 
 
 def combine_rows(x, idx, w, keff, w_gate, w_up, w_down, *, I: int, ws_gate=None, ws_up=None, ws_down=None,
-                 ws_gvec=None, rows=None, nthreads: int = 1) -> np.ndarray:
+                 ws_gvec=None, rows=None, nthreads: int = 1, scales=None, shared_scales=None) -> np.ndarray:
     """Expert FFN + weighted combine (+ gated shared expert) for GIVEN routing
     (idx/w/keff, e.g. after a budget), for the listed token rows.  Weights as
     in forward().  Returns out [n_rows, H] float64."""
@@ -304,8 +323,9 @@ def combine_rows(x, idx, w, keff, w_gate, w_up, w_down, *, I: int, ws_gate=None,
         ws_gate = ws_up = ws_down = ws_gvec = np.zeros(1, np.uint16)
     rows = np.arange(T, dtype=np.int32) if rows is None else _c(rows, np.int32)
     out = np.empty((max(rows.shape[0], 1), H), np.float64)
+    ps, pss, _keep = _scale_ptrs(scales, shared_scales, E)
     _check(_load().oracle_combine_rows(T, H, I, k, Is, _ptr(x), _ptr(idx), _ptr(w), _ptr(keff), pg, pu, pd,
-                                       _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec),
+                                       _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(ws_gvec), ps, pss,
                                        rows.shape[0], _ptr(rows), _ptr(out), nthreads), "combine_rows")
     return out[: rows.shape[0]]
 
@@ -415,3 +435,31 @@ def forward_mxfp8(x, logits, w_gate, w_up, w_down, *, ws_gate=None, ws_up=None, 
         shared = dict(ws_gate=mxfp8_weights(ws_gate), ws_up=mxfp8_weights(ws_up), ws_down=mxfp8_weights(ws_down))
     return forward(x, logits, mxfp8_weights(w_gate), mxfp8_weights(w_up), mxfp8_weights(w_down),
                    **shared, **kw)
+
+
+def nvfp4_weights(w):
+    """Expert matrices [..., rows, K] (bf16 bits, reduction axis last) stored
+    as NVFP4, one fp32 matrix scale per leading index: (the bf16 bit patterns
+    of element x block scale, exact in bf16, and the matrix scales)."""
+    w = _c(w, np.uint16)
+    lead = w.shape[:-2]
+    flat = w.reshape((-1,) + w.shape[-2:])
+    vals, sts = [], []
+    for m in flat:
+        codes, scales, st = nvfp4_quantize(m)
+        vals.append(f64_to_bf16_exact(nvfp4_dequantize(codes, scales, 1.0)))
+        sts.append(st)
+    return np.stack(vals).reshape(w.shape), np.array(sts, np.float64).reshape(lead)
+
+
+def forward_nvfp4(x, logits, w_gate, w_up, w_down, *, ws_gate=None, ws_up=None, ws_down=None, **kw):
+    """The layer with NVFP4 expert weights (routed and shared; the shared gate
+    vector stays bf16): each expert matrix quantised along its reduction axis
+    with its own fp32 scale; the projections take element x block scale as
+    their weights and multiply their outputs by the matrix scale."""
+    (wg, sg), (wu, su), (wd, sd) = (nvfp4_weights(a) for a in (w_gate, w_up, w_down))
+    extra = {}
+    if ws_gate is not None:
+        (g2, s2g), (u2, s2u), (d2, s2d) = (nvfp4_weights(a) for a in (ws_gate, ws_up, ws_down))
+        extra = dict(ws_gate=g2, ws_up=u2, ws_down=d2, shared_scales=np.array([s2g, s2u, s2d], np.float64))
+    return forward(x, logits, wg, wu, wd, scales=np.stack([sg, su, sd], axis=-1), **extra, **kw)

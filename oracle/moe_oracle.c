@@ -283,10 +283,15 @@ int oracle_dispatch(int32_t T, int32_t E, int32_t k, const int32_t *idx, const i
 /* ---------------------------------------------------------------------- */
 /* y = W_down . ( silu(W_gate . x) * (W_up . x) ),  silu(g) = g / (1 + e^-g).
  * W_gate, W_up: [I, H] row-major; W_down: [H, I] row-major; x: [H].
- * Everything accumulates in fp64. */
+ * Everything accumulates in fp64.  `scale` (NULL: none) holds one factor per
+ * projection {gate, up, down} that multiplies its output: the fp32 matrix
+ * scale of weights stored in a block-scaled format (quant_oracle.c), whose
+ * element-times-block-scale values are what W holds.  A factor of 1 leaves
+ * every value bit-identical. */
 static void swiglu_ffn(int32_t H, int32_t I, const uint16_t *wg, const uint16_t *wu,
-                       const uint16_t *wd, const uint16_t *x, double *hbuf, double *y)
+                       const uint16_t *wd, const double *scale, const uint16_t *x, double *hbuf, double *y)
 {
+    const double sg = scale ? scale[0] : 1.0, su = scale ? scale[1] : 1.0, sd = scale ? scale[2] : 1.0;
     for (int32_t i = 0; i < I; ++i) {
         double g = 0.0, u = 0.0;
         const uint16_t *rg = wg + (size_t)i * H, *ru = wu + (size_t)i * H;
@@ -295,13 +300,15 @@ static void swiglu_ffn(int32_t H, int32_t I, const uint16_t *wg, const uint16_t 
             g += bf16_to_f64(rg[c]) * xc;
             u += bf16_to_f64(ru[c]) * xc;
         }
+        g *= sg;
+        u *= su;
         hbuf[i] = g / (1.0 + exp(-g)) * u;
     }
     for (int32_t o = 0; o < H; ++o) {
         double a = 0.0;
         const uint16_t *rd = wd + (size_t)o * I;
         for (int32_t i = 0; i < I; ++i) a += bf16_to_f64(rd[i]) * hbuf[i];
-        y[o] = a;
+        y[o] = sd * a;
     }
 }
 
@@ -321,7 +328,7 @@ int oracle_expert_rows(int32_t H, int32_t I, const uint16_t *wg, const uint16_t 
         } else {
 #pragma omp for schedule(dynamic, 1)
             for (int32_t r = 0; r < n; ++r)
-                swiglu_ffn(H, I, wg, wu, wd, x + (size_t)r * H, hbuf, y + (size_t)r * H);
+                swiglu_ffn(H, I, wg, wu, wd, NULL, x + (size_t)r * H, hbuf, y + (size_t)r * H);
         }
         free(hbuf);
     }
@@ -347,13 +354,14 @@ double oracle_shared_gate_row(int32_t H, const uint16_t *g, const uint16_t *x)
  * Weights: w_gate[e], w_up[e] point to expert e's [I, H] projections and
  * w_down[e] to its [H, I] projection (an entry may be NULL when no listed
  * row routes to e); ws_gate, ws_up [Is, H]; ws_down [H, Is]; ws_gvec [H]
- * (all bf16 bit patterns, row-major). */
+ * (all bf16 bit patterns, row-major).  scales [E][3] and shared_scales [3]
+ * (NULL: none) are the per-projection output factors of swiglu_ffn. */
 int oracle_combine_rows(int32_t T, int32_t H, int32_t I, int32_t k, int32_t Is,
                         const uint16_t *x, const int32_t *idx, const float *w, const int32_t *keff,
                         const uint16_t *const *w_gate, const uint16_t *const *w_up,
                         const uint16_t *const *w_down,
                         const uint16_t *ws_gate, const uint16_t *ws_up, const uint16_t *ws_down,
-                        const uint16_t *ws_gvec,
+                        const uint16_t *ws_gvec, const double *scales, const double *shared_scales,
                         int32_t n_rows, const int32_t *rows, double *out, int32_t nthreads)
 {
     if (T < 0 || H < 1 || I < 1 || k < 1 || Is < 0 || n_rows < 0) return ORACLE_EINVAL;
@@ -385,9 +393,10 @@ int oracle_combine_rows(int32_t T, int32_t H, int32_t I, int32_t k, int32_t Is,
                         err = 2;
                         continue;
                     }
-                    swiglu_ffn(H, I, w_gate[e], w_up[e], w_down[e], xt, hbuf, y);
+                    swiglu_ffn(H, I, w_gate[e], w_up[e], w_down[e], scales ? scales + (size_t)e * 3 : NULL, xt,
+                               hbuf, y);
                 } else {
-                    swiglu_ffn(H, Is, ws_gate, ws_up, ws_down, xt, hbuf, y);
+                    swiglu_ffn(H, Is, ws_gate, ws_up, ws_down, shared_scales, xt, hbuf, y);
                 }
             }
         }
@@ -424,7 +433,7 @@ int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_
                    const uint16_t *const *w_gate, const uint16_t *const *w_up,
                    const uint16_t *const *w_down,
                    const uint16_t *ws_gate, const uint16_t *ws_up, const uint16_t *ws_down,
-                   const uint16_t *ws_gvec,
+                   const uint16_t *ws_gvec, const double *scales, const double *shared_scales,
                    int32_t n_rows, const int32_t *rows, double *out,
                    int32_t *idx, float *w, int32_t *keff, uint8_t *kept, int32_t *n_dropped,
                    int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *slot_pos,
@@ -441,7 +450,8 @@ int oracle_forward(int32_t T, int32_t H, int32_t E, int32_t I, int32_t k, int32_
     rc = oracle_dispatch(T, E, k, idx, keff, counts, offsets, perm, slot_pos);
     if (rc) return rc;
     return oracle_combine_rows(T, H, I, k, Is, x, idx, w, keff, w_gate, w_up, w_down,
-                               ws_gate, ws_up, ws_down, ws_gvec, n_rows, rows, out, nthreads);
+                               ws_gate, ws_up, ws_down, ws_gvec, scales, shared_scales, n_rows, rows, out,
+                               nthreads);
 }
 
 int oracle_max_threads(void)

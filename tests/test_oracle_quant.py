@@ -218,9 +218,71 @@ def pin_forward_mxfp8(o):
     np.testing.assert_array_equal(_bf16_value(q[0][0]).reshape(I, H), d)
 
 
+def _exact_nvfp4_matrix(o, rng, rows, K, st_exp):
+    """Values NVFP4 holds exactly, whose quantisation gives back s_t = 2^st_exp:
+    every block reaches 6 x its scale and one block has the largest scale."""
+    e2 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    mag = e2[rng.integers(0, 8, (rows, K))]
+    mag[:, ::16] = 6.0
+    sign = np.where(rng.integers(0, 2, (rows, K)) == 1, -1.0, 1.0)
+    sbv = o.e4m3_decode(rng.integers(0x30, 0x7E, (rows, K // 16)).astype(np.uint8))
+    sbv[0, 0] = 448.0
+    return sign * mag * np.repeat(sbv, 16, axis=1) * 2.0 ** st_exp
+
+
+def _small_layer(rng, T=12, H=64, E=4, I=32, k=2, Is=32, sigma=0.1):
+    x = _bf16_bits(rng.standard_normal((T, H)))
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    mk = lambda *s: _bf16_bits(rng.standard_normal(s) * sigma)
+    return x, logits, [mk(E, I, H), mk(E, I, H), mk(E, H, I)], [mk(Is, H), mk(Is, H), mk(H, Is)], mk(H)
+
+
+def pin_forward_output_scales(o):
+    rng = np.random.default_rng(9)
+    x, logits, (wg, wu, wd), (sg, su, sd), gv = _small_layer(rng)
+    E = wg.shape[0]
+    base = o.forward(x, logits, wg, wu, wd, ws_gate=sg, ws_up=su, ws_down=sd, ws_gvec=gv, k=2).out
+    up = lambda a, p: _bf16_bits(_bf16_value(a).reshape(a.shape) * 2.0 ** p)
+    # weights times 2, 4, 8 (gate, up, down), output factors 1/2, 1/4, 1/8: the same layer, bit for bit
+    scaled = o.forward(x, logits, up(wg, 1), up(wu, 2), up(wd, 3), ws_gate=up(sg, 1), ws_up=up(su, 2),
+                       ws_down=up(sd, 3), ws_gvec=gv, k=2, scales=np.tile([0.5, 0.25, 0.125], (E, 1)),
+                       shared_scales=[0.5, 0.25, 0.125]).out
+    np.testing.assert_array_equal(scaled, base)
+    ones = o.forward(x, logits, wg, wu, wd, ws_gate=sg, ws_up=su, ws_down=sd, ws_gvec=gv, k=2,
+                     scales=np.ones((E, 3)), shared_scales=np.ones(3)).out
+    np.testing.assert_array_equal(ones, base)
+    # per-expert factors: expert 1's down factor 2 doubles exactly its routed contribution
+    w2 = np.ones((E, 3))
+    w2[1, 2] = 2.0
+    f = o.forward(x, logits, wg, wu, wd, k=2, scales=w2)
+    plain = o.forward(x, logits, wg, wu, wd, k=2)
+    only1 = o.combine_rows(x, plain.idx, plain.w, plain.keff, np.where(np.arange(E)[:, None, None] == 1, wg, 0),
+                           wu, wd, I=wg.shape[1])
+    np.testing.assert_allclose(f.out - plain.out, only1, rtol=1e-12, atol=1e-15)
+
+
+def pin_forward_nvfp4(o):
+    rng = np.random.default_rng(10)
+    x, logits, (wg, wu, wd), (sg, su, sd), gv = _small_layer(rng)
+    kw = dict(ws_gvec=gv, k=2)
+    base = o.forward(x, logits, wg, wu, wd, ws_gate=sg, ws_up=su, ws_down=sd, **kw).out
+    quant = o.forward_nvfp4(x, logits, wg, wu, wd, ws_gate=sg, ws_up=su, ws_down=sd, **kw).out
+    rel = np.linalg.norm(quant - base) / np.linalg.norm(base)
+    assert 0 < rel < 0.5  # one mantissa bit: tens of percent, never exact here
+    # weights that NVFP4 holds with power-of-two matrix scales: the quantised layer is the bf16 layer
+    E, I, H = wg.shape
+    ex = lambda shape, p: _bf16_bits(np.stack([_exact_nvfp4_matrix(o, rng, *shape, p) for _ in range(E)]))
+    eg, eu, ed = ex((I, H), -8), ex((I, H), -9), ex((H, I), -7)
+    es = [_bf16_bits(_exact_nvfp4_matrix(o, rng, *s, p)) for s, p in (((32, H), -8), ((32, H), -6), ((H, 32), -9))]
+    want = o.forward(x, logits, eg, eu, ed, ws_gate=es[0], ws_up=es[1], ws_down=es[2], **kw).out
+    got = o.forward_nvfp4(x, logits, eg, eu, ed, ws_gate=es[0], ws_up=es[1], ws_down=es[2], **kw).out
+    np.testing.assert_array_equal(got, want)
+
+
 PINS = [pin_e4m3_constants, pin_e4m3_decode_matches_torch, pin_e4m3_encode_nearest_even, pin_e2m1_table,
         pin_ue8m0_matches_torch, pin_mxfp8_scale_rule, pin_mxfp8_error_bound, pin_mxfp8_exact_identity,
-        pin_nvfp4_scale_rule, pin_nvfp4_error_bound, pin_nvfp4_exact_identity_and_packing, pin_forward_mxfp8]
+        pin_nvfp4_scale_rule, pin_nvfp4_error_bound, pin_nvfp4_exact_identity_and_packing, pin_forward_mxfp8,
+        pin_forward_output_scales, pin_forward_nvfp4]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -230,31 +292,37 @@ def test_pin(oracle_mod, pin):
 
 # -------------------------------------------------------------- mutants --
 MUTANTS = {
-    "e4m3_bias_8": ("ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
-    "e4m3_subnormal_exp": ("ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)"),
-    "ties_to_larger": ("(d == best_d && (c & 1) == 0 && (best & 1) != 0)", "(d == best_d)"),
-    "ieee_style_top_exponent": ("if (e == 15 && m == 7) return NAN;", "if (e == 15) return NAN;"),
-    "sign_dropped": ("return signbit(x) ? (uint8_t)(c | 0x80) : c;", "return c;"),
-    "e2m1_bias_0": ("ldexp(1.0 + 0.5 * (double)m, e - 1)", "ldexp(1.0 + 0.5 * (double)m, e)"),
-    "mx_scale_ceil": ("se = e2 - 1 - 8;", "se = e2 - 8;"),
-    "mx_scale_emax_7": ("se = e2 - 1 - 8;", "se = e2 - 1 - 7;"),
-    "nvfp4_global_448x4": ("amax / 2688.0f", "amax / 1792.0f"),
-    "nvfp4_block_max_4": ("amax_b / (6.0f * st)", "amax_b / (4.0f * st)"),
-    "nvfp4_nibbles_swapped": ("codes[at / 2] |= (uint8_t)(at % 2 == 0 ? q : q << 4);",
+    "e4m3_bias_8": ("quant", "ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)"),
+    "e4m3_subnormal_exp": ("quant", "ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)"),
+    "ties_to_larger": ("quant", "(d == best_d && (c & 1) == 0 && (best & 1) != 0)", "(d == best_d)"),
+    "ieee_style_top_exponent": ("quant", "if (e == 15 && m == 7) return NAN;", "if (e == 15) return NAN;"),
+    "sign_dropped": ("quant", "return signbit(x) ? (uint8_t)(c | 0x80) : c;", "return c;"),
+    "e2m1_bias_0": ("quant", "ldexp(1.0 + 0.5 * (double)m, e - 1)", "ldexp(1.0 + 0.5 * (double)m, e)"),
+    "mx_scale_ceil": ("quant", "se = e2 - 1 - 8;", "se = e2 - 8;"),
+    "mx_scale_emax_7": ("quant", "se = e2 - 1 - 8;", "se = e2 - 1 - 7;"),
+    "nvfp4_global_448x4": ("quant", "amax / 2688.0f", "amax / 1792.0f"),
+    "nvfp4_block_max_4": ("quant", "amax_b / (6.0f * st)", "amax_b / (4.0f * st)"),
+    "nvfp4_nibbles_swapped": ("quant", "codes[at / 2] |= (uint8_t)(at % 2 == 0 ? q : q << 4);",
                               "codes[at / 2] |= (uint8_t)(at % 2 == 0 ? q << 4 : q);"),
-    "mx_dequant_wrong_block": ("(int)scales[r * (K / 32) + i / 32] - 127", "(int)scales[r * (K / 32) + i / 16 % (K / 32)] - 127"),
+    "mx_dequant_wrong_block": ("quant", "(int)scales[r * (K / 32) + i / 32] - 127", "(int)scales[r * (K / 32) + i / 16 % (K / 32)] - 127"),
+    "scale_gate_up_swapped": ("moe", "g *= sg;\n        u *= su;", "g *= su;\n        u *= sg;"),
+    "scale_down_dropped": ("moe", "y[o] = sd * a;", "y[o] = a;"),
+    "shared_scales_ignored": ("moe", "swiglu_ffn(H, Is, ws_gate, ws_up, ws_down, shared_scales, xt, hbuf, y);",
+                              "swiglu_ffn(H, Is, ws_gate, ws_up, ws_down, NULL, xt, hbuf, y);"),
+    "scales_of_expert_0": ("moe", "scales ? scales + (size_t)e * 3 : NULL", "scales"),
 }
 
 
 def _load_mutant(name, tmp):
-    old, new = MUTANTS[name]
-    src = open(QSRC).read()
+    which, old, new = MUTANTS[name]
+    target, other = (QSRC, MSRC) if which == "quant" else (MSRC, QSRC)
+    src = open(target).read()
     assert src.count(old) == 1, f"mutant {name}: anchor not found exactly once"
     path_c = os.path.join(tmp, f"{name}.c")
     path_so = os.path.join(tmp, f"lib{name}.so")
     with open(path_c, "w") as f:
         f.write(src.replace(old, new))
-    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fopenmp", MSRC, path_c, "-o", path_so, "-lm"],
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fopenmp", other, path_c, "-o", path_so, "-lm"],
                    check=True)
     spec = importlib.util.spec_from_file_location(f"oracle_qmutant_{name}", os.path.join(ROOT, "oracle", "__init__.py"))
     mod = importlib.util.module_from_spec(spec)
