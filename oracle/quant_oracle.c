@@ -81,9 +81,13 @@ static double e2m1_value(uint8_t c)
 }
 
 /* Nearest code among the non-negative finite codes 0..n_pos-1 (values
- * strictly increasing with the code), ties to the even code. */
+ * strictly increasing with the code), ties to the even code.  At or beyond
+ * the largest value that value is the nearest (saturation); it is returned
+ * directly, since far beyond it the distances to the top codes round to the
+ * same double. */
 static uint8_t nearest_code(double mag, double (*value)(uint8_t), int n_pos)
 {
+    if (mag >= value((uint8_t)(n_pos - 1))) return (uint8_t)(n_pos - 1);
     int best = 0;
     double best_d = fabs(mag - value(0));
     for (int c = 1; c < n_pos; ++c) {

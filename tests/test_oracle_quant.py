@@ -56,7 +56,8 @@ def pin_e4m3_encode_nearest_even(o):
     gap = pv[1:] - pv[:-1]
     np.testing.assert_array_equal(o.e4m3_encode(mid - gap / 8), pos[:-1])
     np.testing.assert_array_equal(o.e4m3_encode(mid + gap / 8), pos[1:])
-    assert o.e4m3_encode([449.0, 464.0, 500.0, 1e9, -1e9]).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+    assert o.e4m3_encode([449.0, 464.0, 500.0, 1e9, -1e9, 1.2e18, 3e38, -3e38]).tolist() == \
+        [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x7E, 0x7E, 0xFE]
     assert o.e4m3_encode([-0.0, -1e-6, 1e-6]).tolist() == [0x80, 0x80, 0x00]
     x = np.random.default_rng(0).standard_normal(4096) * np.exp2(np.random.default_rng(1).integers(-12, 8, 4096))
     x = np.clip(x, -448, 448).astype(np.float32)
@@ -71,7 +72,7 @@ def pin_e2m1_table(o):
     assert o.e2m1_encode(np.array(mags)).tolist() == list(range(8))
     # ties between neighbours go to the even code; beyond 6 saturates
     assert o.e2m1_encode([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 100.0]).tolist() == [0, 2, 2, 4, 4, 6, 6, 7, 7]
-    assert o.e2m1_encode([0.26, 0.74, 2.4, 5.1, -5.1, -0.0]).tolist() == [1, 1, 4, 7, 15, 8]
+    assert o.e2m1_encode([0.26, 0.74, 2.4, 5.1, -5.1, -0.0, 1e18, -3e38]).tolist() == [1, 1, 4, 7, 15, 8, 7, 15]
 
 
 def pin_ue8m0_matches_torch(o):
