@@ -249,6 +249,44 @@ int moe_status_clear(void *ws, void *stream);
 /* Static text for a return code. */
 const char *moe_error_string(int code);
 
+/* ---------------------------------------------------------------------
+ * Block-scaled expert weights: the pack step (run once when the weights are
+ * loaded).  The formats are the FP8 and NVFP4 expert weights of DeepGEMM
+ * fork PR #5 "big M opt: splitT1 + L2 scatter + 2 stream" (its megamoe_nvfp4
+ * kernels, its B200 FP8 x FP4 policy), with the published definitions:
+ * E4M3 without infinities (largest finite 448), E2M1 (magnitudes 0, 0.5, 1,
+ * 1.5, 2, 3, 4, 6), UE8M0 (2^(c - 127)).  Rounding is to nearest, ties to
+ * the even code, saturating; the sign bit copies the input's.  The blocks
+ * run along the last (reduction) axis of a row-major matrix: rows of
+ * W_gate / W_up [I, H] and of W_down [H, I].  The layer does not consume
+ * these formats yet.
+ * --------------------------------------------------------------------- */
+
+/* MXFP8: blocks of 32 consecutive elements share a UE8M0 scale
+ * X = 2^(floor(log2(amax)) - 8) (clamped to [2^-127, 2^127]; an all-zero
+ * block takes 2^-127), each element is x / X rounded to E4M3.
+ * w      [rows, K] bf16, K a multiple of 32 (device, 16-byte aligned);
+ * codes  [rows, K] uint8 E4M3 (device, 16-byte aligned, written);
+ * scales [rows, K / 32] uint8 UE8M0 (device, written).
+ * Enqueued on `stream`; MOE_ERR_INVALID_ARG for a bad size or pointer. */
+int moe_quantize_mxfp8(int64_t rows, int32_t K, const moe_bf16_t *w, uint8_t *codes, uint8_t *scales,
+                       void *stream);
+
+/* NVFP4: nmat matrices of [rows, K], stored one after another.  Each matrix
+ * has an fp32 scale s_t = amax / (6 * 448) (1 when all zero); blocks of 16
+ * consecutive elements share an E4M3 scale s_b = E4M3(amax_b / (6 * s_t));
+ * each element is E2M1(x / (s_b * s_t)), all in IEEE fp32 in that order.
+ * w            [nmat, rows, K] bf16, K a multiple of 16 (device, 16-byte aligned);
+ * codes        [nmat, rows, K / 2] uint8, two E2M1 codes per byte, element 2i
+ *              in the low nibble (device, 16-byte aligned, written);
+ * scales       [nmat, rows, K / 16] uint8 E4M3 (device, written);
+ * tensor_scale [nmat] fp32 (device, 4-byte aligned, written; also the
+ *              reduction's scratch while the call runs).
+ * 1 <= nmat <= 65535.  Enqueued on `stream`; MOE_ERR_INVALID_ARG for a bad
+ * size or pointer. */
+int moe_quantize_nvfp4(int32_t nmat, int64_t rows, int32_t K, const moe_bf16_t *w, uint8_t *codes, uint8_t *scales,
+                       float *tensor_scale, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

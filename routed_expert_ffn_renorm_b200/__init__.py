@@ -25,7 +25,7 @@ __all__ = [
     "MoEConfig", "MoEWeights", "MoEError", "load_library", "workspace_bytes", "moe_router_logits", "moe_route",
     "moe_budget",
     "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn_noalloc",
-    "moe_combine", "moe_forward",
+    "moe_combine", "moe_forward", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
     "status_read", "status_clear",
     "EXPORTED_SYMBOLS", "MOE_STATUS_TIMEOUT",
 ]
@@ -36,7 +36,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_route", "moe_budget", "moe_dispatch", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_status_read", "moe_status_clear", "moe_error_string", "moe_expert_gate_up",
-    "moe_expert_down", "moe_expert_ffn_noalloc", "moe_router_logits",
+    "moe_expert_down", "moe_expert_ffn_noalloc", "moe_router_logits", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 MOE_STATUS_TIMEOUT = 1
@@ -134,6 +134,9 @@ def load_library(build_if_stale: bool = True):
         lib.moe_forward.argtypes = [cfg, i32, P, P, ctypes.POINTER(_Weights), P, ctypes.POINTER(_Aux), P, sz, P]
         lib.moe_status_read.argtypes = [P, ctypes.POINTER(i32), P]
         lib.moe_status_clear.argtypes = [P, P]
+        i64 = ctypes.c_int64
+        lib.moe_quantize_mxfp8.argtypes = [i64, i32, P, P, P, P]
+        lib.moe_quantize_nvfp4.argtypes = [i32, i64, i32, P, P, P, P, P]
         lib.moe_error_string.restype = ctypes.c_char_p
         lib.moe_error_string.argtypes = [ctypes.c_int]
         for name in EXPORTED_SYMBOLS:
@@ -183,6 +186,23 @@ def moe_router_logits(cfg: MoEConfig, x, w_router, logits, ws, stream=None):
     _check("moe_router_logits", load_library().moe_router_logits(
         ctypes.byref(cfg._c()), T, _ptr(x), _ptr(w_router), _ptr(logits), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def moe_quantize_mxfp8(w, codes, scales, stream=None):
+    """MXFP8 weights: w [..., K] bf16 -> codes [..., K] uint8 (E4M3) and
+    scales [..., K // 32] uint8 (UE8M0), blocks along the last axis."""
+    K = w.shape[-1]
+    _check("moe_quantize_mxfp8", load_library().moe_quantize_mxfp8(
+        w.numel() // K, K, _ptr(w), _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def moe_quantize_nvfp4(w, codes, scales, tensor_scale, stream=None):
+    """NVFP4 weights: w [nmat, rows, K] bf16 -> codes [nmat, rows, K // 2]
+    uint8 (two E2M1 per byte, element 2i low), scales [nmat, rows, K // 16]
+    uint8 (E4M3), tensor_scale [nmat] fp32 (one per matrix)."""
+    nmat, rows, K = w.shape
+    _check("moe_quantize_nvfp4", load_library().moe_quantize_nvfp4(
+        nmat, rows, K, _ptr(w), _ptr(codes), _ptr(scales), _ptr(tensor_scale), _stream(stream)))
 
 
 def moe_route(cfg: MoEConfig, logits, topk_idx, topk_w, *, x=None, ws_gate_vec=None, sgate=None, keff=None,

@@ -346,6 +346,23 @@ int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, cons
                                   keff, out, as_stream(stream)));
 }
 
+int moe_quantize_mxfp8(int64_t rows, int32_t K, const moe_bf16_t *w, uint8_t *codes, uint8_t *scales,
+                       void *stream) {
+    if (rows < 0 || K < 32 || K % 32 != 0) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!aligned(w) || !aligned(codes) || !scales) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_quantize_mxfp8(rows, K, w, codes, scales, as_stream(stream)));
+}
+
+int moe_quantize_nvfp4(int32_t nmat, int64_t rows, int32_t K, const moe_bf16_t *w, uint8_t *codes, uint8_t *scales,
+                       float *tensor_scale, void *stream) {
+    if (nmat < 1 || nmat > 65535 || rows < 0 || K < 16 || K % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (!tensor_scale || (reinterpret_cast<uintptr_t>(tensor_scale) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!aligned(w) || !aligned(codes) || !scales) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_quantize_nvfp4(nmat, rows, K, w, codes, scales, tensor_scale, as_stream(stream)));
+}
+
 int moe_router_logits(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *w_router,
                       float *logits, void *ws, size_t ws_bytes, void *stream) {
     int rc = check_config(cfg, T);

@@ -93,6 +93,13 @@ size_t rp_partial_bytes(int T, int E, int H);
 cudaError_t launch_router_proj(int T, int E, int H, const uint16_t *x, const uint16_t *w_router, float *logits,
                                float *part, int32_t *status, cudaStream_t st);
 
+// Weight quantisers (quant.cu): MXFP8 over rows x K (K % 32 == 0), NVFP4 over
+// nmat matrices of rows x K (K % 16 == 0); all pointers 16-byte aligned.
+cudaError_t launch_quantize_mxfp8(long long rows, int K, const uint16_t *w, uint8_t *codes, uint8_t *scales,
+                                  cudaStream_t st);
+cudaError_t launch_quantize_nvfp4(int nmat, long long rows, int K, const uint16_t *w, uint8_t *codes,
+                                  uint8_t *scales, float *tensor_scale, cudaStream_t st);
+
 // Combine.
 cudaError_t launch_combine(int T, int k, int H, int has_shared, const uint16_t *ybuf,
                            const int32_t *keff, uint16_t *out, cudaStream_t st);

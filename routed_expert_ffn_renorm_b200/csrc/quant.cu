@@ -1,0 +1,128 @@
+// Weight quantisers for block-scaled expert weights (MXFP8, NVFP4): the
+// pack step that turns bf16 expert matrices into the FP8 / NVFP4 formats of
+// DeepGEMM fork PR #5 "big M opt: splitT1 + L2 scatter + 2 stream" (see
+// quant_codec.cuh for the formats and their rounding).  Run once when the
+// weights are loaded, not per layer call; every block goes through the one
+// per-block function of quant_codec.cuh, which the host test builds too.
+//
+// MXFP8: one thread per 32-element block (its 64 bytes of bf16 in, 32 code
+// bytes and one scale byte out), blocks strided over the grid.
+// NVFP4: (1) the largest |x| of each matrix, an integer max of the fp32
+// bits (order-independent), accumulated with atomicMax into tensor_scale
+// reused as uint32; (2) one thread per matrix turns it into the fp32 matrix
+// scale in place; (3) one thread per 16-element block.
+#include <algorithm>
+
+#include "moe_internal.cuh"
+#include "quant_codec.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kQuantThreads = 256;
+
+__global__ void __launch_bounds__(kQuantThreads) mxfp8_quantize_kernel(long long nblocks, const uint16_t *__restrict__ w,
+                                                                        uint8_t *__restrict__ codes,
+                                                                        uint8_t *__restrict__ scales) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+        uint16_t x[quant::kMxBlock];
+        const uint4 *src = reinterpret_cast<const uint4 *>(w + b * quant::kMxBlock);
+#pragma unroll
+        for (int v = 0; v < quant::kMxBlock / 8; ++v) {
+            const uint4 q = __ldg(src + v);
+            memcpy(x + 8 * v, &q, sizeof q);
+        }
+        uint8_t c[quant::kMxBlock];
+        scales[b] = quant::mxfp8_block(x, c);
+        uint4 *dst = reinterpret_cast<uint4 *>(codes + b * quant::kMxBlock);
+#pragma unroll
+        for (int v = 0; v < quant::kMxBlock / 16; ++v) {
+            uint4 q;
+            memcpy(&q, c + 16 * v, sizeof q);
+            dst[v] = q;
+        }
+    }
+}
+
+// amax_bits[m] = max over matrix m of |x| as fp32 bits; per_mat_vec 16-byte
+// vectors per matrix, blockIdx.y = matrix.
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_amax_kernel(long long per_mat_vec, const uint16_t *__restrict__ w,
+                                                                    uint32_t *__restrict__ amax_bits) {
+    const int m = blockIdx.y;
+    const uint4 *src = reinterpret_cast<const uint4 *>(w) + (long long)m * per_mat_vec;
+    uint32_t mx = 0;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < per_mat_vec; i += stride) {
+        uint16_t x[8];
+        const uint4 q = __ldg(src + i);
+        memcpy(x, &q, sizeof q);
+        const uint32_t a = quant::bf16_amax_bits(x, 8);
+        mx = a > mx ? a : mx;
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if ((threadIdx.x & 31) == 0 && mx != 0) atomicMax(amax_bits + m, mx);
+}
+
+__global__ void nvfp4_scale_kernel(int nmat, float *__restrict__ tensor_scale) {
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m < nmat) tensor_scale[m] = quant::nvfp4_tensor_scale(__float_as_uint(tensor_scale[m]));
+}
+
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_quantize_kernel(long long nblocks, long long per_mat_blocks,
+                                                                        const uint16_t *__restrict__ w,
+                                                                        const float *__restrict__ tensor_scale,
+                                                                        uint8_t *__restrict__ codes,
+                                                                        uint8_t *__restrict__ scales) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+        uint16_t x[quant::kNvBlock];
+        const uint4 *src = reinterpret_cast<const uint4 *>(w + b * quant::kNvBlock);
+#pragma unroll
+        for (int v = 0; v < quant::kNvBlock / 8; ++v) {
+            const uint4 q = __ldg(src + v);
+            memcpy(x + 8 * v, &q, sizeof q);
+        }
+        uint8_t c[quant::kNvBlock / 2];
+        scales[b] = quant::nvfp4_block(x, __ldg(tensor_scale + b / per_mat_blocks), c);
+        uint2 q;
+        memcpy(&q, c, sizeof q);
+        reinterpret_cast<uint2 *>(codes)[b] = q;
+    }
+}
+
+int grid_for(long long work) {
+    const long long g = (work + kQuantThreads - 1) / kQuantThreads;
+    const long long cap = 8LL * device_sm_count();
+    return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_mxfp8(long long rows, int K, const uint16_t *w, uint8_t *codes, uint8_t *scales,
+                                  cudaStream_t st) {
+    const long long nblocks = rows * (K / quant::kMxBlock);
+    mxfp8_quantize_kernel<<<grid_for(nblocks), kQuantThreads, 0, st>>>(nblocks, w, codes, scales);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_nvfp4(int nmat, long long rows, int K, const uint16_t *w, uint8_t *codes,
+                                  uint8_t *scales, float *tensor_scale, cudaStream_t st) {
+    const long long per_mat = rows * K;
+    cudaError_t e = cudaMemsetAsync(tensor_scale, 0, sizeof(float) * (size_t)nmat, st);
+    if (e != cudaSuccess) return e;
+    const long long per_mat_vec = per_mat / 8;
+    const int gx = std::min(grid_for(per_mat_vec), 1024);
+    nvfp4_amax_kernel<<<dim3(gx, nmat), kQuantThreads, 0, st>>>(per_mat_vec, w,
+                                                                 reinterpret_cast<uint32_t *>(tensor_scale));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    nvfp4_scale_kernel<<<(nmat + 127) / 128, 128, 0, st>>>(nmat, tensor_scale);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long per_mat_blocks = per_mat / quant::kNvBlock, nblocks = (long long)nmat * per_mat_blocks;
+    nvfp4_quantize_kernel<<<grid_for(nblocks), kQuantThreads, 0, st>>>(nblocks, per_mat_blocks, w, tensor_scale,
+                                                                        codes, scales);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

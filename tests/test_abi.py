@@ -17,7 +17,7 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 def _declared():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_and_binding_agree():
@@ -93,3 +93,23 @@ def test_workspace_grows_with_tokens():
     a = lib.moe_workspace_bytes(ctypes.byref(c), 16)
     b = lib.moe_workspace_bytes(ctypes.byref(c), 1024)
     assert 0 < a < b and b % 256 == 0
+
+
+def test_quantiser_argument_checks():
+    lib = moe.load_library()
+    # sizes: K must be a positive multiple of the block (32 for MXFP8, 16 for NVFP4)
+    for K in (0, 16, 33, -32):
+        assert lib.moe_quantize_mxfp8(4, K, FAKE, FAKE, FAKE, None) == -1
+    assert lib.moe_quantize_mxfp8(-1, 64, FAKE, FAKE, FAKE, None) == -1
+    for nmat, K in ((0, 16), (65536, 16), (1, 8), (1, 24)):
+        assert lib.moe_quantize_nvfp4(nmat, 4, K, FAKE, FAKE, FAKE, FAKE, None) == -1
+    # pointers: unaligned or missing
+    assert lib.moe_quantize_mxfp8(4, 64, MISALIGNED, FAKE, FAKE, None) == -1
+    assert lib.moe_quantize_mxfp8(4, 64, FAKE, MISALIGNED, FAKE, None) == -1
+    assert lib.moe_quantize_mxfp8(4, 64, FAKE, FAKE, None, None) == -1
+    assert lib.moe_quantize_nvfp4(2, 4, 32, FAKE, FAKE, FAKE, ctypes.c_void_p(FAKE.value + 2), None) == -1
+    assert lib.moe_quantize_nvfp4(2, 4, 32, FAKE, FAKE, None, FAKE, None) == -1
+    assert lib.moe_quantize_nvfp4(2, 4, 32, FAKE, FAKE, FAKE, None, None) == -1
+    # no rows: nothing to do, whatever the data pointers
+    assert lib.moe_quantize_mxfp8(0, 64, None, None, None, None) == 0
+    assert lib.moe_quantize_nvfp4(3, 0, 32, None, None, None, FAKE, None) == 0
