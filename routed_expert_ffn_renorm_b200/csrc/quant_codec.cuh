@@ -144,5 +144,38 @@ MOE_HD uint8_t nvfp4_block(const uint16_t *x, float st, uint8_t *packed) {
     return sc;
 }
 
+// ------------------------------------------------------------ decoders --
+// The weight a block-scaled code stands for, as the bf16 value the tensor
+// cores take (exact: these values have at most 6 significant bits).
+
+// E4M3 code c times 2^se as bf16 bits, built from the code's bits.  Exact
+// for every finite code while se lies in [-117, 119] (a normal bf16); an
+// MXFP8 scale is outside that only for blocks whose largest |x| is below
+// 2^-109.
+MOE_HD uint16_t e4m3_scaled_bf16(uint8_t c, int se) {
+    const uint32_t sign = (uint32_t)(c & 0x80u) << 8;
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    if (e == 0 && m == 0) return (uint16_t)sign;
+    if (e != 0) return (uint16_t)(sign | ((uint32_t)((int)e + 120 + se) << 7) | (m << 4));
+    // subnormal code: m 2^-9 = (1.f) 2^p 2^-9 with p = floor(log2 m); the
+    // leading bit of m becomes the implicit one
+    const uint32_t p = m >= 4u ? 2u : (m >= 2u ? 1u : 0u);
+    return (uint16_t)(sign | ((uint32_t)((int)p + 118 + se) << 7) | ((m << (7u - p)) & 0x7Fu));
+}
+
+// Value of an E2M1 code (low nibble).
+MOE_HD float e2m1_decode(uint8_t c) {
+    const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    const float mag = e == 0 ? 0.5f * (float)m : bits_f32(((e + 126u) << 23) | (m << 22));
+    return (c & 0x8u) ? -mag : mag;
+}
+
+// E2M1 code q times the E4M3 block scale sc, as bf16 bits (the NVFP4 weight
+// without its fp32 matrix scale, which multiplies the projection's output).
+// The fp32 product is exact and its low 16 bits are zero.
+MOE_HD uint16_t nvfp4_scaled_bf16(uint8_t q, uint8_t sc) {
+    return (uint16_t)(f32_bits(e2m1_decode(q) * e4m3_decode(sc)) >> 16);
+}
+
 }  // namespace quant
 }  // namespace moe

@@ -39,4 +39,21 @@ void host_nvfp4_quantize(int32_t nmat, int64_t rows, int32_t K, const uint16_t *
         scales[b] = nvfp4_block(w + b * kNvBlock, tensor_scale[b / per_mat_blocks], codes + b * (kNvBlock / 2));
 }
 
+// out[r, i] = bf16 bits of codes[r, i] x 2^(scales[r, i / 32] - 127)
+void host_mxfp8_to_bf16(int64_t rows, int32_t K, const uint8_t *codes, const uint8_t *scales, uint16_t *out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t i = 0; i < K; ++i)
+            out[r * K + i] = e4m3_scaled_bf16(codes[r * K + i], (int)scales[r * (K / kMxBlock) + i / kMxBlock] - 127);
+}
+
+// out[r, i] = bf16 bits of the E2M1 element (packed, 2i low) x its E4M3 block scale
+void host_nvfp4_to_bf16(int64_t rows, int32_t K, const uint8_t *codes, const uint8_t *scales, uint16_t *out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t i = 0; i < K; ++i) {
+            const int64_t at = r * K + i;
+            const uint8_t q = (uint8_t)((at & 1) ? codes[at / 2] >> 4 : codes[at / 2] & 15);
+            out[at] = nvfp4_scaled_bf16(q, scales[r * (K / kNvBlock) + i / kNvBlock]);
+        }
+}
+
 }  // extern "C"

@@ -6,7 +6,8 @@ quantiser kernels call for every block index; it uses integer and IEEE fp32
 arithmetic only, so a host build takes the kernels' decisions.  This test
 compiles it with g++ (tests/native/quant_codec_host.cpp) and compares every
 code, scale and matrix scale bit for bit with oracle/quant_oracle.c, which
-rounds by searching its code tables instead.
+rounds by searching its code tables instead; and the exact bf16 decoders
+(code x block scale, built from the bits) with the oracle's dequantisers.
 """
 import ctypes
 import os
@@ -32,6 +33,8 @@ def host():
             getattr(lib, name).restype = None
         lib.host_mxfp8_quantize.argtypes = [i64, i32, P, P, P]
         lib.host_nvfp4_quantize.argtypes = [i32, i64, i32, P, P, P, P]
+        lib.host_mxfp8_to_bf16.argtypes = [i64, i32, P, P, P]
+        lib.host_nvfp4_to_bf16.argtypes = [i64, i32, P, P, P]
         yield lib
 
 
@@ -135,3 +138,29 @@ def test_nvfp4_blocks_match_oracle(host, oracle_mod, kind):
         assert st[m] == np.float32(ost)
         np.testing.assert_array_equal(scales[m], os_)
         np.testing.assert_array_equal(codes[m], oc)
+
+
+def test_mxfp8_decode_to_bf16_is_exact(host, oracle_mod):
+    """Every finite E4M3 code at every scale exponent in [-117, 119]: the
+    bf16 built from the bits equals the oracle's fp64 dequantisation."""
+    se = np.arange(-117, 120)
+    codes = np.tile(np.arange(256, dtype=np.uint8), (se.size, 1))
+    codes[:, [0x7F, 0xFF]] = 0  # the NaN codes are never produced
+    scales = np.repeat((se + 127).astype(np.uint8)[:, None], 256 // 32, axis=1)
+    out = np.empty(codes.shape, np.uint16)
+    host.host_mxfp8_to_bf16(codes.shape[0], 256, _p(codes), _p(scales), _p(out))
+    want = oracle_mod.f64_to_bf16_exact(oracle_mod.mxfp8_dequantize(codes, scales))
+    np.testing.assert_array_equal(out, want)
+
+
+def test_nvfp4_decode_to_bf16_is_exact(host, oracle_mod):
+    """Every E2M1 code with every finite E4M3 block scale: element x block
+    scale as bf16 equals the oracle's dequantisation (matrix scale 1)."""
+    sc = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    q = np.arange(16, dtype=np.uint8)
+    codes = np.tile((q[0::2] | (q[1::2] << 4)).astype(np.uint8), (sc.size, 1))  # 16 elements per row
+    scales = sc[:, None]
+    out = np.empty((sc.size, 16), np.uint16)
+    host.host_nvfp4_to_bf16(sc.size, 16, _p(codes), _p(scales), _p(out))
+    want = oracle_mod.f64_to_bf16_exact(oracle_mod.nvfp4_dequantize(codes, scales, 1.0))
+    np.testing.assert_array_equal(out, want)
