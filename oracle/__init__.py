@@ -61,6 +61,7 @@ def _load():
     lib.oracle_route.argtypes = [i32, i32, i32, i32, P, P, P]
     lib.oracle_router_logits.argtypes = [i32, i32, i32, P, P, P]
     lib.oracle_budget.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P]
+    lib.oracle_budget_apply.argtypes = [i32, i32, i32, P, P, P, P]
     lib.oracle_topp.argtypes = [i32, i32, i32, ctypes.c_float, P, P, P]
     lib.oracle_dispatch.argtypes = [i32, i32, i32, P, P, P, P, P, P]
     lib.oracle_expert_rows.argtypes = [i32, i32, P, P, P, i32, P, P, i32]
@@ -155,6 +156,28 @@ def budget(idx: np.ndarray, w: np.ndarray, E: int, N: int, norm_topk: bool = Tru
     _check(_load().oracle_budget(T, E, k, N, int(bool(norm_topk)), _ptr(idx), _ptr(w), _ptr(keff),
                                  _ptr(kept), _ptr(nd)), "budget")
     return idx, w, keff, kept, int(nd[0])
+
+
+def budget_apply(idx: np.ndarray, w: np.ndarray, kept: np.ndarray, norm_topk: bool = True):
+    """Step 4 of the budget for a GIVEN kept set (copies; inputs untouched):
+    each token's slots of kept experts move to the front in order, the tail
+    becomes (-1, 0), and a token that lost a valid slot is renormalised when
+    norm_topk.  budget() is this step after choosing the kept set; a test
+    uses it to check a near-tie that the GPU decided the other way.
+
+    Returns (idx, w, keff [T])."""
+    idx = np.array(idx, np.int32, copy=True, order="C")
+    w = np.array(w, np.float32, copy=True, order="C")
+    kept = _c(kept, np.uint8)
+    T, k = idx.shape
+    if idx.size and int(idx.max()) >= kept.shape[0]:
+        raise ValueError("routing names an expert outside the kept mask")
+    keff = np.ascontiguousarray((idx >= 0).sum(axis=1), dtype=np.int32)
+    if T == 0:
+        keff = np.zeros(1, np.int32)
+    _check(_load().oracle_budget_apply(T, k, int(bool(norm_topk)), _ptr(kept), _ptr(idx), _ptr(w), _ptr(keff)),
+           "budget_apply")
+    return idx, w, keff[:T]
 
 
 def dispatch(idx: np.ndarray, keff: np.ndarray, E: int):

@@ -192,6 +192,34 @@ static int agg_cmp(const void *a, const void *b)
     return (x->id < y->id) ? -1 : (x->id > y->id); /* equal -> lower id first */
 }
 
+/* Step 4 of the budget on its own, for a given kept set: every token's
+ * slots whose expert is kept move to the front in their original order, the
+ * tail becomes (idx -1, w 0), and a token that lost a valid slot has its
+ * kept weights divided by their sum (slot order, fp32) when norm_topk.
+ * keff[t] holds the token's valid slots on entry and its kept slots on exit.
+ * oracle_budget calls this with the kept set of steps 1-3; a test may call
+ * it with another kept set (a near-tie that the GPU decided the other way). */
+int oracle_budget_apply(int32_t T, int32_t k, int32_t norm_topk, const uint8_t *kept,
+                        int32_t *idx, float *w, int32_t *keff)
+{
+    if (T < 0 || k < 1) return ORACLE_EINVAL;
+    for (int32_t t = 0; t < T; ++t) {
+        int32_t *ti = idx + (size_t)t * k;
+        float *tw = w + (size_t)t * k;
+        int32_t c = 0;
+        for (int32_t j = 0; j < k; ++j)
+            if (ti[j] >= 0 && kept[ti[j]]) { ti[c] = ti[j]; tw[c] = tw[j]; ++c; }
+        for (int32_t j = c; j < k; ++j) { ti[j] = -1; tw[j] = 0.0f; }
+        if (norm_topk && c > 0 && c < keff[t]) {
+            float s = 0.0f;
+            for (int32_t j = 0; j < c; ++j) s += tw[j];
+            for (int32_t j = 0; j < c; ++j) tw[j] = tw[j] / s;
+        }
+        keff[t] = c;
+    }
+    return ORACLE_OK;
+}
+
 int oracle_budget(int32_t T, int32_t E, int32_t k, int32_t N, int32_t norm_topk,
                   int32_t *idx, float *w, int32_t *keff, uint8_t *kept, int32_t *n_dropped)
 {
@@ -227,20 +255,7 @@ int oracle_budget(int32_t T, int32_t E, int32_t k, int32_t N, int32_t norm_topk,
     for (int32_t r = 0; r < N; ++r) kept[order[r].id] = 1;
     /* step 4: remove dropped experts from each token's list, renormalise the
      * tokens that lost a slot (keff[t] holds the valid slots before) */
-    for (int32_t t = 0; t < T; ++t) {
-        int32_t *ti = idx + (size_t)t * k;
-        float *tw = w + (size_t)t * k;
-        int32_t c = 0;
-        for (int32_t j = 0; j < k; ++j)
-            if (ti[j] >= 0 && kept[ti[j]]) { ti[c] = ti[j]; tw[c] = tw[j]; ++c; }
-        for (int32_t j = c; j < k; ++j) { ti[j] = -1; tw[j] = 0.0f; }
-        if (norm_topk && c > 0 && c < keff[t]) {
-            float s = 0.0f;
-            for (int32_t j = 0; j < c; ++j) s += tw[j];
-            for (int32_t j = 0; j < c; ++j) tw[j] = tw[j] / s;
-        }
-        keff[t] = c;
-    }
+    oracle_budget_apply(T, k, norm_topk, kept, idx, w, keff);
     /* step 5: the union is now the kept experts */
     *n_dropped = nu - N;
     free(agg);

@@ -157,6 +157,28 @@ def test_budget_worked_example(oracle_mod):
     assert perm.tolist() == d["perm"] and slot_pos.tolist() == d["slot_pos"]
 
 
+def test_budget_apply_worked_example(oracle_mod):
+    """Step 4 for a given kept set: the hand-worked other side of the example's tie."""
+    g = _gold("budget_worked_example.json")
+    idx = np.array(g["idx"], np.int32)
+    w = np.array(g["w"], np.float32)
+    alt = g["alternative_kept"]
+    for norm, key in ((True, "expect_norm"), (False, "expect_no_norm")):
+        i2, w2, keff = oracle_mod.budget_apply(idx, w, np.array(alt["kept"], np.uint8), norm_topk=norm)
+        assert i2.tolist() == alt[key]["idx"] and w2.tolist() == alt[key]["w"] and keff.tolist() == alt[key]["keff"]
+
+
+@pytest.mark.parametrize("norm", [True, False])
+def test_budget_apply_with_own_kept_set_is_budget(oracle_mod, norm):
+    """budget() = choose the kept set, then step 4: applying step 4 to the
+    router output with budget()'s kept set gives its outputs bit for bit."""
+    for seed, N in ((3, 4), (4, 12), (5, 20)):
+        idx, w = _route_for_budget(oracle_mod, 32, 128, 8, seed)
+        i2, w2, keff, kept, nd = oracle_mod.budget(idx, w, 128, N, norm_topk=norm)
+        i3, w3, keff3 = oracle_mod.budget_apply(idx, w, kept, norm_topk=norm)
+        assert (i3 == i2).all() and (w3.view(np.uint32) == w2.view(np.uint32)).all() and (keff3 == keff).all()
+
+
 # ----------------------------------------------------------------- top-p --
 
 def test_topp_worked_example(oracle_mod):
