@@ -58,6 +58,8 @@ def workload_from_args(args):
         kw["topp"] = args.topp
     if args.router_proj:
         kw["router_proj"] = True
+    if args.E is not None:
+        kw["E"] = args.E
     return cfg.with_(**kw) if kw else cfg
 
 
@@ -580,6 +582,8 @@ def run_ours(args, cfg):
         "gpu_launches": (launches_forward(cfg) + launches_stages(cfg)) * args.steps,
         "clocks": sampler.summary(),
         "stages_ms": per_stage,
+        "stages_GB_per_s": {sn: work[sn]["bytes"] / (per_stage[sn] * 1e-3) / 1e9 for sn in stages
+                            if work[sn]["bytes"] and per_stage[sn] > 0},
         **({"router_proj_roofline": roofline("router_proj", work, per_stage["router_proj"], peaks, peak_kind,
                                              long_run, None)} if cfg.router_proj else {}),
         "layer": {"touched_experts": work["touched"], "kept_slots": work["slots"],
@@ -645,11 +649,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="drafter_16x1024")
+    ap.add_argument("--workload", default="large_256e",
+                    help="named workload (default: the 256-expert top-8 layer, T = 16384, the largest one-GPU "
+                         "configuration); drafter_16x1024 / drafter_512x512 / budget_s32 / tiny for the others")
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--topp", type=float, default=None, help="per-token top-p trim (0 = off)")
+    ap.add_argument("--E", type=int, default=None,
+                    help="override the number of routed experts (a scaled stand-in of a workload for ncu captures)")
     ap.add_argument("--router-proj", action="store_true",
                     help="compute the logits with the router projection x . W_r^T inside the layer")
     ap.add_argument("--no-e2e", action="store_true")

@@ -207,7 +207,10 @@ int moe_expert_down(const moe_config_t *cfg, int32_t T, const int32_t *offsets, 
  *     that loads the library until the process exits.
  *   - The first call on a device looks the array's address up (a CUDA
  *     runtime query); make that first call before capturing a stream into a
- *     CUDA graph.
+ *     CUDA graph.  The address is kept for the life of the process: after a
+ *     cudaDeviceReset (or any teardown of the device's primary context) the
+ *     library's device array is reloaded elsewhere and this entry point must
+ *     not be used on that device again in the same process.
  *   - All calls share the one array: calls whose work overlaps on the GPU
  *     (e.g. on two streams at once) race and corrupt each other.  Each call
  *     re-zeroes the counters it needs (an async memset on `stream`); nothing
@@ -256,7 +259,10 @@ const char *moe_error_string(int code);
  * kernels, its B200 FP8 x FP4 policy), with the published definitions:
  * E4M3 without infinities (largest finite 448), E2M1 (magnitudes 0, 0.5, 1,
  * 1.5, 2, 3, 4, 6), UE8M0 (2^(c - 127)).  Rounding is to nearest, ties to
- * the even code, saturating; the sign bit copies the input's.  The blocks
+ * the even code, saturating; the sign bit copies the input's.  Inputs must
+ * be finite: a NaN or infinite weight has no defined code (a NaN counts as
+ * the largest magnitude, so in NVFP4 it spoils its whole matrix's scale);
+ * the quantisers do not check for them.  The blocks
  * run along the last (reduction) axis of a row-major matrix: rows of
  * W_gate / W_up [I, H] and of W_down [H, I].  The layer does not consume
  * these formats yet.

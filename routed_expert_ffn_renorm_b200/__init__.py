@@ -161,6 +161,14 @@ def _ptr(t, allow_none: bool = False):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _expect(t, dtype, numel: int, name: str):
+    """Host-side size check of a tensor the library writes or reads in full:
+    a wrong dtype or a short buffer would otherwise become an out-of-bounds
+    device access."""
+    if t.dtype != dtype or t.numel() != numel:
+        raise ValueError(f"{name}: expected {numel} elements of {dtype}, got {t.numel()} of {t.dtype}")
+
+
 def _stream(stream):
     import torch
     s = torch.cuda.current_stream() if stream is None else stream
@@ -191,7 +199,11 @@ def moe_router_logits(cfg: MoEConfig, x, w_router, logits, ws, stream=None):
 def moe_quantize_mxfp8(w, codes, scales, stream=None):
     """MXFP8 weights: w [..., K] bf16 -> codes [..., K] uint8 (E4M3) and
     scales [..., K // 32] uint8 (UE8M0), blocks along the last axis."""
+    import torch
     K = w.shape[-1]
+    _expect(w, torch.bfloat16, w.numel(), "w")
+    _expect(codes, torch.uint8, w.numel(), "codes")
+    _expect(scales, torch.uint8, w.numel() // 32, "scales")
     _check("moe_quantize_mxfp8", load_library().moe_quantize_mxfp8(
         w.numel() // K, K, _ptr(w), _ptr(codes), _ptr(scales), _stream(stream)))
 
@@ -200,7 +212,12 @@ def moe_quantize_nvfp4(w, codes, scales, tensor_scale, stream=None):
     """NVFP4 weights: w [nmat, rows, K] bf16 -> codes [nmat, rows, K // 2]
     uint8 (two E2M1 per byte, element 2i low), scales [nmat, rows, K // 16]
     uint8 (E4M3), tensor_scale [nmat] fp32 (one per matrix)."""
+    import torch
     nmat, rows, K = w.shape
+    _expect(w, torch.bfloat16, w.numel(), "w")
+    _expect(codes, torch.uint8, w.numel() // 2, "codes")
+    _expect(scales, torch.uint8, w.numel() // 16, "scales")
+    _expect(tensor_scale, torch.float32, nmat, "tensor_scale")
     _check("moe_quantize_nvfp4", load_library().moe_quantize_nvfp4(
         nmat, rows, K, _ptr(w), _ptr(codes), _ptr(scales), _ptr(tensor_scale), _stream(stream)))
 

@@ -123,7 +123,7 @@ struct FfnParams {
     uint16_t *h_shared;  // [T, Is]
     uint16_t *ybuf;      // [T, k+1, H]
     int32_t *status;     // status word
-    int32_t *sched;      // [0] items claimed past the first grid's worth, [1] CTAs done; zero between launches
+    int32_t *sched;      // [0] items claimed, [1] CTAs done; zero between launches
     int32_t *hdone;      // [E+2] finished gate/up items per group (E = shared), [E+1] in all; zero between launches
 };
 
@@ -439,6 +439,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     }
     if constexpr (kPair) cluster_sync();  // both CTAs' barriers initialised before any cross-CTA arrive
     pdl_wait();  // the dispatch outputs and activations are ready past this point
+    // the producer's first claim, issued now so that its round trip overlaps the
+    // schedule set-up below (the counter is zero here: the previous launch's last
+    // CTA, or the dispatch kernel, left it so)
+    int first_claim = 0;
+    if (warp == 0 && lane == 0 && (!kPair || rank == 0)) first_claim = atomicAdd(p.sched, 1);
     // dispatch offsets to shared memory, then the per-expert prefix sums of token
     // tiles and of down items
     for (int e = threadIdx.x; e <= p.E; e += kThreads) offs[e] = __ldg(p.offsets + e);
@@ -481,14 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             // instead of 3.7 GB from DRAM).
             const uint64_t wpol = policy_evict_first();
             const uint64_t bpol = policy_evict_normal();  // token rows (pair loads take a policy)
-            // items are claimed one ahead: a CTA (pair) takes item blockIdx (cluster
-            // index) first, then from the counter, past the first grid's worth
-            // (the counter's value is only added to when the next claim is made, so the
-            // atomic's round trip -- long at launch, when every CTA claims at once -- never
-            // stalls this lane's in-order issue)
-            const int claimers = kPair ? (int)gridDim.x / 2 : (int)gridDim.x;
-            int pending = -1;  // counter value of the claim in flight; -1: the first, static item
-            bool all_ready = false;                       // every gate/up item of the launch is done
+            // Items are claimed from the counter, one ahead: the next claim's atomic
+            // is issued when an item is taken, so its round trip overlaps that item's
+            // loads.  Every item, the first included, comes from the counter, so the
+            // items claimed so far are exactly those of CTAs that are running: a down
+            // item waits only on gate/up items that running CTAs hold, even when not
+            // every CTA of the grid is resident at once.
+            int pending = first_claim;  // counter value of the claim in flight
+            bool all_ready = false;     // every gate/up item of the launch is done
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 const uint32_t qph = (uint32_t)(li / kQueue) & 1u;
@@ -496,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 Item it{};
                 if (!kPair || rank == 0) {
                     if (!mbar_wait<kPair>(&qempty[slot], qph ^ 1u, abort_flag, p.status, true)) break;
-                    item = pending < 0 ? (kPair ? (int)blockIdx.x / 2 : (int)blockIdx.x) : claimers + pending;
+                    item = pending;
                     if (item >= total_items) item = -1;
                     if (item >= 0) pending = atomicAdd(p.sched, 1);  // latency overlaps this item's loads
                     if (item >= 0) it = decode_item(item, sc, p);  // decoded once, for all roles

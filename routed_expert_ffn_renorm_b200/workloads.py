@@ -71,7 +71,7 @@ class MoEConfig:
 TINY = MoEConfig("tiny", T=16, H=256, E=8, I=128, k=2)
 DRAFTER_16x1024 = MoEConfig("drafter_16x1024", T=224, H=5120, E=16, I=1024, k=2, Is=2048)
 DRAFTER_512x512 = MoEConfig("drafter_512x512", T=224, H=5120, E=512, I=512, k=10, Is=2048, zipf_alpha=1.0)
-LARGE_256E = MoEConfig("large_256e", T=512, H=7168, E=256, I=2048, k=8)
+LARGE_256E = MoEConfig("large_256e", T=16384, H=7168, E=256, I=2048, k=8)  # T swept over LARGE_T_SWEEP
 BUDGET_S32 = MoEConfig("budget_s32", T=32, H=4096, E=128, I=1536, k=8, budget=12, zipf_alpha=1.2)
 
 WORKLOADS = {c.name: c for c in (TINY, DRAFTER_16x1024, DRAFTER_512x512, LARGE_256E, BUDGET_S32)}

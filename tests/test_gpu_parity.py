@@ -2,10 +2,13 @@
 
 Bit-exact for routing indices, budget drops, counts, offsets, perm and
 slot_pos; fp32-ulp close for routing weights and the shared gate; relative
-L2 <= 5e-3 on the bf16 layer output.  Small shapes compare every output
-row and span several weight tiles, several token tiles and ragged tails;
-the full-size workloads compare seeded sample rows (routing and dispatch
-always in full).
+L2 <= 5e-3 on the bf16 layer output (and <= 1e-2 on every compared row).
+Small shapes compare every output row and span several weight tiles, several
+token tiles and ragged tails; the full-size workloads compare a stratified
+set of rows -- one from every (expert group, 256-row token tile), the first
+and last row of every group, one from every shared-expert tile, and seeded
+extra tokens -- so every work item of both GEMM phases is reached (routing
+and dispatch always in full).
 """
 import os
 
@@ -17,7 +20,7 @@ import routed_expert_ffn_renorm_b200 as moe
 from routed_expert_ffn_renorm_b200 import workloads as W
 
 import oracle
-from parity_util import check_layer, gpu_forward, lib_config, logits_bound, sample_rows, weights_of
+from parity_util import check_layer, gpu_forward, lib_config, logits_bound, sample_rows, stratified_rows, weights_of
 
 pytestmark = pytest.mark.gpu
 
@@ -357,13 +360,45 @@ def test_zero_tokens_is_noop():
 
 # ------------------------------------------------------------ full sizes --
 
-@pytest.mark.parametrize("cfg,nrows", [(W.DRAFTER_16x1024, 64), (W.DRAFTER_512x512, 16),
-                                       (W.DRAFTER_512x512.with_(zipf_alpha=0.0), 12)],
-                         ids=["drafter_16x1024", "drafter_512x512_a1", "drafter_512x512_a0"])
-def test_drafter_layers(cfg, nrows):
-    rows = sample_rows(cfg.T, nrows)
-    diag, g, _ = _run(cfg, gen_device="cuda", rows=rows)
+def _strat(cfg, n_random):
+    """Row chooser for check_layer: every (group, token tile), group ends, shared tiles."""
+    return lambda offsets, perm: stratified_rows(cfg.T, cfg.k, offsets, perm, tile=256, n_random=n_random,
+                                                 shared_tile=128 if cfg.Is else 0)
+
+
+DRAFTERS = [W.DRAFTER_16x1024, W.DRAFTER_512x512, W.DRAFTER_512x512.with_(zipf_alpha=0.0),
+            W.DRAFTER_512x512.with_(topp=0.8)]
+
+
+@pytest.mark.parametrize("cfg", DRAFTERS, ids=["drafter_16x1024", "drafter_512x512_a1", "drafter_512x512_a0",
+                                               "drafter_512x512_a1_topp0.8"])
+def test_drafter_layers(cfg):
+    diag, g, _ = _run(cfg, gen_device="cuda", rows=_strat(cfg, 32))
     print(cfg.label, diag)
+
+
+def test_drafter_layer_router_projection():
+    """The 512 x 512 drafter layer with its logits from the router projection
+    inside moe_forward: the projection's logits within the fp32 bound of the
+    oracle's, then the whole layer on those logits."""
+    cfg = W.DRAFTER_512x512.with_(router_proj=True)
+    inp = W.make_inputs(cfg, device="cuda")
+    c = lib_config(cfg)
+    ws = torch.zeros(moe.workspace_bytes(c, cfg.T), dtype=torch.uint8, device="cuda")
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    lg = torch.full((cfg.T, cfg.E), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_forward(c, inp.x, None, weights_of(inp), out, ws, aux={"logits": lg})
+    torch.cuda.synchronize()
+    assert moe.status_read(ws) == 0
+    xb, wb = W.bf16_bits(inp.x), W.bf16_bits(inp.w_router)
+    g_lg = lg.cpu().numpy()
+    assert (np.abs(g_lg.astype(np.float64) - oracle.router_logits(xb, wb)) <= logits_bound(xb, wb)).all()
+    inp_l = W.MoEInputs(inp.x, lg, inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down,
+                        inp.ws_gvec)
+    g = gpu_forward(cfg.with_(router_proj=False), inp_l)
+    assert (g.out_bits == W.bf16_bits(out)).all(), "moe_forward with the projection differs from given logits"
+    diag = check_layer(cfg, inp_l, g, rows=_strat(cfg, 32))
+    print(cfg.label, diag, "touched", int((g.counts > 0).sum()))
 
 
 @pytest.mark.parametrize("N", W.BUDGETS)
@@ -376,24 +411,27 @@ def test_budget_layer(N):
 
 @pytest.fixture(scope="module")
 def large_inputs():
-    """256 experts x 2048 x 7168 (22.5 GB bf16) drawn once; logits N(0,1) for the largest T."""
+    """256 experts x 2048 x 7168 (22.5 GB bf16) drawn once; logits N(0,1) for the
+    largest T; host copies of expert weights shared by the tests."""
     cfg = W.LARGE_256E.with_(T=max(W.LARGE_T_SWEEP))
     inp = W.make_inputs(cfg, device="cuda")
-    yield cfg, inp
+    yield cfg, inp, {}
     del inp
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("T,alpha,nrows", [(64, 0.0, 16), (64, 1.5, 16), (512, 1.0, 12), (4096, 1.5, 8),
-                                           (16384, 0.0, 6), (16384, 1.0, 6)])
-def test_large_layer(large_inputs, T, alpha, nrows):
-    base_cfg, base = large_inputs
+@pytest.mark.parametrize("T", W.LARGE_T_SWEEP)
+@pytest.mark.parametrize("alpha", W.LARGE_ALPHAS)
+def test_large_layer(large_inputs, T, alpha):
+    """Every (T, alpha) point of the 256-expert sweep, rows stratified over every
+    (expert group, token tile) plus >= 256 seeded tokens at T >= 4096."""
+    base_cfg, base, cache = large_inputs
     cfg = base_cfg.with_(T=T, zipf_alpha=alpha)
     logits = base.logits[:T] + W.zipf_bias(cfg.E, alpha, "cuda")
     inp = W.MoEInputs(base.x[:T].contiguous(), logits.contiguous(), base.w_gate, base.w_up, base.w_down)
     g = gpu_forward(cfg, inp)
-    diag = check_layer(cfg, inp, g, rows=sample_rows(T, nrows))
-    print(cfg.label, diag, "max group", int(g.counts.max()))
+    diag = check_layer(cfg, inp, g, rows=_strat(cfg, 256 if T >= 4096 else 64), weight_cache=cache)
+    print(cfg.label, diag, "max group", int(g.counts.max()), "touched", int((g.counts > 0).sum()))
 
 
 @pytest.mark.parametrize("cfg", [W.MoEConfig("phases", T=300, H=256, E=8, I=192, k=2, Is=128, zipf_alpha=1.0),
