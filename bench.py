@@ -74,23 +74,26 @@ def workload_desc(cfg) -> dict:
 
 
 # -------------------------------------------------------- accounting --
-def stage_work(cfg, counts):
+def stage_work(cfg, counts, wfmt: str = "bf16"):
     """Algorithmic flops and HBM bytes per launch of each stage.
 
     Bytes count what a kernel must move at least once: the touched experts'
-    weights, its input activations and its output; flops are 2 per MAC."""
+    weights (2 bytes a weight in bf16; 1 + 1/32 in MXFP8: a code and its
+    share of a block scale), its input activations and its output; flops
+    are 2 per MAC."""
     H, I, Is, T, k, E = cfg.H, cfg.I, cfg.Is, cfg.T, cfg.k, cfg.E
+    wb = 2.0 if wfmt == "bf16" else 1.0 + 1.0 / 32
     touched = int(sum(1 for c in counts if c > 0))
     slots = int(sum(counts))
     sh = 1 if Is else 0
     gate_up = dict(
         flops=4 * H * I * slots + 4 * H * Is * T,
-        bytes=touched * 2 * I * H * 2 + sh * 2 * Is * H * 2 + slots * H * 2 + sh * T * H * 2 + (slots * I + T * Is) * 2)
+        bytes=touched * 2 * I * H * wb + sh * 2 * Is * H * wb + slots * H * 2 + sh * T * H * 2 + (slots * I + T * Is) * 2)
     down = dict(
         flops=2 * H * I * slots + 2 * H * Is * T,
-        bytes=touched * H * I * 2 + sh * H * Is * 2 + (slots * I + T * Is) * 2 + (slots + sh * T) * H * 2)
+        bytes=touched * H * I * wb + sh * H * Is * wb + (slots * I + T * Is) * 2 + (slots + sh * T) * H * 2)
     ffn = dict(flops=gate_up["flops"] + down["flops"],
-               bytes=touched * 3 * H * I * 2 + sh * 3 * H * Is * 2 + slots * H * 2 + sh * T * H * 2
+               bytes=touched * 3 * H * I * wb + sh * 3 * H * Is * wb + slots * H * 2 + sh * T * H * 2
                + (slots + sh * T) * H * 2)
     route = dict(flops=0, bytes=T * E * 4 + T * k * 8 + sh * (T * H * 2 + H * 2 + T * 4))
     proj = cfg.router_proj
@@ -99,7 +102,7 @@ def stage_work(cfg, counts):
     dispatch = dict(flops=0, bytes=T * k * 4 * 3 + slots * H * 2 * 2)
     combine = dict(flops=0, bytes=(slots + sh * T) * H * 2 + T * H * 2)
     layer = dict(flops=gate_up["flops"] + down["flops"] + router_proj["flops"],
-                 bytes=touched * 3 * H * I * 2 + sh * (3 * H * Is * 2 + H * 2) + 2 * T * H * 2
+                 bytes=touched * 3 * H * I * wb + sh * (3 * H * Is * wb + H * 2) + 2 * T * H * 2
                  + (E * H * 2 if proj else T * E * 4))
     return dict(router_proj=router_proj, route=route, budget=budget, dispatch=dispatch, gate_up=gate_up, down=down,
                 ffn=ffn, combine=combine, layer=layer, touched=touched, slots=slots)
@@ -301,35 +304,41 @@ def oracle_rows_per_s(cfg, inp_host, target_s: float, max_rows: int, repeat: boo
     return n * passes / dt, n, passes, dt, nthreads
 
 
-def host_inputs(cfg, inp, max_rows: int):
+def host_inputs(cfg, inp, max_rows: int, wfmt: str = "bf16"):
     """Host copies for the oracle: x, logits, and the weights -- all experts
     when they fit in 2 GB, else only the experts the first max_rows sample
-    rows route to (routing after the budget is a subset of routing before)."""
+    rows route to (routing after the budget is a subset of routing before).
+    MXFP8: every expert matrix as the oracle's MXFP8 weights (quantised and
+    dequantised by the oracle, once, before any timing)."""
     import oracle
     from routed_expert_ffn_renorm_b200 import workloads as W
+    bits = W.bf16_bits if wfmt == "bf16" else (lambda t: oracle.mxfp8_weights(W.bf16_bits(t)))
     x = W.bf16_bits(inp.x)
     if cfg.router_proj:  # the projection's logits, computed once before the timed oracle runs
         logits = oracle.router_logits(x, W.bf16_bits(inp.w_router))
     else:
         logits = inp.logits.float().cpu().numpy()
-    if 3 * cfg.E * cfg.H * cfg.I * 2 <= (2 << 30):
+    if 3 * cfg.E * cfg.H * cfg.I * 2 <= (2 << 30) and wfmt == "bf16":
         wg, wu, wd = W.bf16_bits(inp.w_gate), W.bf16_bits(inp.w_up), W.bf16_bits(inp.w_down)
     else:
         idx, _ = oracle.route(logits, cfg.k, cfg.norm_topk)
         need = sorted(set(idx[sample_order(cfg.T)[:max_rows]].ravel().tolist()))
-        wg = {e: W.bf16_bits(inp.w_gate[e]) for e in need}
-        wu = {e: W.bf16_bits(inp.w_up[e]) for e in need}
-        wd = {e: W.bf16_bits(inp.w_down[e]) for e in need}
+        wg = {e: bits(inp.w_gate[e]) for e in need}
+        wu = {e: bits(inp.w_up[e]) for e in need}
+        wd = {e: bits(inp.w_down[e]) for e in need}
     shared = {}
     if cfg.Is:
-        shared = dict(ws_gate=W.bf16_bits(inp.ws_gate), ws_up=W.bf16_bits(inp.ws_up),
-                      ws_down=W.bf16_bits(inp.ws_down), ws_gvec=W.bf16_bits(inp.ws_gvec))
+        shared = dict(ws_gate=bits(inp.ws_gate), ws_up=bits(inp.ws_up),
+                      ws_down=bits(inp.ws_down), ws_gvec=W.bf16_bits(inp.ws_gvec))
     return x, logits, wg, wu, wd, shared
 
 
-def cpu_max_rows(cfg) -> int:
+def cpu_max_rows(cfg, wfmt: str = "bf16") -> int:
     """Largest CPU sample: the whole batch for small layers, 16 rows when the
-    expert weights do not fit a 2 GB host copy."""
+    expert weights do not fit a 2 GB host copy; with MXFP8 weights (which the
+    oracle quantises itself, about a second per expert matrix) 2 rows."""
+    if wfmt != "bf16":
+        return min(cfg.T, 2)
     return cfg.T if 3 * cfg.E * cfg.H * cfg.I * 2 <= (2 << 30) else min(cfg.T, 16)
 
 
@@ -372,7 +381,14 @@ def run_ours(args, cfg):
     pc = ctypes.byref(c._c())
     wts = moe.MoEWeights(inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec,
                          inp.w_router)
-    pw = ctypes.byref(wts._c())
+    mx = args.weights == "mxfp8"
+    if mx:  # the weight pack step, once, before anything is timed
+        wts = moe.pack_mxfp8(wts)
+        torch.cuda.synchronize(dev)
+    wts_c = wts._c()
+    pw = ctypes.byref(wts_c)
+    ffn_fn = lib.moe_expert_ffn_mxfp8 if mx else lib.moe_expert_ffn
+    fwd_fn = lib.moe_forward_mxfp8 if mx else lib.moe_forward
     p = {n: P(t.data_ptr()) for n, t in dict(idx=idx, tw=tw, sgate=sgate, keff=keff, kept=kept, nd=nd,
                                                 counts=counts, offsets=offsets, perm=perm, slot_pos=slot_pos,
                                                 x_perm=x_perm, ybuf=ybuf, out=out, ws=ws, x=inp.x,
@@ -406,8 +422,8 @@ def run_ours(args, cfg):
         chk("moe_dispatch", lib.moe_dispatch(pc, T, p["idx"], p["keff"], p["x"], p["counts"], p["offsets"], p["perm"],
                                              p["slot_pos"], p["x_perm"], p["ws"], wsb, sp))
         ev[pr + 3].record(st)
-        chk("moe_expert_ffn", lib.moe_expert_ffn(pc, T, p["x"], p["x_perm"], p["offsets"], p["perm"], p["tw"], sg, pw,
-                                                 p["ybuf"], p["ws"], wsb, sp))
+        chk("moe_expert_ffn", ffn_fn(pc, T, p["x"], p["x_perm"], p["offsets"], p["perm"], p["tw"], sg, pw,
+                                     p["ybuf"], p["ws"], wsb, sp))
         ev[pr + 4].record(st)
         chk("moe_combine", lib.moe_combine(pc, T, p["ybuf"], p["keff"], p["out"], sp))
         ev[pr + 5].record(st)
@@ -431,7 +447,7 @@ def run_ours(args, cfg):
     if status:
         raise RuntimeError(f"device status {status} after warm-up")
     counts_h = counts.cpu().tolist()
-    work = stage_work(cfg, counts_h)
+    work = stage_work(cfg, counts_h, args.weights)
 
     # ---- eager launches (diagnostic): K steps back to back from the host
     evs = [mk() for _ in range(args.steps)]
@@ -459,9 +475,8 @@ def run_ours(args, cfg):
     def fwd_step(e0, e1):
         st = torch.cuda.current_stream(dev)
         e0.record(st)
-        chk("moe_forward", lib.moe_forward(pc, T, p["x"], None if cfg.router_proj else p["logits"], pw, p["out"],
-                                           ctypes.byref(aux_c), p["ws"],
-                                           wsb, P(st.cuda_stream)))
+        chk("moe_forward", fwd_fn(pc, T, p["x"], None if cfg.router_proj else p["logits"], pw, p["out"],
+                                  ctypes.byref(aux_c), p["ws"], wsb, P(st.cuda_stream)))
         e1.record(st)
 
     fev = mk(ext=True)[:2]
@@ -524,7 +539,8 @@ def run_ours(args, cfg):
             xd.copy_(xh, non_blocking=True)
             if not cfg.router_proj:  # else the layer computes its logits from x
                 ld.copy_(lh, non_blocking=True)
-            moe.moe_forward(c, xd, None if cfg.router_proj else ld, wts, out, ws, stream=st)
+            (moe.moe_forward_mxfp8 if mx else moe.moe_forward)(c, xd, None if cfg.router_proj else ld, wts, out, ws,
+                                                               stream=st)
             oh.copy_(out, non_blocking=True)
             e1.record(st)
 
@@ -559,14 +575,14 @@ def run_ours(args, cfg):
     # the power cap held the clocks down during the timed region
     long_run = (total_ms * 1e-3) > 1.0 or "sw_power_cap" in sampler.summary().get("reasons", [])
     rl = roofline(dom, work, per_stage[dom], peaks, peak_kind, long_run,
-                  recorded_traffic(dom, cfg.label))
+                  recorded_traffic(dom, cfg.label + (":mxfp8" if mx else "")))
     layer_bw = work["layer"]["bytes"] / (step_ms * 1e-3) / 1e9
     layer_tf = work["layer"]["flops"] / (step_ms * 1e-3) / 1e12
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        mr = cpu_max_rows(cfg)
-        hi = host_inputs(cfg, inp, mr)
+        mr = cpu_max_rows(cfg, args.weights)
+        hi = host_inputs(cfg, inp, mr, args.weights)
         rps, nrows, passes, secs, thr = oracle_rows_per_s(cfg, hi, args.cpu_seconds, mr, repeat=True)
         cpu = {"value": rps, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                "sample": f"{nrows} of {T} tokens of {cfg.label}: routing, budget and dispatch over all {T} tokens, "
@@ -575,9 +591,12 @@ def run_ours(args, cfg):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic: seeded N(0,0.02) bf16 x and weights, N(0,1) fp32 "
-        "router logits + Zipf popularity bias",
-        "config": {**workload_desc(cfg), "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,0.02) bf16 x and weights, N(0,1) fp32 router logits + Zipf popularity bias"
+                + ("; expert weights packed to MXFP8 (E4M3 codes + UE8M0 scales per 32) by the library's quantiser"
+                   if mx else ""),
+        "config": {**workload_desc(cfg), "expert_weights": args.weights,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": rl, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": (launches_forward(cfg) + launches_stages(cfg)) * args.steps,
         "clocks": sampler.summary(),
@@ -612,8 +631,8 @@ def run_reference(args, cfg):
         return
     inp = W.make_inputs(cfg, device="cuda" if torch.cuda.is_available() and cfg.E * cfg.I * cfg.H > (1 << 28)
                         else "cpu")
-    mr = cpu_max_rows(cfg)
-    hi = host_inputs(cfg, inp, mr)
+    mr = cpu_max_rows(cfg, args.weights)
+    hi = host_inputs(cfg, inp, mr, args.weights)
     per_step = min(5.0, 150.0 / max(args.steps + args.warmup, 1))  # whole run within a few minutes
     rps, nrows, _, secs, thr = oracle_rows_per_s(cfg, hi, per_step, mr)
     import oracle
@@ -637,7 +656,7 @@ def run_reference(args, cfg):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (same seeded inputs as the GPU arm)",
-            "config": {**workload_desc(cfg), "parallelism": "CPU oracle, rank 0"},
+            "config": {**workload_desc(cfg), "expert_weights": args.weights, "parallelism": "CPU oracle, rank 0"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -660,6 +679,9 @@ def main(argv=None):
                     help="override the number of routed experts (a scaled stand-in of a workload for ncu captures)")
     ap.add_argument("--router-proj", action="store_true",
                     help="compute the logits with the router projection x . W_r^T inside the layer")
+    ap.add_argument("--weights", choices=["bf16", "mxfp8"], default="bf16",
+                    help="expert weight format: bf16, or MXFP8 (E4M3 codes + a power-of-two scale per 32 weights, "
+                         "converted to bf16 on chip; half the weight bytes)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -225,6 +225,58 @@ int moe_expert_ffn_noalloc(const moe_config_t *cfg, int32_t T, const moe_bf16_t 
                            const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
                            const moe_weights_t *w, moe_bf16_t *ybuf, int32_t *device_status, void *stream);
 
+/* ---------------------------------------------------------------------
+ * The expert FFN with MXFP8 expert weights (block-scaled FP8: E4M3 codes,
+ * one UE8M0 power-of-two scale per 32 consecutive weights along the
+ * reduction axis), the FP8 expert weights that DeepGEMM fork PR #5 "big M
+ * opt: splitT1 + L2 scatter + 2 stream" names against its W8A8 reference.
+ * Weights only: activations stay bf16.  Each weight tile is turned into bf16
+ * in shared memory on its way to the tensor cores; every E4M3 code times its
+ * block's power of two is a bf16 value (for scales 2^-117 .. 2^119), so the
+ * layer computes exactly what moe_expert_ffn computes on the dequantised
+ * weights, while half the weight bytes cross HBM.
+ *   Codes: moe_quantize_mxfp8 of each matrix, in the bf16 weights' shapes.
+ *   Scales: moe_quantize_mxfp8's [rows, K / 32] scales repacked once by
+ *   moe_mxfp8_pack_scales (below) -- rows is E * I for w_gate / w_up and
+ *   E * H for w_down, K the matrix's reduction size.
+ * Limits on top of the general ones: H, I and Is multiples of 128.
+ * --------------------------------------------------------------------- */
+typedef struct {
+    const uint8_t *w_gate;          /* [E, I, H] E4M3 codes */
+    const uint8_t *w_up;            /* [E, I, H] E4M3 codes */
+    const uint8_t *w_down;          /* [E, H, I] E4M3 codes */
+    const uint8_t *w_gate_scale;    /* packed UE8M0 scales of w_gate (E * I rows, K = H) */
+    const uint8_t *w_up_scale;      /* packed scales of w_up */
+    const uint8_t *w_down_scale;    /* packed scales of w_down (E * H rows, K = I) */
+    const uint8_t *ws_gate;         /* [Is, H] shared-expert codes, NULL if Is = 0 */
+    const uint8_t *ws_up;           /* [Is, H], NULL if Is = 0 */
+    const uint8_t *ws_down;         /* [H, Is], NULL if Is = 0 */
+    const uint8_t *ws_gate_scale;   /* packed scales of ws_gate (Is rows, K = H), NULL if Is = 0 */
+    const uint8_t *ws_up_scale;     /* packed scales of ws_up, NULL if Is = 0 */
+    const uint8_t *ws_down_scale;   /* packed scales of ws_down (H rows, K = Is), NULL if Is = 0 */
+    const moe_bf16_t *ws_gate_vec;  /* [H] bf16 shared-expert gate vector, NULL if Is = 0 */
+    const moe_bf16_t *w_router;     /* [E, H] bf16 router projection (moe_forward_mxfp8 without logits) */
+} moe_weights_mxfp8_t;
+
+/* Repack MXFP8 scales [rows, K / 32] (as moe_quantize_mxfp8 writes them) into
+ * the layout the FFN reads: [rows / 64][K / 128][64][4] -- for every group of
+ * 64 rows and every 128 weights along K, the group's 64 x 4 scales as one
+ * 256-byte run.  rows % 64 == 0, K % 128 == 0; both pointers device,
+ * 16-byte aligned; same byte count in and out.  Run once per weight load. */
+int moe_mxfp8_pack_scales(int64_t rows, int32_t K, const uint8_t *scales, uint8_t *packed, void *stream);
+
+/* moe_expert_ffn with MXFP8 expert weights; arguments and results as
+ * moe_expert_ffn (the same workspace size). */
+int moe_expert_ffn_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                         const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                         const moe_weights_mxfp8_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_forward with MXFP8 expert weights: routing, budget, dispatch and
+ * combine as moe_forward, the expert FFN as moe_expert_ffn_mxfp8. */
+int moe_forward_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
+                      const moe_weights_mxfp8_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
+                      size_t ws_bytes, void *stream);
+
 /* Combine: out[t, :] = bf16( sum_{j < keff[t]} ybuf[t, j, :] + [Is > 0] ybuf[t, k, :] ),
  * summed in fp32 in slot order and rounded once (a token with no kept slot
  * and no shared expert gets 0).  keff == NULL means k.
@@ -264,8 +316,9 @@ const char *moe_error_string(int code);
  * the largest magnitude, so in NVFP4 it spoils its whole matrix's scale);
  * the quantisers do not check for them.  The blocks
  * run along the last (reduction) axis of a row-major matrix: rows of
- * W_gate / W_up [I, H] and of W_down [H, I].  The layer does not consume
- * these formats yet.
+ * W_gate / W_up [I, H] and of W_down [H, I].  The layer consumes MXFP8
+ * (moe_expert_ffn_mxfp8 / moe_forward_mxfp8 above); NVFP4 is the pack step
+ * only.
  * --------------------------------------------------------------------- */
 
 /* MXFP8: blocks of 32 consecutive elements share a UE8M0 scale

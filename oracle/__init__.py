@@ -436,7 +436,9 @@ def f64_to_bf16_exact(v) -> np.ndarray:
     v = np.asarray(v, np.float64)
     f = v.astype(np.float32)
     bits = f.view(np.uint32)
-    if not np.array_equal(f.astype(np.float64), v, equal_nan=True) or np.any(bits & 0xFFFF):
+    back = f.astype(np.float64)
+    exact = np.array_equal(back, v) or np.array_equal(back, v, equal_nan=True)  # the NaN-aware pass only if needed
+    if not exact or np.any(bits & 0xFFFF):
         raise ValueError("value not representable in bf16")
     return (bits >> 16).astype(np.uint16)
 

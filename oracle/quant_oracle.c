@@ -143,6 +143,8 @@ void oracle_ue8m0_decode(int64_t n, const uint8_t *codes, double *out)
 int oracle_mxfp8_quantize(int64_t rows, int64_t K, const uint16_t *w, uint8_t *codes, uint8_t *scales)
 {
     if (rows < 0 || K < 32 || K % 32 != 0) return ORACLE_EINVAL;
+    /* rows are independent: split over the host threads (no effect on any value) */
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t b = 0; b < K / 32; ++b) {
             const uint16_t *x = w + r * K + b * 32;
@@ -186,6 +188,8 @@ int oracle_nvfp4_quantize(int64_t rows, int64_t K, const uint16_t *w, uint8_t *c
     const float st = amax > 0.0f ? amax / 2688.0f : 1.0f; /* 2688 = 6 * 448 */
     *tensor_scale = st;
     memset(codes, 0, (size_t)(rows * K / 2));
+    /* rows are independent (K is even, so no code byte spans two rows) */
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t b = 0; b < K / 16; ++b) {
             const uint16_t *x = w + r * K + b * 16;

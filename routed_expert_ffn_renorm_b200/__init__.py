@@ -26,6 +26,7 @@ __all__ = [
     "moe_budget",
     "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn_noalloc",
     "moe_combine", "moe_forward", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
+    "MoEWeightsMXFP8", "moe_mxfp8_pack_scales", "moe_expert_ffn_mxfp8", "moe_forward_mxfp8", "pack_mxfp8",
     "status_read", "status_clear",
     "EXPORTED_SYMBOLS", "MOE_STATUS_TIMEOUT",
 ]
@@ -37,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_route", "moe_budget", "moe_dispatch", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_status_read", "moe_status_clear", "moe_error_string", "moe_expert_gate_up",
     "moe_expert_down", "moe_expert_ffn_noalloc", "moe_router_logits", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
+    "moe_mxfp8_pack_scales", "moe_expert_ffn_mxfp8", "moe_forward_mxfp8",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 MOE_STATUS_TIMEOUT = 1
@@ -57,6 +59,12 @@ class _Config(ctypes.Structure):
 class _Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec", "w_router")]
+
+
+class _WeightsMXFP8(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_gate", "w_up", "w_down", "w_gate_scale", "w_up_scale", "w_down_scale", "ws_gate", "ws_up", "ws_down",
+        "ws_gate_scale", "ws_up_scale", "ws_down_scale", "ws_gate_vec", "w_router")]
 
 
 class _Aux(ctypes.Structure):
@@ -101,6 +109,32 @@ class MoEWeights:
             "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "ws_gate_vec", "w_router")))
 
 
+@dataclass
+class MoEWeightsMXFP8:
+    """Device MXFP8 expert weights: E4M3 codes (uint8) in the bf16 weights'
+    shapes -- w_gate, w_up [E, I, H], w_down [E, H, I], optional shared
+    ws_gate, ws_up [Is, H], ws_down [H, Is] -- and each matrix's UE8M0 scales
+    in the FFN's packed layout (moe_mxfp8_pack_scales); ws_gate_vec [H] and
+    w_router [E, H] stay bf16.  pack_mxfp8() builds one from MoEWeights."""
+    w_gate: "torch.Tensor"
+    w_up: "torch.Tensor"
+    w_down: "torch.Tensor"
+    w_gate_scale: "torch.Tensor"
+    w_up_scale: "torch.Tensor"
+    w_down_scale: "torch.Tensor"
+    ws_gate: Optional["torch.Tensor"] = None
+    ws_up: Optional["torch.Tensor"] = None
+    ws_down: Optional["torch.Tensor"] = None
+    ws_gate_scale: Optional["torch.Tensor"] = None
+    ws_up_scale: Optional["torch.Tensor"] = None
+    ws_down_scale: Optional["torch.Tensor"] = None
+    ws_gate_vec: Optional["torch.Tensor"] = None
+    w_router: Optional["torch.Tensor"] = None
+
+    def _c(self) -> _WeightsMXFP8:
+        return _WeightsMXFP8(*(_ptr(getattr(self, n), allow_none=True) for n, _ in _WeightsMXFP8._fields_))
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -137,6 +171,10 @@ def load_library(build_if_stale: bool = True):
         i64 = ctypes.c_int64
         lib.moe_quantize_mxfp8.argtypes = [i64, i32, P, P, P, P]
         lib.moe_quantize_nvfp4.argtypes = [i32, i64, i32, P, P, P, P, P]
+        lib.moe_mxfp8_pack_scales.argtypes = [i64, i32, P, P, P]
+        lib.moe_expert_ffn_mxfp8.argtypes = [cfg, i32, P, P, P, P, P, P, ctypes.POINTER(_WeightsMXFP8), P, P, sz, P]
+        lib.moe_forward_mxfp8.argtypes = [cfg, i32, P, P, ctypes.POINTER(_WeightsMXFP8), P, ctypes.POINTER(_Aux), P,
+                                          sz, P]
         lib.moe_error_string.restype = ctypes.c_char_p
         lib.moe_error_string.argtypes = [ctypes.c_int]
         for name in EXPORTED_SYMBOLS:
@@ -220,6 +258,64 @@ def moe_quantize_nvfp4(w, codes, scales, tensor_scale, stream=None):
     _expect(tensor_scale, torch.float32, nmat, "tensor_scale")
     _check("moe_quantize_nvfp4", load_library().moe_quantize_nvfp4(
         nmat, rows, K, _ptr(w), _ptr(codes), _ptr(scales), _ptr(tensor_scale), _stream(stream)))
+
+
+def moe_mxfp8_pack_scales(scales, packed, stream=None):
+    """MXFP8 scales [rows, K // 32] uint8 -> the FFN's layout
+    [rows / 64][K / 128][64][4] (rows % 64 == 0, K % 128 == 0)."""
+    import torch
+    kb = scales.shape[-1]
+    _expect(scales, torch.uint8, scales.numel(), "scales")
+    _expect(packed, torch.uint8, scales.numel(), "packed")
+    _check("moe_mxfp8_pack_scales", load_library().moe_mxfp8_pack_scales(
+        scales.numel() // kb, kb * 32, _ptr(scales), _ptr(packed), _stream(stream)))
+
+
+def pack_mxfp8(weights: MoEWeights, stream=None) -> MoEWeightsMXFP8:
+    """Quantise every expert matrix of `weights` to MXFP8 on the GPU
+    (moe_quantize_mxfp8, then moe_mxfp8_pack_scales); the gate vector and
+    the router projection are passed through.  Allocates the outputs."""
+    import torch
+
+    def one(w):
+        codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+        scales = torch.empty(w.shape[:-1] + (w.shape[-1] // 32,), dtype=torch.uint8, device=w.device)
+        moe_quantize_mxfp8(w, codes, scales, stream=stream)
+        packed = torch.empty_like(scales)
+        moe_mxfp8_pack_scales(scales, packed, stream=stream)
+        return codes, packed
+
+    (g, gs), (u, us), (d, ds) = one(weights.w_gate), one(weights.w_up), one(weights.w_down)
+    out = MoEWeightsMXFP8(g, u, d, gs, us, ds, ws_gate_vec=weights.ws_gate_vec, w_router=weights.w_router)
+    if weights.ws_gate is not None:
+        (out.ws_gate, out.ws_gate_scale), (out.ws_up, out.ws_up_scale), (out.ws_down, out.ws_down_scale) = (
+            one(weights.ws_gate), one(weights.ws_up), one(weights.ws_down))
+    return out
+
+
+def moe_expert_ffn_mxfp8(cfg: MoEConfig, x, x_perm, offsets, perm, topk_w, weights: MoEWeightsMXFP8, ybuf, ws, *,
+                         sgate=None, stream=None):
+    """moe_expert_ffn with MXFP8 expert weights."""
+    T = x.shape[0]
+    w = weights._c()
+    _check("moe_expert_ffn_mxfp8", load_library().moe_expert_ffn_mxfp8(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(perm), _ptr(topk_w),
+        _ptr(sgate, True), ctypes.byref(w), _ptr(ybuf), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_forward_mxfp8(cfg: MoEConfig, x, logits, weights: MoEWeightsMXFP8, out, ws, *, aux: Optional[dict] = None,
+                      stream=None):
+    """moe_forward with MXFP8 expert weights (arguments as moe_forward)."""
+    T = x.shape[0]
+    w = weights._c()
+    a = _Aux()
+    if aux:
+        for name, t in aux.items():
+            setattr(a, name, _ptr(t))
+    _check("moe_forward_mxfp8", load_library().moe_forward_mxfp8(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(logits, True), ctypes.byref(w), _ptr(out), ctypes.byref(a),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_route(cfg: MoEConfig, logits, topk_idx, topk_w, *, x=None, ws_gate_vec=None, sgate=None, keff=None,

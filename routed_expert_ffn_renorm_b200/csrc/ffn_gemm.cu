@@ -84,12 +84,21 @@ constexpr int kBlockK = 64;                    // K elements per step (128 B row
 constexpr int kTileM = 128;                    // weight rows per tile (MMA M)
 constexpr int kABytes = kTileM * kBlockK * 2;  // 16 KB
 constexpr int kNumBox = 5;                     // token box heights 16 << i
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;                  // bf16 weights: producer, MMA, 4 epilogue warps
+// Block-scaled (MXFP8) weights: converter warps after the epilogue warps turn
+// each ring step's FP8 codes into the bf16 A operand in shared memory.
+constexpr int kConvWarps = 4;
+constexpr int kThreadsQ = kThreads + 32 * kConvWarps;
+constexpr int kQKStep = 128;                   // K elements per FP8 ring step (one 128-byte code box row)
+constexpr int kQCodePages = kTileM * kQKStep / 2048;  // 8 pages: 128 rows x 128 codes
+constexpr int kQScaleBytes = 512;              // 128 rows x 4 UE8M0 scales (blocks of 32) per step
+constexpr int kCbufBytes = 2 * 2 * kABytes;    // two conversion buffers, each two bf16 K slices of 64
 constexpr int kPageBytes = 2048;               // ring unit: 16 token rows of 128 B
 constexpr int kAPages = kABytes / kPageBytes;  // 8 pages of weights per K step
 constexpr int kMaxStepPages = kAPages + 256 * 128 / kPageBytes;  // 24: weights + 256 token rows
 constexpr int kTwoSlicePages = 32;  // two K slices per ring step up to here, when the ring holds 4 slices
 constexpr int kMaxPages = 112;
+constexpr int kQMaxStepPages = kQCodePages + 1 + 2 * (256 * 128 / 2048);  // 41: codes, scales, 2 token boxes
 constexpr int kTickets = 32;                   // K steps in flight at most (barrier pairs)
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
 constexpr int kXchgStride = 33;                // fp32 exchange row stride (bank-conflict free)
@@ -115,6 +124,11 @@ struct FfnParams {
     int phases;         // bit 0: gate/up items, bit 1: down items
     int R[2], Rs[2];    // weight tiles per routed / shared expert, per phase
     int nk[2], nks[2];  // K steps routed / shared, per phase
+    // MXFP8 weights only: the packed UE8M0 scales of each matrix, [phase][0: gate
+    // or down, 1: up], routed and shared; 256 bytes per (64-row group, 128-wide K
+    // step), row-group major (see moe_mxfp8_pack_scales)
+    const uint8_t *sf[2][2];
+    const uint8_t *sfs[2][2];
     const int32_t *offsets;
     const int32_t *perm;
     const float *topk_w;
@@ -231,10 +245,10 @@ __device__ __forceinline__ Item decode_item(int item, const Schedule &sc, const 
 // Exclusive block scan over the experts of two counts at once:
 // a[e] = sum_{e' < e} f(e').x, b[e] likewise with .y; a[E], b[E] = the totals.
 // Every thread of the block calls it.
-template <class F>
+template <int NT, class F>
 __device__ __forceinline__ void expert_scan2(int E, int *a, int *b, int2 *scan_tmp, F f) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int per = (E + kThreads - 1) / kThreads;
+    const int per = (E + NT - 1) / NT;
     const int e0 = threadIdx.x * per, e1 = min(E, e0 + per);
     int2 local = make_int2(0, 0);
     for (int e = e0; e < e1; ++e) {
@@ -244,12 +258,12 @@ __device__ __forceinline__ void expert_scan2(int E, int *a, int *b, int2 *scan_t
     }
     scan_tmp[threadIdx.x] = local;
     __syncthreads();
-    if (warp == 0) {  // kThreads partials, kThreads / 32 per lane
-        int2 v[kThreads / 32];
+    if (warp == 0) {  // NT partials, NT / 32 per lane
+        int2 v[NT / 32];
         int2 sum = make_int2(0, 0);
 #pragma unroll
-        for (int q = 0; q < kThreads / 32; ++q) {
-            v[q] = scan_tmp[lane * (kThreads / 32) + q];
+        for (int q = 0; q < NT / 32; ++q) {
+            v[q] = scan_tmp[lane * (NT / 32) + q];
             sum.x += v[q].x;
             sum.y += v[q].y;
         }
@@ -264,8 +278,8 @@ __device__ __forceinline__ void expert_scan2(int E, int *a, int *b, int2 *scan_t
         }
         int2 run = make_int2(incl.x - sum.x, incl.y - sum.y);
 #pragma unroll
-        for (int q = 0; q < kThreads / 32; ++q) {
-            scan_tmp[lane * (kThreads / 32) + q] = run;
+        for (int q = 0; q < NT / 32; ++q) {
+            scan_tmp[lane * (NT / 32) + q] = run;
             run.x += v[q].x;
             run.y += v[q].y;
         }
@@ -338,7 +352,111 @@ __device__ __forceinline__ StepShape step_shape(const Item &it, const FfnParams 
     return sh;
 }
 
+// MXFP8 ring step: 128 K elements -- the codes of one weight tile (8 pages),
+// their scales (one page, 512 bytes used) and the token rows as two bf16
+// boxes of 64 K (sub_pages = 2^bi pages each).  ns = 2 slices, nk counts
+// 64-wide slices (even: K is a multiple of 128).
+__device__ __forceinline__ StepShape qstep_shape(const Item &it, const FfnParams &p) {
+    StepShape sh;
+    sh.bi = box_index(it.nvalid);
+    sh.sub_pages = 1u << sh.bi;
+    sh.ns = 2;
+    sh.nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
+    return sh;
+}
+__device__ __forceinline__ uint32_t qstep_pages(const StepShape &sh) { return kQCodePages + 1 + 2 * sh.sub_pages; }
+
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
+
+// ------------------------------------------------- MXFP8 weight conversion --
+// An MXFP8 weight is an E4M3 code times its block's power of two 2^se (one
+// UE8M0 scale per 32 consecutive K elements).  Every such value with se in
+// [-117, 119] is a bf16 value, so the conversion below is exact and the MMA
+// then runs on exactly the weights the format stands for.
+//
+// Two codes at once, bf16x2: the code's sign goes to bit 15 of its 16-bit
+// lane and its 7 magnitude bits (eeee mmm) to bits 10..4, i.e. the low four
+// exponent bits and the top three mantissa bits of a bf16.  As a bf16 that
+// lane is 2^(e - 127) * 1.mmm for e > 0 and the subnormal 0.mmm * 2^-126 for
+// e = 0; one multiply by 2^(120 + se) makes both the code's value
+// (2^(e - 7) * 1.mmm, or 0.mmm * 2^-6) times 2^se.  The byte permute with
+// sign replication puts each code's sign in the high byte of its lane, the
+// shift and mask keep bit 15 and bits 10..4.
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t e4m3x2_lanes(uint32_t w, uint32_t sel) {
+    return (prmt_b32(w, 0u, sel) << 4) & 0x87F087F0u;
+}
+
+// 16 codes (one 16-byte chunk) and their scale code -> 16 bf16 (two chunks).
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &q, uint32_t sc, uint4 &o0, uint4 &o1) {
+    uint32_t m1, m2 = 0;
+    const bool one = sc <= 134u;  // 2^(120 + se) is a normal bf16: one multiply
+    if (one) {
+        m1 = (sc + 120u) << 7;
+    } else {  // 2^127 first, then 2^(se - 7)
+        m1 = 254u << 7;
+        m2 = (sc - 7u) << 7;
+        m2 |= m2 << 16;
+    }
+    m1 |= m1 << 16;
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t r[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        r[2 * i] = bf16x2_mul(e4m3x2_lanes(w[i], 0x9180u), m1);      // codes 4i, 4i + 1
+        r[2 * i + 1] = bf16x2_mul(e4m3x2_lanes(w[i], 0xB3A2u), m1);  // codes 4i + 2, 4i + 3
+    }
+    if (!one) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r[i] = bf16x2_mul(r[i], m2);
+    }
+    o0 = make_uint4(r[0], r[1], r[2], r[3]);
+    o1 = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+// One ring step's weight tile: 128 rows x 128 E4M3 codes, as TMA left them
+// (row r at r * 128 bytes, 16-byte chunk c at (c ^ (r & 7)) * 16: the 128-byte
+// swizzle), with their scales (row r's four at byte 4r), into two K-major bf16
+// slices of 64 in the same swizzle (slice s at dst + s * 16 KB), the MMA's A
+// operand.  Thread ct of nt takes units u = ct, ct + nt, ...; unit u is row
+// (u / 64) * 8 + u % 8, chunk (u / 8) % 8, so the 8 lanes of a shared-memory
+// phase share a chunk over 8 consecutive rows and, swizzled, hit 8 distinct
+// 16-byte bank groups on every load and store.
+template <int kNt>
+__device__ __forceinline__ void convert_mxfp8_tile(uint32_t codes, uint32_t scales, uint32_t dst, int ct) {
+#pragma unroll 4
+    for (int i = 0; i < 1024 / kNt; ++i) {
+        const int u = ct + i * kNt;
+        const int r = ((u >> 6) << 3) | (u & 7);
+        const int c = (u >> 3) & 7;
+        const int sw = r & 7;
+        uint4 q;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
+                     : "r"(codes + (uint32_t)(r * 128 + ((c ^ sw) << 4))));
+        uint32_t sc;
+        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sc) : "r"(scales + (uint32_t)(r * 4 + (c >> 1))));
+        uint4 o0, o1;
+        e4m3x16_to_bf16(q, sc, o0, o1);
+        const uint32_t row = dst + (uint32_t)((c >> 2) * kABytes + r * 128);
+        const int cc = (c & 3) << 1;  // first of the two bf16 chunks in the slice
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)((cc ^ sw) << 4)), "r"(o0.x),
+                     "r"(o0.y), "r"(o0.z), "r"(o0.w)
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)(((cc + 1) ^ sw) << 4)),
+                     "r"(o1.x), "r"(o1.y), "r"(o1.z), "r"(o1.w)
+                     : "memory");
+    }
+}
 
 // Down item, token n of the tile: its ybuf row (t*(k+1) + j, or t*(k+1) + k for
 // the shared expert) and the weight applied to it.
@@ -358,12 +476,20 @@ __device__ __forceinline__ void down_dest(const Item &it, int n, const FfnParams
 }
 
 // --------------------------------------------------------------- kernel --
-template <bool kPair>
-__global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant__ FfnMaps maps, const FfnParams p) {
+// kFmt: 0 bf16 weights; 1 MXFP8 weights (E4M3 codes + UE8M0 block scales),
+// converted to bf16 in shared memory by kConvWarps converter warps (single
+// CTAs only).
+template <bool kPair, int kFmt>
+__global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
+    ffn_kernel(const __grid_constant__ FfnMaps maps, const FfnParams p) {
+    constexpr int NT = kFmt ? kThreadsQ : kThreads;
+    static_assert(!(kPair && kFmt), "block-scaled weights run on single CTAs");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t P = (uint32_t)p.pages;
-    uint8_t *ring = smem;
+    // MXFP8: two conversion buffers (bf16 A operands of a ring step) ahead of the ring
+    uint8_t *cbuf = smem;
+    uint8_t *ring = smem + (kFmt ? kCbufBytes : 0);
     float *xchg = reinterpret_cast<float *>(smem + (size_t)P * kPageBytes);
     int *tile_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
     int *dbase = tile_base + (p.E + 1);                                 // [E + 1]
@@ -373,14 +499,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     uint64_t *full = bars, *empty = bars + kTickets, *tfull = bars + 2 * kTickets, *tempty = tfull + 2;
     uint64_t *mma_done = tfull + 4;
     uint64_t *qfull = tfull + 5, *qempty = qfull + kQueue;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qempty + kQueue);
+    uint64_t *cfull = qempty + kQueue, *cempty = cfull + 2;  // MXFP8: conversion buffer converted / free
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // elected -> epilogue: 0 go, -1 stop
     ItemSlot *qdesc = reinterpret_cast<ItemSlot *>(tmem_slot + 4);  // [kQueue], written by the producer
     ItemSlot *epi_desc = qdesc + kQueue;                             // the epilogue's current item
-    int *scan_tmp = reinterpret_cast<int *>(                          // [2 * kThreads] (int2 partials)
-        (reinterpret_cast<uintptr_t>(epi_desc + 1) + 7) & ~uintptr_t(7));
-    uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + 2 * kThreads);  // [kReadyWords], producer-private
+    ItemSlot *conv_desc = epi_desc + 1;                              // the converters' current item
+    int *scan_tmp = reinterpret_cast<int *>(                          // [2 * NT] (int2 partials)
+        (reinterpret_cast<uintptr_t>(conv_desc + 1) + 7) & ~uintptr_t(7));
+    uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + 2 * NT);  // [kReadyWords], producer-private
     uint32_t *ticket_start = ready_bits + kReadyWords;  // [kTickets] first ring page (virtual) of each step; producer-private
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -402,8 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         for (int q = 0; q < kQueue; ++q) {
             mbar_init(&qfull[q], 1);
             // the MMA lane and the elected epilogue thread (pair: and the other CTA's
-            // producer and epilogue)
-            mbar_init(&qempty[q], kPair ? 4 : 2);
+            // producer and epilogue; MXFP8: and the elected converter thread)
+            mbar_init(&qempty[q], kPair ? 4 : (kFmt ? 3 : 2));
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&cfull[b], kConvWarps);  // one arrival per converter warp
+            mbar_init(&cempty[b], 1);          // the MMA lane's commit
         }
         *abort_flag = 0;
         for (int w = 0; w < kReadyWords; ++w) ready_bits[w] = 0;
@@ -446,19 +578,20 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
     if (warp == 0 && lane == 0 && (!kPair || rank == 0)) first_claim = atomicAdd(p.sched, 1);
     // dispatch offsets to shared memory, then the per-expert prefix sums of token
     // tiles and of down items
-    for (int e = threadIdx.x; e <= p.E; e += kThreads) offs[e] = __ldg(p.offsets + e);
+    for (int e = threadIdx.x; e <= p.E; e += NT) offs[e] = __ldg(p.offsets + e);
     __syncthreads();
     Schedule sc;
     sc.shared_ntt = p.Is > 0 ? (p.T + p.BNs - 1) / p.BNs : 0;
     {
         const int BN = p.BN, R1 = p.R[1];
         const int *o = offs;
-        expert_scan2(p.E, tile_base, dbase, reinterpret_cast<int2 *>(scan_tmp), [=](int e) {
+        expert_scan2<NT>(p.E, tile_base, dbase, reinterpret_cast<int2 *>(scan_tmp), [=](int e) {
             const int cnt = o[e + 1] - o[e];
             return make_int2((cnt + BN - 1) / BN, merged_down_items(cnt, BN, R1));
         });
         // every CTA takes the same decision from the same offsets
-        sc.merge = !kPair && (tile_base[p.E] * R1 + p.Rs[1] * sc.shared_ntt) >= kMergePerCta * (int)gridDim.x;
+        sc.merge = !kPair && kFmt == 0 &&
+                   (tile_base[p.E] * R1 + p.Rs[1] * sc.shared_ntt) >= kMergePerCta * (int)gridDim.x;
     }
     tc_fence_after();
     sc.shared_merge = p.Is > 0 && sc.shared_ntt == 1 && down_merged(p.T, p.BN, sc.merge);
@@ -553,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 const PhaseMaps &pm = maps.ph[it.ph];
                 const CUtensorMap *ma0 = it.shared ? &pm.s0 : &pm.a0;
                 const CUtensorMap *ma1 = it.shared ? &pm.s1 : &pm.a1;
-                const StepShape sh = step_shape<kPair>(it, p);
+                const StepShape sh = kFmt ? qstep_shape(it, p) : step_shape<kPair>(it, p);
                 const CUtensorMap *mb = it.shared ? &pm.bs[sh.bi] : &pm.b[sh.bi];
                 // pair: this CTA's weight tile of the two, and its half of the token rows
                 const int rt = kPair ? 2 * it.r + (int)rank : it.r;
@@ -564,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 bool ok = true;
                 for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
                     const int nsub = min(sh.ns, sh.nk - k0);
-                    const uint32_t need = (uint32_t)nsub * sh.sub_pages;
+                    const uint32_t need = kFmt ? qstep_pages(sh) : (uint32_t)nsub * sh.sub_pages;
                     const uint32_t first = ring_alloc(vhead, off, need, P);
                     // Free a ticket and the pages of this step: retire the oldest steps
                     // until the steps in flight and this one lie within P consecutive
@@ -582,7 +715,26 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                     const uint32_t tk = issued % kTickets;
                     if (issued == retired) oldest = vhead - need;
                     ticket_start[tk] = vhead - need;
-                    if constexpr (kPair) {
+                    if constexpr (kFmt != 0) {
+                        // codes of the weight tile, their scales, two token boxes
+                        mbar_arrive_expect_tx(&full[tk], (kQCodePages + 2 * sh.sub_pages) * kPageBytes + kQScaleBytes);
+                        uint8_t *sA = ring + (size_t)first * kPageBytes;
+                        const int kx = k0 * kBlockK;  // = 128 * (K step)
+                        const int ks = k0 >> 1;
+                        tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, apol);  // gate: 64 rows; down: 128 rows
+                        if (it.ph == 0) tma_load_2d_hint(ma1, &full[tk], sA + kQCodePages * kPageBytes / 2, kx, a_row, apol);
+                        uint8_t *sS = sA + kQCodePages * kPageBytes;
+                        const size_t ksteps = (size_t)(sh.nk >> 1);
+                        const size_t rg = (size_t)(a_row >> 6);  // 64-row group of the tile's first row
+                        const uint8_t *const *sfp = it.shared ? p.sfs[it.ph] : p.sf[it.ph];
+                        bulk_load(sS, sfp[0] + (rg * ksteps + ks) * 256, 256, &full[tk]);
+                        // gate/up: the up rows' scales; down: the tile's second 64-row group
+                        bulk_load(sS + 256, it.ph == 0 ? sfp[1] + (rg * ksteps + ks) * 256 : sfp[0] + ((rg + 1) * ksteps + ks) * 256,
+                                  256, &full[tk]);
+                        uint8_t *sB = sS + kPageBytes;
+                        tma_load_2d(mb, &full[tk], sB, kx, it.row0);
+                        tma_load_2d(mb, &full[tk], sB + sh.sub_pages * kPageBytes, kx + kBlockK, it.row0);
+                    } else if constexpr (kPair) {
                         // both CTAs' loads complete on CTA 0's barrier, armed there with both halves
                         if (rank == 0) mbar_arrive_expect_tx(&full[tk], 2 * need * kPageBytes);
                         const uint32_t bar0 = mapa(smem_u32(&full[tk]), 0);
@@ -632,6 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
         if (lane == 0 && (!kPair || rank == 0)) {  // a pair's MMAs are issued by CTA 0
             uint32_t vhead = 0, off = 0, step = 0;  // the producer's page sequence, replayed
             const uint64_t desc0 = sw128_desc(smem_u32(ring));  // ring page 0; other pages by addition
+            const uint64_t cdesc0 = sw128_desc(smem_u32(cbuf));  // MXFP8: conversion buffer 0
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 if (!mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) break;
@@ -639,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 const Item it = qdesc[slot].it;
                 mbar_arrive(&qempty[slot]);
                 if (item < 0) break;
-                const StepShape sh = step_shape<kPair>(it, p);
+                const StepShape sh = kFmt ? qstep_shape(it, p) : step_shape<kPair>(it, p);
                 const uint32_t idesc = idesc_bf16((it.nvalid + 15) & ~15, kPair ? 2 * kTileM : kTileM);
                 const int acc = li & 1;
                 const uint32_t use = (uint32_t)(li >> 1);
@@ -649,11 +802,35 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
                 bool ok = true;
                 for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
                     const int nsub = min(sh.ns, sh.nk - k0);
-                    const uint32_t first = ring_alloc(vhead, off, (uint32_t)nsub * sh.sub_pages, P);
+                    const uint32_t first =
+                        ring_alloc(vhead, off, kFmt ? qstep_pages(sh) : (uint32_t)nsub * sh.sub_pages, P);
                     const uint32_t tk = step % kTickets;
                     if (!mbar_wait_fast<kPair>(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true)) {
                         ok = false;
                         break;
+                    }
+                    if constexpr (kFmt != 0) {
+                        // the converted weights of this step (conversion buffer step & 1), and
+                        // the token boxes in the ring
+                        const uint32_t cb = step & 1u;
+                        if (!mbar_wait_fast(&cfull[cb], (step >> 1) & 1u, abort_flag, p.status, true)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t db = desc0 + (first + kQCodePages + 1) * (kPageBytes / 16);
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const uint64_t da = cdesc0 + (cb * 2 + j) * (kABytes / 16);
+                            const uint64_t dbj = db + j * sh.sub_pages * (kPageBytes / 16);
+#pragma unroll
+                            for (int kk = 0; kk < kBlockK / 16; ++kk)
+                                umma_bf16(d, da + 2 * kk, dbj + 2 * kk, idesc, (k0 | j | kk) != 0);
+                        }
+                        umma_commit(&empty[tk]);  // the ring pages (codes, scales, tokens)
+                        umma_commit(&cempty[cb]);  // the conversion buffer
+                        ++step;
+                        continue;
                     }
                     tc_fence_after();
                     for (int j = 0; j < nsub; ++j) {
@@ -689,6 +866,50 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             if constexpr (kPair) umma_commit_pair_local(mma_done);  // completes once every MMA above has
             else umma_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.status, false);
+        }
+    } else if (kFmt != 0 && warp >= 6) {
+        // ================= MXFP8 converters (warps 6 ..) =================
+        // Walk the producer's step sequence: once a step's codes and scales have
+        // landed and the MMAs of the step two back have released conversion buffer
+        // step & 1, write that step's bf16 weights there and hand it to the MMA lane.
+        // Every converter thread takes the same waits and a warp leaves a step loop
+        // only as a whole (a vote after the waits); a failed wait sets the abort
+        // flag, and the elected thread then publishes "stop" at the next queue read,
+        // so every converter thread reaches the same named barriers.
+        const int ct = threadIdx.x - kThreads;  // 0 .. 32 * kConvWarps - 1
+        const bool elected = ct == 0;
+        uint32_t vhead = 0, off = 0, step = 0;
+        for (int li = 0;; ++li) {
+            const int slot = li % kQueue;
+            if (elected) {
+                if (!*abort_flag && mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) {
+                    *conv_desc = qdesc[slot];
+                    mbar_arrive(&qempty[slot]);
+                } else {
+                    conv_desc->item = -2;
+                }
+            }
+            named_bar_sync(2, 32 * kConvWarps);
+            const int item = conv_desc->item;
+            const Item it = conv_desc->it;
+            named_bar_sync(2, 32 * kConvWarps);  // read by all before the elected thread's next write
+            if (item < 0) break;
+            const StepShape sh = qstep_shape(it, p);
+            const uint32_t need = qstep_pages(sh);
+            for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
+                const uint32_t first = ring_alloc(vhead, off, need, P);
+                const uint32_t tk = step % kTickets, cb = step & 1u;
+                const bool ok = mbar_wait_fast(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true) &&
+                                mbar_wait_fast(&cempty[cb], ((step >> 1) & 1u) ^ 1u, abort_flag, p.status, true);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                const uint32_t codes = smem_u32(ring + (size_t)first * kPageBytes);
+                convert_mxfp8_tile<32 * kConvWarps>(codes, codes + kQCodePages * kPageBytes,
+                                                    smem_u32(cbuf + cb * 2 * kABytes), ct);
+                fence_proxy_async_shared();  // the stores, visible to the tensor cores' reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cfull[cb]);
+                ++step;
+            }
         }
     } else {
         // ================= epilogue (warps 2..5) =================
@@ -801,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
             atomicExch(p.sched + 1, 0);
         }
         if (fused)
-            for (int g = threadIdx.x; g <= p.E + 1; g += kThreads) atomicExch(p.hdone + g, 0);
+            for (int g = threadIdx.x; g <= p.E + 1; g += NT) atomicExch(p.hdone + g, 0);
         __threadfence();
     }
 }
@@ -811,7 +1032,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const __grid_constant_
 // shared-memory cost follows its real token count (the paged ring), so a
 // wide tile costs nothing for small groups and saves re-reading a weight
 // tile for every 128 tokens of large ones.
-int pick_bn() { return 256; }
+// MXFP8 weights: 128, so that a ring step (codes, scales, two token boxes)
+// stays at 25 pages and the smaller ring that the conversion buffers leave
+// still holds three of them.
+int pick_bn(int fmt) { return fmt ? 128 : 256; }
 
 // Token tile of the shared expert, which sees all T tokens.  One 256-token
 // tile streams each weight tile once, but its items then run about twice as
@@ -824,14 +1048,17 @@ int pick_bns(const FfnArgs &a, int bn, int sms) {
     return est >= 4LL * sms ? bn : std::min(bn, 128);
 }
 
-size_t smem_bytes_for(int E, int pages) {
-    return 1024 + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 + 3 * (size_t)(E + 1) * 4 + 8 +
-           (size_t)(2 * kTickets + 5 + 2 * kQueue) * 8 + 16 + (kQueue + 1) * sizeof(ItemSlot) + 8 + 2 * kThreads * 4 +
-           kReadyWords * 4 + kTickets * 4;
+size_t smem_bytes_for(int E, int pages, int fmt) {
+    const int nt = fmt ? kThreadsQ : kThreads;
+    return 1024 + (fmt ? (size_t)kCbufBytes : 0) + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 +
+           3 * (size_t)(E + 1) * 4 + 8 + (size_t)(2 * kTickets + 5 + 2 * kQueue + 4) * 8 + 16 +
+           (kQueue + 2) * sizeof(ItemSlot) + 8 + 2 * (size_t)nt * 4 + kReadyWords * 4 + kTickets * 4;
 }
 
-int pick_pages(int E) {
-    const size_t fixed = smem_bytes_for(E, 0);
+int min_pages(int fmt) { return fmt ? kQMaxStepPages : kMaxStepPages; }
+
+int pick_pages(int E, int fmt) {
+    const size_t fixed = smem_bytes_for(E, 0, fmt);
     if (fixed >= (size_t)kSmemLimit) return 0;
     return (int)std::min<size_t>(kMaxPages, ((size_t)kSmemLimit - fixed) / kPageBytes);
 }
@@ -857,7 +1084,7 @@ DeviceInfo device_info() {
 // Benchmark/test overrides: MOE_FORCE_BN and MOE_FORCE_BNS in {32, 64, 128,
 // 256} (routed / shared token tile, BNS <= BN) and MOE_FORCE_PAGES in
 // [24, 112] (ring size in 2 KB pages, capped by shared memory; 24 holds one
-// widest K step); any other value is rejected.
+// widest K step; 41 with MXFP8 weights); any other value is rejected.
 int parse_tile(const char *f, int *out) {
     char *end = nullptr;
     const long v = strtol(f, &end, 10);
@@ -867,21 +1094,21 @@ int parse_tile(const char *f, int *out) {
 }
 
 int choose_tiles(const FfnArgs &a, int sms, int *bn, int *bns, int *pages) {
-    *bn = pick_bn();
+    *bn = pick_bn(a.fmt);
     if (const char *f = getenv("MOE_FORCE_BN"))
         if (int rc = parse_tile(f, bn)) return rc;
     *bns = pick_bns(a, *bn, sms);
     if (const char *f = getenv("MOE_FORCE_BNS"))
         if (int rc = parse_tile(f, bns)) return rc;
     if (*bns > *bn) return MOE_ERR_INVALID_ARG;
-    *pages = pick_pages(a.E);
+    *pages = pick_pages(a.E, a.fmt);
     if (const char *f = getenv("MOE_FORCE_PAGES")) {
         char *end = nullptr;
         const long v = strtol(f, &end, 10);
-        if (*f == 0 || *end != 0 || v < kMaxStepPages || v > kMaxPages) return MOE_ERR_INVALID_ARG;
+        if (*f == 0 || *end != 0 || v < min_pages(a.fmt) || v > kMaxPages) return MOE_ERR_INVALID_ARG;
         *pages = std::min<int>((int)v, *pages);
     }
-    return *pages >= kMaxStepPages ? MOE_OK : MOE_ERR_UNSUPPORTED;
+    return *pages >= min_pages(a.fmt) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -901,7 +1128,7 @@ int choose_pair(const FfnArgs &a, int phases, int sms, bool *pair) {
     }
     const bool even = ((phases & 1) == 0 || ((a.I / 64) % 2 == 0 && (a.Is / 64) % 2 == 0)) &&
                       ((phases & 2) == 0 || (a.H / kTileM) % 2 == 0);
-    *pair = want && even && sms >= 2;
+    *pair = want && even && sms >= 2 && a.fmt == 0;  // block-scaled weights: single CTAs
     return MOE_OK;
 }
 
@@ -927,7 +1154,9 @@ cudaError_t launch_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t 
 int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     const DeviceInfo di = device_info();
     if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
-    if (phases < 1 || phases > 3) return MOE_ERR_INVALID_ARG;
+    if (phases < 1 || phases > 3 || a.fmt < 0 || a.fmt > 1) return MOE_ERR_INVALID_ARG;
+    // MXFP8: 128-wide K steps and 64-row scale groups
+    if (a.fmt && (a.H % 128 != 0 || a.I % 128 != 0 || a.Is % 128 != 0)) return MOE_ERR_UNSUPPORTED;
     FfnParams p{};
     if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
     bool pair = false;
@@ -959,42 +1188,54 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     p.Rs[1] = a.H / kTileM / per;
     p.nk[1] = a.I / kBlockK;
     p.nks[1] = a.Is / kBlockK;
+    p.sf[0][0] = a.sf_gate;
+    p.sf[0][1] = a.sf_up;
+    p.sf[1][0] = a.sf_down;
+    p.sfs[0][0] = a.sfs_gate;
+    p.sfs[0][1] = a.sfs_up;
+    p.sfs[1][0] = a.sfs_down;
 
     static FfnMaps zero_maps;  // unused maps stay zero
     FfnMaps m = zero_maps;
     const uint64_t Tk = (uint64_t)a.T * a.k;
     bool ok = true;
+    // weight maps: bf16 boxes of 64 K, or MXFP8 code boxes of 128 K (bytes)
+    auto wmap = [&](CUtensorMap *mp, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+        return a.fmt ? encode_2d_u8(mp, base, rows, cols, box_rows) : encode_2d(mp, base, rows, cols, box_rows);
+    };
     if (phases & 1) {
         PhaseMaps &g = m.ph[0];
-        ok = ok && encode_2d(&g.a0, a.w_gate, (uint64_t)a.E * a.I, a.H, 64) &&
-             encode_2d(&g.a1, a.w_up, (uint64_t)a.E * a.I, a.H, 64);
+        ok = ok && wmap(&g.a0, a.w_gate, (uint64_t)a.E * a.I, a.H, 64) &&
+             wmap(&g.a1, a.w_up, (uint64_t)a.E * a.I, a.H, 64);
         for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&g.b[b], a.x_perm, Tk, a.H, 16 << b);
         if (a.Is > 0) {
-            ok = ok && encode_2d(&g.s0, a.ws_gate, a.Is, a.H, 64) && encode_2d(&g.s1, a.ws_up, a.Is, a.H, 64);
+            ok = ok && wmap(&g.s0, a.ws_gate, a.Is, a.H, 64) && wmap(&g.s1, a.ws_up, a.Is, a.H, 64);
             for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&g.bs[b], a.x, a.T, a.H, 16 << b);
         }
     }
     if (phases & 2) {
         PhaseMaps &d = m.ph[1];
-        ok = ok && encode_2d(&d.a0, a.w_down, (uint64_t)a.E * a.H, a.I, kTileM);
+        ok = ok && wmap(&d.a0, a.w_down, (uint64_t)a.E * a.H, a.I, kTileM);
         for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b) ok = ok && encode_2d(&d.b[b], a.h_perm, Tk, a.I, 16 << b);
         if (a.Is > 0) {
-            ok = ok && encode_2d(&d.s0, a.ws_down, a.H, a.Is, kTileM);
+            ok = ok && wmap(&d.s0, a.ws_down, a.H, a.Is, kTileM);
             for (int b = 0; b < kNumBox && (16 << b) <= BN; ++b)
                 ok = ok && encode_2d(&d.bs[b], a.h_shared, a.T, a.Is, 16 << b);
         }
     }
     if (!ok) return MOE_ERR_CUDA;
 
-    const size_t smem = smem_bytes_for(a.E, p.pages);
+    const size_t smem = smem_bytes_for(a.E, p.pages, a.fmt);
     if (smem > (size_t)kSmemLimit) return MOE_ERR_UNSUPPORTED;
     static std::atomic<int> attr_set[64];  // per device: opted in to the full shared memory
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
     if (!attr_set[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+        if (cudaFuncSetAttribute(ffn_kernel<false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+            cudaFuncSetAttribute(ffn_kernel<true, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(ffn_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
                 cudaSuccess)
             return MOE_ERR_CUDA;
         attr_set[dev].store(1, std::memory_order_release);
@@ -1008,12 +1249,18 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
         if ((phases >> ph) & 1) items += tiles * p.R[ph] + st_tiles * p.Rs[ph];
     if (pair) {  // clusters of two CTAs: an even grid
         const int grid = 2 * (int)std::max<long long>(1, std::min<long long>(di.sms / 2, items));
-        return launch_pair(ffn_kernel<true>, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess ? MOE_OK
-                                                                                                          : MOE_ERR_CUDA;
+        return launch_pair(ffn_kernel<true, 0>, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess
+                   ? MOE_OK
+                   : MOE_ERR_CUDA;
     }
     const int grid = (int)std::max<long long>(1, std::min<long long>(di.sms, items));
-    return launch_pdl(ffn_kernel<false>, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess ? MOE_OK
-                                                                                                   : MOE_ERR_CUDA;
+    if (a.fmt == 1)
+        return launch_pdl(ffn_kernel<false, 1>, dim3(grid), dim3(kThreadsQ), smem, st, m, p) == cudaSuccess
+                   ? MOE_OK
+                   : MOE_ERR_CUDA;
+    return launch_pdl(ffn_kernel<false, 0>, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
 }
 
 int device_sm_count() { return device_info().sms; }

@@ -201,6 +201,44 @@ int ffn_args(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_
     return MOE_OK;
 }
 
+// The MXFP8 expert FFN's argument block: the bf16 block with the weight
+// pointers replaced by E4M3 codes and the packed scales added.
+int ffn_args_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                   const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                   const moe_weights_mxfp8_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, FfnArgs *a) {
+    if (!w) return MOE_ERR_INVALID_ARG;
+    const bool sh = cfg->shared_intermediate_size > 0;
+    if (!aligned(w->w_gate) || !aligned(w->w_up) || !aligned(w->w_down) || !aligned(w->w_gate_scale) ||
+        !aligned(w->w_up_scale) || !aligned(w->w_down_scale))
+        return MOE_ERR_INVALID_ARG;
+    if (sh && (!aligned(w->ws_gate) || !aligned(w->ws_up) || !aligned(w->ws_down) || !aligned(w->ws_gate_scale) ||
+               !aligned(w->ws_up_scale) || !aligned(w->ws_down_scale)))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->hidden % 128 != 0 || cfg->moe_intermediate_size % 128 != 0 || cfg->shared_intermediate_size % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;
+    // the bf16 block's checks and fields, with the code pointers standing in for the weights
+    moe_weights_t wb{};
+    wb.w_gate = reinterpret_cast<const moe_bf16_t *>(w->w_gate);
+    wb.w_up = reinterpret_cast<const moe_bf16_t *>(w->w_up);
+    wb.w_down = reinterpret_cast<const moe_bf16_t *>(w->w_down);
+    wb.ws_gate = reinterpret_cast<const moe_bf16_t *>(w->ws_gate);
+    wb.ws_up = reinterpret_cast<const moe_bf16_t *>(w->ws_up);
+    wb.ws_down = reinterpret_cast<const moe_bf16_t *>(w->ws_down);
+    FfnArgs b;
+    int rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, &wb, ybuf, ws, ws_bytes, true, a);
+    if (rc) return rc;
+    rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, &wb, ybuf, ws, ws_bytes, false, &b);
+    if (rc) return rc;
+    a->fmt = 1;
+    a->sf_gate = w->w_gate_scale;
+    a->sf_up = w->w_up_scale;
+    a->sf_down = w->w_down_scale;
+    a->sfs_gate = sh ? w->ws_gate_scale : nullptr;
+    a->sfs_up = sh ? w->ws_up_scale : nullptr;
+    a->sfs_down = sh ? w->ws_down_scale : nullptr;
+    return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -336,6 +374,25 @@ int moe_expert_ffn_noalloc(const moe_config_t *cfg, int32_t T, const moe_bf16_t 
     return MOE_OK;
 }
 
+int moe_mxfp8_pack_scales(int64_t rows, int32_t K, const uint8_t *scales, uint8_t *packed, void *stream) {
+    if (rows < 0 || rows % 64 != 0 || K < 128 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!aligned(scales) || !aligned(packed)) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_mxfp8_pack_scales(rows, K, scales, packed, as_stream(stream)));
+}
+
+int moe_expert_ffn_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                         const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                         const moe_weights_mxfp8_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    FfnArgs a;
+    rc = ffn_args_mxfp8(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, &a);
+    if (rc) return rc;
+    return ffn_launch_both(a, as_stream(stream));
+}
+
 int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, const int32_t *keff, moe_bf16_t *out,
                 void *stream) {
     int rc = check_config(cfg, T);
@@ -375,15 +432,24 @@ int moe_router_logits(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, c
                                       at<float>(ws, L.rpart), at<int32_t>(ws, L.status), as_stream(stream)));
 }
 
-int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits, const moe_weights_t *w,
-                moe_bf16_t *out, const moe_aux_t *aux, void *ws, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The layer around an expert FFN: [router projection] -> route -> [budget]
+// -> dispatch -> ffn(...) -> combine.  `ffn` enqueues the expert FFN of the
+// dispatched batch (bf16 or MXFP8 weights).
+template <class Ffn>
+int forward_impl(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
+                 const moe_bf16_t *w_router, const moe_bf16_t *ws_gate_vec, moe_bf16_t *out, const moe_aux_t *aux,
+                 void *ws, size_t ws_bytes, void *stream, Ffn ffn) {
     int rc = check_config(cfg, T);
     if (rc) return rc;
     if (T == 0) return MOE_OK;
     const bool sh = cfg->shared_intermediate_size > 0;
-    if (!aligned(x) || !aligned_or_null(logits) || !aligned(out) || !aligned(ws) || !w) return MOE_ERR_INVALID_ARG;
-    if (!logits && !aligned(w->w_router)) return MOE_ERR_INVALID_ARG;  // no logits: the projection makes them
-    if (sh && !aligned(w->ws_gate_vec)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x) || !aligned_or_null(logits) || !aligned(out) || !aligned(ws)) return MOE_ERR_INVALID_ARG;
+    if (!logits && !aligned(w_router)) return MOE_ERR_INVALID_ARG;  // no logits: the projection makes them
+    if (sh && !aligned(ws_gate_vec)) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(*cfg, T);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     moe_aux_t a{};
@@ -391,7 +457,7 @@ int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const f
     if (a.logits && !aligned(a.logits)) return MOE_ERR_INVALID_ARG;
     if (!logits) {  // router projection first
         float *lg = a.logits ? a.logits : at<float>(ws, L.logits);
-        rc = moe_router_logits(cfg, T, x, w->w_router, lg, ws, ws_bytes, stream);
+        rc = moe_router_logits(cfg, T, x, w_router, lg, ws, ws_bytes, stream);
         if (rc) return rc;
         logits = lg;
     }
@@ -414,12 +480,12 @@ int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const f
     // launches measured faster for the drafter layers.)
     if (cfg->budget > 0 && front_fits(T, E, k)) {
         rc = cuda_rc(launch_front(T, E, k, cfg->budget, cfg->norm_topk, cfg->topp, cfg->hidden, logits, x,
-                                  sh ? w->ws_gate_vec : nullptr, idx, tw, sgate, keff, kept, ndrop, counts, offsets,
+                                  sh ? ws_gate_vec : nullptr, idx, tw, sgate, keff, kept, ndrop, counts, offsets,
                                   perm, slot_pos, x_perm, at<int32_t>(ws, L.status),
                                   at<int32_t>(ws, L.status + kHdoneOffset), as_stream(stream)));
         if (rc) return rc;
     } else {
-        rc = moe_route(cfg, T, logits, x, sh ? w->ws_gate_vec : nullptr, idx, tw, sgate, keff, stream);
+        rc = moe_route(cfg, T, logits, x, sh ? ws_gate_vec : nullptr, idx, tw, sgate, keff, stream);
         if (rc) return rc;
         if (cfg->budget > 0) {
             rc = moe_budget(cfg, T, idx, tw, keff, kept, ndrop, ws, ws_bytes, stream);
@@ -428,9 +494,42 @@ int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const f
         rc = moe_dispatch(cfg, T, idx, keff, x, counts, offsets, perm, slot_pos, x_perm, ws, ws_bytes, stream);
         if (rc) return rc;
     }
-    rc = moe_expert_ffn(cfg, T, x, x_perm, offsets, perm, tw, sgate, w, ybuf, ws, ws_bytes, stream);
+    rc = ffn(x_perm, offsets, perm, tw, sgate, ybuf);
     if (rc) return rc;
     return moe_combine(cfg, T, ybuf, keff, out, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_forward(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits, const moe_weights_t *w,
+                moe_bf16_t *out, const moe_aux_t *aux, void *ws, size_t ws_bytes, void *stream) {
+    const int rc = check_config(cfg, T);
+    if (rc || T == 0) return rc;
+    if (!w) return MOE_ERR_INVALID_ARG;
+    return forward_impl(cfg, T, x, logits, w->w_router, w->ws_gate_vec, out, aux, ws, ws_bytes, stream,
+                        [&](const moe_bf16_t *x_perm, const int32_t *offsets, const int32_t *perm, const float *tw,
+                            const float *sgate, moe_bf16_t *ybuf) {
+                            return moe_expert_ffn(cfg, T, x, x_perm, offsets, perm, tw, sgate, w, ybuf, ws, ws_bytes,
+                                                  stream);
+                        });
+}
+
+int moe_forward_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
+                      const moe_weights_mxfp8_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
+                      size_t ws_bytes, void *stream) {
+    const int rc = check_config(cfg, T);
+    if (rc || T == 0) return rc;
+    if (!w) return MOE_ERR_INVALID_ARG;
+    if (cfg->hidden % 128 != 0 || cfg->moe_intermediate_size % 128 != 0 || cfg->shared_intermediate_size % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;  // before anything is launched
+    return forward_impl(cfg, T, x, logits, w->w_router, w->ws_gate_vec, out, aux, ws, ws_bytes, stream,
+                        [&](const moe_bf16_t *x_perm, const int32_t *offsets, const int32_t *perm, const float *tw,
+                            const float *sgate, moe_bf16_t *ybuf) {
+                            return moe_expert_ffn_mxfp8(cfg, T, x, x_perm, offsets, perm, tw, sgate, w, ybuf, ws,
+                                                        ws_bytes, stream);
+                        });
 }
 
 int moe_status_read(const void *ws, int32_t *status_out, void *stream) {

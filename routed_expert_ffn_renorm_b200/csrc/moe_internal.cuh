@@ -99,6 +99,9 @@ cudaError_t launch_quantize_mxfp8(long long rows, int K, const uint16_t *w, uint
                                   cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(int nmat, long long rows, int K, const uint16_t *w, uint8_t *codes,
                                   uint8_t *scales, float *tensor_scale, cudaStream_t st);
+// MXFP8 scales [rows, K / 32] -> the FFN's layout [rows / 64][K / 128][64][4]
+// (rows % 64 == 0, K % 128 == 0).
+cudaError_t launch_mxfp8_pack_scales(long long rows, int K, const uint8_t *scales, uint8_t *packed, cudaStream_t st);
 
 // Combine.
 cudaError_t launch_combine(int T, int k, int H, int has_shared, const uint16_t *ybuf,
@@ -111,6 +114,10 @@ struct FfnArgs {
     const int32_t *offsets, *perm;
     const float *topk_w, *sgate;
     const uint16_t *w_gate, *w_up, *w_down, *ws_gate, *ws_up, *ws_down;
+    // fmt 1 (MXFP8 weights): the w_* / ws_* pointers above hold E4M3 codes (one
+    // byte per weight, same shapes) and these the packed UE8M0 scales
+    int fmt;
+    const uint8_t *sf_gate, *sf_up, *sf_down, *sfs_gate, *sfs_up, *sfs_down;
     uint16_t *h_perm, *h_shared, *ybuf;
     int32_t *status;  // the workspace's status block: [0] status word,
                       // [4..5] gate/up (or fused) and [8..9] down work-item counters

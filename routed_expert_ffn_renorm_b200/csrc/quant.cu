@@ -98,7 +98,34 @@ int grid_for(long long work) {
     return (int)(g < 1 ? 1 : (g > cap ? cap : g));
 }
 
+// MXFP8 scales [rows, K / 32] -> [rows / 64][K / 128][64][4]: for every
+// 64-row group and 128-wide K step, the 4 block scales of each of its 64
+// rows in one contiguous 256-byte run, which the expert FFN's producer loads
+// with one bulk copy per ring step.  One thread per 4-byte run.
+__global__ void __launch_bounds__(kQuantThreads) mxfp8_pack_scales_kernel(long long rows, int K,
+                                                                           const uint8_t *__restrict__ in,
+                                                                           uint32_t *__restrict__ out) {
+    const int kb = K / 32, ksteps = K / 128;
+    const long long n = rows * ksteps;  // 4-byte runs
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long o = (long long)blockIdx.x * blockDim.x + threadIdx.x; o < n; o += stride) {
+        const long long rgks = o >> 6;  // (row group, K step)
+        const int r = (int)(o & 63);
+        const long long rg = rgks / ksteps;
+        const int ks = (int)(rgks - rg * ksteps);
+        const uint8_t *src = in + (rg * 64 + r) * kb + ks * 4;
+        out[o] = (uint32_t)src[0] | ((uint32_t)src[1] << 8) | ((uint32_t)src[2] << 16) | ((uint32_t)src[3] << 24);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_mxfp8_pack_scales(long long rows, int K, const uint8_t *scales, uint8_t *packed, cudaStream_t st) {
+    const long long n = rows * (K / 128);
+    mxfp8_pack_scales_kernel<<<grid_for(n), kQuantThreads, 0, st>>>(rows, K, scales,
+                                                                     reinterpret_cast<uint32_t *>(packed));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_mxfp8(long long rows, int K, const uint16_t *w, uint8_t *codes, uint8_t *scales,
                                   cudaStream_t st) {

@@ -85,7 +85,9 @@ class GpuResult:
     out_bits: np.ndarray  # raw bf16 bits, for bit-identity checks
 
 
-def gpu_forward(cfg: W.MoEConfig, inp: W.MoEInputs, ws: Optional[torch.Tensor] = None) -> GpuResult:
+def gpu_forward(cfg: W.MoEConfig, inp: W.MoEInputs, ws: Optional[torch.Tensor] = None, weights=None,
+                fwd=None) -> GpuResult:
+    """moe_forward (or `fwd`, e.g. moe_forward_mxfp8, with `weights`) on the inputs."""
     dev = inp.x.device
     T, k, E = cfg.T, cfg.k, cfg.E
     c = lib_config(cfg)
@@ -106,7 +108,8 @@ def gpu_forward(cfg: W.MoEConfig, inp: W.MoEInputs, ws: Optional[torch.Tensor] =
     if cfg.Is:
         aux["sgate"] = torch.empty(T, dtype=torch.float32, device=dev)
     out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
-    moe.moe_forward(c, inp.x, inp.logits, weights_of(inp), out, ws, aux=aux)
+    (fwd or moe.moe_forward)(c, inp.x, inp.logits, weights if weights is not None else weights_of(inp), out, ws,
+                             aux=aux)
     status = moe.status_read(ws)
     torch.cuda.synchronize()
     h = {n: t.cpu().numpy() for n, t in aux.items()}
@@ -170,10 +173,11 @@ def sample_rows(T: int, n: int, seed: int = 1) -> np.ndarray:
     return np.unique(np.concatenate([[0, T - 1], mid])).astype(np.int32)
 
 
-def _expert_dicts(inp: W.MoEInputs, experts, cache: Optional[dict] = None):
-    """Host copies of the listed experts' weights; `cache` (keyed by expert)
-    keeps them across calls on the same weight tensors."""
-    bits = W.bf16_bits
+def _expert_dicts(inp: W.MoEInputs, experts, cache: Optional[dict] = None, wmap=None):
+    """Host copies of the listed experts' weights (through `wmap`, e.g. the
+    oracle's MXFP8 weights, when given); `cache` (keyed by expert) keeps them
+    across calls on the same weight tensors."""
+    bits = W.bf16_bits if wmap is None else (lambda t: wmap(W.bf16_bits(t)))
     cache = {} if cache is None else cache
     for e in experts:
         if e not in cache:
@@ -183,8 +187,10 @@ def _expert_dicts(inp: W.MoEInputs, experts, cache: Optional[dict] = None):
 
 
 def check_layer(cfg: W.MoEConfig, inp: W.MoEInputs, g: GpuResult, rows=None,
-                nthreads: Optional[int] = None, weight_cache: Optional[dict] = None) -> dict:
-    """Compare a GPU forward with the oracle; returns diagnostics, asserts."""
+                nthreads: Optional[int] = None, weight_cache: Optional[dict] = None, wmap=None) -> dict:
+    """Compare a GPU forward with the oracle; returns diagnostics, asserts.
+    `wmap` maps each expert matrix's bf16 bits to the weights the oracle
+    uses (e.g. oracle.mxfp8_weights for the MXFP8 layer); default: as is."""
     assert g.status == 0, f"device status {g.status}"
     T, k, E = cfg.T, cfg.k, cfg.E
     nthreads = nthreads or oracle.max_threads()
@@ -250,10 +256,11 @@ def check_layer(cfg: W.MoEConfig, inp: W.MoEInputs, g: GpuResult, rows=None,
     elif callable(rows):  # rows chosen from the (now verified) dispatch
         rows = rows(offsets, perm)
     need = sorted({int(idx_b[t, j]) for t in rows for j in range(int(keff_b[t]))})
-    wg, wu, wd = _expert_dicts(inp, need, weight_cache)
+    wg, wu, wd = _expert_dicts(inp, need, weight_cache, wmap)
     kw = {}
     if cfg.Is:
-        kw = dict(ws_gate=W.bf16_bits(inp.ws_gate), ws_up=W.bf16_bits(inp.ws_up), ws_down=W.bf16_bits(inp.ws_down),
+        sb = W.bf16_bits if wmap is None else (lambda t: wmap(W.bf16_bits(t)))
+        kw = dict(ws_gate=sb(inp.ws_gate), ws_up=sb(inp.ws_up), ws_down=sb(inp.ws_down),
                   ws_gvec=W.bf16_bits(inp.ws_gvec))
     ref = oracle.combine_rows(W.bf16_bits(inp.x), idx_b, w_b, keff_b, wg, wu, wd, I=cfg.I, rows=rows,
                               nthreads=nthreads, **kw)

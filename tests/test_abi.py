@@ -113,3 +113,35 @@ def test_quantiser_argument_checks():
     # no rows: nothing to do, whatever the data pointers
     assert lib.moe_quantize_mxfp8(0, 64, None, None, None, None) == 0
     assert lib.moe_quantize_nvfp4(3, 0, 32, None, None, None, FAKE, None) == 0
+
+
+def test_mxfp8_argument_checks():
+    """The MXFP8 entry points reject bad shapes and pointers before any launch."""
+    lib = moe.load_library()
+    P = ctypes.c_void_p
+    # scale repacking: rows a multiple of 64, K of 128, aligned pointers
+    assert lib.moe_mxfp8_pack_scales(63, 256, FAKE, FAKE, None) == -1
+    assert lib.moe_mxfp8_pack_scales(64, 192, FAKE, FAKE, None) == -1
+    assert lib.moe_mxfp8_pack_scales(64, 256, MISALIGNED, FAKE, None) == -1
+    assert lib.moe_mxfp8_pack_scales(0, 256, None, None, None) == 0
+    full = moe._WeightsMXFP8(*([FAKE.value] * 12 + [FAKE.value, FAKE.value]))
+    ws_bytes = lib.moe_workspace_bytes(ctypes.byref(_cfg()), 16)
+    args = (16, FAKE, FAKE, FAKE, FAKE, FAKE, None)
+    # I = 64 is a legal bf16 shape but not an MXFP8 one (128-wide K steps)
+    c = _cfg(moe_intermediate_size=64)
+    assert lib.moe_expert_ffn_mxfp8(ctypes.byref(c), *args, ctypes.byref(full), FAKE, FAKE, 1 << 40, None) == -2
+    assert lib.moe_forward_mxfp8(ctypes.byref(c), 16, FAKE, FAKE, ctypes.byref(full), FAKE, None, FAKE, 1 << 40,
+                                 None) == -2
+    c = _cfg()
+    assert lib.moe_expert_ffn_mxfp8(ctypes.byref(c), *args, None, FAKE, FAKE, ws_bytes, None) == -1
+    bad = moe._WeightsMXFP8(*([FAKE.value] * 3 + [MISALIGNED.value] + [FAKE.value] * 10))
+    assert lib.moe_expert_ffn_mxfp8(ctypes.byref(c), *args, ctypes.byref(bad), FAKE, FAKE, ws_bytes, None) == -1
+    assert lib.moe_expert_ffn_mxfp8(ctypes.byref(c), *args, ctypes.byref(full), FAKE, FAKE, ws_bytes - 1,
+                                    None) == -3
+    # a shared expert needs its codes and scales
+    cs = _cfg(shared_intermediate_size=128)
+    noshared = moe._WeightsMXFP8(*([FAKE.value] * 6 + [None] * 6 + [FAKE.value, FAKE.value]))
+    ws_s = lib.moe_workspace_bytes(ctypes.byref(cs), 16)
+    assert lib.moe_expert_ffn_mxfp8(ctypes.byref(cs), *args[:-1], FAKE, ctypes.byref(noshared), FAKE, FAKE, ws_s,
+                                    None) == -1
+    assert lib.moe_forward_mxfp8(ctypes.byref(c), 0, None, None, ctypes.byref(full), None, None, None, 0, None) == 0
