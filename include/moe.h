@@ -65,6 +65,11 @@ typedef uint16_t moe_bf16_t; /* bf16 bit pattern */
 
 /* Bits of the device status word (see moe_status_read). */
 #define MOE_STATUS_TIMEOUT 1       /* a pipeline wait ran past its limit; results invalid */
+#define MOE_STATUS_BOUNDS 2        /* checked library only (libmoe_checked.so, built with
+                                      MOE_DEBUG_BOUNDS): an input index was out of range --
+                                      an expert id outside [-1, E) in a kept slot, dispatch
+                                      offsets not a prefix sum within T*k, a perm entry outside
+                                      [0, T*k); the access was skipped, results invalid */
 
 typedef struct {
     int32_t hidden;                   /* H */
@@ -279,7 +284,8 @@ int moe_forward_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, c
 
 /* Combine: out[t, :] = bf16( sum_{j < keff[t]} ybuf[t, j, :] + [Is > 0] ybuf[t, k, :] ),
  * summed in fp32 in slot order and rounded once (a token with no kept slot
- * and no shared expert gets 0).  keff == NULL means k.
+ * and no shared expert gets 0).  keff == NULL means k; a keff entry outside
+ * [0, k] counts as the nearest end (a token's own rows are all it reads).
  * ybuf [T, k+1, H]; keff [T]; out [T, H]. */
 int moe_combine(const moe_config_t *cfg, int32_t T, const moe_bf16_t *ybuf, const int32_t *keff,
                 moe_bf16_t *out, void *stream);

@@ -33,6 +33,7 @@ __all__ = [
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libmoe_checked.so")  # built with MOE_DEBUG_BOUNDS
 
 EXPORTED_SYMBOLS = (
     "moe_workspace_bytes", "moe_route", "moe_budget", "moe_dispatch", "moe_expert_ffn", "moe_combine",
@@ -42,6 +43,7 @@ EXPORTED_SYMBOLS = (
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 MOE_STATUS_TIMEOUT = 1
+MOE_STATUS_BOUNDS = 2
 
 
 class MoEError(RuntimeError):
@@ -136,22 +138,30 @@ class MoEWeightsMXFP8:
 
 
 _lib = None
+_checked = None
 _lock = threading.Lock()
 
 
-def load_library(build_if_stale: bool = True):
-    """Load libmoe.so (building it first when missing or older than its sources)."""
-    global _lib
+def load_library(build_if_stale: bool = True, variant: str = "release"):
+    """Load libmoe.so (building it first when missing or older than its
+    sources).  variant="checked" loads libmoe_checked.so instead, the same
+    library built with MOE_DEBUG_BOUNDS (range checks on the caller's index
+    inputs, reported as MOE_STATUS_BOUNDS); the functions below always call
+    the release library unless a test swaps it in."""
+    global _lib, _checked
     with _lock:
-        if _lib is not None:
+        if variant == "release" and _lib is not None:
             return _lib
+        if variant == "checked" and _checked is not None:
+            return _checked
+        path = LIB_PATH if variant == "release" else CHECKED_LIB_PATH
         if build_if_stale:
             from . import _build
-            if _build.stale():
-                _build.build()
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m routed_expert_ffn_renorm_b200._build`")
-        lib = ctypes.CDLL(LIB_PATH)
+            if _build.stale(variant):
+                _build.build(variant=variant)
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m routed_expert_ffn_renorm_b200._build`")
+        lib = ctypes.CDLL(path)
         P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
         cfg = ctypes.POINTER(_Config)
         lib.moe_workspace_bytes.restype = sz
@@ -180,7 +190,10 @@ def load_library(build_if_stale: bool = True):
         for name in EXPORTED_SYMBOLS:
             if name not in ("moe_workspace_bytes", "moe_error_string"):
                 getattr(lib, name).restype = ctypes.c_int
-        _lib = lib
+        if variant == "release":
+            _lib = lib
+        else:
+            _checked = lib
         return lib
 
 

@@ -32,6 +32,14 @@ def _nvcc() -> str:
     return cand
 
 
+# The bounds-checked variant (libmoe_checked.so): the same sources with
+# MOE_DEBUG_BOUNDS, whose kernels range-check the index inputs a caller
+# passes and report MOE_STATUS_BOUNDS instead of touching memory out of range.
+VARIANTS = {"release": (LIB, BUILD_DIR, []),
+            "checked": (os.path.join(HERE, "libmoe_checked.so"), os.path.join(BUILD_DIR, "checked"),
+                        ["-DMOE_DEBUG_BOUNDS"])}
+
+
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -40,24 +48,26 @@ def _deps():
     return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "moe.h"), __file__]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(variant: str = "release") -> bool:
+    lib = VARIANTS[variant][0]
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, variant: str = "release") -> str:
+    lib, build_dir, defs = VARIANTS[variant]
+    if not force and not stale(variant):
+        return lib
     nvcc = _nvcc()
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    os.makedirs(build_dir, exist_ok=True)
     hdr_t = max(os.path.getmtime(p) for p in _deps() if not p.endswith(".cu"))
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr_t):
-            cmd = [nvcc, *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
+            cmd = [nvcc, *ARCH, *NVCC_FLAGS, *defs, "-I", INCLUDE, "-c", src, "-o", obj]
             r = subprocess.run(cmd, capture_output=True, text=True)
             if r.returncode != 0:
                 sys.stderr.write(r.stdout + r.stderr)
@@ -65,16 +75,16 @@ def build(force: bool = False, verbose: bool = False) -> str:
             if verbose:
                 sys.stderr.write(r.stderr)
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-ldl", "-lpthread", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("linking libmoe.so failed")
-    os.replace(tmp, LIB)
-    return LIB
+        raise RuntimeError(f"linking {os.path.basename(lib)} failed")
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    variant = "checked" if "--checked" in sys.argv else "release"
+    print(build(force="--force" in sys.argv, verbose=True, variant=variant))

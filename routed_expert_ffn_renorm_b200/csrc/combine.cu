@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int k, int vec, int
 #pragma unroll
     for (int u = 0; u < 4; ++u) v[u] = u < k ? __ldg(rows + (size_t)u * vec) : make_uint4(0, 0, 0, 0);
     const uint4 vs = has_shared ? __ldg(rows + (size_t)k * vec) : make_uint4(0, 0, 0, 0);
-    const int ke = keff ? __ldg(keff + t) : k;
+    const int ke = keff ? min(max(__ldg(keff + t), 0), k) : k;  // a token's rows only, whatever keff holds
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;

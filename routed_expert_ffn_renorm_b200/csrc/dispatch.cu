@@ -51,7 +51,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums) {
 }
 
 __global__ void __launch_bounds__(256) hist_kernel(int T, int E, int k, const int32_t *__restrict__ idx,
-                                                   const int32_t *__restrict__ keff, int32_t *__restrict__ hist) {
+                                                   const int32_t *__restrict__ keff, int32_t *__restrict__ hist,
+                                                   int32_t *__restrict__ status) {
     __shared__ int h[kMaxExperts];
     pdl_launch_dependents();
     pdl_wait();
@@ -64,6 +65,7 @@ __global__ void __launch_bounds__(256) hist_kernel(int T, int E, int k, const in
         if (j < ke) {
             const int e = idx[s];
             if (e >= 0 && e < E) atomicAdd(&h[e], 1);
+            else if (kDebugBounds && e != -1 && status) atomicOr(status, MOE_STATUS_BOUNDS);
         }
     }
     __syncthreads();
@@ -180,7 +182,9 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(int T, int E, int 
             if (s < s_end) {
                 const int t = s / k, j = s - t * k;
                 const int e = __ldg(idx + s);
-                if (j < (keff ? __ldg(keff + t) : k) && e >= 0 && e < E) key = e;
+                const bool kept = j < (keff ? __ldg(keff + t) : k);
+                if (kept && e >= 0 && e < E) key = e;
+                else if (kDebugBounds && kept && e != -1 && writer && sched) atomicOr(sched, MOE_STATUS_BOUNDS);
             }
             const unsigned peers = __match_any_sync(0xffffffffu, key);
             if (key >= 0 && lane == __ffs(peers) - 1) hist[warp * E + key] += __popc(peers);
@@ -291,7 +295,7 @@ cudaError_t launch_dispatch(int T, int E, int k, const int32_t *idx, const int32
                           perm, slot_pos, status_block, hdone);
     }
     const int nchunks = dispatch_chunks(T);
-    cudaError_t e = launch_pdl(hist_kernel, dim3(nchunks), dim3(256), 0, st, T, E, k, idx, keff, hist);
+    cudaError_t e = launch_pdl(hist_kernel, dim3(nchunks), dim3(256), 0, st, T, E, k, idx, keff, hist, status_block);
     if (e != cudaSuccess) return e;
     e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, E, nchunks, hist, counts, offsets, status_block, hdone);
     if (e != cudaSuccess) return e;

@@ -129,6 +129,12 @@ struct FfnParams {
     // step), row-group major (see moe_mxfp8_pack_scales)
     const uint8_t *sf[2][2];
     const uint8_t *sfs[2][2];
+    // the group-readiness wait's limit (kWaitLimitNs), and a group whose
+    // readiness target is one past what its gate/up items can reach (-1: none)
+    // -- both only changed by the test hooks MOE_TEST_WAIT_LIMIT_US and
+    // MOE_TEST_STALL_GROUP, to make a wait run out on purpose
+    unsigned long long wait_limit_ns;
+    int stall_group;
     const int32_t *offsets;
     const int32_t *perm;
     const float *topk_w;
@@ -470,6 +476,11 @@ __device__ __forceinline__ void down_dest(const Item &it, int n, const FfnParams
         mw = __ldg(p.sgate + t);
     } else {
         const int slot = __ldg(p.perm + it.row0 + n);
+        if (kDebugBounds && (slot < 0 || slot >= p.T * p.k)) {  // skip the token's store
+            atomicOr(p.status, MOE_STATUS_BOUNDS);
+            mrow = -1;
+            return;
+        }
         mrow = slot + slot / p.k;  // t*(k+1) + j
         mw = __ldg(p.topk_w + slot);
     }
@@ -580,6 +591,19 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     // tiles and of down items
     for (int e = threadIdx.x; e <= p.E; e += NT) offs[e] = __ldg(p.offsets + e);
     __syncthreads();
+    if constexpr (kDebugBounds) {
+        // the offsets must be a prefix sum from 0 to at most T*k; otherwise no
+        // routed item runs (every CTA reads the same offsets and decides alike)
+        bool bad = false;
+        for (int e = threadIdx.x; e <= p.E; e += NT)
+            bad |= (e == 0 && offs[0] != 0) || (e < p.E && offs[e] > offs[e + 1]) ||
+                   (e == p.E && offs[e] > p.T * p.k);
+        if (__syncthreads_or(bad)) {
+            if (threadIdx.x == 0) atomicOr(p.status, MOE_STATUS_BOUNDS);
+            for (int e = threadIdx.x; e <= p.E; e += NT) offs[e] = 0;
+            __syncthreads();
+        }
+    }
     Schedule sc;
     sc.shared_ntt = p.Is > 0 ? (p.T + p.BNs - 1) / p.BNs : 0;
     {
@@ -656,15 +680,16 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 }
                 if (item < 0) break;
                 const int grp = it.shared ? p.E : it.e;
-                if (fused && it.ph == 1 && !all_ready && !((ready_bits[grp >> 5] >> (grp & 31)) & 1u)) {
+                const bool stalled = grp == p.stall_group;
+                if (fused && it.ph == 1 && (!all_ready || stalled) && !((ready_bits[grp >> 5] >> (grp & 31)) & 1u)) {
                     // wait until every gate/up tile of the group has stored its h rows
                     // (or every gate/up item of the launch is done)
                     const int32_t *flag = p.hdone + grp;
-                    const int target = (it.shared ? p.Rs[0] : p.R[0]) * it.ntt;
+                    const int target = (it.shared ? p.Rs[0] : p.R[0]) * it.ntt + (stalled ? 1 : 0);
                     auto check = [&]() {
                         const int all = ld_acquire(p.hdone + p.E + 1), mine = ld_acquire(flag);
-                        if (all >= sc.n[0]) all_ready = true;
-                        return all_ready || mine >= target;
+                        if (!stalled && all >= sc.n[0]) all_ready = true;
+                        return (all_ready && !stalled) || mine >= target;
                     };
                     bool ready = check();
                     const unsigned long long t0 = ready ? 0ull : globaltimer();
@@ -672,7 +697,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                         ready = check();
                         if (!ready && (spin & 63u) == 0) {
                             if (*abort_flag) break;
-                            if (globaltimer() - t0 > kWaitLimitNs) {
+                            if (globaltimer() - t0 > p.wait_limit_ns) {
                                 *abort_flag = 1;
                                 atomicOr(p.status, MOE_STATUS_TIMEOUT);
                                 break;
@@ -976,7 +1001,8 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                         for (int i = 0; i < 32; ++i) {
                             const int rr = __shfl_sync(0xffffffffu, mrow, i);
                             const float ww = __shfl_sync(0xffffffffu, mw, i);
-                            if (c0 + i < it.nvalid) out[(size_t)rr * p.H] = f32_to_bf16_bits(v[i] * ww);
+                            if (c0 + i < it.nvalid && (!kDebugBounds || rr >= 0))
+                                out[(size_t)rr * p.H] = f32_to_bf16_bits(v[i] * ww);
                         }
                     }
                 }
@@ -1111,6 +1137,29 @@ int choose_tiles(const FfnArgs &a, int sms, int *bn, int *bns, int *pages) {
     return *pages >= min_pages(a.fmt) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
+// Test hooks (failure-path tests only): MOE_TEST_WAIT_LIMIT_US in [1, 4e6]
+// shortens the fused launch's group-readiness wait, MOE_TEST_STALL_GROUP in
+// [0, E] (E: the shared expert) gives that group's down items a readiness
+// target its gate/up items never reach, so their wait runs out and the
+// launch ends with MOE_STATUS_TIMEOUT after the limit.  Unset: 4 s, none.
+int test_hooks(const FfnArgs &a, unsigned long long *limit_ns, int *stall) {
+    *limit_ns = kWaitLimitNs;
+    *stall = -1;
+    if (const char *f = getenv("MOE_TEST_WAIT_LIMIT_US")) {
+        char *end = nullptr;
+        const long long v = strtoll(f, &end, 10);
+        if (*f == 0 || *end != 0 || v < 1 || v > 4000000) return MOE_ERR_INVALID_ARG;
+        *limit_ns = (unsigned long long)v * 1000ull;
+    }
+    if (const char *f = getenv("MOE_TEST_STALL_GROUP")) {
+        char *end = nullptr;
+        const long v = strtol(f, &end, 10);
+        if (*f == 0 || *end != 0 || v < 0 || v > a.E) return MOE_ERR_INVALID_ARG;
+        *stall = (int)v;
+    }
+    return MOE_OK;
+}
+
 }  // namespace
 
 // CTA pairs (cta_group::2) for a single-phase launch whose groups fill wide
@@ -1159,6 +1208,7 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     if (a.fmt && (a.H % 128 != 0 || a.I % 128 != 0 || a.Is % 128 != 0)) return MOE_ERR_UNSUPPORTED;
     FfnParams p{};
     if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
+    if (int rc = test_hooks(a, &p.wait_limit_ns, &p.stall_group)) return rc;
     bool pair = false;
     if (int rc = choose_pair(a, phases, di.sms, &pair)) return rc;
     const int BN = p.BN;

@@ -22,6 +22,17 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
     return *reinterpret_cast<uint16_t *>(&b);
 }
 
+// Bounds-checked build (-DMOE_DEBUG_BOUNDS, libmoe_checked.so): index inputs
+// that come from the caller are range-checked where they are used; a bad one
+// sets MOE_STATUS_BOUNDS in the status word and the access is skipped (no
+// trap).  kDebugBounds is false in the release build, so the checks compile
+// away there.
+#ifdef MOE_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+
 // Programmatic dependent launch: every kernel of the layer lets the next one
 // launch as soon as all of its CTAs are running, and waits for its own
 // predecessor (grid completion and memory flush) before it reads anything
