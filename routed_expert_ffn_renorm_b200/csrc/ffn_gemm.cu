@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     // MXFP8: two conversion buffers (bf16 A operands of a ring step) ahead of the ring
     uint8_t *cbuf = smem;
     uint8_t *ring = smem + (kFmt ? kCbufBytes : 0);
-    float *xchg = reinterpret_cast<float *>(smem + (size_t)P * kPageBytes);
+    float *xchg = reinterpret_cast<float *>(ring + (size_t)P * kPageBytes);  // after the ring, whichever format
     int *tile_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
     int *dbase = tile_base + (p.E + 1);                                 // [E + 1]
     int *offs = dbase + (p.E + 1);                                      // [E + 1]
