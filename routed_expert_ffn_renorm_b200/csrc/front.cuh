@@ -49,7 +49,9 @@ __device__ __forceinline__ int route_token_impl(int t, int E, int k, int norm_to
     const float *l = logits + (size_t)t * E;
     // expert of slot i of this lane
     auto expert = [&](int i) { return kVec ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i; };
-    float v[V];
+    // only the keys stay live: a logit comes back from its key exactly (up to
+    // the sign of a zero, which neither the max nor exp sees), so the V
+    // logits need no registers of their own
     uint32_t key[V];
     if constexpr (kVec) {
 #pragma unroll
@@ -57,20 +59,19 @@ __device__ __forceinline__ int route_token_impl(int t, int E, int k, int norm_to
             const int e0 = 128 * c + 4 * lane;  // E % 4 == 0: all four present or none
             float4 q = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
             if (e0 < E) q = kGlobal ? __ldg(reinterpret_cast<const float4 *>(l + e0)) : *reinterpret_cast<const float4 *>(l + e0);
-            v[4 * c] = q.x;
-            v[4 * c + 1] = q.y;
-            v[4 * c + 2] = q.z;
-            v[4 * c + 3] = q.w;
+            const bool in = e0 < E;
+            key[4 * c] = in ? float_order_key(q.x) : 0u;
+            key[4 * c + 1] = in ? float_order_key(q.y) : 0u;
+            key[4 * c + 2] = in ? float_order_key(q.z) : 0u;
+            key[4 * c + 3] = in ? float_order_key(q.w) : 0u;
         }
     } else {
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int e = expert(i);
-            v[i] = e < E ? (kGlobal ? __ldg(l + e) : l[e]) : -INFINITY;
+            key[i] = e < E ? float_order_key(kGlobal ? __ldg(l + e) : l[e]) : 0u;
         }
     }
-#pragma unroll
-    for (int i = 0; i < V; ++i) key[i] = expert(i) < E ? float_order_key(v[i]) : 0u;
     // softmax denominator: the largest logit, then sum of exp(l - max) over all E
     uint32_t km = key[0];
 #pragma unroll
@@ -79,7 +80,7 @@ __device__ __forceinline__ int route_token_impl(int t, int E, int k, int norm_to
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < V; ++i)
-        if (expert(i) < E) s += expf(v[i] - m);
+        if (expert(i) < E) s += expf(order_key_float(key[i]) - m);
 #pragma unroll
     for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
 

@@ -17,8 +17,10 @@ namespace {
 
 constexpr int kRouteThreads = 32 + kGateThreads;  // one token per block: warp 0 routes, warps 1.. dot
 
+// V >= 16 wants more registers than the default occupancy target leaves
+// (that build spilled); the narrower routers keep a high block occupancy.
 template <int V>  // logits per lane: V * 32 >= E
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(int T, int E, int k, int norm_topk, float topp,
+__global__ void __launch_bounds__(kRouteThreads, V >= 16 ? 1 : 8) route_kernel(int T, int E, int k, int norm_topk, float topp,
                                                               const float *__restrict__ logits,
                                                               int32_t *__restrict__ idx, float *__restrict__ w,
                                                               int32_t *__restrict__ keff,
