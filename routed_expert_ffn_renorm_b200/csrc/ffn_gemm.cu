@@ -87,7 +87,7 @@ constexpr int kNumBox = 5;                     // token box heights 16 << i
 constexpr int kThreads = 192;                  // bf16 weights: producer, MMA, 4 epilogue warps
 // Block-scaled (MXFP8) weights: converter warps after the epilogue warps turn
 // each ring step's FP8 codes into the bf16 A operand in shared memory.
-constexpr int kConvWarps = 4;
+constexpr int kConvWarps = 8;  // two per SM sub-partition, so one hides the other's shared-memory latency
 constexpr int kThreadsQ = kThreads + 32 * kConvWarps;
 constexpr int kQKStep = 128;                   // K elements per FP8 ring step (one 128-byte code box row)
 constexpr int kQCodePages = kTileM * kQKStep / 2048;  // 8 pages: 128 rows x 128 codes
@@ -439,20 +439,28 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &q, uint32_t sc, uin
 // 16-byte bank groups on every load and store.
 template <int kNt>
 __device__ __forceinline__ void convert_mxfp8_tile(uint32_t codes, uint32_t scales, uint32_t dst, int ct) {
-#pragma unroll 4
-    for (int i = 0; i < 1024 / kNt; ++i) {
+    constexpr int N = 1024 / kNt;  // units per thread
+    // every load first, so that a thread has all its N loads in flight at once
+    uint4 q[N];
+    uint32_t sc[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int u = ct + i * kNt;
+        const int r = ((u >> 6) << 3) | (u & 7);
+        const int c = (u >> 3) & 7;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(q[i].x), "=r"(q[i].y), "=r"(q[i].z), "=r"(q[i].w)
+                     : "r"(codes + (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4))));
+        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sc[i]) : "r"(scales + (uint32_t)(r * 4 + (c >> 1))));
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
         const int u = ct + i * kNt;
         const int r = ((u >> 6) << 3) | (u & 7);
         const int c = (u >> 3) & 7;
         const int sw = r & 7;
-        uint4 q;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
-                     : "r"(codes + (uint32_t)(r * 128 + ((c ^ sw) << 4))));
-        uint32_t sc;
-        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sc) : "r"(scales + (uint32_t)(r * 4 + (c >> 1))));
         uint4 o0, o1;
-        e4m3x16_to_bf16(q, sc, o0, o1);
+        e4m3x16_to_bf16(q[i], sc[i], o0, o1);
         const uint32_t row = dst + (uint32_t)((c >> 2) * kABytes + r * 128);
         const int cc = (c & 3) << 1;  // first of the two bf16 chunks in the slice
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)((cc ^ sw) << 4)), "r"(o0.x),
