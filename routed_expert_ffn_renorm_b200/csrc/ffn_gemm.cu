@@ -135,6 +135,7 @@ struct FfnParams {
     // MOE_TEST_STALL_GROUP, to make a wait run out on purpose
     unsigned long long wait_limit_ns;
     int stall_group;
+    int prefetch;  // 1: L2-prefetch the next item's first K step near the end of each item
     const int32_t *offsets;
     const int32_t *perm;
     const float *topk_w;
@@ -402,72 +403,85 @@ __device__ __forceinline__ uint32_t e4m3x2_lanes(uint32_t w, uint32_t sel) {
     return (prmt_b32(w, 0u, sel) << 4) & 0x87F087F0u;
 }
 
-// 16 codes (one 16-byte chunk) and their scale code -> 16 bf16 (two chunks).
-__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &q, uint32_t sc, uint4 &o0, uint4 &o1) {
-    uint32_t m1, m2 = 0;
-    const bool one = sc <= 134u;  // 2^(120 + se) is a normal bf16: one multiply
-    if (one) {
-        m1 = (sc + 120u) << 7;
-    } else {  // 2^127 first, then 2^(se - 7)
-        m1 = 254u << 7;
-        m2 = (sc - 7u) << 7;
-        m2 |= m2 << 16;
-    }
-    m1 |= m1 << 16;
+// 16 codes (one 16-byte chunk) -> 16 bf16 (two chunks): each pair of codes
+// as two bf16 lanes, times the bf16x2 multiplier m.
+__device__ __forceinline__ void e4m3x16_times(const uint4 &q, uint32_t m, uint32_t (&r)[8]) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    uint32_t r[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        r[2 * i] = bf16x2_mul(e4m3x2_lanes(w[i], 0x9180u), m1);      // codes 4i, 4i + 1
-        r[2 * i + 1] = bf16x2_mul(e4m3x2_lanes(w[i], 0xB3A2u), m1);  // codes 4i + 2, 4i + 3
+        r[2 * i] = bf16x2_mul(e4m3x2_lanes(w[i], 0x9180u), m);      // codes 4i, 4i + 1
+        r[2 * i + 1] = bf16x2_mul(e4m3x2_lanes(w[i], 0xB3A2u), m);  // codes 4i + 2, 4i + 3
     }
-    if (!one) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) r[i] = bf16x2_mul(r[i], m2);
-    }
-    o0 = make_uint4(r[0], r[1], r[2], r[3]);
-    o1 = make_uint4(r[4], r[5], r[6], r[7]);
 }
+// bf16x2 of 2^(120 + se) from the UE8M0 code sc = se + 127, sc <= 134: the
+// exponent field sc + 120 in both halves, one multiply-add.
+__device__ __forceinline__ uint32_t mx_mult(uint32_t sc) { return sc * 0x00800080u + 120u * 0x00800080u; }
+
+// A converter thread's units of a ring step: unit u = ct + i * kNt is row
+// (u / 64) * 8 + u % 8, chunk c = (u / 8) % 8; the 8 lanes of a shared-memory
+// phase share a chunk over 8 consecutive rows and, swizzled, hit 8 distinct
+// 16-byte bank groups on every load and store.  Their byte offsets do not
+// change from step to step and are computed once.
+template <int kNt>
+struct ConvUnits {
+    static constexpr int N = 1024 / kNt;
+    uint32_t src[N];  // code chunk in the code box: r * 128 + ((c ^ (r & 7)) << 4)
+    uint32_t sc[N];   // scale byte: r * 4 + c / 2
+    uint32_t dst[N];  // first bf16 chunk in the conversion buffer; the second is dst ^ 16
+    __device__ __forceinline__ explicit ConvUnits(int ct) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const int u = ct + i * kNt;
+            const int r = ((u >> 6) << 3) | (u & 7), c = (u >> 3) & 7, sw = r & 7;
+            src[i] = (uint32_t)(r * 128 + ((c ^ sw) << 4));
+            sc[i] = (uint32_t)(r * 4 + (c >> 1));
+            // slice c / 4, bf16 chunks 2 (c % 4) and 2 (c % 4) + 1 of row r
+            dst[i] = (uint32_t)((c >> 2) * kABytes + r * 128 + (((2 * (c & 3)) ^ sw) << 4));
+        }
+    }
+};
 
 // One ring step's weight tile: 128 rows x 128 E4M3 codes, as TMA left them
 // (row r at r * 128 bytes, 16-byte chunk c at (c ^ (r & 7)) * 16: the 128-byte
 // swizzle), with their scales (row r's four at byte 4r), into two K-major bf16
 // slices of 64 in the same swizzle (slice s at dst + s * 16 KB), the MMA's A
-// operand.  Thread ct of nt takes units u = ct, ct + nt, ...; unit u is row
-// (u / 64) * 8 + u % 8, chunk (u / 8) % 8, so the 8 lanes of a shared-memory
-// phase share a chunk over 8 consecutive rows and, swizzled, hit 8 distinct
-// 16-byte bank groups on every load and store.
+// operand.  Every load is issued before the first conversion, so a thread has
+// all of them in flight at once.  A block scale above 2^7 needs two
+// multiplies; a warp takes that path only when one of its blocks needs it.
 template <int kNt>
-__device__ __forceinline__ void convert_mxfp8_tile(uint32_t codes, uint32_t scales, uint32_t dst, int ct) {
-    constexpr int N = 1024 / kNt;  // units per thread
-    // every load first, so that a thread has all its N loads in flight at once
+__device__ __forceinline__ void convert_mxfp8_tile(uint32_t codes, uint32_t scales, uint32_t dst,
+                                                   const ConvUnits<kNt> &cu) {
+    constexpr int N = ConvUnits<kNt>::N;
     uint4 q[N];
     uint32_t sc[N];
 #pragma unroll
     for (int i = 0; i < N; ++i) {
-        const int u = ct + i * kNt;
-        const int r = ((u >> 6) << 3) | (u & 7);
-        const int c = (u >> 3) & 7;
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(q[i].x), "=r"(q[i].y), "=r"(q[i].z), "=r"(q[i].w)
-                     : "r"(codes + (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4))));
-        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sc[i]) : "r"(scales + (uint32_t)(r * 4 + (c >> 1))));
+                     : "r"(codes + cu.src[i]));
+        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sc[i]) : "r"(scales + cu.sc[i]));
     }
+    bool small = true;
+#pragma unroll
+    for (int i = 0; i < N; ++i) small &= sc[i] <= 134u;
+    const bool fast = __all_sync(0xffffffffu, small);
 #pragma unroll
     for (int i = 0; i < N; ++i) {
-        const int u = ct + i * kNt;
-        const int r = ((u >> 6) << 3) | (u & 7);
-        const int c = (u >> 3) & 7;
-        const int sw = r & 7;
-        uint4 o0, o1;
-        e4m3x16_to_bf16(q[i], sc[i], o0, o1);
-        const uint32_t row = dst + (uint32_t)((c >> 2) * kABytes + r * 128);
-        const int cc = (c & 3) << 1;  // first of the two bf16 chunks in the slice
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)((cc ^ sw) << 4)), "r"(o0.x),
-                     "r"(o0.y), "r"(o0.z), "r"(o0.w)
+        uint32_t r[8];
+        if (fast) {
+            e4m3x16_times(q[i], mx_mult(sc[i]), r);
+        } else {  // 2^(120 + se) as 2^127 (or 2^(120 + se) itself) times 2^(se - 7) (or 1)
+            const bool one = sc[i] <= 134u;
+            uint32_t m1 = one ? (sc[i] + 120u) << 7 : 254u << 7, m2 = one ? 127u << 7 : (sc[i] - 7u) << 7;
+            e4m3x16_times(q[i], m1 | (m1 << 16), r);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) r[j] = bf16x2_mul(r[j], m2 | (m2 << 16));
+        }
+        const uint32_t d = dst + cu.dst[i];
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
                      : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (uint32_t)(((cc + 1) ^ sw) << 4)),
-                     "r"(o1.x), "r"(o1.y), "r"(o1.z), "r"(o1.w)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d ^ 16u), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                     "r"(r[7])
                      : "memory");
     }
 }
@@ -799,6 +813,32 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                         }
                     }
                     ++issued;
+                    // Four steps before the item's end, the next item's first step goes to
+                    // L2 (its weights, and for gate/up its token rows): a new item starts
+                    // in new DRAM pages and translations, whose first load otherwise
+                    // lands well after the previous item's last one (about 2 us on the
+                    // 16-expert layer).  h rows of a down item may not be written yet and
+                    // are left out.
+                    if (p.prefetch && k0 == max(sh.ns, sh.nk - 4 * sh.ns) / sh.ns * sh.ns && pending < total_items) {
+                        const Item nx = decode_item(pending, sc, p);
+                        const PhaseMaps &pn = maps.ph[nx.ph];
+                        const int nrt = kPair ? 2 * nx.r + (int)rank : nx.r;
+                        const int nrow = nx.ph == 0 ? (nx.shared ? 0 : nx.e * p.I) + nrt * 64
+                                                    : (nx.shared ? 0 : nx.e * p.H) + nrt * kTileM;
+                        const StepShape nsh = kFmt ? qstep_shape(nx, p) : step_shape<kPair>(nx, p);
+                        const int nslices = kFmt ? 2 : min(nsh.ns, nsh.nk);
+                        for (int j = 0; j < nslices; ++j) {
+                            const int kx = kFmt ? 0 : j * kBlockK;  // an FP8 code box spans both slices
+                            if (kFmt && j > 0) break;
+                            tma_prefetch_2d(nx.shared ? &pn.s0 : &pn.a0, kx, nrow);
+                            if (nx.ph == 0) tma_prefetch_2d(nx.shared ? &pn.s1 : &pn.a1, kx, nrow);
+                        }
+                        if (nx.ph == 0) {
+                            const int nb = nx.row0 + (kPair ? (int)rank * pair_half(nx.nvalid) : 0);
+                            const CUtensorMap *nmb = nx.shared ? &pn.bs[nsh.bi] : &pn.b[nsh.bi];
+                            for (int j = 0; j < min(2, nsh.nk); ++j) tma_prefetch_2d(nmb, j * kBlockK, nb);
+                        }
+                    }
                 }
                 if (!ok) break;
             }
@@ -911,6 +951,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
         // so every converter thread reaches the same named barriers.
         const int ct = threadIdx.x - kThreads;  // 0 .. 32 * kConvWarps - 1
         const bool elected = ct == 0;
+        const ConvUnits<32 * kConvWarps> cu(ct);
         uint32_t vhead = 0, off = 0, step = 0;
         for (int li = 0;; ++li) {
             const int slot = li % kQueue;
@@ -937,7 +978,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const uint32_t codes = smem_u32(ring + (size_t)first * kPageBytes);
                 convert_mxfp8_tile<32 * kConvWarps>(codes, codes + kQCodePages * kPageBytes,
-                                                    smem_u32(cbuf + cb * 2 * kABytes), ct);
+                                                    smem_u32(cbuf + cb * 2 * kABytes), cu);
                 fence_proxy_async_shared();  // the stores, visible to the tensor cores' reads
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cfull[cb]);
@@ -1217,6 +1258,11 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     FfnParams p{};
     if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
     if (int rc = test_hooks(a, &p.wait_limit_ns, &p.stall_group)) return rc;
+    p.prefetch = 1;
+    if (const char *f = getenv("MOE_FORCE_PREFETCH")) {  // benchmark override: 0 / 1
+        if ((f[0] != '0' && f[0] != '1') || f[1] != 0) return MOE_ERR_INVALID_ARG;
+        p.prefetch = f[0] == '1';
+    }
     bool pair = false;
     if (int rc = choose_pair(a, phases, di.sms, &pair)) return rc;
     const int BN = p.BN;
