@@ -135,7 +135,6 @@ struct FfnParams {
     // MOE_TEST_STALL_GROUP, to make a wait run out on purpose
     unsigned long long wait_limit_ns;
     int stall_group;
-    int prefetch;  // 1: L2-prefetch the next item's first K step near the end of each item
     const int32_t *offsets;
     const int32_t *perm;
     const float *topk_w;
@@ -813,32 +812,6 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                         }
                     }
                     ++issued;
-                    // Four steps before the item's end, the next item's first step goes to
-                    // L2 (its weights, and for gate/up its token rows): a new item starts
-                    // in new DRAM pages and translations, whose first load otherwise
-                    // lands well after the previous item's last one (about 2 us on the
-                    // 16-expert layer).  h rows of a down item may not be written yet and
-                    // are left out.
-                    if (p.prefetch && k0 == max(sh.ns, sh.nk - 4 * sh.ns) / sh.ns * sh.ns && pending < total_items) {
-                        const Item nx = decode_item(pending, sc, p);
-                        const PhaseMaps &pn = maps.ph[nx.ph];
-                        const int nrt = kPair ? 2 * nx.r + (int)rank : nx.r;
-                        const int nrow = nx.ph == 0 ? (nx.shared ? 0 : nx.e * p.I) + nrt * 64
-                                                    : (nx.shared ? 0 : nx.e * p.H) + nrt * kTileM;
-                        const StepShape nsh = kFmt ? qstep_shape(nx, p) : step_shape<kPair>(nx, p);
-                        const int nslices = kFmt ? 2 : min(nsh.ns, nsh.nk);
-                        for (int j = 0; j < nslices; ++j) {
-                            const int kx = kFmt ? 0 : j * kBlockK;  // an FP8 code box spans both slices
-                            if (kFmt && j > 0) break;
-                            tma_prefetch_2d(nx.shared ? &pn.s0 : &pn.a0, kx, nrow);
-                            if (nx.ph == 0) tma_prefetch_2d(nx.shared ? &pn.s1 : &pn.a1, kx, nrow);
-                        }
-                        if (nx.ph == 0) {
-                            const int nb = nx.row0 + (kPair ? (int)rank * pair_half(nx.nvalid) : 0);
-                            const CUtensorMap *nmb = nx.shared ? &pn.bs[nsh.bi] : &pn.b[nsh.bi];
-                            for (int j = 0; j < min(2, nsh.nk); ++j) tma_prefetch_2d(nmb, j * kBlockK, nb);
-                        }
-                    }
                 }
                 if (!ok) break;
             }
@@ -1258,11 +1231,6 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     FfnParams p{};
     if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
     if (int rc = test_hooks(a, &p.wait_limit_ns, &p.stall_group)) return rc;
-    p.prefetch = 1;
-    if (const char *f = getenv("MOE_FORCE_PREFETCH")) {  // benchmark override: 0 / 1
-        if ((f[0] != '0' && f[0] != '1') || f[1] != 0) return MOE_ERR_INVALID_ARG;
-        p.prefetch = f[0] == '1';
-    }
     bool pair = false;
     if (int rc = choose_pair(a, phases, di.sms, &pair)) return rc;
     const int BN = p.BN;
