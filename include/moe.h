@@ -282,6 +282,46 @@ int moe_forward_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, c
                       const moe_weights_mxfp8_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
                       size_t ws_bytes, void *stream);
 
+/* ---------------------------------------------------------------------
+ * Expert parallelism: the E experts split over W ranks (one GPU each), rank
+ * r holding experts [r * epr, (r + 1) * epr), epr = E / W -- the layout of
+ * the multi-rank MegaMoE of DeepGEMM PR #381 ("B200 performance", EP8) and
+ * DeepGEMM fork PR #5, whose dispatch sends each token's routed rows to the
+ * ranks holding its experts and whose combine brings the weighted expert
+ * outputs back.  The exchange is the caller's collective (NCCL all-to-all);
+ * these three calls are the per-rank steps around it (see the package's
+ * ep.py for the whole layer):
+ *   1. moe_route, then moe_ep_rank_ids, then moe_dispatch with W "experts"
+ *      on the rank ids: slots grouped by destination rank (perm, counts) and
+ *      the rows to send (x_perm, in that order);
+ *   2. moe_ep_pack: for each row to send, the expert id local to its rank
+ *      and the routing weight;
+ *   3. (exchange; at the destination moe_dispatch + moe_expert_ffn with k = 1
+ *      on the received rows and their local ids and weights, moe_combine to
+ *      make the weighted outputs contiguous; exchange back)
+ *   4. moe_ep_unpack: the returned rows, in send order, to the token-ordered
+ *      ybuf rows; the shared expert on the home rank; moe_combine.
+ * --------------------------------------------------------------------- */
+
+/* rank_idx[s] = topk_idx[s] / experts_per_rank for s < T*k (-1 stays -1).
+ * topk_idx, rank_idx [T, k] i32 (device). */
+int moe_ep_rank_ids(int32_t T, int32_t k, int32_t experts_per_rank, const int32_t *topk_idx, int32_t *rank_idx,
+                    void *stream);
+
+/* For p < *n_sent (device int: the dispatch's offsets[W]), with s = perm[p]:
+ * local_idx[p] = topk_idx[s] % experts_per_rank, local_w[p] = topk_w[s].
+ * n_max >= *n_sent bounds the launch (T*k).  perm from moe_dispatch on the
+ * rank ids; local_idx, local_w [n_max] (device). */
+int moe_ep_pack(int32_t n_max, const int32_t *n_sent, int32_t experts_per_rank, const int32_t *perm,
+                const int32_t *topk_idx, const float *topk_w, int32_t *local_idx, float *local_w, void *stream);
+
+/* ybuf[s + s / k, :] = rows[p, :] for p < *n_returned (device int), s =
+ * perm[p]: the weighted expert outputs, returned in send order, to the
+ * token-ordered rows moe_combine adds.  rows [n_max, H]; ybuf [T, k+1, H];
+ * n_max <= T*k. */
+int moe_ep_unpack(const moe_config_t *cfg, int32_t T, int32_t n_max, const int32_t *n_returned, const int32_t *perm,
+                  const moe_bf16_t *rows, moe_bf16_t *ybuf, void *stream);
+
 /* Combine: out[t, :] = bf16( sum_{j < keff[t]} ybuf[t, j, :] + [Is > 0] ybuf[t, k, :] ),
  * summed in fp32 in slot order and rounded once (a token with no kept slot
  * and no shared expert gets 0).  keff == NULL means k; a keff entry outside

@@ -27,6 +27,7 @@ __all__ = [
     "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn_noalloc",
     "moe_combine", "moe_forward", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
     "MoEWeightsMXFP8", "moe_mxfp8_pack_scales", "moe_expert_ffn_mxfp8", "moe_forward_mxfp8", "pack_mxfp8",
+    "moe_ep_rank_ids", "moe_ep_pack", "moe_ep_unpack",
     "status_read", "status_clear",
     "EXPORTED_SYMBOLS", "MOE_STATUS_TIMEOUT",
 ]
@@ -40,6 +41,7 @@ EXPORTED_SYMBOLS = (
     "moe_forward", "moe_status_read", "moe_status_clear", "moe_error_string", "moe_expert_gate_up",
     "moe_expert_down", "moe_expert_ffn_noalloc", "moe_router_logits", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
     "moe_mxfp8_pack_scales", "moe_expert_ffn_mxfp8", "moe_forward_mxfp8",
+    "moe_ep_rank_ids", "moe_ep_pack", "moe_ep_unpack",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 MOE_STATUS_TIMEOUT = 1
@@ -182,6 +184,9 @@ def load_library(build_if_stale: bool = True, variant: str = "release"):
         lib.moe_quantize_mxfp8.argtypes = [i64, i32, P, P, P, P]
         lib.moe_quantize_nvfp4.argtypes = [i32, i64, i32, P, P, P, P, P]
         lib.moe_mxfp8_pack_scales.argtypes = [i64, i32, P, P, P]
+        lib.moe_ep_rank_ids.argtypes = [i32, i32, i32, P, P, P]
+        lib.moe_ep_pack.argtypes = [i32, P, i32, P, P, P, P, P, P]
+        lib.moe_ep_unpack.argtypes = [cfg, i32, i32, P, P, P, P, P]
         lib.moe_expert_ffn_mxfp8.argtypes = [cfg, i32, P, P, P, P, P, P, ctypes.POINTER(_WeightsMXFP8), P, P, sz, P]
         lib.moe_forward_mxfp8.argtypes = [cfg, i32, P, P, ctypes.POINTER(_WeightsMXFP8), P, ctypes.POINTER(_Aux), P,
                                           sz, P]
@@ -329,6 +334,28 @@ def moe_forward_mxfp8(cfg: MoEConfig, x, logits, weights: MoEWeightsMXFP8, out, 
     _check("moe_forward_mxfp8", load_library().moe_forward_mxfp8(
         ctypes.byref(cfg._c()), T, _ptr(x), _ptr(logits, True), ctypes.byref(w), _ptr(out), ctypes.byref(a),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_ep_rank_ids(topk_idx, rank_idx, experts_per_rank: int, stream=None):
+    """rank_idx = topk_idx // experts_per_rank (-1 stays -1): the rank holding each slot's expert."""
+    T, k = topk_idx.shape
+    _check("moe_ep_rank_ids", load_library().moe_ep_rank_ids(T, k, experts_per_rank, _ptr(topk_idx), _ptr(rank_idx),
+                                                             _stream(stream)))
+
+
+def moe_ep_pack(n_sent, perm, topk_idx, topk_w, local_idx, local_w, experts_per_rank: int, stream=None):
+    """For the first n_sent[0] (device) entries p of perm: local_idx[p] =
+    topk_idx[perm[p]] % experts_per_rank, local_w[p] = topk_w[perm[p]]."""
+    _check("moe_ep_pack", load_library().moe_ep_pack(
+        local_idx.numel(), _ptr(n_sent), experts_per_rank, _ptr(perm), _ptr(topk_idx), _ptr(topk_w), _ptr(local_idx),
+        _ptr(local_w), _stream(stream)))
+
+
+def moe_ep_unpack(cfg: MoEConfig, T: int, n_returned, perm, rows, ybuf, stream=None):
+    """ybuf[s + s // k] = rows[p] for p < n_returned[0] (device), s = perm[p]."""
+    _check("moe_ep_unpack", load_library().moe_ep_unpack(
+        ctypes.byref(cfg._c()), T, rows.shape[0], _ptr(n_returned), _ptr(perm), _ptr(rows), _ptr(ybuf),
+        _stream(stream)))
 
 
 def moe_route(cfg: MoEConfig, logits, topk_idx, topk_w, *, x=None, ws_gate_vec=None, sgate=None, keff=None,

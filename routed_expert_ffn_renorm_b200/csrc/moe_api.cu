@@ -374,6 +374,36 @@ int moe_expert_ffn_noalloc(const moe_config_t *cfg, int32_t T, const moe_bf16_t 
     return MOE_OK;
 }
 
+int moe_ep_rank_ids(int32_t T, int32_t k, int32_t experts_per_rank, const int32_t *topk_idx, int32_t *rank_idx,
+                    void *stream) {
+    if (T < 0 || k < 1 || experts_per_rank < 1) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!aligned(topk_idx) || !aligned(rank_idx)) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_ep_rank_ids(T * k, experts_per_rank, topk_idx, rank_idx, as_stream(stream)));
+}
+
+int moe_ep_pack(int32_t n_max, const int32_t *n_sent, int32_t experts_per_rank, const int32_t *perm,
+                const int32_t *topk_idx, const float *topk_w, int32_t *local_idx, float *local_w, void *stream) {
+    if (n_max < 0 || experts_per_rank < 1) return MOE_ERR_INVALID_ARG;
+    if (n_max == 0) return MOE_OK;
+    if (!n_sent || !aligned(perm) || !aligned(topk_idx) || !aligned(topk_w) || !aligned(local_idx) ||
+        !aligned(local_w))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_ep_pack(n_max, n_sent, experts_per_rank, perm, topk_idx, topk_w, local_idx, local_w,
+                                  as_stream(stream)));
+}
+
+int moe_ep_unpack(const moe_config_t *cfg, int32_t T, int32_t n_max, const int32_t *n_returned, const int32_t *perm,
+                  const moe_bf16_t *rows, moe_bf16_t *ybuf, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (n_max < 0 || n_max > T * cfg->num_experts_per_tok) return MOE_ERR_INVALID_ARG;
+    if (T == 0 || n_max == 0) return MOE_OK;
+    if (!n_returned || !aligned(perm) || !aligned(rows) || !aligned(ybuf)) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_ep_unpack(n_max, n_returned, cfg->num_experts_per_tok, cfg->hidden, perm, rows, ybuf,
+                                    as_stream(stream)));
+}
+
 int moe_mxfp8_pack_scales(int64_t rows, int32_t K, const uint8_t *scales, uint8_t *packed, void *stream) {
     if (rows < 0 || rows % 64 != 0 || K < 128 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
     if (rows == 0) return MOE_OK;

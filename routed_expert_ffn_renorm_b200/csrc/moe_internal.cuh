@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -113,6 +115,15 @@ cudaError_t launch_quantize_nvfp4(int nmat, long long rows, int K, const uint16_
 // MXFP8 scales [rows, K / 32] -> the FFN's layout [rows / 64][K / 128][64][4]
 // (rows % 64 == 0, K % 128 == 0).
 cudaError_t launch_mxfp8_pack_scales(long long rows, int K, const uint8_t *scales, uint8_t *packed, cudaStream_t st);
+
+// Expert parallelism (ep.cu): destination ranks of slots, the send metadata
+// in send order, and the returned rows back to token order.  n_dev: the
+// number of sent (returned) rows, on the device (the dispatch's offsets[W]).
+cudaError_t launch_ep_rank_ids(int n, int epr, const int32_t *idx, int32_t *rank_idx, cudaStream_t st);
+cudaError_t launch_ep_pack(int n_max, const int32_t *n_dev, int epr, const int32_t *perm, const int32_t *idx,
+                           const float *w, int32_t *local_idx, float *local_w, cudaStream_t st);
+cudaError_t launch_ep_unpack(int n_max, const int32_t *n_dev, int k, int H, const int32_t *perm, const uint16_t *rows,
+                             uint16_t *ybuf, cudaStream_t st);
 
 // Combine.
 cudaError_t launch_combine(int T, int k, int H, int has_shared, const uint16_t *ybuf,
