@@ -86,13 +86,18 @@ constexpr int kABytes = kTileM * kBlockK * 2;  // 16 KB
 constexpr int kNumBox = 5;                     // token box heights 16 << i
 constexpr int kThreads = 192;                  // bf16 weights: producer, MMA, 4 epilogue warps
 // Block-scaled (MXFP8) weights: converter warps after the epilogue warps turn
-// each ring step's FP8 codes into the bf16 A operand in shared memory.
+// each ring step's FP8 codes into the bf16 A operand in tensor memory.
 constexpr int kConvWarps = 8;  // two per SM sub-partition, so one hides the other's shared-memory latency
 constexpr int kThreadsQ = kThreads + 32 * kConvWarps;
 constexpr int kQKStep = 128;                   // K elements per FP8 ring step (one 128-byte code box row)
 constexpr int kQCodePages = kTileM * kQKStep / 2048;  // 8 pages: 128 rows x 128 codes
 constexpr int kQScaleBytes = 512;              // 128 rows x 4 UE8M0 scales (blocks of 32) per step
-constexpr int kCbufBytes = 2 * 2 * kABytes;    // two conversion buffers, each two bf16 K slices of 64
+// MXFP8: a step's converted A operand (two bf16 K slices of 64: 64 TMEM
+// columns) goes to one of kConvBufs buffers after the accumulators (from
+// column kConvCol0 on; the token tile is at most 128 wide then).
+constexpr int kConvBufs = 4;
+constexpr int kConvCols = 64;
+constexpr int kConvCol0 = 256;
 constexpr int kPageBytes = 2048;               // ring unit: 16 token rows of 128 B
 constexpr int kAPages = kABytes / kPageBytes;  // 8 pages of weights per K step
 constexpr int kMaxStepPages = kAPages + 256 * 128 / kPageBytes;  // 24: weights + 256 token rows
@@ -416,72 +421,48 @@ __device__ __forceinline__ void e4m3x16_times(const uint4 &q, uint32_t m, uint32
 // exponent field sc + 120 in both halves, one multiply-add.
 __device__ __forceinline__ uint32_t mx_mult(uint32_t sc) { return sc * 0x00800080u + 120u * 0x00800080u; }
 
-// A converter thread's units of a ring step: unit u = ct + i * kNt is row
-// (u / 64) * 8 + u % 8, chunk c = (u / 8) % 8; the 8 lanes of a shared-memory
-// phase share a chunk over 8 consecutive rows and, swizzled, hit 8 distinct
-// 16-byte bank groups on every load and store.  Their byte offsets do not
-// change from step to step and are computed once.
-template <int kNt>
-struct ConvUnits {
-    static constexpr int N = 1024 / kNt;
-    uint32_t src[N];  // code chunk in the code box: r * 128 + ((c ^ (r & 7)) << 4)
-    uint32_t sc[N];   // scale byte: r * 4 + c / 2
-    uint32_t dst[N];  // first bf16 chunk in the conversion buffer; the second is dst ^ 16
-    __device__ __forceinline__ explicit ConvUnits(int ct) {
+// One converter thread's share of a ring step.  The step's weight tile is 128
+// rows x 128 E4M3 codes as TMA left them (row r at r * 128 bytes, 16-byte chunk
+// c at (c ^ (r & 7)) * 16: the 128-byte swizzle) with row r's four UE8M0 scales
+// at byte 4r.  The thread turns row r into 128 bf16, two consecutive K per
+// 32-bit column (the lower K in the low half), and stores them to 64 columns of
+// TMEM lane r: the MMA's A operand.  The 8 lanes of a shared-memory phase read
+// one chunk index of 8 consecutive rows, which the swizzle puts in 8 distinct
+// 16-byte bank groups.  A block scale above 2^7 needs two multiplies; a warp
+// takes that path only when one of its blocks needs it.
+__device__ __forceinline__ void convert_mxfp8_row(uint32_t codes, uint32_t scales, int r, uint32_t taddr) {
+    uint4 q[8];
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-            const int u = ct + i * kNt;
-            const int r = ((u >> 6) << 3) | (u & 7), c = (u >> 3) & 7, sw = r & 7;
-            src[i] = (uint32_t)(r * 128 + ((c ^ sw) << 4));
-            sc[i] = (uint32_t)(r * 4 + (c >> 1));
-            // slice c / 4, bf16 chunks 2 (c % 4) and 2 (c % 4) + 1 of row r
-            dst[i] = (uint32_t)((c >> 2) * kABytes + r * 128 + (((2 * (c & 3)) ^ sw) << 4));
-        }
-    }
-};
-
-// One ring step's weight tile: 128 rows x 128 E4M3 codes, as TMA left them
-// (row r at r * 128 bytes, 16-byte chunk c at (c ^ (r & 7)) * 16: the 128-byte
-// swizzle), with their scales (row r's four at byte 4r), into two K-major bf16
-// slices of 64 in the same swizzle (slice s at dst + s * 16 KB), the MMA's A
-// operand.  Every load is issued before the first conversion, so a thread has
-// all of them in flight at once.  A block scale above 2^7 needs two
-// multiplies; a warp takes that path only when one of its blocks needs it.
-template <int kNt>
-__device__ __forceinline__ void convert_mxfp8_tile(uint32_t codes, uint32_t scales, uint32_t dst,
-                                                   const ConvUnits<kNt> &cu) {
-    constexpr int N = ConvUnits<kNt>::N;
-    uint4 q[N];
-    uint32_t sc[N];
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
+    for (int j = 0; j < 8; ++j)
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(q[i].x), "=r"(q[i].y), "=r"(q[i].z), "=r"(q[i].w)
-                     : "r"(codes + cu.src[i]));
-        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sc[i]) : "r"(scales + cu.sc[i]));
-    }
-    bool small = true;
+                     : "=r"(q[j].x), "=r"(q[j].y), "=r"(q[j].z), "=r"(q[j].w)
+                     : "r"(codes + (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4))));
+    uint32_t s4;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(s4) : "r"(scales + (uint32_t)(r * 4)));
+    uint32_t sc[4];
 #pragma unroll
-    for (int i = 0; i < N; ++i) small &= sc[i] <= 134u;
-    const bool fast = __all_sync(0xffffffffu, small);
+    for (int b = 0; b < 4; ++b) sc[b] = (s4 >> (8 * b)) & 0xffu;
+    const bool fast = __all_sync(0xffffffffu, sc[0] <= 134u && sc[1] <= 134u && sc[2] <= 134u && sc[3] <= 134u);
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-        uint32_t r[8];
-        if (fast) {
-            e4m3x16_times(q[i], mx_mult(sc[i]), r);
-        } else {  // 2^(120 + se) as 2^127 (or 2^(120 + se) itself) times 2^(se - 7) (or 1)
-            const bool one = sc[i] <= 134u;
-            uint32_t m1 = one ? (sc[i] + 120u) << 7 : 254u << 7, m2 = one ? 127u << 7 : (sc[i] - 7u) << 7;
-            e4m3x16_times(q[i], m1 | (m1 << 16), r);
+    for (int h = 0; h < 2; ++h) {
+        uint32_t o[32];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) r[j] = bf16x2_mul(r[j], m2 | (m2 << 16));
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t c = sc[2 * h + (j >> 1)];
+            uint32_t t[8];
+            if (fast) {
+                e4m3x16_times(q[4 * h + j], mx_mult(c), t);
+            } else {  // 2^(120 + se) as 2^127 (or 2^(120 + se) itself) times 2^(se - 7) (or 1)
+                const bool one = c <= 134u;
+                const uint32_t m1 = one ? (c + 120u) << 7 : 254u << 7, m2 = one ? 127u << 7 : (c - 7u) << 7;
+                e4m3x16_times(q[4 * h + j], m1 | (m1 << 16), t);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t[i] = bf16x2_mul(t[i], m2 | (m2 << 16));
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[8 * j + i] = t[i];
         }
-        const uint32_t d = dst + cu.dst[i];
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d ^ 16u), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-                     "r"(r[7])
-                     : "memory");
+        tmem_st32(taddr + (uint32_t)(32 * h), o);
     }
 }
 
@@ -519,10 +500,8 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t P = (uint32_t)p.pages;
-    // MXFP8: two conversion buffers (bf16 A operands of a ring step) ahead of the ring
-    uint8_t *cbuf = smem;
-    uint8_t *ring = smem + (kFmt ? kCbufBytes : 0);
-    float *xchg = reinterpret_cast<float *>(ring + (size_t)P * kPageBytes);  // after the ring, whichever format
+    uint8_t *ring = smem;
+    float *xchg = reinterpret_cast<float *>(ring + (size_t)P * kPageBytes);
     int *tile_base = reinterpret_cast<int *>(xchg + 64 * kXchgStride);  // [E + 1]
     int *dbase = tile_base + (p.E + 1);                                 // [E + 1]
     int *offs = dbase + (p.E + 1);                                      // [E + 1]
@@ -531,20 +510,21 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     uint64_t *full = bars, *empty = bars + kTickets, *tfull = bars + 2 * kTickets, *tempty = tfull + 2;
     uint64_t *mma_done = tfull + 4;
     uint64_t *qfull = tfull + 5, *qempty = qfull + kQueue;
-    uint64_t *cfull = qempty + kQueue, *cempty = cfull + 2;  // MXFP8: conversion buffer converted / free
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cempty + 2);
+    // MXFP8: conversion buffer (in TMEM) converted / free
+    uint64_t *cfull = qempty + kQueue, *cempty = cfull + kConvBufs;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cempty + kConvBufs);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // elected -> epilogue: 0 go, -1 stop
     ItemSlot *qdesc = reinterpret_cast<ItemSlot *>(tmem_slot + 4);  // [kQueue], written by the producer
     ItemSlot *epi_desc = qdesc + kQueue;                             // the epilogue's current item
-    ItemSlot *conv_desc = epi_desc + 1;                              // the converters' current item
+    ItemSlot *conv_desc = epi_desc + 1;                              // [2] each converter group's current item
     int *scan_tmp = reinterpret_cast<int *>(                          // [2 * NT] (int2 partials)
-        (reinterpret_cast<uintptr_t>(conv_desc + 1) + 7) & ~uintptr_t(7));
+        (reinterpret_cast<uintptr_t>(conv_desc + 2) + 7) & ~uintptr_t(7));
     uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + 2 * NT);  // [kReadyWords], producer-private
     uint32_t *ticket_start = ready_bits + kReadyWords;  // [kTickets] first ring page (virtual) of each step; producer-private
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tmem_cols = 2 * p.BN;
+    const int tmem_cols = kFmt ? 512 : 2 * p.BN;  // MXFP8: accumulators, then the conversion buffers
     const uint32_t rank = kPair ? cluster_ctarank() : 0u;  // 0: the pair's MMA issuer
     pdl_launch_dependents();
 
@@ -562,11 +542,11 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
         for (int q = 0; q < kQueue; ++q) {
             mbar_init(&qfull[q], 1);
             // the MMA lane and the elected epilogue thread (pair: and the other CTA's
-            // producer and epilogue; MXFP8: and the elected converter thread)
-            mbar_init(&qempty[q], kPair ? 4 : (kFmt ? 3 : 2));
+            // producer and epilogue; MXFP8: and the two converter groups' elected threads)
+            mbar_init(&qempty[q], kPair ? 4 : (kFmt ? 4 : 2));
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&cfull[b], kConvWarps);  // one arrival per converter warp
+        for (int b = 0; b < kConvBufs; ++b) {
+            mbar_init(&cfull[b], kConvWarps / 2);  // one arrival per warp of the converting group
             mbar_init(&cempty[b], 1);          // the MMA lane's commit
         }
         *abort_flag = 0;
@@ -830,7 +810,6 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
         if (lane == 0 && (!kPair || rank == 0)) {  // a pair's MMAs are issued by CTA 0
             uint32_t vhead = 0, off = 0, step = 0;  // the producer's page sequence, replayed
             const uint64_t desc0 = sw128_desc(smem_u32(ring));  // ring page 0; other pages by addition
-            const uint64_t cdesc0 = sw128_desc(smem_u32(cbuf));  // MXFP8: conversion buffer 0
             for (int li = 0;; ++li) {
                 const int slot = li % kQueue;
                 if (!mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) break;
@@ -856,22 +835,23 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                         break;
                     }
                     if constexpr (kFmt != 0) {
-                        // the converted weights of this step (conversion buffer step & 1), and
-                        // the token boxes in the ring
-                        const uint32_t cb = step & 1u;
-                        if (!mbar_wait_fast(&cfull[cb], (step >> 1) & 1u, abort_flag, p.status, true)) {
+                        // the converted weights of this step (TMEM buffer step % kConvBufs, A read
+                        // from tensor memory: 8 columns per K 16), and the token boxes in the ring
+                        const uint32_t cb = step % kConvBufs;
+                        if (!mbar_wait_fast(&cfull[cb], (step / kConvBufs) & 1u, abort_flag, p.status, true)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint64_t db = desc0 + (first + kQCodePages + 1) * (kPageBytes / 16);
+                        const uint32_t ta = tmem_base + (uint32_t)(kConvCol0 + cb * kConvCols);
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            const uint64_t da = cdesc0 + (cb * 2 + j) * (kABytes / 16);
                             const uint64_t dbj = db + j * sh.sub_pages * (kPageBytes / 16);
 #pragma unroll
                             for (int kk = 0; kk < kBlockK / 16; ++kk)
-                                umma_bf16(d, da + 2 * kk, dbj + 2 * kk, idesc, (k0 | j | kk) != 0);
+                                umma_bf16_ts(d, ta + (uint32_t)(j * 32 + kk * 8), dbj + 2 * kk, idesc,
+                                             (k0 | j | kk) != 0);
                         }
                         umma_commit(&empty[tk]);  // the ring pages (codes, scales, tokens)
                         umma_commit(&cempty[cb]);  // the conversion buffer
@@ -915,47 +895,58 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
         }
     } else if (kFmt != 0 && warp >= 6) {
         // ================= MXFP8 converters (warps 6 ..) =================
-        // Walk the producer's step sequence: once a step's codes and scales have
-        // landed and the MMAs of the step two back have released conversion buffer
-        // step & 1, write that step's bf16 weights there and hand it to the MMA lane.
-        // Every converter thread takes the same waits and a warp leaves a step loop
-        // only as a whole (a vote after the waits); a failed wait sets the abort
-        // flag, and the elected thread then publishes "stop" at the next queue read,
-        // so every converter thread reaches the same named barriers.
+        // Two groups of kConvWarps / 2 warps take alternate steps, so that one
+        // group's conversion overlaps the other's loads and TMEM stores.  Each
+        // group walks the producer's step sequence: once one of its steps' codes
+        // and scales have landed and the MMAs of the step kConvBufs back have
+        // released TMEM buffer step % kConvBufs, it writes that step's bf16
+        // weights there and hands it to the MMA lane.  Thread lane of warp w
+        // converts row 32 (w % 4) + lane: a warp reaches only its own quarter of
+        // the TMEM lanes, and a group's warps cover the four quarters.
+        // Every thread of a group takes the same waits and a warp leaves a step
+        // loop only as a whole (a vote after the waits); a failed wait sets the
+        // abort flag, and the group's elected thread then publishes "stop" at the
+        // next queue read, so every thread of the group reaches the same named
+        // barriers.
         const int ct = threadIdx.x - kThreads;  // 0 .. 32 * kConvWarps - 1
-        const bool elected = ct == 0;
-        const ConvUnits<32 * kConvWarps> cu(ct);
+        const uint32_t g = (uint32_t)(ct / (16 * kConvWarps));  // group: steps with step % 2 == g
+        const bool elected = ct % (16 * kConvWarps) == 0;
+        ItemSlot *desc = conv_desc + g;
+        const int cq = warp & 3, crow = 32 * cq + lane;
+        const uint32_t tlane = tmem_base + ((uint32_t)(32 * cq) << 16) + (uint32_t)kConvCol0;
         uint32_t vhead = 0, off = 0, step = 0;
         for (int li = 0;; ++li) {
             const int slot = li % kQueue;
             if (elected) {
                 if (!*abort_flag && mbar_wait(&qfull[slot], (uint32_t)(li / kQueue) & 1u, abort_flag, p.status, true)) {
-                    *conv_desc = qdesc[slot];
+                    *desc = qdesc[slot];
                     mbar_arrive(&qempty[slot]);
                 } else {
-                    conv_desc->item = -2;
+                    desc->item = -2;
                 }
             }
-            named_bar_sync(2, 32 * kConvWarps);
-            const int item = conv_desc->item;
-            const Item it = conv_desc->it;
-            named_bar_sync(2, 32 * kConvWarps);  // read by all before the elected thread's next write
+            named_bar_sync(2 + g, 16 * kConvWarps);
+            const int item = desc->item;
+            const Item it = desc->it;
+            named_bar_sync(2 + g, 16 * kConvWarps);  // read by all before the elected thread's next write
             if (item < 0) break;
             const StepShape sh = qstep_shape(it, p);
             const uint32_t need = qstep_pages(sh);
-            for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
+            bool ok = true;
+            for (int k0 = 0; k0 < sh.nk; k0 += sh.ns, ++step) {
                 const uint32_t first = ring_alloc(vhead, off, need, P);
-                const uint32_t tk = step % kTickets, cb = step & 1u;
-                const bool ok = mbar_wait_fast(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true) &&
-                                mbar_wait_fast(&cempty[cb], ((step >> 1) & 1u) ^ 1u, abort_flag, p.status, true);
+                if ((step & 1u) != g) continue;  // the other group's step
+                const uint32_t tk = step % kTickets, cb = step % kConvBufs;
+                ok = mbar_wait_fast(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true) &&
+                     mbar_wait_fast(&cempty[cb], ((step / kConvBufs) & 1u) ^ 1u, abort_flag, p.status, true);
                 if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after();
                 const uint32_t codes = smem_u32(ring + (size_t)first * kPageBytes);
-                convert_mxfp8_tile<32 * kConvWarps>(codes, codes + kQCodePages * kPageBytes,
-                                                    smem_u32(cbuf + cb * 2 * kABytes), cu);
-                fence_proxy_async_shared();  // the stores, visible to the tensor cores' reads
+                convert_mxfp8_row(codes, codes + kQCodePages * kPageBytes, crow, tlane + cb * kConvCols);
+                tmem_wait_st();  // this thread's stores done, before the arrival
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cfull[cb]);
-                ++step;
             }
         }
     } else {
@@ -1098,9 +1089,9 @@ int pick_bns(const FfnArgs &a, int bn, int sms) {
 
 size_t smem_bytes_for(int E, int pages, int fmt) {
     const int nt = fmt ? kThreadsQ : kThreads;
-    return 1024 + (fmt ? (size_t)kCbufBytes : 0) + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 +
-           3 * (size_t)(E + 1) * 4 + 8 + (size_t)(2 * kTickets + 5 + 2 * kQueue + 4) * 8 + 16 +
-           (kQueue + 2) * sizeof(ItemSlot) + 8 + 2 * (size_t)nt * 4 + kReadyWords * 4 + kTickets * 4;
+    return 1024 + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 +
+           3 * (size_t)(E + 1) * 4 + 8 + (size_t)(2 * kTickets + 5 + 2 * kQueue + 2 * kConvBufs) * 8 + 16 +
+           (kQueue + 3) * sizeof(ItemSlot) + 8 + 2 * (size_t)nt * 4 + kReadyWords * 4 + kTickets * 4;
 }
 
 int min_pages(int fmt) { return fmt ? kQMaxStepPages : kMaxStepPages; }
@@ -1230,6 +1221,7 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     if (a.fmt && (a.H % 128 != 0 || a.I % 128 != 0 || a.Is % 128 != 0)) return MOE_ERR_UNSUPPORTED;
     FfnParams p{};
     if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
+    if (a.fmt && 2 * p.BN > kConvCol0) return MOE_ERR_UNSUPPORTED;  // MXFP8: accumulators end where the A buffers start
     if (int rc = test_hooks(a, &p.wait_limit_ns, &p.stall_group)) return rc;
     bool pair = false;
     if (int rc = choose_pair(a, phases, di.sms, &pair)) return rc;
