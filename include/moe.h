@@ -236,7 +236,7 @@ int moe_expert_ffn_noalloc(const moe_config_t *cfg, int32_t T, const moe_bf16_t 
  * reduction axis), the FP8 expert weights that DeepGEMM fork PR #5 "big M
  * opt: splitT1 + L2 scatter + 2 stream" names against its W8A8 reference.
  * Weights only: activations stay bf16.  Each weight tile is turned into bf16
- * in shared memory on its way to the tensor cores; every E4M3 code times its
+ * in tensor memory on its way to the tensor cores; every E4M3 code times its
  * block's power of two is a bf16 value (for scales 2^-117 .. 2^119), so the
  * layer computes exactly what moe_expert_ffn computes on the dequantised
  * weights, while half the weight bytes cross HBM.
@@ -280,6 +280,66 @@ int moe_expert_ffn_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x
  * combine as moe_forward, the expert FFN as moe_expert_ffn_mxfp8. */
 int moe_forward_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
                       const moe_weights_mxfp8_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
+                      size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------
+ * The expert FFN with NVFP4 expert weights (E2M1 codes, an E4M3 scale per 16
+ * consecutive weights along the reduction axis, an fp32 scale per matrix):
+ * the FP4 expert weights of DeepGEMM fork PR #5 "big M opt: splitT1 + L2
+ * scatter + 2 stream" (megamoe_nvfp4) and of DeepGEMM PR #381's B200 FP8 x
+ * FP4 policy, here with bf16 activations.  Each weight tile is turned into
+ * bf16 in tensor memory on its way to the tensor cores: an E2M1 code times
+ * its E4M3 block scale is always a bf16 value, so the MMAs see exactly the
+ * weights the format stands for, and the matrix scale multiplies each
+ * projection's fp32 output (gate and up before the SwiGLU, down before the
+ * gate weight).  A quarter of the bf16 weight bytes cross HBM.
+ *   Codes: moe_quantize_nvfp4 of each weight array (nmat = E for the routed
+ *   experts, 1 for each shared matrix), [rows, K / 2] bytes per matrix.
+ *   Scales: moe_quantize_nvfp4's [rows, K / 16] block scales repacked once
+ *   by moe_nvfp4_pack_scales (below) -- rows is E * I for w_gate / w_up and
+ *   E * H for w_down, K the matrix's reduction size.
+ *   Matrix scales: moe_quantize_nvfp4's tensor_scale output.
+ * Limits on top of the general ones: H, I and Is multiples of 128.
+ * --------------------------------------------------------------------- */
+typedef struct {
+    const uint8_t *w_gate;          /* [E, I, H / 2] E2M1 codes, two per byte (lower K in the low nibble) */
+    const uint8_t *w_up;            /* [E, I, H / 2] */
+    const uint8_t *w_down;          /* [E, H, I / 2] */
+    const uint8_t *w_gate_scale;    /* packed E4M3 block scales of w_gate (E * I rows, K = H) */
+    const uint8_t *w_up_scale;      /* packed block scales of w_up */
+    const uint8_t *w_down_scale;    /* packed block scales of w_down (E * H rows, K = I) */
+    const float *w_gate_tscale;     /* [E] fp32 matrix scales of w_gate (4-byte aligned) */
+    const float *w_up_tscale;       /* [E] of w_up */
+    const float *w_down_tscale;     /* [E] of w_down */
+    const uint8_t *ws_gate;         /* [Is, H / 2] shared-expert codes, NULL if Is = 0 */
+    const uint8_t *ws_up;           /* [Is, H / 2], NULL if Is = 0 */
+    const uint8_t *ws_down;         /* [H, Is / 2], NULL if Is = 0 */
+    const uint8_t *ws_gate_scale;   /* packed block scales of ws_gate (Is rows, K = H), NULL if Is = 0 */
+    const uint8_t *ws_up_scale;     /* packed block scales of ws_up, NULL if Is = 0 */
+    const uint8_t *ws_down_scale;   /* packed block scales of ws_down (H rows, K = Is), NULL if Is = 0 */
+    const float *ws_tscale;         /* [3] fp32 matrix scales of ws_gate, ws_up, ws_down; NULL if Is = 0 */
+    const moe_bf16_t *ws_gate_vec;  /* [H] bf16 shared-expert gate vector, NULL if Is = 0 */
+    const moe_bf16_t *w_router;     /* [E, H] bf16 router projection (moe_forward_nvfp4 without logits) */
+} moe_weights_nvfp4_t;
+
+/* Repack NVFP4 block scales [rows, K / 16] (as moe_quantize_nvfp4 writes
+ * them) into the layout the FFN reads: [rows / 64][K / 128][64][8] -- for
+ * every group of 64 rows and every 128 weights along K, the group's 64 x 8
+ * scales as one 512-byte run.  rows % 64 == 0, K % 128 == 0; both pointers
+ * device, 16-byte aligned; same byte count in and out.  Run once per weight
+ * load. */
+int moe_nvfp4_pack_scales(int64_t rows, int32_t K, const uint8_t *scales, uint8_t *packed, void *stream);
+
+/* moe_expert_ffn with NVFP4 expert weights; arguments and results as
+ * moe_expert_ffn (the same workspace size). */
+int moe_expert_ffn_nvfp4(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                         const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                         const moe_weights_nvfp4_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, void *stream);
+
+/* moe_forward with NVFP4 expert weights: routing, budget, dispatch and
+ * combine as moe_forward, the expert FFN as moe_expert_ffn_nvfp4. */
+int moe_forward_nvfp4(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
+                      const moe_weights_nvfp4_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
                       size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------
@@ -362,9 +422,9 @@ const char *moe_error_string(int code);
  * the largest magnitude, so in NVFP4 it spoils its whole matrix's scale);
  * the quantisers do not check for them.  The blocks
  * run along the last (reduction) axis of a row-major matrix: rows of
- * W_gate / W_up [I, H] and of W_down [H, I].  The layer consumes MXFP8
- * (moe_expert_ffn_mxfp8 / moe_forward_mxfp8 above); NVFP4 is the pack step
- * only.
+ * W_gate / W_up [I, H] and of W_down [H, I].  The layer consumes both
+ * (moe_expert_ffn_mxfp8 / moe_forward_mxfp8, moe_expert_ffn_nvfp4 /
+ * moe_forward_nvfp4 above).
  * --------------------------------------------------------------------- */
 
 /* MXFP8: blocks of 32 consecutive elements share a UE8M0 scale

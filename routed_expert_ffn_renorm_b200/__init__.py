@@ -27,6 +27,7 @@ __all__ = [
     "moe_dispatch", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_expert_ffn_noalloc",
     "moe_combine", "moe_forward", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
     "MoEWeightsMXFP8", "moe_mxfp8_pack_scales", "moe_expert_ffn_mxfp8", "moe_forward_mxfp8", "pack_mxfp8",
+    "MoEWeightsNVFP4", "moe_nvfp4_pack_scales", "moe_expert_ffn_nvfp4", "moe_forward_nvfp4", "pack_nvfp4",
     "moe_ep_rank_ids", "moe_ep_pack", "moe_ep_unpack",
     "status_read", "status_clear",
     "EXPORTED_SYMBOLS", "MOE_STATUS_TIMEOUT",
@@ -41,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "moe_forward", "moe_status_read", "moe_status_clear", "moe_error_string", "moe_expert_gate_up",
     "moe_expert_down", "moe_expert_ffn_noalloc", "moe_router_logits", "moe_quantize_mxfp8", "moe_quantize_nvfp4",
     "moe_mxfp8_pack_scales", "moe_expert_ffn_mxfp8", "moe_forward_mxfp8",
+    "moe_nvfp4_pack_scales", "moe_expert_ffn_nvfp4", "moe_forward_nvfp4",
     "moe_ep_rank_ids", "moe_ep_pack", "moe_ep_unpack",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
@@ -69,6 +71,13 @@ class _WeightsMXFP8(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "w_gate", "w_up", "w_down", "w_gate_scale", "w_up_scale", "w_down_scale", "ws_gate", "ws_up", "ws_down",
         "ws_gate_scale", "ws_up_scale", "ws_down_scale", "ws_gate_vec", "w_router")]
+
+
+class _WeightsNVFP4(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_gate", "w_up", "w_down", "w_gate_scale", "w_up_scale", "w_down_scale", "w_gate_tscale", "w_up_tscale",
+        "w_down_tscale", "ws_gate", "ws_up", "ws_down", "ws_gate_scale", "ws_up_scale", "ws_down_scale",
+        "ws_tscale", "ws_gate_vec", "w_router")]
 
 
 class _Aux(ctypes.Structure):
@@ -139,6 +148,38 @@ class MoEWeightsMXFP8:
         return _WeightsMXFP8(*(_ptr(getattr(self, n), allow_none=True) for n, _ in _WeightsMXFP8._fields_))
 
 
+@dataclass
+class MoEWeightsNVFP4:
+    """Device NVFP4 expert weights: E2M1 codes (uint8, two per byte, the
+    lower K in the low nibble) -- w_gate, w_up [E, I, H // 2], w_down
+    [E, H, I // 2], optional shared ws_gate, ws_up [Is, H // 2], ws_down
+    [H, Is // 2] -- each matrix's E4M3 block scales in the FFN's packed
+    layout (moe_nvfp4_pack_scales), and the fp32 matrix scales: w_*_tscale
+    [E] and ws_tscale [3] (shared gate, up, down).  ws_gate_vec [H] and
+    w_router [E, H] stay bf16.  pack_nvfp4() builds one from MoEWeights."""
+    w_gate: "torch.Tensor"
+    w_up: "torch.Tensor"
+    w_down: "torch.Tensor"
+    w_gate_scale: "torch.Tensor"
+    w_up_scale: "torch.Tensor"
+    w_down_scale: "torch.Tensor"
+    w_gate_tscale: "torch.Tensor"
+    w_up_tscale: "torch.Tensor"
+    w_down_tscale: "torch.Tensor"
+    ws_gate: Optional["torch.Tensor"] = None
+    ws_up: Optional["torch.Tensor"] = None
+    ws_down: Optional["torch.Tensor"] = None
+    ws_gate_scale: Optional["torch.Tensor"] = None
+    ws_up_scale: Optional["torch.Tensor"] = None
+    ws_down_scale: Optional["torch.Tensor"] = None
+    ws_tscale: Optional["torch.Tensor"] = None
+    ws_gate_vec: Optional["torch.Tensor"] = None
+    w_router: Optional["torch.Tensor"] = None
+
+    def _c(self) -> _WeightsNVFP4:
+        return _WeightsNVFP4(*(_ptr(getattr(self, n), allow_none=True) for n, _ in _WeightsNVFP4._fields_))
+
+
 _lib = None
 _checked = None
 _lock = threading.Lock()
@@ -189,6 +230,10 @@ def load_library(build_if_stale: bool = True, variant: str = "release"):
         lib.moe_ep_unpack.argtypes = [cfg, i32, i32, P, P, P, P, P]
         lib.moe_expert_ffn_mxfp8.argtypes = [cfg, i32, P, P, P, P, P, P, ctypes.POINTER(_WeightsMXFP8), P, P, sz, P]
         lib.moe_forward_mxfp8.argtypes = [cfg, i32, P, P, ctypes.POINTER(_WeightsMXFP8), P, ctypes.POINTER(_Aux), P,
+                                          sz, P]
+        lib.moe_nvfp4_pack_scales.argtypes = [i64, i32, P, P, P]
+        lib.moe_expert_ffn_nvfp4.argtypes = [cfg, i32, P, P, P, P, P, P, ctypes.POINTER(_WeightsNVFP4), P, P, sz, P]
+        lib.moe_forward_nvfp4.argtypes = [cfg, i32, P, P, ctypes.POINTER(_WeightsNVFP4), P, ctypes.POINTER(_Aux), P,
                                           sz, P]
         lib.moe_error_string.restype = ctypes.c_char_p
         lib.moe_error_string.argtypes = [ctypes.c_int]
@@ -332,6 +377,71 @@ def moe_forward_mxfp8(cfg: MoEConfig, x, logits, weights: MoEWeightsMXFP8, out, 
         for name, t in aux.items():
             setattr(a, name, _ptr(t))
     _check("moe_forward_mxfp8", load_library().moe_forward_mxfp8(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(logits, True), ctypes.byref(w), _ptr(out), ctypes.byref(a),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_nvfp4_pack_scales(scales, packed, stream=None):
+    """NVFP4 block scales [rows, K // 16] uint8 -> the FFN's layout
+    [rows / 64][K / 128][64][8] (rows % 64 == 0, K % 128 == 0)."""
+    import torch
+    kb = scales.shape[-1]
+    _expect(scales, torch.uint8, scales.numel(), "scales")
+    _expect(packed, torch.uint8, scales.numel(), "packed")
+    _check("moe_nvfp4_pack_scales", load_library().moe_nvfp4_pack_scales(
+        scales.numel() // kb, kb * 16, _ptr(scales), _ptr(packed), _stream(stream)))
+
+
+def pack_nvfp4(weights: MoEWeights, stream=None) -> MoEWeightsNVFP4:
+    """Quantise every expert matrix of `weights` to NVFP4 on the GPU
+    (moe_quantize_nvfp4 with one matrix scale per expert matrix, then
+    moe_nvfp4_pack_scales); the gate vector and the router projection are
+    passed through.  Allocates the outputs."""
+    import torch
+
+    def one(w, tscale):
+        w3 = w.reshape((-1,) + tuple(w.shape[-2:]))
+        codes = torch.empty(w.shape[:-1] + (w.shape[-1] // 2,), dtype=torch.uint8, device=w.device)
+        scales = torch.empty(w.shape[:-1] + (w.shape[-1] // 16,), dtype=torch.uint8, device=w.device)
+        moe_quantize_nvfp4(w3, codes, scales, tscale, stream=stream)
+        packed = torch.empty_like(scales)
+        moe_nvfp4_pack_scales(scales, packed, stream=stream)
+        return codes, packed
+
+    E = weights.w_gate.shape[0]
+    ts = torch.empty(3, E, dtype=torch.float32, device=weights.w_gate.device)
+    (g, gs), (u, us), (d, ds) = (one(weights.w_gate, ts[0]), one(weights.w_up, ts[1]), one(weights.w_down, ts[2]))
+    out = MoEWeightsNVFP4(g, u, d, gs, us, ds, ts[0], ts[1], ts[2], ws_gate_vec=weights.ws_gate_vec,
+                          w_router=weights.w_router)
+    if weights.ws_gate is not None:
+        out.ws_tscale = torch.empty(3, dtype=torch.float32, device=weights.ws_gate.device)
+        (out.ws_gate, out.ws_gate_scale), (out.ws_up, out.ws_up_scale), (out.ws_down, out.ws_down_scale) = (
+            one(weights.ws_gate, out.ws_tscale[0:1]), one(weights.ws_up, out.ws_tscale[1:2]),
+            one(weights.ws_down, out.ws_tscale[2:3]))
+    return out
+
+
+def moe_expert_ffn_nvfp4(cfg: MoEConfig, x, x_perm, offsets, perm, topk_w, weights: MoEWeightsNVFP4, ybuf, ws, *,
+                         sgate=None, stream=None):
+    """moe_expert_ffn with NVFP4 expert weights."""
+    T = x.shape[0]
+    w = weights._c()
+    _check("moe_expert_ffn_nvfp4", load_library().moe_expert_ffn_nvfp4(
+        ctypes.byref(cfg._c()), T, _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(perm), _ptr(topk_w),
+        _ptr(sgate, True), ctypes.byref(w), _ptr(ybuf), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_forward_nvfp4(cfg: MoEConfig, x, logits, weights: MoEWeightsNVFP4, out, ws, *, aux: Optional[dict] = None,
+                      stream=None):
+    """moe_forward with NVFP4 expert weights (arguments as moe_forward)."""
+    T = x.shape[0]
+    w = weights._c()
+    a = _Aux()
+    if aux:
+        for name, t in aux.items():
+            setattr(a, name, _ptr(t))
+    _check("moe_forward_nvfp4", load_library().moe_forward_nvfp4(
         ctypes.byref(cfg._c()), T, _ptr(x), _ptr(logits, True), ctypes.byref(w), _ptr(out), ctypes.byref(a),
         _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 

@@ -85,16 +85,19 @@ constexpr int kTileM = 128;                    // weight rows per tile (MMA M)
 constexpr int kABytes = kTileM * kBlockK * 2;  // 16 KB
 constexpr int kNumBox = 5;                     // token box heights 16 << i
 constexpr int kThreads = 192;                  // bf16 weights: producer, MMA, 4 epilogue warps
-// Block-scaled (MXFP8) weights: converter warps after the epilogue warps turn
-// each ring step's FP8 codes into the bf16 A operand in tensor memory.
-constexpr int kConvWarps = 8;  // two per SM sub-partition, so one hides the other's shared-memory latency
+// Block-scaled weights (kFmt 1: MXFP8, 2: NVFP4): converter warps after the
+// epilogue warps turn each ring step's codes into the bf16 A operand in
+// tensor memory.  A ring step covers 128 K of a 128-row weight tile: its
+// codes (MXFP8: 128 B a row, 8 pages; NVFP4: 64 B a row, 4 pages), its
+// block scales (one page: two runs of 64 rows, MXFP8 4 UE8M0 bytes a row,
+// NVFP4 8 E4M3 bytes a row) and two token boxes.
+constexpr int kConvWarps = 8;  // two groups of four, one warp of each per SM sub-partition
 constexpr int kThreadsQ = kThreads + 32 * kConvWarps;
-constexpr int kQKStep = 128;                   // K elements per FP8 ring step (one 128-byte code box row)
-constexpr int kQCodePages = kTileM * kQKStep / 2048;  // 8 pages: 128 rows x 128 codes
-constexpr int kQScaleBytes = 512;              // 128 rows x 4 UE8M0 scales (blocks of 32) per step
-// MXFP8: a step's converted A operand (two bf16 K slices of 64: 64 TMEM
-// columns) goes to one of kConvBufs buffers after the accumulators (from
-// column kConvCol0 on; the token tile is at most 128 wide then).
+template <int kFmt> constexpr int qcode_pages() { return kFmt == 2 ? 4 : 8; }
+template <int kFmt> constexpr int qscale_run() { return kFmt == 2 ? 512 : 256; }  // bytes per 64 rows
+// A step's converted A operand (two bf16 K slices of 64: 64 TMEM columns) goes
+// to one of kConvBufs buffers after the accumulators (from column kConvCol0
+// on; the token tile is at most 128 wide then).
 constexpr int kConvBufs = 4;
 constexpr int kConvCols = 64;
 constexpr int kConvCol0 = 256;
@@ -103,7 +106,7 @@ constexpr int kAPages = kABytes / kPageBytes;  // 8 pages of weights per K step
 constexpr int kMaxStepPages = kAPages + 256 * 128 / kPageBytes;  // 24: weights + 256 token rows
 constexpr int kTwoSlicePages = 32;  // two K slices per ring step up to here, when the ring holds 4 slices
 constexpr int kMaxPages = 112;
-constexpr int kQMaxStepPages = kQCodePages + 1 + 2 * (256 * 128 / 2048);  // 41: codes, scales, 2 token boxes
+constexpr int kQMaxStepPages = 8 + 1 + 2 * (256 * 128 / 2048);  // 41: codes, scales, 2 token boxes (at most)
 constexpr int kTickets = 32;                   // K steps in flight at most (barrier pairs)
 constexpr int kSmemLimit = 232448;             // 227 KB opt-in per CTA
 constexpr int kXchgStride = 33;                // fp32 exchange row stride (bank-conflict free)
@@ -129,11 +132,16 @@ struct FfnParams {
     int phases;         // bit 0: gate/up items, bit 1: down items
     int R[2], Rs[2];    // weight tiles per routed / shared expert, per phase
     int nk[2], nks[2];  // K steps routed / shared, per phase
-    // MXFP8 weights only: the packed UE8M0 scales of each matrix, [phase][0: gate
-    // or down, 1: up], routed and shared; 256 bytes per (64-row group, 128-wide K
-    // step), row-group major (see moe_mxfp8_pack_scales)
+    // block-scaled weights only: the packed block scales of each matrix, [phase][0:
+    // gate or down, 1: up], routed and shared; one run (qscale_run bytes) per
+    // (64-row group, 128-wide K step), row-group major (moe_mxfp8_pack_scales,
+    // moe_nvfp4_pack_scales)
     const uint8_t *sf[2][2];
     const uint8_t *sfs[2][2];
+    // NVFP4 only: the fp32 matrix scales, [phase][0: gate or down, 1: up] with
+    // one per expert, and the shared expert's {gate, up, down}
+    const float *ts[2][2];
+    const float *tss;
     // the group-readiness wait's limit (kWaitLimitNs), and a group whose
     // readiness target is one past what its gate/up items can reach (-1: none)
     // -- both only changed by the test hooks MOE_TEST_WAIT_LIMIT_US and
@@ -375,7 +383,10 @@ __device__ __forceinline__ StepShape qstep_shape(const Item &it, const FfnParams
     sh.nk = it.shared ? p.nks[it.ph] : p.nk[it.ph];
     return sh;
 }
-__device__ __forceinline__ uint32_t qstep_pages(const StepShape &sh) { return kQCodePages + 1 + 2 * sh.sub_pages; }
+template <int kFmt>
+__device__ __forceinline__ uint32_t qstep_pages(const StepShape &sh) {
+    return qcode_pages<kFmt>() + 1 + 2 * sh.sub_pages;
+}
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + __expf(-g)); }
 
@@ -466,6 +477,79 @@ __device__ __forceinline__ void convert_mxfp8_row(uint32_t codes, uint32_t scale
     }
 }
 
+// ------------------------------------------------- NVFP4 weight conversion --
+// An NVFP4 weight is an E2M1 code c (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6)
+// times its block's E4M3 scale s (one per 16 consecutive K elements), times
+// the matrix's fp32 scale, which the epilogue applies.  c * s has at most 6
+// significant bits and lies in [2^-10, 2688]: a bf16 value, so the
+// conversion is exact.
+//
+// The hardware unpacks two codes into f16x2 exactly.  The f16 of a nonzero c
+// is normal with its 9 low mantissa bits zero, so shifting the pair right by
+// 3 and clearing the bits the signs leave behind gives, read as bf16x2, the
+// magnitudes c * 2^-112 (exponent rebiased from 15 to 127).  One multiply by
+// the block's 2^112 * s (at most 2^121: no overflow) makes c * s; the signs
+// are put back last.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+}
+__device__ __forceinline__ uint32_t e2m1_f16x2_times(uint32_t x, uint32_t m) {
+    return bf16x2_mul((x >> 3) & 0x0FFF0FFFu, m) | (x & 0x80008000u);
+}
+// bf16x2 of 2^112 * s for the two E4M3 scales in bytes 0 and 2 of `two`:
+// each byte's 7 magnitude bits placed at bits 10..4 of its lane read as
+// s * 2^-120 (the subnormal scales as bf16 subnormals), and two exact
+// multiplies by 2^116 follow.  Block scales are never negative.
+__device__ __forceinline__ uint32_t nv_mult2(uint32_t two) {
+    constexpr uint32_t c116 = ((127u + 116u) << 7) * 0x00010001u;
+    return bf16x2_mul(bf16x2_mul(two << 4, c116), c116);
+}
+
+// One converter thread's share of an NVFP4 ring step.  The step's weight tile
+// is 128 rows x 64 bytes of codes (128 K, two codes a byte, the lower K in the
+// low nibble) as TMA left them with the 64-byte swizzle (row r at r * 64,
+// 16-byte chunk c at (c ^ ((r >> 1) & 3)) * 16), and row r's eight E4M3 block
+// scales at byte 8r.  The thread turns row r into 128 bf16 and stores them to
+// 64 columns of TMEM lane r, as convert_mxfp8_row does.  The 8 lanes of a
+// shared-memory phase read one chunk index of 8 consecutive rows, which the
+// swizzle puts in 8 distinct 16-byte bank groups.
+__device__ __forceinline__ void convert_nvfp4_row(uint32_t codes, uint32_t scales, int r, uint32_t taddr) {
+    uint4 q[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(q[j].x), "=r"(q[j].y), "=r"(q[j].z), "=r"(q[j].w)
+                     : "r"(codes + (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4))));
+    uint32_t s0, s1;  // block scales 0..3, 4..7
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(s0), "=r"(s1) : "r"(scales + (uint32_t)(r * 8)));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t o[32];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int j = 2 * h + jj;  // chunk j: K 32 j .. 32 j + 31, blocks 2 j and 2 j + 1
+            const uint32_t m2 = nv_mult2(prmt_b32(j < 2 ? s0 : s1, 0u, (j & 1) ? 0x4342u : 0x4140u));
+            const uint32_t ma = prmt_b32(m2, 0u, 0x1010u), mb = prmt_b32(m2, 0u, 0x3232u);
+            const uint32_t w[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // word i: K 32 j + 8 i .. + 7
+                uint32_t x[4];
+                e2m1x8_to_f16x2(w[i], x);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) o[16 * jj + 4 * i + t] = e2m1_f16x2_times(x[t], i < 2 ? ma : mb);
+            }
+        }
+        tmem_st32(taddr + (uint32_t)(32 * h), o);
+    }
+}
+
 // Down item, token n of the tile: its ybuf row (t*(k+1) + j, or t*(k+1) + k for
 // the shared expert) and the weight applied to it.
 __device__ __forceinline__ void down_dest(const Item &it, int n, const FfnParams &p, int &mrow, float &mw) {
@@ -489,9 +573,10 @@ __device__ __forceinline__ void down_dest(const Item &it, int n, const FfnParams
 }
 
 // --------------------------------------------------------------- kernel --
-// kFmt: 0 bf16 weights; 1 MXFP8 weights (E4M3 codes + UE8M0 block scales),
-// converted to bf16 in shared memory by kConvWarps converter warps (single
-// CTAs only).
+// kFmt: 0 bf16 weights; 1 MXFP8 weights (E4M3 codes + UE8M0 block scales);
+// 2 NVFP4 weights (E2M1 codes + E4M3 block scales + an fp32 scale per
+// matrix).  Block-scaled weights are converted to bf16 in tensor memory by
+// kConvWarps converter warps (single CTAs only).
 template <bool kPair, int kFmt>
 __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     ffn_kernel(const __grid_constant__ FfnMaps maps, const FfnParams p) {
@@ -713,6 +798,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 const CUtensorMap *ma0 = it.shared ? &pm.s0 : &pm.a0;
                 const CUtensorMap *ma1 = it.shared ? &pm.s1 : &pm.a1;
                 const StepShape sh = kFmt ? qstep_shape(it, p) : step_shape<kPair>(it, p);
+                constexpr int kCP = qcode_pages<kFmt>(), kRun = qscale_run<kFmt>();
                 const CUtensorMap *mb = it.shared ? &pm.bs[sh.bi] : &pm.b[sh.bi];
                 // pair: this CTA's weight tile of the two, and its half of the token rows
                 const int rt = kPair ? 2 * it.r + (int)rank : it.r;
@@ -723,7 +809,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 bool ok = true;
                 for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
                     const int nsub = min(sh.ns, sh.nk - k0);
-                    const uint32_t need = kFmt ? qstep_pages(sh) : (uint32_t)nsub * sh.sub_pages;
+                    const uint32_t need = kFmt ? qstep_pages<kFmt>(sh) : (uint32_t)nsub * sh.sub_pages;
                     const uint32_t first = ring_alloc(vhead, off, need, P);
                     // Free a ticket and the pages of this step: retire the oldest steps
                     // until the steps in flight and this one lie within P consecutive
@@ -743,20 +829,21 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                     ticket_start[tk] = vhead - need;
                     if constexpr (kFmt != 0) {
                         // codes of the weight tile, their scales, two token boxes
-                        mbar_arrive_expect_tx(&full[tk], (kQCodePages + 2 * sh.sub_pages) * kPageBytes + kQScaleBytes);
+                        mbar_arrive_expect_tx(&full[tk], (kCP + 2 * sh.sub_pages) * kPageBytes + 2 * kRun);
                         uint8_t *sA = ring + (size_t)first * kPageBytes;
                         const int kx = k0 * kBlockK;  // = 128 * (K step)
+                        const int kc = kFmt == 2 ? kx / 2 : kx;  // the codes' byte column
                         const int ks = k0 >> 1;
-                        tma_load_2d_hint(ma0, &full[tk], sA, kx, a_row, apol);  // gate: 64 rows; down: 128 rows
-                        if (it.ph == 0) tma_load_2d_hint(ma1, &full[tk], sA + kQCodePages * kPageBytes / 2, kx, a_row, apol);
-                        uint8_t *sS = sA + kQCodePages * kPageBytes;
+                        tma_load_2d_hint(ma0, &full[tk], sA, kc, a_row, apol);  // gate: 64 rows; down: 128 rows
+                        if (it.ph == 0) tma_load_2d_hint(ma1, &full[tk], sA + kCP * kPageBytes / 2, kc, a_row, apol);
+                        uint8_t *sS = sA + kCP * kPageBytes;
                         const size_t ksteps = (size_t)(sh.nk >> 1);
                         const size_t rg = (size_t)(a_row >> 6);  // 64-row group of the tile's first row
                         const uint8_t *const *sfp = it.shared ? p.sfs[it.ph] : p.sf[it.ph];
-                        bulk_load(sS, sfp[0] + (rg * ksteps + ks) * 256, 256, &full[tk]);
+                        bulk_load(sS, sfp[0] + (rg * ksteps + ks) * kRun, kRun, &full[tk]);
                         // gate/up: the up rows' scales; down: the tile's second 64-row group
-                        bulk_load(sS + 256, it.ph == 0 ? sfp[1] + (rg * ksteps + ks) * 256 : sfp[0] + ((rg + 1) * ksteps + ks) * 256,
-                                  256, &full[tk]);
+                        bulk_load(sS + kRun, it.ph == 0 ? sfp[1] + (rg * ksteps + ks) * kRun : sfp[0] + ((rg + 1) * ksteps + ks) * kRun,
+                                  kRun, &full[tk]);
                         uint8_t *sB = sS + kPageBytes;
                         tma_load_2d(mb, &full[tk], sB, kx, it.row0);
                         tma_load_2d(mb, &full[tk], sB + sh.sub_pages * kPageBytes, kx + kBlockK, it.row0);
@@ -828,7 +915,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 for (int k0 = 0; k0 < sh.nk; k0 += sh.ns) {
                     const int nsub = min(sh.ns, sh.nk - k0);
                     const uint32_t first =
-                        ring_alloc(vhead, off, kFmt ? qstep_pages(sh) : (uint32_t)nsub * sh.sub_pages, P);
+                        ring_alloc(vhead, off, kFmt ? qstep_pages<kFmt>(sh) : (uint32_t)nsub * sh.sub_pages, P);
                     const uint32_t tk = step % kTickets;
                     if (!mbar_wait_fast<kPair>(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true)) {
                         ok = false;
@@ -843,7 +930,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                        const uint64_t db = desc0 + (first + kQCodePages + 1) * (kPageBytes / 16);
+                        const uint64_t db = desc0 + (first + qcode_pages<kFmt>() + 1) * (kPageBytes / 16);
                         const uint32_t ta = tmem_base + (uint32_t)(kConvCol0 + cb * kConvCols);
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
@@ -931,7 +1018,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
             named_bar_sync(2 + g, 16 * kConvWarps);  // read by all before the elected thread's next write
             if (item < 0) break;
             const StepShape sh = qstep_shape(it, p);
-            const uint32_t need = qstep_pages(sh);
+            const uint32_t need = qstep_pages<kFmt>(sh);
             bool ok = true;
             for (int k0 = 0; k0 < sh.nk; k0 += sh.ns, ++step) {
                 const uint32_t first = ring_alloc(vhead, off, need, P);
@@ -942,7 +1029,10 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const uint32_t codes = smem_u32(ring + (size_t)first * kPageBytes);
-                convert_mxfp8_row(codes, codes + kQCodePages * kPageBytes, crow, tlane + cb * kConvCols);
+                if constexpr (kFmt == 2)
+                    convert_nvfp4_row(codes, codes + qcode_pages<kFmt>() * kPageBytes, crow, tlane + cb * kConvCols);
+                else
+                    convert_mxfp8_row(codes, codes + qcode_pages<kFmt>() * kPageBytes, crow, tlane + cb * kConvCols);
                 tmem_wait_st();  // this thread's stores done, before the arrival
                 tc_fence_before();
                 __syncwarp();
@@ -974,6 +1064,12 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
             int mrow0 = 0;
             float mw0 = 0.f;
             if (it.ph == 1) down_dest(it, lane, p, mrow0, mw0);
+            // NVFP4: the matrix scales of this item's projections (gate or down, up)
+            float ts0 = 1.f, ts1 = 1.f;
+            if constexpr (kFmt == 2) {
+                ts0 = it.shared ? p.tss[2 * it.ph] : __ldg(p.ts[it.ph][0] + it.e);
+                if (it.ph == 0) ts1 = it.shared ? p.tss[1] : __ldg(p.ts[0][1] + it.e);
+            }
             if (elected) *epi_flag = mbar_wait<kPair>(&tfull[acc], use & 1u, abort_flag, p.status, true) ? 0 : -1;
             named_bar_sync(1, 128);
             if (*epi_flag) break;
@@ -984,6 +1080,11 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 if (it.ph == 0) {
                     float v[32];
                     tmem_ld32(tbase + (uint32_t)c0, v);
+                    if constexpr (kFmt == 2) {
+                        const float ts = q < 2 ? ts0 : ts1;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= ts;
+                    }
                     if (q < 2) {  // gate rows 0..63: silu(g) to the exchange buffer
                         float *xr = xchg + (q * 32 + lane) * kXchgStride;
 #pragma unroll
@@ -1006,6 +1107,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                     int mrow = mrow0;
                     float mw = mw0;
                     if (c0 > 0) down_dest(it, c0 + lane, p, mrow, mw);
+                    if constexpr (kFmt == 2) mw *= ts0;
                     for (int t = 0; t < it.m; ++t) {  // weight tile r + t: accumulator columns t * BN/2
                         float v[32];
                         tmem_ld32(tbase + (uint32_t)(t * (p.BN >> 1) + c0), v);
@@ -1094,7 +1196,7 @@ size_t smem_bytes_for(int E, int pages, int fmt) {
            (kQueue + 3) * sizeof(ItemSlot) + 8 + 2 * (size_t)nt * 4 + kReadyWords * 4 + kTickets * 4;
 }
 
-int min_pages(int fmt) { return fmt ? kQMaxStepPages : kMaxStepPages; }
+int min_pages(int fmt) { return fmt == 2 ? 4 + 1 + 2 * (256 * 128 / 2048) : fmt ? kQMaxStepPages : kMaxStepPages; }
 
 int pick_pages(int E, int fmt) {
     const size_t fixed = smem_bytes_for(E, 0, fmt);
@@ -1216,12 +1318,12 @@ cudaError_t launch_pair(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t 
 int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     const DeviceInfo di = device_info();
     if (di.cc_major != 10) return MOE_ERR_UNSUPPORTED;
-    if (phases < 1 || phases > 3 || a.fmt < 0 || a.fmt > 1) return MOE_ERR_INVALID_ARG;
-    // MXFP8: 128-wide K steps and 64-row scale groups
+    if (phases < 1 || phases > 3 || a.fmt < 0 || a.fmt > 2) return MOE_ERR_INVALID_ARG;
+    // block-scaled weights: 128-wide K steps and 64-row scale groups
     if (a.fmt && (a.H % 128 != 0 || a.I % 128 != 0 || a.Is % 128 != 0)) return MOE_ERR_UNSUPPORTED;
     FfnParams p{};
     if (int rc = choose_tiles(a, di.sms, &p.BN, &p.BNs, &p.pages)) return rc;
-    if (a.fmt && 2 * p.BN > kConvCol0) return MOE_ERR_UNSUPPORTED;  // MXFP8: accumulators end where the A buffers start
+    if (a.fmt && 2 * p.BN > kConvCol0) return MOE_ERR_UNSUPPORTED;  // accumulators end where the A buffers start
     if (int rc = test_hooks(a, &p.wait_limit_ns, &p.stall_group)) return rc;
     bool pair = false;
     if (int rc = choose_pair(a, phases, di.sms, &pair)) return rc;
@@ -1258,14 +1360,20 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     p.sfs[0][0] = a.sfs_gate;
     p.sfs[0][1] = a.sfs_up;
     p.sfs[1][0] = a.sfs_down;
+    p.ts[0][0] = a.ts_gate;
+    p.ts[0][1] = a.ts_up;
+    p.ts[1][0] = a.ts_down;
+    p.tss = a.tss;
 
     static FfnMaps zero_maps;  // unused maps stay zero
     FfnMaps m = zero_maps;
     const uint64_t Tk = (uint64_t)a.T * a.k;
     bool ok = true;
-    // weight maps: bf16 boxes of 64 K, or MXFP8 code boxes of 128 K (bytes)
+    // weight maps: bf16 boxes of 64 K, or code boxes of 128 K (MXFP8: 128 bytes
+    // a row, 128-byte swizzle; NVFP4: 64 bytes a row, 64-byte swizzle)
     auto wmap = [&](CUtensorMap *mp, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-        return a.fmt ? encode_2d_u8(mp, base, rows, cols, box_rows) : encode_2d(mp, base, rows, cols, box_rows);
+        if (a.fmt == 2) return encode_2d_u8(mp, base, rows, cols / 2, box_rows, 64);
+        return a.fmt ? encode_2d_u8(mp, base, rows, cols, box_rows, 128) : encode_2d(mp, base, rows, cols, box_rows);
     };
     if (phases & 1) {
         PhaseMaps &g = m.ph[0];
@@ -1300,6 +1408,8 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
             cudaFuncSetAttribute(ffn_kernel<true, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
                 cudaSuccess ||
             cudaFuncSetAttribute(ffn_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(ffn_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
                 cudaSuccess)
             return MOE_ERR_CUDA;
         attr_set[dev].store(1, std::memory_order_release);
@@ -1320,6 +1430,10 @@ int ffn_launch(const FfnArgs &a, int phases, cudaStream_t st) {
     const int grid = (int)std::max<long long>(1, std::min<long long>(di.sms, items));
     if (a.fmt == 1)
         return launch_pdl(ffn_kernel<false, 1>, dim3(grid), dim3(kThreadsQ), smem, st, m, p) == cudaSuccess
+                   ? MOE_OK
+                   : MOE_ERR_CUDA;
+    if (a.fmt == 2)
+        return launch_pdl(ffn_kernel<false, 2>, dim3(grid), dim3(kThreadsQ), smem, st, m, p) == cudaSuccess
                    ? MOE_OK
                    : MOE_ERR_CUDA;
     return launch_pdl(ffn_kernel<false, 0>, dim3(grid), dim3(kThreads), smem, st, m, p) == cudaSuccess

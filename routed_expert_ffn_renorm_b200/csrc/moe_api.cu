@@ -201,41 +201,71 @@ int ffn_args(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_
     return MOE_OK;
 }
 
-// The MXFP8 expert FFN's argument block: the bf16 block with the weight
-// pointers replaced by E4M3 codes and the packed scales added.
-int ffn_args_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
-                   const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
-                   const moe_weights_mxfp8_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, FfnArgs *a) {
-    if (!w) return MOE_ERR_INVALID_ARG;
+// A block-scaled expert FFN's argument block: the bf16 block with the weight
+// pointers replaced by the codes and the packed block scales added.  codes /
+// scales: gate, up, down, shared gate, shared up, shared down.
+int ffn_args_scaled(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                    const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                    const uint8_t *const (&codes)[6], const uint8_t *const (&scales)[6], int fmt, moe_bf16_t *ybuf,
+                    void *ws, size_t ws_bytes, FfnArgs *a) {
     const bool sh = cfg->shared_intermediate_size > 0;
-    if (!aligned(w->w_gate) || !aligned(w->w_up) || !aligned(w->w_down) || !aligned(w->w_gate_scale) ||
-        !aligned(w->w_up_scale) || !aligned(w->w_down_scale))
-        return MOE_ERR_INVALID_ARG;
-    if (sh && (!aligned(w->ws_gate) || !aligned(w->ws_up) || !aligned(w->ws_down) || !aligned(w->ws_gate_scale) ||
-               !aligned(w->ws_up_scale) || !aligned(w->ws_down_scale)))
-        return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < (sh ? 6 : 3); ++i)
+        if (!aligned(codes[i]) || !aligned(scales[i])) return MOE_ERR_INVALID_ARG;
     if (cfg->hidden % 128 != 0 || cfg->moe_intermediate_size % 128 != 0 || cfg->shared_intermediate_size % 128 != 0)
         return MOE_ERR_UNSUPPORTED;
     // the bf16 block's checks and fields, with the code pointers standing in for the weights
     moe_weights_t wb{};
-    wb.w_gate = reinterpret_cast<const moe_bf16_t *>(w->w_gate);
-    wb.w_up = reinterpret_cast<const moe_bf16_t *>(w->w_up);
-    wb.w_down = reinterpret_cast<const moe_bf16_t *>(w->w_down);
-    wb.ws_gate = reinterpret_cast<const moe_bf16_t *>(w->ws_gate);
-    wb.ws_up = reinterpret_cast<const moe_bf16_t *>(w->ws_up);
-    wb.ws_down = reinterpret_cast<const moe_bf16_t *>(w->ws_down);
+    wb.w_gate = reinterpret_cast<const moe_bf16_t *>(codes[0]);
+    wb.w_up = reinterpret_cast<const moe_bf16_t *>(codes[1]);
+    wb.w_down = reinterpret_cast<const moe_bf16_t *>(codes[2]);
+    wb.ws_gate = reinterpret_cast<const moe_bf16_t *>(codes[3]);
+    wb.ws_up = reinterpret_cast<const moe_bf16_t *>(codes[4]);
+    wb.ws_down = reinterpret_cast<const moe_bf16_t *>(codes[5]);
     FfnArgs b;
     int rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, &wb, ybuf, ws, ws_bytes, true, a);
     if (rc) return rc;
     rc = ffn_args(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, &wb, ybuf, ws, ws_bytes, false, &b);
     if (rc) return rc;
-    a->fmt = 1;
-    a->sf_gate = w->w_gate_scale;
-    a->sf_up = w->w_up_scale;
-    a->sf_down = w->w_down_scale;
-    a->sfs_gate = sh ? w->ws_gate_scale : nullptr;
-    a->sfs_up = sh ? w->ws_up_scale : nullptr;
-    a->sfs_down = sh ? w->ws_down_scale : nullptr;
+    a->fmt = fmt;
+    a->sf_gate = scales[0];
+    a->sf_up = scales[1];
+    a->sf_down = scales[2];
+    a->sfs_gate = sh ? scales[3] : nullptr;
+    a->sfs_up = sh ? scales[4] : nullptr;
+    a->sfs_down = sh ? scales[5] : nullptr;
+    return MOE_OK;
+}
+
+int ffn_args_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                   const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                   const moe_weights_mxfp8_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, FfnArgs *a) {
+    if (!w) return MOE_ERR_INVALID_ARG;
+    const uint8_t *const codes[6] = {w->w_gate, w->w_up, w->w_down, w->ws_gate, w->ws_up, w->ws_down};
+    const uint8_t *const scales[6] = {w->w_gate_scale,  w->w_up_scale,  w->w_down_scale,
+                                      w->ws_gate_scale, w->ws_up_scale, w->ws_down_scale};
+    return ffn_args_scaled(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, codes, scales, 1, ybuf, ws, ws_bytes, a);
+}
+
+bool f32_aligned(const float *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int ffn_args_nvfp4(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                   const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                   const moe_weights_nvfp4_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, FfnArgs *a) {
+    if (!w) return MOE_ERR_INVALID_ARG;
+    const bool sh = cfg->shared_intermediate_size > 0;
+    if (!f32_aligned(w->w_gate_tscale) || !f32_aligned(w->w_up_tscale) || !f32_aligned(w->w_down_tscale) ||
+        (sh && !f32_aligned(w->ws_tscale)))
+        return MOE_ERR_INVALID_ARG;
+    const uint8_t *const codes[6] = {w->w_gate, w->w_up, w->w_down, w->ws_gate, w->ws_up, w->ws_down};
+    const uint8_t *const scales[6] = {w->w_gate_scale,  w->w_up_scale,  w->w_down_scale,
+                                      w->ws_gate_scale, w->ws_up_scale, w->ws_down_scale};
+    const int rc =
+        ffn_args_scaled(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, codes, scales, 2, ybuf, ws, ws_bytes, a);
+    if (rc) return rc;
+    a->ts_gate = w->w_gate_tscale;
+    a->ts_up = w->w_up_tscale;
+    a->ts_down = w->w_down_tscale;
+    a->tss = sh ? w->ws_tscale : nullptr;
     return MOE_OK;
 }
 
@@ -411,6 +441,25 @@ int moe_mxfp8_pack_scales(int64_t rows, int32_t K, const uint8_t *scales, uint8_
     return cuda_rc(launch_mxfp8_pack_scales(rows, K, scales, packed, as_stream(stream)));
 }
 
+int moe_nvfp4_pack_scales(int64_t rows, int32_t K, const uint8_t *scales, uint8_t *packed, void *stream) {
+    if (rows < 0 || rows % 64 != 0 || K < 128 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!aligned(scales) || !aligned(packed)) return MOE_ERR_INVALID_ARG;
+    return cuda_rc(launch_nvfp4_pack_scales(rows, K, scales, packed, as_stream(stream)));
+}
+
+int moe_expert_ffn_nvfp4(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
+                         const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
+                         const moe_weights_nvfp4_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_config(cfg, T);
+    if (rc) return rc;
+    if (T == 0) return MOE_OK;
+    FfnArgs a;
+    rc = ffn_args_nvfp4(cfg, T, x, x_perm, offsets, perm, topk_w, sgate, w, ybuf, ws, ws_bytes, &a);
+    if (rc) return rc;
+    return ffn_launch_both(a, as_stream(stream));
+}
+
 int moe_expert_ffn_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const moe_bf16_t *x_perm,
                          const int32_t *offsets, const int32_t *perm, const float *topk_w, const float *sgate,
                          const moe_weights_mxfp8_t *w, moe_bf16_t *ybuf, void *ws, size_t ws_bytes, void *stream) {
@@ -468,7 +517,7 @@ namespace {
 
 // The layer around an expert FFN: [router projection] -> route -> [budget]
 // -> dispatch -> ffn(...) -> combine.  `ffn` enqueues the expert FFN of the
-// dispatched batch (bf16 or MXFP8 weights).
+// dispatched batch (bf16, MXFP8 or NVFP4 weights).
 template <class Ffn>
 int forward_impl(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
                  const moe_bf16_t *w_router, const moe_bf16_t *ws_gate_vec, moe_bf16_t *out, const moe_aux_t *aux,
@@ -558,6 +607,22 @@ int moe_forward_mxfp8(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, c
                         [&](const moe_bf16_t *x_perm, const int32_t *offsets, const int32_t *perm, const float *tw,
                             const float *sgate, moe_bf16_t *ybuf) {
                             return moe_expert_ffn_mxfp8(cfg, T, x, x_perm, offsets, perm, tw, sgate, w, ybuf, ws,
+                                                        ws_bytes, stream);
+                        });
+}
+
+int moe_forward_nvfp4(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const float *logits,
+                      const moe_weights_nvfp4_t *w, moe_bf16_t *out, const moe_aux_t *aux, void *ws,
+                      size_t ws_bytes, void *stream) {
+    const int rc = check_config(cfg, T);
+    if (rc || T == 0) return rc;
+    if (!w) return MOE_ERR_INVALID_ARG;
+    if (cfg->hidden % 128 != 0 || cfg->moe_intermediate_size % 128 != 0 || cfg->shared_intermediate_size % 128 != 0)
+        return MOE_ERR_UNSUPPORTED;  // before anything is launched
+    return forward_impl(cfg, T, x, logits, w->w_router, w->ws_gate_vec, out, aux, ws, ws_bytes, stream,
+                        [&](const moe_bf16_t *x_perm, const int32_t *offsets, const int32_t *perm, const float *tw,
+                            const float *sgate, moe_bf16_t *ybuf) {
+                            return moe_expert_ffn_nvfp4(cfg, T, x, x_perm, offsets, perm, tw, sgate, w, ybuf, ws,
                                                         ws_bytes, stream);
                         });
 }

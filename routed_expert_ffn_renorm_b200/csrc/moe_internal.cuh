@@ -115,6 +115,7 @@ cudaError_t launch_quantize_nvfp4(int nmat, long long rows, int K, const uint16_
 // MXFP8 scales [rows, K / 32] -> the FFN's layout [rows / 64][K / 128][64][4]
 // (rows % 64 == 0, K % 128 == 0).
 cudaError_t launch_mxfp8_pack_scales(long long rows, int K, const uint8_t *scales, uint8_t *packed, cudaStream_t st);
+cudaError_t launch_nvfp4_pack_scales(long long rows, int K, const uint8_t *scales, uint8_t *packed, cudaStream_t st);
 
 // Expert parallelism (ep.cu): destination ranks of slots, the send metadata
 // in send order, and the returned rows back to token order.  n_dev: the
@@ -137,9 +138,13 @@ struct FfnArgs {
     const float *topk_w, *sgate;
     const uint16_t *w_gate, *w_up, *w_down, *ws_gate, *ws_up, *ws_down;
     // fmt 1 (MXFP8 weights): the w_* / ws_* pointers above hold E4M3 codes (one
-    // byte per weight, same shapes) and these the packed UE8M0 scales
+    // byte per weight, same shapes) and sf_* the packed UE8M0 scales; fmt 2
+    // (NVFP4): they hold E2M1 codes (two per byte), sf_* the packed E4M3 block
+    // scales, ts_* the fp32 matrix scales ([E] each) and tss the shared
+    // expert's {gate, up, down}
     int fmt;
     const uint8_t *sf_gate, *sf_up, *sf_down, *sfs_gate, *sfs_up, *sfs_down;
+    const float *ts_gate, *ts_up, *ts_down, *tss;
     uint16_t *h_perm, *h_shared, *ybuf;
     int32_t *status;  // the workspace's status block: [0] status word,
                       // [4..5] gate/up (or fused) and [8..9] down work-item counters

@@ -118,7 +118,35 @@ __global__ void __launch_bounds__(kQuantThreads) mxfp8_pack_scales_kernel(long l
     }
 }
 
+// NVFP4 block scales [rows, K / 16] -> [rows / 64][K / 128][64][8]: for each
+// 64-row group and 128-wide K step, the 8 block scales of each of its 64 rows
+// in one contiguous 512-byte run.  One thread per 8-byte run.
+__global__ void __launch_bounds__(kQuantThreads) nvfp4_pack_scales_kernel(long long rows, int K,
+                                                                          const uint8_t *__restrict__ in,
+                                                                          uint2 *__restrict__ out) {
+    const int kb = K / 16, ksteps = K / 128;
+    const long long n = rows * ksteps;  // 8-byte runs
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long o = (long long)blockIdx.x * blockDim.x + threadIdx.x; o < n; o += stride) {
+        const long long rgks = o >> 6;  // (row group, K step)
+        const int r = (int)(o & 63);
+        const long long rg = rgks / ksteps;
+        const int ks = (int)(rgks - rg * ksteps);
+        const uint8_t *src = in + (rg * 64 + r) * kb + ks * 8;
+        uint2 v;
+        v.x = (uint32_t)src[0] | ((uint32_t)src[1] << 8) | ((uint32_t)src[2] << 16) | ((uint32_t)src[3] << 24);
+        v.y = (uint32_t)src[4] | ((uint32_t)src[5] << 8) | ((uint32_t)src[6] << 16) | ((uint32_t)src[7] << 24);
+        out[o] = v;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_nvfp4_pack_scales(long long rows, int K, const uint8_t *scales, uint8_t *packed, cudaStream_t st) {
+    const long long n = rows * (K / 128);
+    nvfp4_pack_scales_kernel<<<grid_for(n), kQuantThreads, 0, st>>>(rows, K, scales, reinterpret_cast<uint2 *>(packed));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_mxfp8_pack_scales(long long rows, int K, const uint8_t *scales, uint8_t *packed, cudaStream_t st) {
     const long long n = rows * (K / 128);

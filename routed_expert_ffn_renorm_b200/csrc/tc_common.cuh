@@ -287,18 +287,21 @@ inline bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
-// 2-D uint8 row-major [rows, cols] tensor (FP8 codes), box = 128 columns
-// (bytes) x box_rows rows, 128-byte swizzle.
-inline bool encode_2d_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D uint8 row-major [rows, cols] tensor (block-scaled weight codes), box =
+// box_bytes columns (bytes: 128 or 64) x box_rows rows, swizzled at the box
+// row's width (128- or 64-byte swizzle).
+inline bool encode_2d_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                         uint32_t box_bytes) {
     auto fn = get_encode_fn();
-    if (!fn) return false;
+    if (!fn || (box_bytes != 128 && box_bytes != 64)) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols};
-    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t box[2] = {box_bytes, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 

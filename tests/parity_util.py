@@ -190,7 +190,9 @@ def check_layer(cfg: W.MoEConfig, inp: W.MoEInputs, g: GpuResult, rows=None,
                 nthreads: Optional[int] = None, weight_cache: Optional[dict] = None, wmap=None) -> dict:
     """Compare a GPU forward with the oracle; returns diagnostics, asserts.
     `wmap` maps each expert matrix's bf16 bits to the weights the oracle
-    uses (e.g. oracle.mxfp8_weights for the MXFP8 layer); default: as is."""
+    uses (e.g. oracle.mxfp8_weights for the MXFP8 layer), or to (weights,
+    matrix scale) pairs (oracle.nvfp4_weights for the NVFP4 layer); default:
+    as is."""
     assert g.status == 0, f"device status {g.status}"
     T, k, E = cfg.T, cfg.k, cfg.E
     nthreads = nthreads or oracle.max_threads()
@@ -258,10 +260,19 @@ def check_layer(cfg: W.MoEConfig, inp: W.MoEInputs, g: GpuResult, rows=None,
     need = sorted({int(idx_b[t, j]) for t in rows for j in range(int(keff_b[t]))})
     wg, wu, wd = _expert_dicts(inp, need, weight_cache, wmap)
     kw = {}
+    if need and isinstance(wg[need[0]], tuple):  # (weights, matrix scale) per expert matrix
+        sc = np.ones((max(max(need), int(idx_b.max(initial=0))) + 1, 3))
+        for e in need:
+            sc[e] = [float(wg[e][1]), float(wu[e][1]), float(wd[e][1])]
+        wg, wu, wd = ({e: m[e][0] for e in need} for m in (wg, wu, wd))
+        kw["scales"] = sc
     if cfg.Is:
         sb = W.bf16_bits if wmap is None else (lambda t: wmap(W.bf16_bits(t)))
-        kw = dict(ws_gate=sb(inp.ws_gate), ws_up=sb(inp.ws_up), ws_down=sb(inp.ws_down),
-                  ws_gvec=W.bf16_bits(inp.ws_gvec))
+        sgw, suw, sdw = sb(inp.ws_gate), sb(inp.ws_up), sb(inp.ws_down)
+        if isinstance(sgw, tuple):
+            kw["shared_scales"] = np.array([float(sgw[1]), float(suw[1]), float(sdw[1])])
+            sgw, suw, sdw = sgw[0], suw[0], sdw[0]
+        kw.update(ws_gate=sgw, ws_up=suw, ws_down=sdw, ws_gvec=W.bf16_bits(inp.ws_gvec))
     ref = oracle.combine_rows(W.bf16_bits(inp.x), idx_b, w_b, keff_b, wg, wu, wd, I=cfg.I, rows=rows,
                               nthreads=nthreads, **kw)
     err = rel_l2(g.out[rows], ref)

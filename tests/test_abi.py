@@ -145,3 +145,43 @@ def test_mxfp8_argument_checks():
     assert lib.moe_expert_ffn_mxfp8(ctypes.byref(cs), *args[:-1], FAKE, ctypes.byref(noshared), FAKE, FAKE, ws_s,
                                     None) == -1
     assert lib.moe_forward_mxfp8(ctypes.byref(c), 0, None, None, ctypes.byref(full), None, None, None, 0, None) == 0
+
+
+def test_nvfp4_argument_checks():
+    """The NVFP4 entry points reject bad shapes and pointers before any launch."""
+    lib = moe.load_library()
+    # scale repacking: rows a multiple of 64, K of 128, aligned pointers
+    assert lib.moe_nvfp4_pack_scales(63, 256, FAKE, FAKE, None) == -1
+    assert lib.moe_nvfp4_pack_scales(64, 192, FAKE, FAKE, None) == -1
+    assert lib.moe_nvfp4_pack_scales(64, 256, FAKE, MISALIGNED, None) == -1
+    assert lib.moe_nvfp4_pack_scales(0, 256, None, None, None) == 0
+    nf = len(moe._WeightsNVFP4._fields_)
+    full = moe._WeightsNVFP4(*([FAKE.value] * nf))
+    ws_bytes = lib.moe_workspace_bytes(ctypes.byref(_cfg()), 16)
+    args = (16, FAKE, FAKE, FAKE, FAKE, FAKE, None)
+    # I = 64 is a legal bf16 shape but not an NVFP4 one (128-wide K steps)
+    c = _cfg(moe_intermediate_size=64)
+    assert lib.moe_expert_ffn_nvfp4(ctypes.byref(c), *args, ctypes.byref(full), FAKE, FAKE, 1 << 40, None) == -2
+    assert lib.moe_forward_nvfp4(ctypes.byref(c), 16, FAKE, FAKE, ctypes.byref(full), FAKE, None, FAKE, 1 << 40,
+                                 None) == -2
+    c = _cfg()
+    assert lib.moe_expert_ffn_nvfp4(ctypes.byref(c), *args, None, FAKE, FAKE, ws_bytes, None) == -1
+    names = [n for n, _ in moe._WeightsNVFP4._fields_]
+    for field, value in (("w_down_scale", MISALIGNED.value), ("w_up_tscale", None),
+                         ("w_gate_tscale", FAKE.value + 2)):  # a matrix-scale pointer must be 4-byte aligned
+        vals = [FAKE.value] * nf
+        vals[names.index(field)] = value
+        bad = moe._WeightsNVFP4(*vals)
+        assert lib.moe_expert_ffn_nvfp4(ctypes.byref(c), *args, ctypes.byref(bad), FAKE, FAKE, ws_bytes,
+                                        None) == -1, field
+    assert lib.moe_expert_ffn_nvfp4(ctypes.byref(c), *args, ctypes.byref(full), FAKE, FAKE, ws_bytes - 1,
+                                    None) == -3
+    # a shared expert needs its codes, block scales and matrix scales
+    cs = _cfg(shared_intermediate_size=128)
+    ws_s = lib.moe_workspace_bytes(ctypes.byref(cs), 16)
+    vals = [FAKE.value] * nf
+    vals[names.index("ws_tscale")] = None
+    noscale = moe._WeightsNVFP4(*vals)
+    assert lib.moe_expert_ffn_nvfp4(ctypes.byref(cs), *args[:-1], FAKE, ctypes.byref(noscale), FAKE, FAKE, ws_s,
+                                    None) == -1
+    assert lib.moe_forward_nvfp4(ctypes.byref(c), 0, None, None, ctypes.byref(full), None, None, None, 0, None) == 0
