@@ -78,11 +78,11 @@ def stage_work(cfg, counts, wfmt: str = "bf16"):
     """Algorithmic flops and HBM bytes per launch of each stage.
 
     Bytes count what a kernel must move at least once: the touched experts'
-    weights (2 bytes a weight in bf16; 1 + 1/32 in MXFP8: a code and its
-    share of a block scale), its input activations and its output; flops
-    are 2 per MAC."""
+    weights (2 bytes a weight in bf16; 1 + 1/32 in MXFP8 and 1/2 + 1/16 in
+    NVFP4: a code and its share of a block scale), its input activations and
+    its output; flops are 2 per MAC."""
     H, I, Is, T, k, E = cfg.H, cfg.I, cfg.Is, cfg.T, cfg.k, cfg.E
-    wb = 2.0 if wfmt == "bf16" else 1.0 + 1.0 / 32
+    wb = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}[wfmt]
     touched = int(sum(1 for c in counts if c > 0))
     slots = int(sum(counts))
     sh = 1 if Is else 0
@@ -308,11 +308,22 @@ def host_inputs(cfg, inp, max_rows: int, wfmt: str = "bf16"):
     """Host copies for the oracle: x, logits, and the weights -- all experts
     when they fit in 2 GB, else only the experts the first max_rows sample
     rows route to (routing after the budget is a subset of routing before).
-    MXFP8: every expert matrix as the oracle's MXFP8 weights (quantised and
-    dequantised by the oracle, once, before any timing)."""
+    MXFP8 / NVFP4: every expert matrix as the oracle's MXFP8 / NVFP4 weights
+    (quantised by the oracle, once, before any timing; NVFP4's matrix scales
+    go to the oracle as its output factors)."""
+    import numpy as np
     import oracle
     from routed_expert_ffn_renorm_b200 import workloads as W
-    bits = W.bf16_bits if wfmt == "bf16" else (lambda t: oracle.mxfp8_weights(W.bf16_bits(t)))
+    scaled = {}  # NVFP4: matrix name -> {expert: matrix scale}
+
+    def bits(t, name=None, e=None):
+        if wfmt == "bf16":
+            return W.bf16_bits(t)
+        if wfmt == "mxfp8":
+            return oracle.mxfp8_weights(W.bf16_bits(t))
+        v, st = oracle.nvfp4_weights(W.bf16_bits(t))
+        scaled.setdefault(name, {})[e] = float(st)
+        return v
     x = W.bf16_bits(inp.x)
     if cfg.router_proj:  # the projection's logits, computed once before the timed oracle runs
         logits = oracle.router_logits(x, W.bf16_bits(inp.w_router))
@@ -323,20 +334,29 @@ def host_inputs(cfg, inp, max_rows: int, wfmt: str = "bf16"):
     else:
         idx, _ = oracle.route(logits, cfg.k, cfg.norm_topk)
         need = sorted(set(idx[sample_order(cfg.T)[:max_rows]].ravel().tolist()))
-        wg = {e: bits(inp.w_gate[e]) for e in need}
-        wu = {e: bits(inp.w_up[e]) for e in need}
-        wd = {e: bits(inp.w_down[e]) for e in need}
+        wg = {e: bits(inp.w_gate[e], "g", e) for e in need}
+        wu = {e: bits(inp.w_up[e], "u", e) for e in need}
+        wd = {e: bits(inp.w_down[e], "d", e) for e in need}
     shared = {}
     if cfg.Is:
-        shared = dict(ws_gate=bits(inp.ws_gate), ws_up=bits(inp.ws_up),
-                      ws_down=bits(inp.ws_down), ws_gvec=W.bf16_bits(inp.ws_gvec))
+        shared = dict(ws_gate=bits(inp.ws_gate, "sg", 0), ws_up=bits(inp.ws_up, "su", 0),
+                      ws_down=bits(inp.ws_down, "sd", 0), ws_gvec=W.bf16_bits(inp.ws_gvec))
+    if wfmt == "nvfp4":
+        sc = np.ones((cfg.E, 3))
+        for j, name in enumerate("gud"):
+            for e, v in scaled.get(name, {}).items():
+                sc[e, j] = v
+        shared["scales"] = sc
+        if cfg.Is:
+            shared["shared_scales"] = np.array([scaled["sg"][0], scaled["su"][0], scaled["sd"][0]])
     return x, logits, wg, wu, wd, shared
 
 
 def cpu_max_rows(cfg, wfmt: str = "bf16") -> int:
     """Largest CPU sample: the whole batch for small layers, 16 rows when the
-    expert weights do not fit a 2 GB host copy; with MXFP8 weights (which the
-    oracle quantises itself, about a second per expert matrix) 2 rows."""
+    expert weights do not fit a 2 GB host copy; with MXFP8 or NVFP4 weights
+    (which the oracle quantises itself, about a second per expert matrix) 2
+    rows."""
     if wfmt != "bf16":
         return min(cfg.T, 2)
     return cfg.T if 3 * cfg.E * cfg.H * cfg.I * 2 <= (2 << 30) else min(cfg.T, 16)
@@ -381,14 +401,16 @@ def run_ours(args, cfg):
     pc = ctypes.byref(c._c())
     wts = moe.MoEWeights(inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up, inp.ws_down, inp.ws_gvec,
                          inp.w_router)
-    mx = args.weights == "mxfp8"
-    if mx:  # the weight pack step, once, before anything is timed
-        wts = moe.pack_mxfp8(wts)
+    fmt = args.weights
+    if fmt != "bf16":  # the weight pack step, once, before anything is timed
+        wts = moe.pack_mxfp8(wts) if fmt == "mxfp8" else moe.pack_nvfp4(wts)
         torch.cuda.synchronize(dev)
     wts_c = wts._c()
     pw = ctypes.byref(wts_c)
-    ffn_fn = lib.moe_expert_ffn_mxfp8 if mx else lib.moe_expert_ffn
-    fwd_fn = lib.moe_forward_mxfp8 if mx else lib.moe_forward
+    sfx = "" if fmt == "bf16" else "_" + fmt
+    ffn_fn = getattr(lib, "moe_expert_ffn" + sfx)
+    fwd_fn = getattr(lib, "moe_forward" + sfx)
+    fwd_py = getattr(moe, "moe_forward" + sfx)
     p = {n: P(t.data_ptr()) for n, t in dict(idx=idx, tw=tw, sgate=sgate, keff=keff, kept=kept, nd=nd,
                                                 counts=counts, offsets=offsets, perm=perm, slot_pos=slot_pos,
                                                 x_perm=x_perm, ybuf=ybuf, out=out, ws=ws, x=inp.x,
@@ -539,8 +561,7 @@ def run_ours(args, cfg):
             xd.copy_(xh, non_blocking=True)
             if not cfg.router_proj:  # else the layer computes its logits from x
                 ld.copy_(lh, non_blocking=True)
-            (moe.moe_forward_mxfp8 if mx else moe.moe_forward)(c, xd, None if cfg.router_proj else ld, wts, out, ws,
-                                                               stream=st)
+            fwd_py(c, xd, None if cfg.router_proj else ld, wts, out, ws, stream=st)
             oh.copy_(out, non_blocking=True)
             e1.record(st)
 
@@ -575,7 +596,7 @@ def run_ours(args, cfg):
     # the power cap held the clocks down during the timed region
     long_run = (total_ms * 1e-3) > 1.0 or "sw_power_cap" in sampler.summary().get("reasons", [])
     rl = roofline(dom, work, per_stage[dom], peaks, peak_kind, long_run,
-                  recorded_traffic(dom, cfg.label + (":mxfp8" if mx else "")))
+                  recorded_traffic(dom, cfg.label + ("" if fmt == "bf16" else ":" + fmt)))
     layer_bw = work["layer"]["bytes"] / (step_ms * 1e-3) / 1e9
     layer_tf = work["layer"]["flops"] / (step_ms * 1e-3) / 1e12
 
@@ -593,8 +614,11 @@ def run_ours(args, cfg):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded N(0,0.02) bf16 x and weights, N(0,1) fp32 router logits + Zipf popularity bias"
-                + ("; expert weights packed to MXFP8 (E4M3 codes + UE8M0 scales per 32) by the library's quantiser"
-                   if mx else ""),
+                + {"bf16": "",
+                   "mxfp8": "; expert weights packed to MXFP8 (E4M3 codes + UE8M0 scales per 32) by the library's "
+                            "quantiser",
+                   "nvfp4": "; expert weights packed to NVFP4 (E2M1 codes + E4M3 scales per 16 + an fp32 scale per "
+                            "matrix) by the library's quantiser"}[fmt],
         "config": {**workload_desc(cfg), "expert_weights": args.weights,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": rl, "cpu_baseline": cpu, "e2e": e2e,
@@ -679,9 +703,10 @@ def main(argv=None):
                     help="override the number of routed experts (a scaled stand-in of a workload for ncu captures)")
     ap.add_argument("--router-proj", action="store_true",
                     help="compute the logits with the router projection x . W_r^T inside the layer")
-    ap.add_argument("--weights", choices=["bf16", "mxfp8"], default="bf16",
-                    help="expert weight format: bf16, or MXFP8 (E4M3 codes + a power-of-two scale per 32 weights, "
-                         "converted to bf16 on chip; half the weight bytes)")
+    ap.add_argument("--weights", choices=["bf16", "mxfp8", "nvfp4"], default="bf16",
+                    help="expert weight format: bf16; MXFP8 (E4M3 codes + a power-of-two scale per 32 weights, "
+                         "converted to bf16 on chip; half the weight bytes); NVFP4 (E2M1 codes + an E4M3 scale per "
+                         "16 weights + an fp32 scale per matrix; a quarter of the weight bytes)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
