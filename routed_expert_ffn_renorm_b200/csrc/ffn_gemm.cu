@@ -84,7 +84,10 @@ constexpr int kBlockK = 64;                    // K elements per step (128 B row
 constexpr int kTileM = 128;                    // weight rows per tile (MMA M)
 constexpr int kABytes = kTileM * kBlockK * 2;  // 16 KB
 constexpr int kNumBox = 5;                     // token box heights 16 << i
-constexpr int kThreads = 192;                  // bf16 weights: producer, MMA, 4 epilogue warps
+// Warps: 0 producer (weights), 1 MMA issuer, 2..5 epilogue, 6 token loader
+// (single CTAs), then the converters of block-scaled weights.
+constexpr int kThreads = 224;
+constexpr int kLoadWarp = 6;
 // Block-scaled weights (kFmt 1: MXFP8, 2: NVFP4): converter warps after the
 // epilogue warps turn each ring step's codes into the bf16 A operand in
 // tensor memory.  A ring step covers 128 K of a 128-row weight tile: its
@@ -118,6 +121,16 @@ struct PhaseMaps {
     CUtensorMap s0, s1;       // shared A: gate/up ws_gate, ws_up [Is, H]; down ws_down [H, Is] (s1 unused)
     CUtensorMap b[kNumBox];   // routed activations [T*k, K], box heights 16 << i
     CUtensorMap bs[kNumBox];  // shared activations [T, K]
+};
+
+// The token copies of one ring step, which the producer hands the loader warp
+// (single CTAs): n slices of `map` at (x + 64 j, y) into dst + j * dst_step.
+struct LoadDesc {
+    const CUtensorMap *map;
+    uint32_t dst, dst_step;
+    int x, y;
+    int n;
+    int fence;  // 1: the slices are h rows other CTAs wrote (a proxy fence first)
 };
 
 struct __align__(64) FfnMaps {
@@ -597,7 +610,8 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     uint64_t *qfull = tfull + 5, *qempty = qfull + kQueue;
     // MXFP8: conversion buffer (in TMEM) converted / free
     uint64_t *cfull = qempty + kQueue, *cempty = cfull + kConvBufs;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cempty + kConvBufs);
+    uint64_t *armed = cempty + kConvBufs;  // [kTickets] single CTAs: a step's token copies handed to the loader
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(armed + kTickets);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // elected -> epilogue: 0 go, -1 stop
     ItemSlot *qdesc = reinterpret_cast<ItemSlot *>(tmem_slot + 4);  // [kQueue], written by the producer
@@ -607,6 +621,10 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
         (reinterpret_cast<uintptr_t>(conv_desc + 2) + 7) & ~uintptr_t(7));
     uint32_t *ready_bits = reinterpret_cast<uint32_t *>(scan_tmp + 2 * NT);  // [kReadyWords], producer-private
     uint32_t *ticket_start = ready_bits + kReadyWords;  // [kTickets] first ring page (virtual) of each step; producer-private
+    LoadDesc *ldesc = reinterpret_cast<LoadDesc *>(                    // [kTickets] producer -> loader
+        (reinterpret_cast<uintptr_t>(ticket_start + kTickets) + 7) & ~uintptr_t(7));
+    volatile int *stop_at = reinterpret_cast<volatile int *>(ldesc + kTickets);  // steps the producer armed, at its exit
+    volatile int *loader_done = stop_at + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tmem_cols = kFmt ? 512 : 2 * p.BN;  // MXFP8: accumulators, then the conversion buffers
@@ -618,7 +636,10 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
         for (int s = 0; s < kTickets; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&armed[s], 1);
         }
+        *stop_at = 0x7fffffff;
+        *loader_done = 0;
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], kPair ? 2 : 1);  // pair: both CTAs' epilogues
@@ -844,9 +865,9 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                         // gate/up: the up rows' scales; down: the tile's second 64-row group
                         bulk_load(sS + kRun, it.ph == 0 ? sfp[1] + (rg * ksteps + ks) * kRun : sfp[0] + ((rg + 1) * ksteps + ks) * kRun,
                                   kRun, &full[tk]);
-                        uint8_t *sB = sS + kPageBytes;
-                        tma_load_2d(mb, &full[tk], sB, kx, it.row0);
-                        tma_load_2d(mb, &full[tk], sB + sh.sub_pages * kPageBytes, kx + kBlockK, it.row0);
+                        // the two token slices: the loader's
+                        ldesc[tk] = LoadDesc{mb, smem_u32(sS + kPageBytes), sh.sub_pages * kPageBytes, kx, it.row0, 2,
+                                             it.ph == 1};
                     } else if constexpr (kPair) {
                         // both CTAs' loads complete on CTA 0's barrier, armed there with both halves
                         if (rank == 0) mbar_arrive_expect_tx(&full[tk], 2 * need * kPageBytes);
@@ -875,12 +896,27 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                                 if (it.m == 2)
                                     tma_load_2d_hint(ma0, &full[tk], sA + kABytes, kx, a_row + kTileM, apol);
                             }
-                            tma_load_2d(mb, &full[tk], sA + it.m * kABytes, kx, it.row0);
                         }
+                        // the token slice of every sub-step: the loader's
+                        ldesc[tk] = LoadDesc{mb, smem_u32(ring + (size_t)first * kPageBytes + it.m * kABytes),
+                                             sh.sub_pages * kPageBytes, k0 * kBlockK, it.row0, nsub, it.ph == 1};
                     }
+                    if constexpr (!kPair) mbar_arrive(&armed[tk]);  // after the full barrier is armed
                     ++issued;
                 }
                 if (!ok) break;
+            }
+            if constexpr (!kPair) {
+                // the loader stops at the first step never armed; its copies of the
+                // armed ones are issued once it says so (bounded wait)
+                *stop_at = (int)issued;
+                const unsigned long long t0 = globaltimer();
+                while (!*loader_done)
+                    if (globaltimer() - t0 > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        atomicOr(p.status, MOE_STATUS_TIMEOUT);
+                        break;
+                    }
             }
             // wait for every copy still in flight before the CTA may exit (pair: the
             // copies complete on CTA 0's barrier; the MMAs that consumed them release
@@ -980,8 +1016,42 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
             else umma_commit(mma_done);
             mbar_wait(mma_done, 0, abort_flag, p.status, false);
         }
-    } else if (kFmt != 0 && warp >= 6) {
-        // ================= MXFP8 converters (warps 6 ..) =================
+    } else if (warp == kLoadWarp) {
+        // ================= token loader (single CTAs) =================
+        // Issues the token copies of every ring step, in step order, once the
+        // producer has armed the step's full barrier and described them: one
+        // thread issuing a TMA copy costs it ~40-50 ns, so at decode sizes the
+        // copies of a step, not HBM, would set the pace of a single producer.
+        // It stops at the first step the producer never armed (stop_at, set
+        // when the producer leaves), so that every armed step's copies are
+        // issued and the producer's final drain sees them all land.
+        if (!kPair && lane == 0) {
+            for (uint32_t step = 0;; ++step) {
+                const uint32_t tk = step % kTickets, par = (step / kTickets) & 1u;
+                bool go = false;
+                const unsigned long long t0 = globaltimer();
+                for (uint32_t spin = 0;; ++spin) {
+                    if (mbar_try_wait(&armed[tk], par)) {
+                        go = true;
+                        break;
+                    }
+                    if ((int)step >= *stop_at) break;
+                    if ((spin & 63u) == 63u && globaltimer() - t0 > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        atomicOr(p.status, MOE_STATUS_TIMEOUT);
+                        break;
+                    }
+                }
+                if (!go) break;
+                const LoadDesc d = ldesc[tk];
+                if (d.fence) fence_proxy_async_global();  // h written by other CTAs (the producer saw it ready)
+                for (int j = 0; j < d.n; ++j)
+                    tma_load_2d_s(d.map, &full[tk], d.dst + (uint32_t)j * d.dst_step, d.x + j * kBlockK, d.y);
+            }
+            *loader_done = 1;
+        }
+    } else if (kFmt != 0 && warp > kLoadWarp) {
+        // ================= MXFP8 converters (warps 7 ..) =================
         // Two groups of kConvWarps / 2 warps take alternate steps, so that one
         // group's conversion overlaps the other's loads and TMEM stores.  Each
         // group walks the producer's step sequence: once one of its steps' codes
@@ -1192,8 +1262,9 @@ int pick_bns(const FfnArgs &a, int bn, int sms) {
 size_t smem_bytes_for(int E, int pages, int fmt) {
     const int nt = fmt ? kThreadsQ : kThreads;
     return 1024 + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 +
-           3 * (size_t)(E + 1) * 4 + 8 + (size_t)(2 * kTickets + 5 + 2 * kQueue + 2 * kConvBufs) * 8 + 16 +
-           (kQueue + 3) * sizeof(ItemSlot) + 8 + 2 * (size_t)nt * 4 + kReadyWords * 4 + kTickets * 4;
+           3 * (size_t)(E + 1) * 4 + 8 + (size_t)(3 * kTickets + 5 + 2 * kQueue + 2 * kConvBufs) * 8 + 16 +
+           (kQueue + 3) * sizeof(ItemSlot) + 8 + 2 * (size_t)nt * 4 + kReadyWords * 4 + kTickets * 4 + 8 +
+           kTickets * sizeof(LoadDesc) + 8;
 }
 
 int min_pages(int fmt) { return fmt == 2 ? 4 + 1 + 2 * (256 * 128 / 2048) : fmt ? kQMaxStepPages : kMaxStepPages; }
