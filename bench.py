@@ -30,6 +30,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import sys
 import threading
 import time
@@ -135,11 +136,18 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:  # the grouped FFN kernel's source
-    h = hashlib.sha256()
-    with open(os.path.join(ROOT, "routed_expert_ffn_renorm_b200", "csrc", "ffn_gemm.cu"), "rb") as f:
-        h.update(f.read())
-    return h.hexdigest()[:16]
+def code_hash(text: str) -> str:
+    """sha256 prefix of C++/CUDA source with its comments and blank lines
+    removed: what a recorded measurement depends on."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
+def kernel_source_hash() -> str:  # the grouped FFN kernel's code
+    with open(os.path.join(ROOT, "routed_expert_ffn_renorm_b200", "csrc", "ffn_gemm.cu")) as f:
+        return code_hash(f.read())
 
 
 def recorded_traffic(kernel: str, workload: str):

@@ -48,9 +48,11 @@
 // (32 KB of weights per barrier round trip), and their loops avoid divisions
 // and out-of-line calls on the common path.
 //
-// Roles (192 threads, one CTA per SM, persistent): warp 0 -- TMA producer
-// (one lane); warp 1 -- TMEM allocation and MMA issue (one lane); warps
-// 2..5 -- epilogue, one TMEM lane quarter each.
+// Roles (224 threads, one CTA per SM, persistent): warp 0 -- TMA producer
+// (one lane; the weight boxes, and all copies of a CTA pair); warp 1 -- TMEM
+// allocation and MMA issue (one lane); warps 2..5 -- epilogue, one TMEM lane
+// quarter each; warp 6 -- the token loader of single CTAs (one lane).
+// Block-scaled weights add eight converter warps (480 threads).
 //
 // Work items are handed out dynamically (a global counter, claimed one item
 // ahead) in the order phase 0 [shared expert, routed experts ascending],
@@ -384,10 +386,11 @@ __device__ __forceinline__ StepShape step_shape(const Item &it, const FfnParams 
     return sh;
 }
 
-// MXFP8 ring step: 128 K elements -- the codes of one weight tile (8 pages),
-// their scales (one page, 512 bytes used) and the token rows as two bf16
-// boxes of 64 K (sub_pages = 2^bi pages each).  ns = 2 slices, nk counts
-// 64-wide slices (even: K is a multiple of 128).
+// Block-scaled ring step: 128 K elements -- the codes of one weight tile
+// (MXFP8 8 pages, NVFP4 4), their scales (one page: 512 or 1024 bytes used)
+// and the token rows as two bf16 boxes of 64 K (sub_pages = 2^bi pages
+// each).  ns = 2 slices, nk counts 64-wide slices (even: K is a multiple of
+// 128).
 __device__ __forceinline__ StepShape qstep_shape(const Item &it, const FfnParams &p) {
     StepShape sh;
     sh.bi = box_index(it.nvalid);
@@ -608,7 +611,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     uint64_t *full = bars, *empty = bars + kTickets, *tfull = bars + 2 * kTickets, *tempty = tfull + 2;
     uint64_t *mma_done = tfull + 4;
     uint64_t *qfull = tfull + 5, *qempty = qfull + kQueue;
-    // MXFP8: conversion buffer (in TMEM) converted / free
+    // block-scaled weights: conversion buffer (in TMEM) converted / free
     uint64_t *cfull = qempty + kQueue, *cempty = cfull + kConvBufs;
     uint64_t *armed = cempty + kConvBufs;  // [kTickets] single CTAs: a step's token copies handed to the loader
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(armed + kTickets);
@@ -627,7 +630,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     volatile int *loader_done = stop_at + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tmem_cols = kFmt ? 512 : 2 * p.BN;  // MXFP8: accumulators, then the conversion buffers
+    const int tmem_cols = kFmt ? 512 : 2 * p.BN;  // block-scaled weights: accumulators, then the conversion buffers
     const uint32_t rank = kPair ? cluster_ctarank() : 0u;  // 0: the pair's MMA issuer
     pdl_launch_dependents();
 
@@ -648,7 +651,8 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
         for (int q = 0; q < kQueue; ++q) {
             mbar_init(&qfull[q], 1);
             // the MMA lane and the elected epilogue thread (pair: and the other CTA's
-            // producer and epilogue; MXFP8: and the two converter groups' elected threads)
+            // producer and epilogue; block-scaled weights: and the two converter groups'
+            // elected threads)
             mbar_init(&qempty[q], kPair ? 4 : (kFmt ? 4 : 2));
         }
         for (int b = 0; b < kConvBufs; ++b) {
@@ -1051,7 +1055,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
             *loader_done = 1;
         }
     } else if (kFmt != 0 && warp > kLoadWarp) {
-        // ================= MXFP8 converters (warps 7 ..) =================
+        // ================= block-scaled weight converters (warps 7 ..) =================
         // Two groups of kConvWarps / 2 warps take alternate steps, so that one
         // group's conversion overlaps the other's loads and TMEM stores.  Each
         // group walks the producer's step sequence: once one of its steps' codes
@@ -1243,9 +1247,8 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
 // shared-memory cost follows its real token count (the paged ring), so a
 // wide tile costs nothing for small groups and saves re-reading a weight
 // tile for every 128 tokens of large ones.
-// MXFP8 weights: 128, so that a ring step (codes, scales, two token boxes)
-// stays at 25 pages and the smaller ring that the conversion buffers leave
-// still holds three of them.
+// Block-scaled weights: 128, so that the two accumulators end where the
+// conversion buffers start in tensor memory (column 256).
 int pick_bn(int fmt) { return fmt ? 128 : 256; }
 
 // Token tile of the shared expert, which sees all T tokens.  One 256-token
@@ -1296,7 +1299,7 @@ DeviceInfo device_info() {
 // Benchmark/test overrides: MOE_FORCE_BN and MOE_FORCE_BNS in {32, 64, 128,
 // 256} (routed / shared token tile, BNS <= BN) and MOE_FORCE_PAGES in
 // [24, 112] (ring size in 2 KB pages, capped by shared memory; 24 holds one
-// widest K step; 41 with MXFP8 weights); any other value is rejected.
+// widest K step; 41 with block-scaled weights); any other value is rejected.
 int parse_tile(const char *f, int *out) {
     char *end = nullptr;
     const long v = strtol(f, &end, 10);
