@@ -126,13 +126,17 @@ struct PhaseMaps {
 };
 
 // The token copies of one ring step, which the producer hands the loader warp
-// (single CTAs): n slices of `map` at (x + 64 j, y) into dst + j * dst_step.
+// (single CTAs): n slices of `map` at (x + 64 j, y) into dst + j * dst_step;
+// with block-scaled weights also the step's two runs of block scales,
+// sc_bytes each from sc_src[i] to sc_dst + i * sc_bytes.
 struct LoadDesc {
     const CUtensorMap *map;
+    const uint8_t *sc_src[2];
     uint32_t dst, dst_step;
     int x, y;
     int n;
     int fence;  // 1: the slices are h rows other CTAs wrote (a proxy fence first)
+    uint32_t sc_dst, sc_bytes;  // sc_bytes 0: no scale runs
 };
 
 struct __align__(64) FfnMaps {
@@ -612,8 +616,10 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
     uint64_t *mma_done = tfull + 4;
     uint64_t *qfull = tfull + 5, *qempty = qfull + kQueue;
     // block-scaled weights: conversion buffer (in TMEM) converted / free
-    uint64_t *cfull = qempty + kQueue, *cempty = cfull + kConvBufs;
-    uint64_t *armed = cempty + kConvBufs;  // [kTickets] single CTAs: a step's token copies handed to the loader
+    // block-scaled weights: TMEM conversion buffer converted (a buffer is free again
+    // once the MMAs of the last step that used it are done: that step's empty barrier)
+    uint64_t *cfull = qempty + kQueue;
+    uint64_t *armed = cfull + kConvBufs;  // [kTickets] single CTAs: a step's token copies handed to the loader
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(armed + kTickets);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // elected -> epilogue: 0 go, -1 stop
@@ -655,10 +661,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
             // elected threads)
             mbar_init(&qempty[q], kPair ? 4 : (kFmt ? 4 : 2));
         }
-        for (int b = 0; b < kConvBufs; ++b) {
-            mbar_init(&cfull[b], kConvWarps / 2);  // one arrival per warp of the converting group
-            mbar_init(&cempty[b], 1);          // the MMA lane's commit
-        }
+        for (int b = 0; b < kConvBufs; ++b) mbar_init(&cfull[b], kConvWarps / 2);  // one arrival per warp of the converting group
         *abort_flag = 0;
         for (int w = 0; w < kReadyWords; ++w) ready_bits[w] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -865,13 +868,21 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                         const size_t ksteps = (size_t)(sh.nk >> 1);
                         const size_t rg = (size_t)(a_row >> 6);  // 64-row group of the tile's first row
                         const uint8_t *const *sfp = it.shared ? p.sfs[it.ph] : p.sf[it.ph];
-                        bulk_load(sS, sfp[0] + (rg * ksteps + ks) * kRun, kRun, &full[tk]);
-                        // gate/up: the up rows' scales; down: the tile's second 64-row group
-                        bulk_load(sS + kRun, it.ph == 0 ? sfp[1] + (rg * ksteps + ks) * kRun : sfp[0] + ((rg + 1) * ksteps + ks) * kRun,
-                                  kRun, &full[tk]);
-                        // the two token slices: the loader's
-                        ldesc[tk] = LoadDesc{mb, smem_u32(sS + kPageBytes), sh.sub_pages * kPageBytes, kx, it.row0, 2,
-                                             it.ph == 1};
+                        // the two runs of block scales (gate/up: the gate and the up rows;
+                        // down: the tile's two 64-row groups) and the two token slices:
+                        // the loader's
+                        ldesc[tk] = LoadDesc{mb,
+                                             {sfp[0] + (rg * ksteps + ks) * kRun,
+                                              it.ph == 0 ? sfp[1] + (rg * ksteps + ks) * kRun
+                                                         : sfp[0] + ((rg + 1) * ksteps + ks) * kRun},
+                                             smem_u32(sS + kPageBytes),
+                                             sh.sub_pages * kPageBytes,
+                                             kx,
+                                             it.row0,
+                                             2,
+                                             it.ph == 1,
+                                             smem_u32(sS),
+                                             (uint32_t)kRun};
                     } else if constexpr (kPair) {
                         // both CTAs' loads complete on CTA 0's barrier, armed there with both halves
                         if (rank == 0) mbar_arrive_expect_tx(&full[tk], 2 * need * kPageBytes);
@@ -902,8 +913,16 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                             }
                         }
                         // the token slice of every sub-step: the loader's
-                        ldesc[tk] = LoadDesc{mb, smem_u32(ring + (size_t)first * kPageBytes + it.m * kABytes),
-                                             sh.sub_pages * kPageBytes, k0 * kBlockK, it.row0, nsub, it.ph == 1};
+                        ldesc[tk] = LoadDesc{mb,
+                                             {nullptr, nullptr},
+                                             smem_u32(ring + (size_t)first * kPageBytes + it.m * kABytes),
+                                             sh.sub_pages * kPageBytes,
+                                             k0 * kBlockK,
+                                             it.row0,
+                                             nsub,
+                                             it.ph == 1,
+                                             0u,
+                                             0u};
                     }
                     if constexpr (!kPair) mbar_arrive(&armed[tk]);  // after the full barrier is armed
                     ++issued;
@@ -957,7 +976,10 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                     const uint32_t first =
                         ring_alloc(vhead, off, kFmt ? qstep_pages<kFmt>(sh) : (uint32_t)nsub * sh.sub_pages, P);
                     const uint32_t tk = step % kTickets;
-                    if (!mbar_wait_fast<kPair>(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true)) {
+                    // block-scaled weights: the converters arrive only after this step's full
+                    // barrier (codes, scales and tokens), so their barrier stands for both
+                    if (kFmt == 0 &&
+                        !mbar_wait_fast<kPair>(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true)) {
                         ok = false;
                         break;
                     }
@@ -980,8 +1002,7 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                                 umma_bf16_ts(d, ta + (uint32_t)(j * 32 + kk * 8), dbj + 2 * kk, idesc,
                                              (k0 | j | kk) != 0);
                         }
-                        umma_commit(&empty[tk]);  // the ring pages (codes, scales, tokens)
-                        umma_commit(&cempty[cb]);  // the conversion buffer
+                        umma_commit(&empty[tk]);  // the ring pages (codes, scales, tokens) and the TMEM buffer
                         ++step;
                         continue;
                     }
@@ -1051,6 +1072,8 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 if (d.fence) fence_proxy_async_global();  // h written by other CTAs (the producer saw it ready)
                 for (int j = 0; j < d.n; ++j)
                     tma_load_2d_s(d.map, &full[tk], d.dst + (uint32_t)j * d.dst_step, d.x + j * kBlockK, d.y);
+                for (int i = 0; i < 2 && d.sc_bytes; ++i)
+                    bulk_load_s(d.sc_dst + (uint32_t)i * d.sc_bytes, d.sc_src[i], d.sc_bytes, &full[tk]);
             }
             *loader_done = 1;
         }
@@ -1098,8 +1121,14 @@ __global__ void __launch_bounds__(kFmt ? kThreadsQ : kThreads, 1)
                 const uint32_t first = ring_alloc(vhead, off, need, P);
                 if ((step & 1u) != g) continue;  // the other group's step
                 const uint32_t tk = step % kTickets, cb = step % kConvBufs;
+                // TMEM buffer cb is free once the MMAs of step - kConvBufs, its last user, are
+                // done: that step's empty barrier.  It cannot have completed another phase
+                // since: that takes the MMAs of step - kConvBufs + kTickets, which this group
+                // converts after this one.
+                const uint32_t prev = step - kConvBufs;
                 ok = mbar_wait_fast(&full[tk], (step / kTickets) & 1u, abort_flag, p.status, true) &&
-                     mbar_wait_fast(&cempty[cb], ((step / kConvBufs) & 1u) ^ 1u, abort_flag, p.status, true);
+                     (step < kConvBufs ||
+                      mbar_wait_fast(&empty[prev % kTickets], (prev / kTickets) & 1u, abort_flag, p.status, true));
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const uint32_t codes = smem_u32(ring + (size_t)first * kPageBytes);
@@ -1265,7 +1294,7 @@ int pick_bns(const FfnArgs &a, int bn, int sms) {
 size_t smem_bytes_for(int E, int pages, int fmt) {
     const int nt = fmt ? kThreadsQ : kThreads;
     return 1024 + (size_t)pages * kPageBytes + 64 * kXchgStride * 4 +
-           3 * (size_t)(E + 1) * 4 + 8 + (size_t)(3 * kTickets + 5 + 2 * kQueue + 2 * kConvBufs) * 8 + 16 +
+           3 * (size_t)(E + 1) * 4 + 8 + (size_t)(3 * kTickets + 5 + 2 * kQueue + kConvBufs) * 8 + 16 +
            (kQueue + 3) * sizeof(ItemSlot) + 8 + 2 * (size_t)nt * 4 + kReadyWords * 4 + kTickets * 4 + 8 +
            kTickets * sizeof(LoadDesc) + 8;
 }
