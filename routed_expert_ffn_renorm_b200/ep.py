@@ -25,6 +25,11 @@ GPU test runs two ranks on one GPU, exchanging in process).  The batch-union
 expert budget couples every rank's tokens and is not supported here
 (budget must be 0); the top-p trim is per token and is.
 
+The weights may be bf16 (MoEWeights) or block-scaled (MoEWeightsMXFP8,
+MoEWeightsNVFP4): the expert FFN calls are then the matching
+moe_expert_ffn_mxfp8 / moe_expert_ffn_nvfp4, and the output is
+moe_forward_mxfp8's / moe_forward_nvfp4's, bit for bit.
+
 The stage methods (dispatch, experts, combine) do no communication; forward()
 puts the exchanges between them.  `exchange` is the only function that talks
 to other ranks.
@@ -34,8 +39,14 @@ from __future__ import annotations
 from dataclasses import dataclass
 from typing import List, Optional, Sequence
 
-from . import (MoEConfig, MoEWeights, moe_combine, moe_dispatch, moe_ep_pack, moe_ep_rank_ids, moe_ep_unpack,
-               moe_expert_ffn, moe_route, workspace_bytes)
+import dataclasses
+
+from . import (MoEConfig, MoEWeights, MoEWeightsMXFP8, MoEWeightsNVFP4, moe_combine, moe_dispatch, moe_ep_pack,
+               moe_ep_rank_ids, moe_ep_unpack, moe_expert_ffn, moe_expert_ffn_mxfp8, moe_expert_ffn_nvfp4, moe_route,
+               workspace_bytes)
+
+# the expert FFN entry point of each weight type
+_FFN = {MoEWeights: moe_expert_ffn, MoEWeightsMXFP8: moe_expert_ffn_mxfp8, MoEWeightsNVFP4: moe_expert_ffn_nvfp4}
 
 
 def exchange(send_counts: Sequence[int], tensors: Sequence["torch.Tensor"], group=None):
@@ -89,16 +100,21 @@ class EPLayer:
     """One rank's share of an expert-parallel routed-MoE layer.
 
     cfg: the whole layer (E = all routed experts, budget 0).  weights: this
-    rank's routed experts (w_gate, w_up [epr, I, H], w_down [epr, H, I]) and
-    the whole shared expert (and its gate vector), device bf16."""
+    rank's routed experts (w_gate, w_up [epr, I, H], w_down [epr, H, I], or
+    their codes and scales) and the whole shared expert (and its gate
+    vector): MoEWeights, MoEWeightsMXFP8 or MoEWeightsNVFP4 on the device
+    (shard_weights cuts them from a whole layer's)."""
 
-    def __init__(self, cfg: MoEConfig, world: int, rank: int, weights: MoEWeights):
+    def __init__(self, cfg: MoEConfig, world: int, rank: int, weights):
         import torch
         if cfg.budget:
             raise ValueError("the batch-union expert budget spans every rank's tokens; expert parallelism needs budget 0")
         if world < 1 or cfg.n_routed_experts % world:
             raise ValueError("n_routed_experts must be a multiple of the number of ranks")
+        if type(weights) not in _FFN:
+            raise TypeError(f"unsupported weight type {type(weights).__name__}")
         self.cfg, self.world, self.rank, self.weights = cfg, world, rank, weights
+        self._ffn = _FFN[type(weights)]
         self.epr = cfg.n_routed_experts // world
         if weights.w_gate.shape[0] != self.epr:
             raise ValueError(f"this rank holds {self.epr} experts, got {weights.w_gate.shape[0]}")
@@ -171,7 +187,7 @@ class EPLayer:
         ybuf = torch.empty((R, 2, H), dtype=torch.bfloat16, device=dev)
         ws = self._ws(cfg, R)
         moe_dispatch(cfg, idx, counts, offsets, perm, slot_pos, ws, x=rows, x_perm=x_perm)
-        moe_expert_ffn(cfg, rows, x_perm, offsets, perm, w, self.weights, ybuf, ws)
+        self._ffn(cfg, rows, x_perm, offsets, perm, w, self.weights, ybuf, ws)
         moe_combine(cfg, ybuf, out)  # k = 1, no shared expert: row r = ybuf[r, 0], exactly
         return out
 
@@ -192,8 +208,8 @@ class EPLayer:
             ws = self._ws(cs, T)
             zero_off = torch.zeros(self.epr + 1, dtype=torch.int32, device=dev)
             x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
-            moe_expert_ffn(cs, state.x, x_perm, zero_off, state.perm, state.w, self.weights, ybuf, ws,
-                           sgate=state.sgate)
+            self._ffn(cs, state.x, x_perm, zero_off, state.perm, state.w, self.weights, ybuf, ws,
+                      sgate=state.sgate)
         moe_combine(cfg, ybuf, out, keff=state.keff)
         return out
 
@@ -208,11 +224,16 @@ class EPLayer:
         return self.combine(state, back)
 
 
-def shard_weights(weights: MoEWeights, world: int, rank: int) -> MoEWeights:
+def shard_weights(weights, world: int, rank: int):
     """Rank `rank`'s share of a whole layer's weights: its routed experts
-    (contiguous views, no copy) and the whole shared expert."""
+    (contiguous views, no copy) and the whole shared expert.  Works for every
+    weight type: the routed arrays (w_gate, w_up, w_down and, block-scaled,
+    their packed scales and matrix scales) all lead with the expert index --
+    the packed scale layout keeps each expert's rows in a contiguous run of
+    64-row groups, as many bytes as its [I, K / block] slice."""
     E = weights.w_gate.shape[0]
     epr = E // world
     sl = slice(rank * epr, (rank + 1) * epr)
-    return MoEWeights(weights.w_gate[sl], weights.w_up[sl], weights.w_down[sl], weights.ws_gate, weights.ws_up,
-                      weights.ws_down, weights.ws_gate_vec, weights.w_router)
+    routed = {f.name: getattr(weights, f.name)[sl] for f in dataclasses.fields(weights)
+              if f.name.startswith("w_") and f.name != "w_router" and getattr(weights, f.name) is not None}
+    return dataclasses.replace(weights, **routed)

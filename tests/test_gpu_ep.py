@@ -22,10 +22,11 @@ def _blocks(counts):
     return [slice(int(off[i]), int(off[i + 1])) for i in range(len(counts))]
 
 
-def ep_emulated(cfg, inp, world):
-    """The layer through EPLayer on `world` emulated ranks; returns out [T, H]."""
+def ep_emulated(cfg, inp, world, full=None):
+    """The layer through EPLayer on `world` emulated ranks (weights `full`,
+    default the bf16 ones); returns out [T, H]."""
     c = lib_config(cfg)
-    full = weights_of(inp)
+    full = weights_of(inp) if full is None else full
     layers = [EPLayer(c, world, r, shard_weights(full, world, r)) for r in range(world)]
     tok = np.array_split(np.arange(cfg.T), world)
     xs = [inp.x[t[0]:t[-1] + 1].contiguous() if len(t) else inp.x[:0] for t in tok]
@@ -63,6 +64,27 @@ def test_ep_equals_single_gpu_layer(cfg, world):
     out = ep_emulated(cfg, inp, world)
     assert (W.bf16_bits(out) == ref.out_bits).all(), "expert-parallel output differs from moe_forward"
     print(cfg.label, "world", world, check_layer(cfg, inp, ref))
+
+
+CASES_Q = [
+    (W.MoEConfig("ep_q_shared", T=64, H=256, E=8, I=128, k=2, Is=128, zipf_alpha=1.0), 2),
+    (W.MoEConfig("ep_q_four", T=100, H=384, E=16, I=256, k=4), 4),
+]
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "nvfp4"])
+@pytest.mark.parametrize("cfg,world", CASES_Q, ids=[c.name for c, _ in CASES_Q])
+def test_ep_block_scaled_equals_single_gpu_layer(cfg, world, fmt):
+    """Block-scaled expert weights, sharded by expert (codes, packed scales,
+    matrix scales): bit for bit the single-GPU block-scaled layer."""
+    inp = W.make_inputs(cfg, device="cuda")
+    pack = moe.pack_mxfp8 if fmt == "mxfp8" else moe.pack_nvfp4
+    fwd = moe.moe_forward_mxfp8 if fmt == "mxfp8" else moe.moe_forward_nvfp4
+    wq = pack(weights_of(inp))
+    ref = gpu_forward(cfg, inp, weights=wq, fwd=fwd)
+    out = ep_emulated(cfg, inp, world, full=wq)
+    assert ref.status == 0
+    assert (W.bf16_bits(out) == ref.out_bits).all(), "expert-parallel output differs from the single-GPU layer"
 
 
 def test_ep_rejects_budget():
