@@ -70,6 +70,10 @@ typedef uint16_t moe_bf16_t; /* bf16 bit pattern */
                                       an expert id outside [-1, E) in a kept slot, dispatch
                                       offsets not a prefix sum within T*k, a perm entry outside
                                       [0, T*k); the access was skipped, results invalid */
+#define MOE_STATUS_NONFINITE 4     /* checked library only: moe_forward's router logits (given
+                                      or projected) held a NaN or an infinity, outside the
+                                      contract (a softmax over them is undefined); results
+                                      invalid.  moe_route alone has no status word to report it */
 
 typedef struct {
     int32_t hidden;                   /* H */

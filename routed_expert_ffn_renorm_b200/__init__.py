@@ -48,6 +48,7 @@ EXPORTED_SYMBOLS = (
 NOALLOC_SCRATCH_BYTES = 8 << 20  # MOE_NOALLOC_SCRATCH_BYTES
 MOE_STATUS_TIMEOUT = 1
 MOE_STATUS_BOUNDS = 2
+MOE_STATUS_NONFINITE = 4
 
 
 class MoEError(RuntimeError):

@@ -554,6 +554,10 @@ int forward_impl(const moe_config_t *cfg, int32_t T, const moe_bf16_t *x, const 
     moe_bf16_t *ybuf = at<moe_bf16_t>(ws, L.ybuf);
 
     const int E = cfg->n_routed_experts, k = cfg->num_experts_per_tok;
+    if constexpr (kDebugBounds) {  // checked library: non-finite logits are reported, not routed silently
+        rc = cuda_rc(launch_check_logits((long long)T * E, logits, at<int32_t>(ws, L.status), as_stream(stream)));
+        if (rc) return rc;
+    }
     // A small batch with an expert budget: route, budget and dispatch in one launch
     // instead of four.  (Without a budget the separate route and dispatch
     // launches measured faster for the drafter layers.)

@@ -63,6 +63,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Every wrapper enqueues on `st` and returns cudaGetLastError().
 
 // Route (one warp per token).
+// Checked library: sets MOE_STATUS_NONFINITE in *status when any of the n
+// logits is a NaN or an infinity.
+cudaError_t launch_check_logits(long long n, const float *logits, int32_t *status, cudaStream_t st);
 cudaError_t launch_route(int T, int E, int k, int norm_topk, float topp, const float *logits, int32_t *idx,
                          float *w, int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H,
                          float *sgate, cudaStream_t st);

@@ -9,6 +9,8 @@
 // (shared_gate_group), side by side.  route_lane_kernel (32 < E <= 64):
 // separate blocks route 32 tokens lane by lane and compute the gates.  Both read the logits (and
 // x) once; they are latency-bound and small next to the expert FFN.
+#include <algorithm>
+
 #include "front.cuh"
 
 namespace moe {
@@ -87,6 +89,27 @@ cudaError_t launch_v(int T, int E, int k, int norm_topk, float topp, const float
 }
 
 }  // namespace
+
+namespace {
+// One pass over the logits (checked library only): a block that sees a NaN or
+// an infinity sets the status bit once.
+__global__ void __launch_bounds__(256) check_logits_kernel(long long n, const float *__restrict__ logits,
+                                                         int32_t *__restrict__ status) {
+    pdl_wait();
+    bool bad = false;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        bad |= !isfinite(__ldg(logits + i));
+    pdl_launch_dependents();
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, MOE_STATUS_NONFINITE);
+}
+}  // namespace
+
+cudaError_t launch_check_logits(long long n, const float *logits, int32_t *status, cudaStream_t st) {
+    const long long blocks = std::min<long long>((n + 255) / 256, 1184);
+    return launch_pdl(check_logits_kernel, dim3((unsigned)std::max<long long>(blocks, 1)), dim3(256), 0, st, n,
+                      logits, status);
+}
 
 cudaError_t launch_route(int T, int E, int k, int norm_topk, float topp, const float *logits, int32_t *idx, float *w,
                          int32_t *keff, const uint16_t *x, const uint16_t *gvec, int H, float *sgate,

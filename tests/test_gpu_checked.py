@@ -130,6 +130,21 @@ def test_bad_perm_reported(launches, checked):
     assert torch.equal(ybuf.view(-1, cfg.H)[rows].view(torch.int16), ref.view(-1, cfg.H)[rows].view(torch.int16))
 
 
+@pytest.mark.parametrize("bad", [float("nan"), float("inf")])
+def test_nonfinite_logits_reported(bad, checked):
+    """The checked library's moe_forward reports a NaN or infinite router logit
+    (MOE_STATUS_NONFINITE) before routing; a clean call leaves the bit clear."""
+    cfg = W.MoEConfig("bad_logit", T=24, H=256, E=8, I=128, k=2, Is=64)
+    inp = W.make_inputs(cfg, device="cuda")
+    g = gpu_forward(cfg, inp)
+    assert g.status == 0
+    logits = inp.logits.clone()
+    logits[5, 3] = bad
+    g = gpu_forward(cfg, W.MoEInputs(inp.x, logits, inp.w_gate, inp.w_up, inp.w_down, inp.ws_gate, inp.ws_up,
+                                     inp.ws_down, inp.ws_gvec))
+    assert g.status & moe.MOE_STATUS_NONFINITE
+
+
 def test_combine_clamps_keff():
     """moe_combine reads a token's own rows only: keff outside [0, k] counts as
     its nearest end (every build)."""
